@@ -1,0 +1,518 @@
+/*
+ * Oracle for the SmoothQuant-smoothed INT8 W8A8 linear path.
+ *
+ * TEST INFRASTRUCTURE ONLY. This is a plain, slow, single-purpose CPU restatement of
+ * what the path computes, written to be checked against the pages by eye. Only the
+ * test-suite, the smoke check and the benchmark's CPU-baseline leg may load it; the
+ * library never calls it, and it shares no code, header, table or helper with the
+ * CUDA library.
+ *
+ * Arithmetic conventions (a reading where the pages are silent; see the design notes):
+ *   - IEEE binary32 with round-to-nearest-even for every float operation, no FMA
+ *     contraction (built with -ffp-contract=off) except where fmaf() is written out.
+ *   - bf16 values travel as raw 16-bit patterns; widening is exact, narrowing is RN-even.
+ *
+ * Sources (page title, section):
+ *   [P2] "INT8 W8A8 ... using SmoothQuant and GPTQ" (arc-codex article 3619...):
+ *        "At its core, quantizing a weight involves 2 steps" -- scale = max|col|/127,
+ *        q = round(w/scale); "The problem with naive quantization" -- per-channel RTN and
+ *        its worked example; "Why activation quantization is hard" -- one dynamic scale per
+ *        token, worked example [1.32, 0.75, 0.91, 153.0]; "How SmoothQuant prevents
+ *        outliers" -- RMSNorm = divide by RMS then multiply by gamma, gamma folding;
+ *        "How the SmoothQuant smoothing factor is computed" -- s_j from max|A_j|, max|W_j|,
+ *        alpha (formula lost in the extract; the SmoothQuant paper's form is used).
+ *   [P3] "INT8 Post-Training Quantization for LLM Inference on NVIDIA GPUs", section
+ *        "1. Min-Max Calibration" -- S = max(|min|,|max|)/127, range [-127, 127].
+ *   [P4] "W8A8 ... accuracy and serving results" (Red Hat developer article), section
+ *        "Inter-token latency (ITL)" -- per layer: measure the range, compute a scale,
+ *        convert to INT8, multiply, convert back to BF16.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ bf16 <-> f32 */
+
+/* Widen a bf16 bit pattern: the 16 bits are the top half of a binary32. */
+float oracle_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Narrow binary32 to bf16 with round-to-nearest, ties to even. NaN stays NaN. */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0u)
+        return (uint16_t)((u >> 16) | 0x0040u); /* quiet NaN */
+    uint32_t lsb = (u >> 16) & 1u;             /* ties go to the even neighbour */
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------ per-token quantization */
+
+/*
+ * Symmetric per-token quantization of one row of fp32 values [P2 "Why activation
+ * quantization is hard"; P3 "1. Min-Max Calibration"]:
+ *   amax = max_j |y_j|,  s = amax / 127,  q_j = clamp(round_half_even(y_j / s), -127, 127).
+ * An all-zero row has no range; it gets s = 0 and q = 0 (the pages are silent).
+ */
+void oracle_quantize_row_f32(const float *y, int64_t K, int8_t *q, float *s_out)
+{
+    float amax = 0.0f;
+    for (int64_t j = 0; j < K; ++j) {
+        float a = fabsf(y[j]);
+        if (a > amax)
+            amax = a;
+    }
+    if (amax == 0.0f) {
+        *s_out = 0.0f;
+        for (int64_t j = 0; j < K; ++j)
+            q[j] = 0;
+        return;
+    }
+    float s = amax / 127.0f;
+    *s_out = s;
+    for (int64_t j = 0; j < K; ++j) {
+        float t = rintf(y[j] / s); /* default rounding mode: nearest, ties to even */
+        if (t > 127.0f)
+            t = 127.0f;
+        if (t < -127.0f)
+            t = -127.0f;
+        q[j] = (int8_t)t;
+    }
+}
+
+/* ------------------------------------------------------------------ parallel rows */
+
+typedef void (*row_fn)(void *ctx, int64_t row);
+struct par_job {
+    row_fn fn;
+    void *ctx;
+    int64_t begin, end;
+};
+
+static void *par_worker(void *arg)
+{
+    struct par_job *j = (struct par_job *)arg;
+    for (int64_t r = j->begin; r < j->end; ++r)
+        j->fn(j->ctx, r);
+    return NULL;
+}
+
+/* Runs fn(ctx, r) for r in [0, n). Rows are independent, so splitting them across threads
+ * changes no arithmetic. */
+static void parallel_rows(row_fn fn, void *ctx, int64_t n, int nthreads)
+{
+    if (nthreads < 1)
+        nthreads = 1;
+    if (nthreads > 256)
+        nthreads = 256;
+    if ((int64_t)nthreads > n)
+        nthreads = (int)(n > 0 ? n : 1);
+    if (nthreads == 1) {
+        for (int64_t r = 0; r < n; ++r)
+            fn(ctx, r);
+        return;
+    }
+    pthread_t tid[256];
+    struct par_job jobs[256];
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].fn = fn;
+        jobs[t].ctx = ctx;
+        jobs[t].begin = n * t / nthreads;
+        jobs[t].end = n * (t + 1) / nthreads;
+        pthread_create(&tid[t], NULL, par_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nthreads; ++t)
+        pthread_join(tid[t], NULL);
+}
+
+/* ------------------------------------------------------------------- quantize_rows */
+
+struct qrows_ctx {
+    const uint16_t *x;
+    const float *sinv;
+    int64_t K;
+    int8_t *q;
+    float *s;
+};
+
+static void qrows_row(void *vctx, int64_t m)
+{
+    struct qrows_ctx *c = (struct qrows_ctx *)vctx;
+    float *y = (float *)malloc((size_t)c->K * sizeof(float));
+    for (int64_t j = 0; j < c->K; ++j) {
+        y[j] = oracle_bf16_to_f32(c->x[m * c->K + j]);
+        if (c->sinv)
+            y[j] = y[j] * c->sinv[j]; /* smoothing folded into X: X' = X diag(1/s) */
+    }
+    oracle_quantize_row_f32(y, c->K, c->q + m * c->K, c->s + m);
+    free(y);
+}
+
+/*
+ * Per-token dynamic quantization of a bf16 activation [M, K] (row-major), optionally
+ * after multiplying channel j by sinv[j] = 1/s_j (SmoothQuant applied to X directly).
+ * [P2 "Why activation quantization is hard"; P3 "1. Min-Max Calibration"]
+ */
+int oracle_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int64_t K, int8_t *q,
+                         float *s, int nthreads)
+{
+    struct qrows_ctx c = {x, sinv, K, q, s};
+    parallel_rows(qrows_row, &c, M, nthreads);
+    return 0;
+}
+
+/* --------------------------------------------------------- smoothed RMSNorm + quant */
+
+struct rms_ctx {
+    const uint16_t *x, *r;
+    uint16_t *h_out;
+    const float *gamma;
+    float eps;
+    int64_t K;
+    int8_t *q;
+    float *s, *ms_out, *y_out;
+    uint8_t *ambiguous;
+    const float *ms_override;
+};
+
+static void rms_row(void *vctx, int64_t m)
+{
+    struct rms_ctx *c = (struct rms_ctx *)vctx;
+    const int64_t K = c->K;
+    float *h = (float *)malloc((size_t)K * sizeof(float));
+    float *y = (float *)malloc((size_t)K * sizeof(float));
+
+    /* Optional residual add; the sum is rounded to bf16 (it is the next residual). */
+    for (int64_t j = 0; j < K; ++j) {
+        float v = oracle_bf16_to_f32(c->x[m * K + j]);
+        if (c->r) {
+            uint16_t hb = oracle_f32_to_bf16(v + oracle_bf16_to_f32(c->r[m * K + j]));
+            if (c->h_out)
+                c->h_out[m * K + j] = hb;
+            v = oracle_bf16_to_f32(hb);
+        }
+        h[j] = v;
+    }
+
+    /* Mean of squares. Each square of a bf16 value is exact in binary32; the sum is
+     * accumulated in binary64 in index order. The order of a binary64 sum is not fixed by
+     * the method, so any order is acceptable: the row is flagged when another order could
+     * round the mean to a different binary32 value. */
+    double sum = 0.0;
+    for (int64_t j = 0; j < K; ++j)
+        sum += (double)(h[j] * h[j]);
+    float ms = (float)(sum / (double)K);
+    if (c->ambiguous) {
+        /* |any-order sum - this sum| <= 2 (K-1) u sum with u = 2^-53 (recursive summation
+         * bound for non-negative terms, applied to both orders); widened by 2x. */
+        double delta = 4.0 * (double)K * ldexp(1.0, -53) * sum;
+        float lo = (float)((sum - delta) / (double)K);
+        float hi = (float)((sum + delta) / (double)K);
+        c->ambiguous[m] = (lo != hi) ? 1 : 0;
+    }
+    if (c->ms_override)
+        ms = c->ms_override[m];
+    if (c->ms_out)
+        c->ms_out[m] = ms;
+
+    float rstd = 1.0f / sqrtf(ms + c->eps);
+    /* [P2 "How SmoothQuant prevents outliers"]: divide by the RMS, then multiply channel
+     * by channel by gamma; here gamma already carries the smoothing (gamma' = gamma / s). */
+    for (int64_t j = 0; j < K; ++j) {
+        float t = h[j] * rstd;
+        y[j] = t * c->gamma[j];
+    }
+    if (c->y_out)
+        memcpy(c->y_out + m * K, y, (size_t)K * sizeof(float));
+    if (c->q)
+        oracle_quantize_row_f32(y, K, c->q + m * K, c->s + m);
+    free(h);
+    free(y);
+}
+
+/*
+ * h = bf16(x + residual) (if residual), rstd = 1/sqrt(mean(h^2) + eps), y = h*rstd*gamma',
+ * then per-token quantization of y. Optional outputs: ms_out (the binary32 mean of
+ * squares used), ambiguous (1 where another summation order could change ms), y_out (the
+ * fp32 normalized row before quantization). ms_override forces ms per row (used to
+ * evaluate the other admissible ms of an ambiguous row). q may be NULL (y_out only).
+ */
+int oracle_smooth_rmsnorm_quant(const uint16_t *x, const uint16_t *residual, uint16_t *h_out,
+                                const float *gamma, float eps, int64_t M, int64_t K, int8_t *q,
+                                float *s, float *ms_out, uint8_t *ambiguous,
+                                const float *ms_override, float *y_out, int nthreads)
+{
+    struct rms_ctx c = {x, residual, h_out, gamma, eps, K, q, s, ms_out, y_out, ambiguous,
+                        ms_override};
+    parallel_rows(rms_row, &c, M, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------ exp and SiLU(gate)*up */
+
+/*
+ * exp for binary32, fixed so that two independent implementations agree bit for bit:
+ * Cody & Waite argument reduction (x = k ln2 + r, ln2 split into a 16-bit head and a
+ * binary32 tail), the degree-7 Taylor polynomial of e^r evaluated by Horner's rule with
+ * fused multiply-adds, and an exact scaling by 2^k done as two power-of-two factors so
+ * that overflow and gradual underflow round once, in the last multiply.
+ *   x > 89 -> +inf;  x < -104 -> +0;  NaN -> NaN.
+ */
+float oracle_exp(float x)
+{
+    if (x != x)
+        return x;
+    if (x > 89.0f)
+        return INFINITY;
+    if (x < -104.0f)
+        return 0.0f;
+    const float log2e = 1.44269502162933349609375f;     /* RN_binary32(1/ln 2) */
+    const float ln2_hi = 0.693145751953125f;            /* ln 2 to 16 significant bits */
+    const float ln2_lo = 1.428606765330187045037746429443359375e-06f; /* RN(ln2 - ln2_hi) */
+    float kf = rintf(x * log2e);
+    int k = (int)kf;
+    float r = fmaf(-kf, ln2_hi, x);
+    r = fmaf(-kf, ln2_lo, r);
+    /* Taylor coefficients 1/i!, i = 7 .. 0, each rounded to binary32. */
+    const float c7 = 1.0f / 5040.0f, c6 = 1.0f / 720.0f, c5 = 1.0f / 120.0f,
+                c4 = 1.0f / 24.0f, c3 = 1.0f / 6.0f, c2 = 0.5f, c1 = 1.0f, c0 = 1.0f;
+    float p = c7;
+    p = fmaf(p, r, c6);
+    p = fmaf(p, r, c5);
+    p = fmaf(p, r, c4);
+    p = fmaf(p, r, c3);
+    p = fmaf(p, r, c2);
+    p = fmaf(p, r, c1);
+    p = fmaf(p, r, c0);
+    int k1 = k / 2; /* truncation toward zero; k1 and k - k1 are both in [-75, 65] */
+    int k2 = k - k1;
+    return (p * ldexpf(1.0f, k1)) * ldexpf(1.0f, k2);
+}
+
+/* silu(g) = g * sigmoid(g) = g / (1 + e^-g), in binary32 with oracle_exp. */
+float oracle_silu(float g)
+{
+    return g / (1.0f + oracle_exp(-g));
+}
+
+struct silu_ctx {
+    const uint16_t *gu;
+    int64_t I;
+    int8_t *q;
+    float *s;
+};
+
+static void silu_row(void *vctx, int64_t m)
+{
+    struct silu_ctx *c = (struct silu_ctx *)vctx;
+    const int64_t I = c->I;
+    float *a = (float *)malloc((size_t)I * sizeof(float));
+    for (int64_t j = 0; j < I; ++j) {
+        float g = oracle_bf16_to_f32(c->gu[m * 2 * I + j]);     /* gate half */
+        float u = oracle_bf16_to_f32(c->gu[m * 2 * I + I + j]); /* up half */
+        a[j] = oracle_silu(g) * u;
+    }
+    oracle_quantize_row_f32(a, I, c->q + m * I, c->s + m);
+    free(a);
+}
+
+/*
+ * Llama MLP activation before the down projection, a = silu(gate) * up on the
+ * concatenated [M, 2I] gate|up output, then per-token quantization of a (fp32, never
+ * rounded to bf16).
+ */
+int oracle_silu_mul_quant(const uint16_t *gate_up, int64_t M, int64_t I, int8_t *q, float *s,
+                          int nthreads)
+{
+    struct silu_ctx c = {gate_up, I, q, s};
+    parallel_rows(silu_row, &c, M, nthreads);
+    return 0;
+}
+
+/* -------------------------------------------------------------- GEMM and dequant */
+
+/* Dequantize one accumulator [P2 "applied and reversed after accumulation"; P4 "converting
+ * back to BF16"]: y = bf16( (float(acc) * s_tok) * s_ch ). */
+uint16_t oracle_dequant(int32_t acc, float s_tok, float s_ch)
+{
+    float f = (float)acc; /* round to nearest even: |acc| may exceed 2^24 */
+    f = f * s_tok;
+    f = f * s_ch;
+    return oracle_f32_to_bf16(f);
+}
+
+struct gemm_ctx {
+    const int8_t *xq;
+    const float *s_tok;
+    const int8_t *wq;
+    const float *s_ch;
+    int64_t N, K;
+    uint16_t *y;
+    int32_t *acc;
+};
+
+static void gemm_row(void *vctx, int64_t m)
+{
+    struct gemm_ctx *c = (struct gemm_ctx *)vctx;
+    for (int64_t n = 0; n < c->N; ++n) {
+        int32_t a = 0;
+        for (int64_t k = 0; k < c->K; ++k)
+            a += (int32_t)c->xq[m * c->K + k] * (int32_t)c->wq[n * c->K + k];
+        if (c->acc)
+            c->acc[m * c->N + n] = a;
+        if (c->y)
+            c->y[m * c->N + n] = oracle_dequant(a, c->s_tok[m], c->s_ch[n]);
+    }
+}
+
+/*
+ * y[m,n] = bf16( (float(sum_k xq[m,k] wq[n,k]) * s_tok[m]) * s_ch[n] ).
+ * xq [M,K] and wq [N,K] are int8, both K-contiguous; the int32 sum is exact for
+ * K <= 2^31 / 127^2 = 133,144. acc (optional) receives the int32 sums [M,N].
+ */
+int oracle_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                        const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y,
+                        int32_t *acc, int nthreads)
+{
+    struct gemm_ctx c = {xq, s_tok, wq, s_ch, N, K, y, acc};
+    parallel_rows(gemm_row, &c, M, nthreads);
+    return 0;
+}
+
+/* The same output at `count` chosen (m, n) positions only, for shapes too large to do whole. */
+int oracle_gemm_dequant_sampled(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                                const float *s_ch, int64_t K, const int64_t *ms,
+                                const int64_t *ns, int64_t count, uint16_t *y, int32_t *acc)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = ms[i], n = ns[i];
+        int32_t a = 0;
+        for (int64_t k = 0; k < K; ++k)
+            a += (int32_t)xq[m * K + k] * (int32_t)wq[n * K + k];
+        if (acc)
+            acc[i] = a;
+        if (y)
+            y[i] = oracle_dequant(a, s_tok[m], s_ch[n]);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------- offline preparation */
+
+/* max_m |A[m, j]| over the rows of a fp32 [M, K] matrix (the calibration statistic of
+ * [P2 "How the SmoothQuant smoothing factor is computed"]). */
+int oracle_column_absmax_f32(const float *a, int64_t M, int64_t K, float *amax)
+{
+    for (int64_t j = 0; j < K; ++j)
+        amax[j] = 0.0f;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = fabsf(a[m * K + j]);
+            if (v > amax[j])
+                amax[j] = v;
+        }
+    return 0;
+}
+
+/* max over rows of |B[m, j]| for a bf16 matrix, e.g. the weight W [N, K] whose input
+ * channel j is column j (the page's "row j" refers to the transposed [K, N] layout). */
+int oracle_column_absmax_bf16(const uint16_t *b, int64_t M, int64_t K, float *amax)
+{
+    for (int64_t j = 0; j < K; ++j)
+        amax[j] = 0.0f;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = fabsf(oracle_bf16_to_f32(b[m * K + j]));
+            if (v > amax[j])
+                amax[j] = v;
+        }
+    return 0;
+}
+
+/*
+ * Smoothing factor per input channel, s_j = max|A_j|^alpha / max|W_j|^(1 - alpha),
+ * evaluated in binary64 and rounded once to binary32. A channel with no activation or no
+ * weight range keeps s_j = 1 (the page is silent).
+ */
+int oracle_smoothing_factors(const float *a_max, const float *w_max, int64_t K, double alpha,
+                             float *s)
+{
+    for (int64_t j = 0; j < K; ++j) {
+        if (a_max[j] == 0.0f || w_max[j] == 0.0f) {
+            s[j] = 1.0f;
+            continue;
+        }
+        double v = pow((double)a_max[j], alpha) / pow((double)w_max[j], 1.0 - alpha);
+        s[j] = (float)v;
+    }
+    return 0;
+}
+
+/* gamma'_j = gamma_j / s_j and the reciprocal 1/s_j used when smoothing X directly
+ * [P2 "How the SmoothQuant smoothing factor is computed", last paragraph]. */
+int oracle_fold_gamma(const float *gamma, const float *s, int64_t K, float *gamma_folded,
+                      float *s_inv)
+{
+    for (int64_t j = 0; j < K; ++j) {
+        if (gamma_folded)
+            gamma_folded[j] = gamma[j] / s[j];
+        if (s_inv)
+            s_inv[j] = 1.0f / s[j];
+    }
+    return 0;
+}
+
+/* W'[n, j] = W[n, j] * s_j: the receiving linear's input channel j scaled up by s_j
+ * [P2 "How the SmoothQuant smoothing factor is computed", last paragraph]. fp32 out. */
+int oracle_smooth_weight(const uint16_t *w, const float *s, int64_t N, int64_t K, float *out)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K; ++j)
+            out[n * K + j] = oracle_bf16_to_f32(w[n * K + j]) * s[j];
+    return 0;
+}
+
+struct rtn_ctx {
+    const uint16_t *w;
+    const float *s;
+    int64_t K;
+    int8_t *wq;
+    float *s_ch;
+};
+
+static void rtn_row(void *vctx, int64_t n)
+{
+    struct rtn_ctx *c = (struct rtn_ctx *)vctx;
+    float *v = (float *)malloc((size_t)c->K * sizeof(float));
+    for (int64_t j = 0; j < c->K; ++j) {
+        v[j] = oracle_bf16_to_f32(c->w[n * c->K + j]);
+        if (c->s)
+            v[j] = v[j] * c->s[j]; /* W' = W diag(s): input channel j scaled up by s_j */
+    }
+    oracle_quantize_row_f32(v, c->K, c->wq + n * c->K, c->s_ch + n);
+    free(v);
+}
+
+/*
+ * Per-output-channel round-to-nearest weight quantization of the smoothed weight
+ * [P2 "The problem with naive quantization"]: for each output channel n (a row of the
+ * [N, K] weight), s_ch[n] = max_j |W'[n, j]| / 127 and wq = round(W' / s_ch).
+ * s may be NULL (no smoothing).
+ */
+int oracle_rtn_weights(const uint16_t *w, const float *s, int64_t N, int64_t K, int8_t *wq,
+                       float *s_ch, int nthreads)
+{
+    struct rtn_ctx c = {w, s, K, wq, s_ch};
+    parallel_rows(rtn_row, &c, N, nthreads);
+    return 0;
+}
