@@ -1,0 +1,608 @@
+#!/usr/bin/env python
+"""Benchmark of the W8A8 SmoothQuant linear path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode8b] [--impl ours]
+
+One step = one pass of the whole hot path over one batch: for each token count M of the
+workload, one Llama decoder block's linear path on its own layer's weights
+(smoothed RMSNorm+quant -> qkv GEMM; attention stand-in -> quant -> o GEMM; residual add ->
+smoothed RMSNorm+quant -> gate_up GEMM; SiLU*up+quant -> down GEMM). The default workload is
+the Llama-3.1-8B decode set, M = 1, 8, 32, 64 (four layers, 872 MB of int8 weights, so
+every step streams its weights from HBM: inputs larger than L2, no flush needed).
+
+The timed region replays a CUDA graph of the step K times between CUDA events on the
+launching stream, after W warm-up steps, bracketed by a barrier and device synchronizations;
+multi-GPU runs are independent replicas (one process per GPU, no data-path collective) and
+report the max time over ranks. Prints one JSON line (rank 0).
+
+`--impl reference` times the CPU oracle instead (host cores, bounded samples of the same
+workload). `--case gemm:M:N:K` runs one GEMM launch repeatedly (for profilers).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "W8A8 linear TOPS & HBM GB/s at Llama-3.1-8B shapes; % of roofline"
+EPS = 1e-5
+ALPHA = 0.5
+CALIB_TOKENS = 128
+
+LLAMA8B = dict(model="llama-3.1-8b", H=4096, I=14336, QKV=6144)
+LLAMA70B = dict(model="llama-3.1-70b", H=8192, I=28672, QKV=10240)
+WORKLOADS = {
+    "decode8b": dict(arch=LLAMA8B, Ms=[1, 8, 32, 64], desc="Llama-3.1-8B decode linear set"),
+    "prefill8b": dict(arch=LLAMA8B, Ms=[2048, 8192], desc="Llama-3.1-8B prefill linear set"),
+    "block8b": dict(arch=LLAMA8B, Ms=[512], desc="Llama-3.1-8B decoder block linear path"),
+    "set70b": dict(arch=LLAMA70B, Ms=[16, 4096], desc="Llama-3.1-70B-shaped linear set"),
+}
+
+# Measured peaks (driver-written); fallbacks are the pool's earlier measurements.
+FALLBACK_HBM_GBS = 6650.0
+INT8_NOMINAL_TOPS = 4500.0
+
+
+# ------------------------------------------------------------------ work model
+
+
+def projections(arch):
+    H, I, Q = arch["H"], arch["I"], arch["QKV"]
+    return {"qkv": (Q, H), "o": (H, H), "gate_up": (2 * I, H), "down": (H, I)}
+
+
+def gemm_bytes(M, N, K):
+    """Algorithmic HBM bytes of one GEMM+dequant: int8 weight and activation, fp32 scales,
+    bf16 output."""
+    return N * K + M * K + 4 * M + 4 * N + 2 * M * N
+
+
+def layer_work(arch, M):
+    """(ops, bytes, gemm_ops, gemm_bytes) of one block's linear path at M tokens."""
+    H, I = arch["H"], arch["I"]
+    P = projections(arch)
+    g_ops = sum(2 * M * N * K for (N, K) in P.values())
+    g_bytes = sum(gemm_bytes(M, N, K) for (N, K) in P.values())
+    row_bytes = ((3 * M * H + 4 * M + 4 * H)          # smoothed RMSNorm + quant (qkv input)
+                 + (3 * M * H + 4 * M + 4 * H)        # quantize_rows (o input, smoothed)
+                 + (7 * M * H + 4 * M + 4 * H)        # residual add + RMSNorm + quant
+                 + (5 * M * I + 4 * M))               # SiLU*up + quant (down input)
+    return g_ops, g_bytes + row_bytes, g_ops, g_bytes
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+def reduce_max(value: float) -> float:
+    """Max of a float over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def combine(units_per_rank: float, seconds_per_rank: float, world: int):
+    """Whole-job throughput of `world` replicas: all units over the slowest rank's time."""
+    t = reduce_max(seconds_per_rank)
+    return units_per_rank * world / t, t
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) in a thread."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index, period_s=0.05):
+        self.samples = []
+        self.err = None
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report why
+            self.err = repr(e)
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception as e:
+                self.err = repr(e)
+            time.sleep(self.period)
+
+    def start(self):
+        if self.h is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.h is not None:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if self.h is None:
+            return {"error": self.err}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "during the timed region"
+        if len(win) < 3:
+            win = [s for s in self.samples if s[0] >= t0]
+            note = "timed region plus the same load replayed right after it"
+        if not win:
+            return {"error": "no samples", "sm_max_mhz": self.max_mhz}
+        reasons = set()
+        for _, _, rs in win:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in win), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(win), "window": note}
+
+
+# ------------------------------------------------------------------ workload on the GPU
+
+
+class Layer:
+    """One decoder block's linear path at M tokens: prepared weights, inputs, outputs."""
+
+    def __init__(self, arch, M, seed, device):
+        import int8_w8a8_quantized_smoothed_b200 as w8
+        from int8_w8a8_quantized_smoothed_b200 import prep, synth
+        self.M, self.arch = M, arch
+        H, I = arch["H"], arch["I"]
+        P = projections(arch)
+        g1 = synth.gamma_device(H, seed + 1, device)
+        g2 = synth.gamma_device(H, seed + 2, device)
+        # calibration batches (separate seeds, same distributions as the served tokens)
+        x_cal = synth.activation_device(CALIB_TOKENS, H, seed + 3, device)
+        a_cal = synth.activation_device(CALIB_TOKENS, H, seed + 4, device)
+        h_cal = synth.activation_device(CALIB_TOKENS, H, seed + 5, device)
+        a_qkv = prep.column_absmax(prep.rmsnorm_calibration(x_cal, g1, EPS))
+        a_o = prep.column_absmax(a_cal)
+        a_gu = prep.column_absmax(prep.rmsnorm_calibration(h_cal, g2, EPS))
+        self.w = {}
+        for i, (name, (N, K)) in enumerate(P.items()):
+            wb = synth.weight_device(N, K, seed + 10 + i, device)
+            if name == "qkv":
+                p = prep.prepare_linear(wb, a_qkv, ALPHA)
+                self.g1f = torch.from_numpy(prep.fold(g1.cpu().numpy(), p["s"])[0]).to(device)
+            elif name == "o":
+                p = prep.prepare_linear(wb, a_o, ALPHA)
+                self.sinv_o = p["s_inv_dev"]
+            elif name == "gate_up":
+                p = prep.prepare_linear(wb, a_gu, ALPHA)
+                self.g2f = torch.from_numpy(prep.fold(g2.cpu().numpy(), p["s"])[0]).to(device)
+            else:  # down: its input is SiLU*up, no norm to fold into
+                wq, sch = w8.w8a8_quantize_rows(wb)
+                p = dict(wq=wq, s_ch=sch)
+            self.w[name] = (p["wq"], p["s_ch"])
+            del wb
+        torch.cuda.synchronize()
+        # inputs (device) and their pinned host copies for the end-to-end measurement
+        self.x = synth.activation_device(M, H, seed + 20, device)
+        self.attn = synth.activation_device(M, H, seed + 21, device)
+        self.x_host = self.x.cpu().pin_memory()
+        self.attn_host = self.attn.cpu().pin_memory()
+        e = dict(device=device)
+        self.q1 = torch.empty(M, H, dtype=torch.int8, **e)
+        self.s1 = torch.empty(M, dtype=torch.float32, **e)
+        self.qkv = torch.empty(M, P["qkv"][0], dtype=torch.bfloat16, **e)
+        self.q2 = torch.empty(M, H, dtype=torch.int8, **e)
+        self.s2 = torch.empty(M, dtype=torch.float32, **e)
+        self.o = torch.empty(M, H, dtype=torch.bfloat16, **e)
+        self.h = torch.empty(M, H, dtype=torch.bfloat16, **e)
+        self.q3 = torch.empty(M, H, dtype=torch.int8, **e)
+        self.s3 = torch.empty(M, dtype=torch.float32, **e)
+        self.gu = torch.empty(M, 2 * I, dtype=torch.bfloat16, **e)
+        self.q4 = torch.empty(M, I, dtype=torch.int8, **e)
+        self.s4 = torch.empty(M, dtype=torch.float32, **e)
+        self.down = torch.empty(M, H, dtype=torch.bfloat16, **e)
+        self.down_host = torch.empty(M, H, dtype=torch.bfloat16).pin_memory()
+
+    def rows(self):
+        import int8_w8a8_quantized_smoothed_b200 as w8
+        w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
+        w8.w8a8_quantize_rows(self.attn, self.sinv_o, q=self.q2, s_tok=self.s2)
+
+    def chain(self, ws, gemms=True, rows=True):
+        import int8_w8a8_quantized_smoothed_b200 as w8
+        if rows:
+            w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
+        if gemms:
+            w8.w8a8_gemm_dequant(self.q1, self.s1, *self.w["qkv"], y=self.qkv, workspace=ws)
+        if rows:
+            w8.w8a8_quantize_rows(self.attn, self.sinv_o, q=self.q2, s_tok=self.s2)
+        if gemms:
+            w8.w8a8_gemm_dequant(self.q2, self.s2, *self.w["o"], y=self.o, workspace=ws)
+        if rows:
+            w8.w8a8_smooth_rmsnorm_quant(self.o, self.g2f, EPS, residual=self.x, h_out=self.h,
+                                         q=self.q3, s_tok=self.s3)
+        if gemms:
+            w8.w8a8_gemm_dequant(self.q3, self.s3, *self.w["gate_up"], y=self.gu, workspace=ws)
+        if rows:
+            w8.w8a8_silu_mul_quant(self.gu, q=self.q4, s_tok=self.s4)
+        if gemms:
+            w8.w8a8_gemm_dequant(self.q4, self.s4, *self.w["down"], y=self.down, workspace=ws)
+
+
+def capture(fn):
+    """CUDA graph of fn() (warmed up on a side stream first)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, steps, warmup):
+    """Seconds for `steps` replays (events on the launching stream), after `warmup`."""
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def run_ours(args, world, rank, local):
+    import int8_w8a8_quantized_smoothed_b200 as w8
+    from int8_w8a8_quantized_smoothed_b200 import build as wbuild
+    wbuild.build()
+    w8.lib()
+    dev = torch.device("cuda", local)
+    wl = WORKLOADS[args.workload]
+    arch = wl["arch"]
+    layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev) for i, M in enumerate(wl["Ms"])]
+    ws = w8.Workspace(dev)
+    max_ws = max(w8.w8a8_gemm_workspace_size(L.M, N, K) for L in layers
+                 for (N, K) in projections(arch).values())
+    ws.get(max_ws)
+
+    def step():
+        for L in layers:
+            L.chain(ws)
+
+    def step_gemms():
+        for L in layers:
+            L.chain(ws, rows=False)
+
+    def step_rows():
+        for L in layers:
+            L.chain(ws, gemms=False)
+
+    def step_e2e():
+        for L in layers:
+            L.x.copy_(L.x_host, non_blocking=True)
+            L.attn.copy_(L.attn_host, non_blocking=True)
+        step()
+        for L in layers:
+            L.down_host.copy_(L.down, non_blocking=True)
+
+    ops = sum(layer_work(arch, L.M)[0] for L in layers)
+    nbytes = sum(layer_work(arch, L.M)[1] for L in layers)
+    g_bytes = sum(layer_work(arch, L.M)[3] for L in layers)
+    launches_per_step = 8 * len(layers)
+    h2d = sum(L.x.numel() * 2 + L.attn.numel() * 2 for L in layers)
+    d2h = sum(L.down.numel() * 2 for L in layers)
+
+    g_step = capture(step)
+    assert w8.w8a8_device_status(reset=True) == 0, "device-side wait ran out"
+
+    clocks = ClockSampler(local).start()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    secs = time_graph(g_step, args.steps, args.warmup)
+    t_wall1 = time.perf_counter()
+    # keep the same load running briefly if the timed region was too short to sample
+    if t_wall1 - t_wall0 < 0.3 and clocks.h is not None:
+        t_end = time.perf_counter() + 0.5
+        while time.perf_counter() < t_end:
+            for _ in range(50):
+                g_step.replay()
+            torch.cuda.synchronize()
+    clocks.stop()
+    value, t_max = combine(nbytes, secs / args.steps, world)
+    ms_per_step = t_max * 1e3
+
+    # dominant kernel: the GEMM launches of the step, timed alone as a graph
+    g_gemm = capture(step_gemms)
+    gsecs = time_graph(g_gemm, args.steps, args.warmup) / args.steps
+    g_rows = capture(step_rows)
+    rsecs = time_graph(g_rows, args.steps, args.warmup) / args.steps
+    g_e2e = capture(step_e2e)
+    esecs = time_graph(g_e2e, args.steps, args.warmup) / args.steps
+    e_value, _ = combine(nbytes, esecs, world)
+    assert w8.w8a8_device_status(reset=True) == 0, "device-side wait ran out"
+
+    hbm_peak, peak_src = read_peaks()
+    gemm_gbs = g_bytes / gsecs / 1e9
+    t_roof = max(ops / (INT8_NOMINAL_TOPS * 1e12), nbytes / (hbm_peak * 1e9))
+    result = {
+        "metric": METRIC, "value": round(value / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8xi8->i32, fp32 scales, bf16 io", "data": "synthetic",
+        "config": {"workload": f"{wl['desc']}, M in {wl['Ms']}: one decoder block's linear "
+                               f"path per M on its own layer's weights",
+                   "tokens": wl["Ms"], "hidden": arch["H"], "intermediate": arch["I"],
+                   "qkv_out": arch["QKV"], "alpha": ALPHA, "parallelism": f"replicas x{world}",
+                   "l2": "no flush: each step streams "
+                         f"{sum(L.w[n][0].numel() for L in layers for n in L.w) / 1e6:.0f} MB "
+                         "of int8 weights (> 126 MB L2)",
+                   "timing": "CUDA graph of one step replayed K times, CUDA events"},
+        "tops": round(ops / t_max / 1e12, 3),
+        "roofline_step": {"t_roof_us": round(t_roof * 1e6, 2),
+                          "t_us": round(t_max * 1e6, 2), "frac": round(t_roof / t_max, 4),
+                          "note": "max(ops/4.5 POPS nominal int8, bytes/HBM peak)"},
+        "roofline": {"kernel": "gemm_decode_kernel (all GEMM launches of the step)",
+                     "bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(gemm_gbs / hbm_peak, 4),
+                     "peak_source": f"{peak_src} copy bandwidth (burst)",
+                     "traffic": None,
+                     "per_launch_us": round(gsecs / (4 * len(layers)) * 1e6, 3)},
+        "breakdown_us": {"step": round(t_max * 1e6, 2), "gemms": round(gsecs * 1e6, 2),
+                         "row_kernels": round(rsecs * 1e6, 2)},
+        "e2e": {"value": round(e_value / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(esecs * 1e3, 5),
+                "how": "CUDA graph: pinned-host inputs H2D, the step's C-ABI calls, output D2H"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(t_wall0, time.perf_counter()),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(arch)
+    if args.traffic is not None:
+        result["roofline"]["traffic"] = args.traffic
+    del g_step, g_gemm, g_rows, g_e2e
+    return result
+
+
+# ------------------------------------------------------------------ oracle (CPU) legs
+
+
+def _oracle_layer(arch, M, seed):
+    """Inputs and prepared int8 weights for the oracle's chain (CPU, seeded)."""
+    from int8_w8a8_quantized_smoothed_b200 import synth
+    H = arch["H"]
+    P = projections(arch)
+    pr = {}
+    for i, (name, (N, K)) in enumerate(P.items()):
+        pr[name] = dict(wq=synth.int8_codes((N, K), seed + i, extremes=False),
+                        s_ch=synth.scales(N, seed + 10 + i, 1e-4, 2e-2))
+    pr["gamma1f"] = synth.gamma(H, seed + 20)
+    pr["gamma2f"] = synth.gamma(H, seed + 21)
+    pr["s_inv_o"] = (1.0 / synth.gamma(H, seed + 22)).astype(np.float32)
+    inputs = dict(x=synth.activation(M, H, seed + 30), attn=synth.activation(M, H, seed + 31))
+    return pr, inputs
+
+
+def cpu_baseline(arch, M=64, min_seconds=10.0):
+    """The oracle, as it stands, on this host's cores: one decoder block's linear path at
+    M tokens, repeated for at least `min_seconds`."""
+    import oracle
+    pr, inputs = _oracle_layer(arch, M, 77)
+    nthreads = oracle.NTHREADS
+    _, nbytes, _, _ = layer_work(arch, M)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.block_reference(inputs, pr, EPS, nthreads=nthreads)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": round(nbytes * passes / el / 1e9, 4), "unit": "GB/s",
+            "cores": min(nthreads, M), "kind": "oracle",
+            "sample": f"one decoder block's linear path at M={M} ({arch['model']} shapes), "
+                      f"{passes} passes in {el:.1f} s; rows split over {min(nthreads, M)} "
+                      f"threads of {os.cpu_count()} host cores"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle timed on the host cores, each step a bounded sample
+    (the M=1 block linear path of the workload's architecture)."""
+    if rank != 0:
+        return None
+    import oracle
+    wl = WORKLOADS[args.workload]
+    arch = wl["arch"]
+    M = 1
+    pr, inputs = _oracle_layer(arch, M, 91)
+    _, nbytes, _, _ = layer_work(arch, M)
+    nth = oracle.NTHREADS
+    for _ in range(args.warmup):
+        oracle.block_reference(inputs, pr, EPS, nthreads=nth)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.block_reference(inputs, pr, EPS, nthreads=nth)
+    el = time.perf_counter() - t0
+    value = nbytes * args.steps / el / 1e9
+    sample = (f"per step: one decoder block's linear path at M={M} ({arch['model']} shapes) "
+              f"through the CPU oracle")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8xi8->i32, fp32 scales, bf16 io",
+        "data": "synthetic",
+        "config": {"workload": f"{wl['desc']} (bounded CPU sample, M=1 per step)",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": min(nth, M),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ single-kernel case
+
+
+def run_case(args):
+    """`--case gemm:M:N:K[:variant]` or `rows:M:K`: one kernel launched repeatedly."""
+    import int8_w8a8_quantized_smoothed_b200 as w8
+    from int8_w8a8_quantized_smoothed_b200 import build as wbuild, synth
+    wbuild.build()
+    parts = args.case.split(":")
+    dev = torch.device("cuda", 0)
+    if parts[0] == "gemm":
+        M, N, K = (int(v) for v in parts[1:4])
+        variant = int(parts[4]) if len(parts) > 4 else 0
+        copies = max(1, math.ceil(4 * 126e6 / (N * K)))  # rotate weights through > 4x L2
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+        st = torch.rand(M, device=dev) * 1e-2
+        ws_ = [torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev)
+               for _ in range(copies)]
+        sc = torch.rand(N, device=dev) * 1e-3
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        wsp = w8.Workspace(dev)
+
+        def launch(i):
+            w8.w8a8_gemm_dequant_ex(xq, st, ws_[i % copies], sc, y=y, workspace=wsp,
+                                    variant=variant)
+        work = gemm_bytes(M, N, K)
+    else:
+        M, K = int(parts[1]), int(parts[2])
+        x = synth.activation_device(M, K, 1, dev)
+        g = torch.ones(K, device=dev)
+        q = torch.empty(M, K, dtype=torch.int8, device=dev)
+        s = torch.empty(M, device=dev)
+
+        def launch(i):
+            w8.w8a8_smooth_rmsnorm_quant(x, g, EPS, q=q, s_tok=s)
+        work = 3 * M * K + 4 * M + 4 * K
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        launch(i)
+    e1.record()
+    torch.cuda.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / args.steps
+    return {"case": args.case, "us_per_launch": round(t * 1e6, 3),
+            "GBps_algorithmic": round(work / t / 1e9, 1),
+            "note": "eager launches: includes launch gaps when the kernel is short"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode8b")
+    ap.add_argument("--case", default=None)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel, if measured")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.case is None:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+    if args.case:
+        print(json.dumps(run_case(args)), flush=True)
+        return 0
+    world, rank, local = dist_setup(args)
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    out = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,178 @@
+/*
+ * w8a8.h -- C ABI of the B200 (sm_100a) W8A8 SmoothQuant linear path.
+ *
+ * The path is the INT8 W8A8 linear layer of a Llama-3-class decoder: per-token symmetric
+ * dynamic activation quantization (fused with an RMSNorm whose gamma carries the SmoothQuant
+ * factors, or with SiLU(gate)*up), an int8 x int8 -> int32 GEMM against per-output-channel
+ * int8 weights, and a dequantization epilogue to bf16. Page citations are by page title and
+ * section:
+ *   [W8A8]  "INT8 W8A8 quantization of Llama 3.1 8B with SmoothQuant and GPTQ" (arc-codex)
+ *   [PTQ]   "INT8 Post-Training Quantization for LLM Inference on NVIDIA GPUs" (devtechtools)
+ *   [SERVE] "W8A8 Llama 3.1 8B: accuracy and serving results" (Red Hat developers)
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; row-major, contiguous.
+ *     The library allocates no device memory in any call; it keeps one small device status
+ *     word per device (see w8a8_device_status) and nothing else.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream). Host-detectable
+ *     errors are returned before anything is launched; a launch failure returns
+ *     W8A8_ERR_CUDA. Device-side problems (a bounded wait that ran out) are reported by
+ *     w8a8_device_status().
+ *   - bf16 values are raw 16-bit patterns (w8a8_bf16). fp32 arithmetic is IEEE binary32 with
+ *     round-to-nearest-even, including division and square root.
+ *   - Base pointers of vectors read or written 16 bytes at a time must be 16-byte aligned
+ *     (stated per argument); otherwise W8A8_ERR_ALIGNMENT.
+ *   - Inputs must be finite; results for NaN or Inf inputs are unspecified.
+ *   - Calls are thread-safe; the only mutable host state is a once-per-process init.
+ *   - There is no CPU fallback: without a B200-class device a call returns
+ *     W8A8_ERR_NO_DEVICE.
+ */
+#ifndef W8A8_H
+#define W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W8A8_API __attribute__((visibility("default")))
+#else
+#define W8A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *w8a8_stream_t; /* identical to cudaStream_t / CUstream */
+typedef uint16_t w8a8_bf16;                /* raw bf16 bit pattern */
+
+enum w8a8_status {
+    W8A8_OK = 0,
+    W8A8_ERR_INVALID_ARG = -1,       /* null pointer, non-positive size, aliasing */
+    W8A8_ERR_ALIGNMENT = -2,         /* a base pointer is not 16-byte aligned */
+    W8A8_ERR_UNSUPPORTED_SHAPE = -3, /* K or N not a supported multiple, or too large */
+    W8A8_ERR_WORKSPACE = -4,         /* workspace missing or smaller than required */
+    W8A8_ERR_CUDA = -5,              /* a CUDA runtime/driver call failed */
+    W8A8_ERR_TIMEOUT = -6,           /* a device-side bounded wait ran out */
+    W8A8_ERR_NO_DEVICE = -7          /* no sm_100 device is current */
+};
+
+/*
+ * Per-token dynamic symmetric quantization of activations [W8A8 "Why activation
+ * quantization is hard"; PTQ "1. Min-Max Calibration"], optionally with the SmoothQuant
+ * factors folded into X (X' = X diag(1/s), [W8A8 "How the SmoothQuant smoothing factor is
+ * computed"]):
+ *   y[m,j]   = float(x[m,j]) * smooth_inv[j]          (or float(x[m,j]) if smooth_inv == NULL)
+ *   s_tok[m] = max_j |y[m,j]| / 127
+ *   q[m,j]   = clamp(round_half_even(y[m,j] / s_tok[m]), -127, 127)
+ *   an all-zero row gives s_tok = 0 and q = 0.
+ * x: bf16 [M,K], 16-byte aligned. smooth_inv: fp32 [K] or NULL, 16-byte aligned.
+ * q: int8 [M,K], 16-byte aligned, must not overlap x. s_tok: fp32 [M].
+ * Requires M >= 1, K >= 16, K % 16 == 0, K <= 32768.
+ * Also serves the offline per-output-channel weight quantization [W8A8 "The problem with
+ * naive quantization"]: with x = W [N,K] and smooth_inv = s (the factors themselves) it
+ * yields the round-to-nearest int8 weights of diag(s)-smoothed W and their scales s_ch.
+ */
+W8A8_API int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, int64_t K,
+                       int8_t *q, float *s_tok, w8a8_stream_t stream);
+
+/*
+ * Smoothed RMSNorm fused with per-token quantization [W8A8 "How SmoothQuant prevents
+ * outliers in activation tensors": RMSNorm divides by the RMS, then multiplies by gamma;
+ * SmoothQuant divides gamma by s]:
+ *   h[m,j]   = bf16(float(x[m,j]) + float(residual[m,j]))  if residual != NULL, written to h_out
+ *              float(x[m,j])                                otherwise
+ *   ms[m]    = float( (sum_j double(h[m,j]^2)) / K )      (binary64 sum, any order)
+ *   rstd[m]  = 1 / sqrt(ms[m] + eps)                       (binary32)
+ *   y[m,j]   = (h[m,j] * rstd[m]) * gamma_smoothed[j]      (binary32, in this order)
+ *   then s_tok, q from y exactly as in w8a8_quantize_rows.
+ * x, residual, h_out: bf16 [M,K], 16-byte aligned; residual and h_out are both NULL or both
+ * non-NULL (h_out may alias residual, not x). gamma_smoothed: fp32 [K] (gamma / s), 16-byte
+ * aligned. q: int8 [M,K], 16-byte aligned. s_tok: fp32 [M].
+ * Requires M >= 1, K >= 16, K % 16 == 0, K <= 32768, eps >= 0.
+ */
+W8A8_API int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a8_bf16 *h_out,
+                              const float *gamma_smoothed, float eps, int64_t M, int64_t K,
+                              int8_t *q, float *s_tok, w8a8_stream_t stream);
+
+/*
+ * SiLU(gate) * up fused with per-token requantization, the input of a Llama MLP's down
+ * projection (not on the pages; the decoder-block workload's MLP):
+ *   g = float(gate_up[m, j]), u = float(gate_up[m, I + j])
+ *   a[m,j] = (g / (1 + w8a8_exp(-g))) * u                  (binary32)
+ *   then s_tok, q from a exactly as in w8a8_quantize_rows.
+ * w8a8_exp is a fixed binary32 exp: Cody-Waite reduction x = k ln2 + r with
+ * k = rint(x * RN(1/ln2)), r = fma(-k, ln2_hi, x) then fma(-k, ln2_lo, r) (ln2_hi = ln2 to 16
+ * significant bits, ln2_lo = RN(ln2 - ln2_hi)), the degree-7 Taylor polynomial of e^r with
+ * coefficients RN(1/i!) by Horner's rule in fmaf, times 2^(k/2) then 2^(k - k/2) (k/2
+ * truncated); x > 89 gives +inf and x < -104 gives +0.
+ * gate_up: bf16 [M, 2I] ([gate | up] halves), 16-byte aligned. q: int8 [M, I], 16-byte
+ * aligned. s_tok: fp32 [M]. Requires M >= 1, I >= 16, I % 16 == 0, I <= 32768.
+ */
+W8A8_API int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *q,
+                        float *s_tok, w8a8_stream_t stream);
+
+/*
+ * Bytes of device workspace w8a8_gemm_dequant needs for this shape (0 if none). The
+ * workspace must be zero-filled before its first use; every call that returns W8A8_OK
+ * leaves it zero-filled again, so one zeroed buffer serves any number of calls issued in
+ * order on one stream. Calls that may run concurrently need separate workspaces.
+ */
+W8A8_API size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * INT8 tensor-core GEMM with the fused dequantization epilogue [W8A8 "How we compressed the
+ * model" (INT8 tensor cores), "Why activation quantization is hard" (one scale per token,
+ * applied and reversed after accumulation); SERVE "Inter-token latency (ITL)" (multiply,
+ * then convert back to BF16)]:
+ *   acc[m,n] = sum_k int32(xq[m,k]) * int32(wq[n,k])        (exact int32)
+ *   y[m,n]   = bf16( (float(acc[m,n]) * s_tok[m]) * s_ch[n] )  (binary32 RN, then RN to bf16)
+ * xq: int8 [M,K] (K contiguous), 16-byte aligned. wq: int8 [N,K] (K contiguous, i.e. the
+ * weight in nn.Linear layout), 16-byte aligned. s_tok: fp32 [M]. s_ch: fp32 [N], 16-byte
+ * aligned. y: bf16 [M,N], 16-byte aligned. acc_out: int32 [M,N] or NULL; when given, the
+ * raw accumulators are written too (a check mode; it adds 4 bytes of traffic per output).
+ * workspace/workspace_bytes: see w8a8_gemm_workspace_size (may be NULL/0 when it returns 0).
+ * Requires M >= 1, N >= 8, N % 8 == 0, K >= 16, K % 16 == 0, K <= 133144 (so that
+ * 127 * 127 * K fits in int32), M, N <= 2^31 - 1.
+ * Small M (at most 256 tokens) runs a swap-AB split-K kernel that streams the weight;
+ * larger M runs a persistent tile kernel. Both give identical results.
+ */
+W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                      const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
+                      int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                      w8a8_stream_t stream);
+
+/*
+ * The same GEMM with the kernel chosen by the caller, for tests and tuning:
+ * variant 0 = automatic (as w8a8_gemm_dequant), 1 = persistent tile kernel, 2 = swap-AB
+ * split-K kernel (M <= 256 only). splits = 0 picks the split count automatically, otherwise
+ * the K range is cut into at most `splits` parts (variant 2). tile_n = 0 automatic, else 128
+ * or 256 (variant 1). The workspace needed is w8a8_gemm_workspace_size_ex() of the same
+ * arguments.
+ */
+W8A8_API int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                         const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
+                         int32_t *acc_out, void *workspace, size_t workspace_bytes,
+                         int variant, int splits, int tile_n, w8a8_stream_t stream);
+W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int splits,
+                                   int tile_n);
+
+/*
+ * Device status: synchronizes the current device, then returns W8A8_OK or
+ * W8A8_ERR_TIMEOUT if any kernel of this library on it gave up a bounded wait (every
+ * mbarrier and ticket wait in the kernels is limited, ~2 s) since the last reset.
+ * reset != 0 clears the word. Returns W8A8_ERR_CUDA if synchronization fails.
+ */
+W8A8_API int w8a8_device_status(int reset);
+
+/* Static, human-readable name of a status code. */
+W8A8_API const char *w8a8_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+W8A8_API int w8a8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H */

@@ -1,0 +1,241 @@
+"""B200 (sm_100a) W8A8 SmoothQuant linear path: thin Python binding of ``libw8a8.so``.
+
+The functions below carry the C ABI's names (``include/w8a8.h``) and only marshal
+arguments: they check dtypes, shapes, devices and contiguity of torch tensors, pass raw
+device pointers and the current CUDA stream, and raise ``W8A8Error`` on a non-zero status.
+Every computation runs in the library's CUDA kernels; there is no CPU path. Importing the
+package does not need a GPU, but every compute call does.
+
+    q, s = w8a8_smooth_rmsnorm_quant(x, gamma_smoothed, eps)
+    y = w8a8_gemm_dequant(q, s, wq, s_ch)
+"""
+import ctypes as C
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "W8A8Error", "lib", "LIB_PATH",
+    "w8a8_quantize_rows", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
+    "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
+    "w8a8_gemm_workspace_size_ex", "w8a8_device_status", "w8a8_status_string", "w8a8_version",
+    "Workspace",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw8a8.so")
+
+STATUS = {0: "W8A8_OK", -1: "W8A8_ERR_INVALID_ARG", -2: "W8A8_ERR_ALIGNMENT",
+          -3: "W8A8_ERR_UNSUPPORTED_SHAPE", -4: "W8A8_ERR_WORKSPACE", -5: "W8A8_ERR_CUDA",
+          -6: "W8A8_ERR_TIMEOUT", -7: "W8A8_ERR_NO_DEVICE"}
+
+# (name, restype, argtypes) of every function declared in include/w8a8.h
+_P, _I64, _I, _F, _SZ = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
+SIGNATURES = [
+    ("w8a8_quantize_rows", _I, [_P, _P, _I64, _I64, _P, _P, _P]),
+    ("w8a8_smooth_rmsnorm_quant", _I, [_P, _P, _P, _P, _F, _I64, _I64, _P, _P, _P]),
+    ("w8a8_silu_mul_quant", _I, [_P, _I64, _I64, _P, _P, _P]),
+    ("w8a8_gemm_workspace_size", _SZ, [_I64, _I64, _I64]),
+    ("w8a8_gemm_dequant", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    ("w8a8_gemm_dequant_ex", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _I, _I,
+                                  _I, _P]),
+    ("w8a8_gemm_workspace_size_ex", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
+    ("w8a8_device_status", _I, [_I]),
+    ("w8a8_status_string", C.c_char_p, [_I]),
+    ("w8a8_version", _I, []),
+]
+
+_lib = None
+_lock = threading.Lock()
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+
+
+def lib():
+    """The loaded CUDA library. Fails loudly when it has not been built: there is no
+    fallback implementation."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise ImportError(
+                        f"{LIB_PATH} is missing; build it with "
+                        "`python -m int8_w8a8_quantized_smoothed_b200.build`")
+                L = C.CDLL(LIB_PATH)
+                for name, res, args in SIGNATURES:
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = L
+    return _lib
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise W8A8Error(fn, rc)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def w8a8_status_string(status: int) -> str:
+    return lib().w8a8_status_string(int(status)).decode()
+
+
+def w8a8_version() -> int:
+    return lib().w8a8_version()
+
+
+def w8a8_device_status(reset: bool = False) -> int:
+    """Synchronizes the current device; returns 0 or -6 (a bounded wait ran out)."""
+    return lib().w8a8_device_status(1 if reset else 0)
+
+
+def w8a8_quantize_rows(x, smooth_inv=None, q=None, s_tok=None, stream=None):
+    """Per-token int8 quantization of bf16 x [M, K] (optionally x * smooth_inv)."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    if smooth_inv is not None:
+        _need(smooth_inv, "smooth_inv", torch.float32, (K,))
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _need(q, "q", torch.int8, (M, K))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_quantize_rows", lib().w8a8_quantize_rows(
+        _ptr(x), _ptr(smooth_inv), M, K, _ptr(q), _ptr(s_tok), _stream(stream)))
+    return q, s_tok
+
+
+def w8a8_smooth_rmsnorm_quant(x, gamma_smoothed, eps, residual=None, h_out=None, q=None,
+                              s_tok=None, stream=None):
+    """RMSNorm with SmoothQuant-folded gamma, fused with per-token quantization.
+    With `residual`, h = bf16(x + residual) is normalized and also returned."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    _need(gamma_smoothed, "gamma_smoothed", torch.float32, (K,))
+    if residual is not None:
+        _need(residual, "residual", torch.bfloat16, (M, K))
+        h_out = torch.empty_like(x) if h_out is None else h_out
+        _need(h_out, "h_out", torch.bfloat16, (M, K))
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _need(q, "q", torch.int8, (M, K))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_smooth_rmsnorm_quant", lib().w8a8_smooth_rmsnorm_quant(
+        _ptr(x), _ptr(residual), _ptr(h_out), _ptr(gamma_smoothed), float(eps), M, K, _ptr(q),
+        _ptr(s_tok), _stream(stream)))
+    if residual is not None:
+        return q, s_tok, h_out
+    return q, s_tok
+
+
+def w8a8_silu_mul_quant(gate_up, q=None, s_tok=None, stream=None):
+    """SiLU(gate) * up over the [M, 2I] gate|up halves, fused with per-token quantization."""
+    _need(gate_up, "gate_up", torch.bfloat16)
+    M, I2 = gate_up.shape
+    if I2 % 2:
+        raise ValueError("gate_up must have an even number of columns")
+    I = I2 // 2
+    q = torch.empty((M, I), dtype=torch.int8, device=gate_up.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=gate_up.device) if s_tok is None else s_tok
+    _need(q, "q", torch.int8, (M, I))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_silu_mul_quant", lib().w8a8_silu_mul_quant(
+        _ptr(gate_up), M, I, _ptr(q), _ptr(s_tok), _stream(stream)))
+    return q, s_tok
+
+
+def w8a8_gemm_workspace_size(M, N, K) -> int:
+    return int(lib().w8a8_gemm_workspace_size(M, N, K))
+
+
+def w8a8_gemm_workspace_size_ex(M, N, K, variant=0, splits=0, tile_n=0) -> int:
+    return int(lib().w8a8_gemm_workspace_size_ex(M, N, K, variant, splits, tile_n))
+
+
+class Workspace:
+    """A zero-filled device workspace that grows on demand (the library never allocates).
+    One instance serves calls issued in order on one stream."""
+
+    def __init__(self, device=None):
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        self.buf = None
+
+    def get(self, nbytes):
+        if nbytes == 0:
+            return None, 0
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=self.device)
+        return self.buf, self.buf.numel()
+
+
+_default_ws = {}
+
+
+def _workspace_for(device):
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _default_ws.get(key)
+    if ws is None:
+        ws = _default_ws[key] = Workspace(device)
+    return ws
+
+
+def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None,
+                         variant=0, splits=0, tile_n=0, stream=None):
+    """y = bf16((float(xq @ wq.T) * s_tok[:, None]) * s_ch[None, :]) on the tensor cores.
+    variant 0 = automatic, 1 = persistent tile kernel, 2 = swap-AB split-K kernel."""
+    _need(xq, "xq", torch.int8)
+    _need(wq, "wq", torch.int8)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2:
+        raise ValueError(f"xq [M,K] and wq [N,K] disagree on K: {K} vs {K2}")
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _need(s_ch, "s_ch", torch.float32, (N,))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N))
+    if acc_out is not None:
+        _need(acc_out, "acc_out", torch.int32, (M, N))
+    need = w8a8_gemm_workspace_size_ex(M, N, K, variant, splits, tile_n)
+    if workspace is None:
+        workspace = _workspace_for(xq.device)
+    if isinstance(workspace, Workspace):
+        wbuf, wbytes = workspace.get(need)
+    else:
+        wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
+                                   * workspace.element_size())
+    _check("w8a8_gemm_dequant", lib().w8a8_gemm_dequant_ex(
+        _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _ptr(acc_out),
+        _ptr(wbuf), wbytes, int(variant), int(splits), int(tile_n), _stream(stream)))
+    return y
+
+
+def w8a8_gemm_dequant(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None, stream=None):
+    return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=y, acc_out=acc_out,
+                                workspace=workspace, stream=stream)

@@ -1,0 +1,478 @@
+// C ABI of the W8A8 SmoothQuant linear path (declared in include/w8a8.h): argument
+// validation, kernel selection, TMA descriptor encoding and launches. Every compute step
+// runs in the kernels of rowquant.cuh and gemm.cuh; there is no host fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "gemm.cuh"
+#include "rowquant.cuh"
+#include "w8a8.h"
+
+namespace {
+
+using namespace w8a8;
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull; // 2 s per bounded wait
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int ok = -1; // -1 unknown, 0 unsupported, 1 sm_100
+    int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+std::set<std::pair<const void *, int>> g_smem_set;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// Current device if it is an sm_100 part; fills its SM count.
+int current_device(int *dev, int *num_sms)
+{
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) {
+        cudaGetLastError();
+        return W8A8_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &info = g_dev[d];
+    if (info.ok < 0) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, d) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) {
+            cudaGetLastError();
+            return W8A8_ERR_NO_DEVICE;
+        }
+        info.ok = (major == 10) ? 1 : 0;
+        info.num_sms = sms;
+    }
+    if (info.ok != 1)
+        return W8A8_ERR_NO_DEVICE;
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                             cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr) {
+            cudaGetLastError();
+            return W8A8_ERR_CUDA;
+        }
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *dev = d;
+    *num_sms = info.num_sms;
+    return W8A8_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+int ensure_smem(const void *kernel, int dev, int bytes)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto key = std::make_pair(kernel, dev);
+    if (g_smem_set.count(key))
+        return W8A8_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    g_smem_set.insert(key);
+    return W8A8_OK;
+}
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+// 2-D int8 [rows, K] K-contiguous tensor, box = 128 bytes of K x box_rows, 128B swizzle,
+// out-of-range elements read as zero.
+int encode_kmajor_i8(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ row kernels
+
+struct RowLaunch {
+    int nch;
+    int threads;
+};
+
+// One CTA per row; each thread holds nch vectors of 8 values (nch <= 4, <= 1024 threads).
+RowLaunch row_launch(int64_t K)
+{
+    const int64_t nvec = K / 8;
+    int nch = static_cast<int>((nvec + 255) / 256);
+    nch = nch < 1 ? 1 : (nch > 4 ? 4 : nch);
+    if (nch == 3)
+        nch = 4;
+    int64_t t = (nvec + nch - 1) / nch;
+    t = ((t + 31) / 32) * 32;
+    return RowLaunch{nch, static_cast<int>(t)};
+}
+
+int check_row_shape(int64_t M, int64_t K)
+{
+    if (M < 1 || K < 16)
+        return W8A8_ERR_INVALID_ARG;
+    if (K % 16 != 0 || K > 32768 || M > 0x7fffffffLL)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    return W8A8_OK;
+}
+
+template <int NCH>
+void launch_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int K, int8_t *q,
+                          float *s, int threads, cudaStream_t st)
+{
+    quantize_rows_kernel<NCH><<<static_cast<unsigned>(M), threads, 0, st>>>(x, sinv, K, q, s);
+}
+
+template <int NCH>
+void launch_rmsnorm(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
+                    int64_t M, int K, int8_t *q, float *s, int threads, cudaStream_t st)
+{
+    if (r)
+        rmsnorm_quant_kernel<NCH, true><<<static_cast<unsigned>(M), threads, 0, st>>>(
+            x, r, h, g, eps, K, q, s);
+    else
+        rmsnorm_quant_kernel<NCH, false><<<static_cast<unsigned>(M), threads, 0, st>>>(
+            x, r, h, g, eps, K, q, s);
+}
+
+template <int NCH>
+void launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int threads,
+                 cudaStream_t st)
+{
+    silu_mul_quant_kernel<NCH><<<static_cast<unsigned>(M), threads, 0, st>>>(gu, I, q, s);
+}
+
+// ------------------------------------------------------------------ GEMM planning
+
+struct GemmPlan {
+    int variant = 0; // 1 prefill, 2 decode
+    int tile_n = 256;
+    int nt = 16;          // decode token tile
+    int splits = 1;       // decode split count
+    int kb_per_split = 0; // decode k-blocks per split
+    size_t ws_bytes = 0;
+    size_t ticket_off = 0;
+};
+
+int decode_nt(int64_t M)
+{
+    return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+}
+
+int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int splits, int tile_n, int num_sms,
+              GemmPlan *p)
+{
+    if (variant < 0 || variant > 2 || splits < 0 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
+        return W8A8_ERR_INVALID_ARG;
+    if (variant == 0)
+        variant = (M <= 64) ? 2 : 1;
+    if (variant == 2 && M > 256)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    p->variant = variant;
+    const int64_t kblocks = (K + kBK - 1) / kBK;
+    if (variant == 1) {
+        if (tile_n == 0) {
+            const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
+            tile_n = tiles256 >= num_sms ? 256 : 128;
+        }
+        p->tile_n = tile_n;
+        p->ws_bytes = 0;
+        return W8A8_OK;
+    }
+    p->nt = decode_nt(M);
+    const int64_t nb = (N + kBM - 1) / kBM;
+    const int64_t per_sm = p->nt <= 128 ? 2 : 1;
+    int64_t sp = splits;
+    if (sp == 0) {
+        sp = (num_sms * per_sm) / nb;
+        if (sp < 1)
+            sp = 1;
+    }
+    if (sp > kblocks)
+        sp = kblocks;
+    if (sp > 65535)
+        sp = 65535;
+    const int64_t kb_per = (kblocks + sp - 1) / sp;
+    sp = (kblocks + kb_per - 1) / kb_per;
+    p->splits = static_cast<int>(sp);
+    p->kb_per_split = static_cast<int>(kb_per);
+    if (sp > 1) {
+        const size_t acc_bytes = static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
+        p->ticket_off = (acc_bytes + 255) & ~static_cast<size_t>(255);
+        p->ws_bytes = p->ticket_off + static_cast<size_t>(nb) * 4u;
+    } else {
+        p->ws_bytes = 0;
+    }
+    return W8A8_OK;
+}
+
+int check_gemm_shape(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 8 || K < 16)
+        return W8A8_ERR_INVALID_ARG;
+    if (N % 8 != 0 || K % 16 != 0 || K > 133144 || M > 0x7fffffffLL || N > 0x7fffffffLL)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    return W8A8_OK;
+}
+
+template <int BN, int STAGES>
+int launch_prefill(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
+                   const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
+                   int dev, int num_sms, cudaStream_t st)
+{
+    using Cfg = PrefillCfg<BN, STAGES>;
+    const void *fn = reinterpret_cast<const void *>(&gemm_prefill_kernel<BN, STAGES>);
+    int rc = ensure_smem(fn, dev, Cfg::kSmemBytes);
+    if (rc)
+        return rc;
+    const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    gemm_prefill_kernel<BN, STAGES><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(
+        ta, tb, s_tok, s_ch, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y, acc,
+        kWaitLimitNs);
+    return launch_status();
+}
+
+template <int NT, int STAGES, int MINB>
+int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
+                  const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
+                  uint16_t *y, int32_t *acc, void *ws, int dev, cudaStream_t st)
+{
+    using Cfg = DecodeCfg<NT, STAGES>;
+    const void *fn = reinterpret_cast<const void *>(&gemm_decode_kernel<NT, STAGES, MINB>);
+    int rc = ensure_smem(fn, dev, Cfg::kSmemBytes);
+    if (rc)
+        return rc;
+    const int64_t nb = (N + kBM - 1) / kBM;
+    dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>(p.splits));
+    int32_t *ws_acc = p.splits > 1 ? static_cast<int32_t *>(ws) : nullptr;
+    unsigned int *ws_ticket =
+        p.splits > 1 ? reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.ticket_off)
+                     : nullptr;
+    gemm_decode_kernel<NT, STAGES, MINB><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(
+        tw, tx, s_tok, s_ch, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+        p.kb_per_split, p.splits, y, acc, ws_acc, ws_ticket, kWaitLimitNs);
+    return launch_status();
+}
+
+} // namespace
+
+extern "C" {
+
+int w8a8_version(void)
+{
+    return (1 << 16) | 0;
+}
+
+const char *w8a8_status_string(int status)
+{
+    switch (status) {
+    case W8A8_OK:
+        return "ok";
+    case W8A8_ERR_INVALID_ARG:
+        return "invalid argument";
+    case W8A8_ERR_ALIGNMENT:
+        return "pointer not 16-byte aligned";
+    case W8A8_ERR_UNSUPPORTED_SHAPE:
+        return "unsupported shape";
+    case W8A8_ERR_WORKSPACE:
+        return "workspace missing or too small";
+    case W8A8_ERR_CUDA:
+        return "CUDA error";
+    case W8A8_ERR_TIMEOUT:
+        return "device-side wait timed out";
+    case W8A8_ERR_NO_DEVICE:
+        return "no sm_100 device";
+    default:
+        return "unknown status";
+    }
+}
+
+int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, int64_t K,
+                       int8_t *q, float *s_tok, w8a8_stream_t stream)
+{
+    if (!x || !q || !s_tok)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, K);
+    if (rc)
+        return rc;
+    if (!aligned16(x) || !aligned16(q) || (smooth_inv && !aligned16(smooth_inv)))
+        return W8A8_ERR_ALIGNMENT;
+    if (static_cast<const void *>(x) == static_cast<const void *>(q))
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    const RowLaunch L = row_launch(K);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (L.nch) {
+    case 1: launch_quantize_rows<1>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, st); break;
+    case 2: launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, st); break;
+    default: launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, st); break;
+    }
+    return launch_status();
+}
+
+int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a8_bf16 *h_out,
+                              const float *gamma_smoothed, float eps, int64_t M, int64_t K,
+                              int8_t *q, float *s_tok, w8a8_stream_t stream)
+{
+    if (!x || !gamma_smoothed || !q || !s_tok || ((residual == nullptr) != (h_out == nullptr)))
+        return W8A8_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f))
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, K);
+    if (rc)
+        return rc;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(gamma_smoothed) ||
+        (residual && (!aligned16(residual) || !aligned16(h_out))))
+        return W8A8_ERR_ALIGNMENT;
+    if (h_out && static_cast<const void *>(h_out) == static_cast<const void *>(x))
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    const RowLaunch L = row_launch(K);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (L.nch) {
+    case 1: launch_rmsnorm<1>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, st); break;
+    case 2: launch_rmsnorm<2>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, st); break;
+    default: launch_rmsnorm<4>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, st); break;
+    }
+    return launch_status();
+}
+
+int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *q, float *s_tok,
+                        w8a8_stream_t stream)
+{
+    if (!gate_up || !q || !s_tok)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, I);
+    if (rc)
+        return rc;
+    if (!aligned16(gate_up) || !aligned16(q))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    const RowLaunch L = row_launch(I);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (L.nch) {
+    case 1: launch_silu<1>(gate_up, M, (int)I, q, s_tok, L.threads, st); break;
+    case 2: launch_silu<2>(gate_up, M, (int)I, q, s_tok, L.threads, st); break;
+    default: launch_silu<4>(gate_up, M, (int)I, q, s_tok, L.threads, st); break;
+    }
+    return launch_status();
+}
+
+size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int splits,
+                                   int tile_n)
+{
+    if (check_gemm_shape(M, N, K))
+        return 0;
+    int dev, sms = 148;
+    if (current_device(&dev, &sms))
+        sms = 148;
+    GemmPlan p;
+    if (plan_gemm(M, N, K, variant, splits, tile_n, sms, &p))
+        return 0;
+    return p.ws_bytes;
+}
+
+size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    return w8a8_gemm_workspace_size_ex(M, N, K, 0, 0, 0);
+}
+
+int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                         const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
+                         int32_t *acc_out, void *workspace, size_t workspace_bytes, int variant,
+                         int splits, int tile_n, w8a8_stream_t stream)
+{
+    if (!xq || !s_tok || !wq || !s_ch || !y)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc)
+        return rc;
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(s_ch) || !aligned16(y) ||
+        (acc_out && !aligned16(acc_out)) || (workspace && !aligned16(workspace)))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    GemmPlan p;
+    if ((rc = plan_gemm(M, N, K, variant, splits, tile_n, sms, &p)))
+        return rc;
+    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
+        return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (p.variant == 1) {
+        CUtensorMap ta, tb;
+        if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, p.tile_n))
+            return W8A8_ERR_CUDA;
+        if (p.tile_n == 256)
+            return launch_prefill<256, 4>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
+        return launch_prefill<128, 6>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
+    }
+    CUtensorMap tw, tx;
+    if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
+        return W8A8_ERR_CUDA;
+    switch (p.nt) {
+    case 16: return launch_decode<16, 6, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
+    case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
+    case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
+    case 128: return launch_decode<128, 3, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
+    default: return launch_decode<256, 4, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
+    }
+}
+
+int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, const float *s_ch,
+                      int64_t M, int64_t N, int64_t K, w8a8_bf16 *y, int32_t *acc_out,
+                      void *workspace, size_t workspace_bytes, w8a8_stream_t stream)
+{
+    return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace,
+                                workspace_bytes, 0, 0, 0, stream);
+}
+
+int w8a8_device_status(int reset)
+{
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    if (reset) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+    }
+    return (word & kStatusTimeout) ? W8A8_ERR_TIMEOUT : W8A8_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,87 @@
+"""Shared test helpers: moving numpy inputs to the device and comparing against the oracle."""
+import numpy as np
+import torch
+
+import oracle
+
+SENTINEL_BF16 = 0x7FC1  # a NaN pattern no kernel writes
+SENTINEL_I8 = -128       # a code the kernels never produce
+
+
+def dev_bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host_bf16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def with_canary(shape, dtype, fill):
+    """An output tensor of `shape` carved from a larger buffer pre-filled with `fill`; the
+    returned `check()` verifies every element beyond the tensor is still `fill`."""
+    n = int(np.prod(shape))
+    buf = torch.full((n + 256,), fill, dtype=dtype, device="cuda")
+    t = buf[:n].view(*shape)
+
+    def check():
+        tail = buf[n:]
+        assert bool((tail == fill).all()), "write past the end of an output"
+    return t, check
+
+
+def bf16_out(shape):
+    n = int(np.prod(shape))
+    buf = torch.full((n + 256,), SENTINEL_BF16, dtype=torch.int16, device="cuda")
+    t = buf[:n].view(torch.bfloat16).view(*shape)
+
+    def check():
+        assert bool((buf[n:] == SENTINEL_BF16).all()), "write past the end of an output"
+    return t, check
+
+
+def i8_out(shape):
+    return with_canary(shape, torch.int8, SENTINEL_I8)
+
+
+def f32_out(shape):
+    return with_canary(shape, torch.float32, float("nan"))
+
+
+def bf16_ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in representable bf16 steps between two bf16 bit-pattern arrays."""
+    def ordered(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, 0x8000 - (u & 0x7FFF), 0x8000 + u)
+    return np.abs(ordered(a) - ordered(b))
+
+
+def assert_rms_rows_match(got_q, got_s, x, gamma, eps, residual=None, ref=None):
+    """GPU smoothed-RMSNorm results against the oracle. Rows whose binary64 mean of squares
+    lies so close to a binary32 rounding boundary that another summation order may round it
+    the other way (oracle flag `ambiguous`) may match either neighbouring binary32 value;
+    every other row must match exactly."""
+    if ref is None:
+        ref = oracle.smooth_rmsnorm_quant(x, gamma, eps, residual=residual)
+    bad = np.where((got_s != ref["s"]) | (got_q != ref["q"]).any(axis=1))[0]
+    for m in bad:
+        assert ref["ambiguous"][m], f"row {m} differs and is not ambiguous"
+        ok = False
+        for direction in (np.inf, -np.inf):
+            ms = ref["ms"].copy()
+            ms[m] = np.nextafter(np.float32(ms[m]), np.float32(direction))
+            alt = oracle.smooth_rmsnorm_quant(x[m:m + 1], gamma, eps,
+                                              residual=None if residual is None
+                                              else residual[m:m + 1],
+                                              ms_override=ms[m:m + 1])
+            if alt["s"][0] == got_s[m] and np.array_equal(alt["q"][0], got_q[m]):
+                ok = True
+        assert ok, f"row {m} matches neither admissible mean of squares"
+    return ref, len(bad)

@@ -1,0 +1,133 @@
+"""Parity of the tcgen05 INT8 GEMM + dequant kernels with the oracle, through the C ABI:
+int32 accumulators and bf16 outputs bit-exact (the bar is 1 bf16 ulp; the epilogue is built
+to the oracle's operation order, so 0 is expected and asserted, and the ulp distance is
+reported on failure). Both kernels (persistent tile / swap-AB split-K) are run on the same
+shapes, including ragged M, N and K tails, several tiles, and extreme accumulators."""
+import numpy as np
+import pytest
+import torch
+
+import int8_w8a8_quantized_smoothed_b200 as w8
+import oracle
+from int8_w8a8_quantized_smoothed_b200 import synth
+from helpers import bf16_out, bf16_ulp_distance, dev, host, host_bf16, with_canary
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(M, N, K, seed):
+    xq = synth.int8_codes((M, K), seed)
+    wq = synth.int8_codes((N, K), seed + 1)
+    st = synth.scales(M, seed + 2, 1e-3, 0.5)
+    sc = synth.scales(N, seed + 3, 1e-4, 2e-2)
+    return xq, st, wq, sc
+
+
+def _run(xq, st, wq, sc, variant, splits=0, tile_n=0):
+    M, N = xq.shape[0], wq.shape[0]
+    y, cy = bf16_out((M, N))
+    acc, ca = with_canary((M, N), torch.int32, -7)
+    w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), y=y, acc_out=acc,
+                            variant=variant, splits=splits, tile_n=tile_n)
+    torch.cuda.synchronize()
+    cy(); ca()
+    return host_bf16(y), host(acc)
+
+
+def _compare(y, acc, y_ref, acc_ref):
+    assert np.array_equal(acc, acc_ref), f"{(acc != acc_ref).sum()} accumulators differ"
+    d = bf16_ulp_distance(y, y_ref)
+    assert d.max() <= 1, f"bf16 differs by up to {d.max()} ulp"
+    assert np.array_equal(y, y_ref), f"{(d > 0).sum()} outputs differ by 1 ulp"
+
+
+DECODE_SHAPES = [(1, 8, 16), (1, 512, 256), (16, 512, 256), (8, 1024, 4096), (3, 136, 400),
+                 (33, 1032, 4096), (64, 1024, 14336), (17, 256, 4112), (100, 384, 1024),
+                 (256, 264, 512), (129, 128, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_decode_kernel_bit_exact(M, N, K, splits):
+    xq, st, wq, sc = _inputs(M, N, K, seed=M + N + K)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    y, acc = _run(xq, st, wq, sc, variant=2, splits=splits)
+    _compare(y, acc, y_ref, acc_ref)
+
+
+PREFILL_SHAPES = [(1, 8, 16), (16, 512, 256), (128, 256, 128), (129, 264, 400), (200, 136, 208),
+                  (300, 1024, 4096), (512, 2048, 1024), (257, 520, 14336), (1000, 3000, 64)]
+
+
+@pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
+@pytest.mark.parametrize("tile_n", [128, 256])
+def test_prefill_kernel_bit_exact(M, N, K, tile_n):
+    xq, st, wq, sc = _inputs(M, N, K, seed=3 * M + N + K)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    y, acc = _run(xq, st, wq, sc, variant=1, tile_n=tile_n)
+    _compare(y, acc, y_ref, acc_ref)
+
+
+def test_persistent_kernel_many_tiles_per_cta():
+    # more tiles than SMs: every CTA loops over several tiles and both TMEM accumulators
+    M, N, K = 2048, 4096, 256
+    xq, st, wq, sc = _inputs(M, N, K, 5)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    for tn in (128, 256):
+        y, acc = _run(xq, st, wq, sc, variant=1, tile_n=tn)
+        _compare(y, acc, y_ref, acc_ref)
+
+
+def test_extreme_accumulators():
+    # |acc| = 127 * 127 * K for K = 14336 (about 2.3e8 > 2^24): int->float rounding matters
+    M, N, K = 4, 16, 14336
+    xq = np.full((M, K), 127, np.int8)
+    xq[1] = -127
+    wq = np.full((N, K), 127, np.int8)
+    wq[3] = -127
+    st = synth.scales(M, 1)
+    sc = synth.scales(N, 2)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    assert acc_ref[0, 0] == 127 * 127 * K
+    for variant in (1, 2):
+        y, acc = _run(xq, st, wq, sc, variant=variant)
+        _compare(y, acc, y_ref, acc_ref)
+
+
+def test_auto_variant_and_workspace_reuse():
+    # the split-K workspace must come back zero-filled: run twice through one workspace
+    for (M, N, K) in [(8, 6144, 4096), (64, 4096, 4096), (512, 1024, 1024)]:
+        xq, st, wq, sc = _inputs(M, N, K, 11)
+        y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+        ws = w8.Workspace()
+        for _ in range(2):
+            y = w8.w8a8_gemm_dequant(dev(xq), dev(st), dev(wq), dev(sc), workspace=ws)
+            torch.cuda.synchronize()
+            assert np.array_equal(host_bf16(y), y_ref)
+        if ws.buf is not None:
+            assert int(ws.buf.count_nonzero()) == 0
+
+
+def test_zero_scales_give_zero():
+    M, N, K = 8, 64, 256
+    xq, st, wq, sc = _inputs(M, N, K, 13)
+    st[2] = 0.0
+    sc[5] = 0.0
+    y_ref, _ = oracle.gemm_dequant(xq, st, wq, sc)
+    for variant in (1, 2):
+        y = w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), variant=variant)
+        yh = host_bf16(y)
+        assert np.array_equal(yh, y_ref)
+        assert not (yh[2] & 0x7FFF).any() and not (yh[:, 5] & 0x7FFF).any()
+
+
+def test_workspace_too_small_is_reported():
+    M, N, K = 8, 1024, 4096
+    xq, st, wq, sc = _inputs(M, N, K, 1)
+    need = w8.w8a8_gemm_workspace_size_ex(M, N, K, 2, 4, 0)
+    assert need > 0
+    small = torch.zeros(need - 4, dtype=torch.uint8, device="cuda")
+    with pytest.raises(w8.W8A8Error, match="WORKSPACE"):
+        w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), workspace=small, variant=2,
+                                splits=4)
+    assert w8.w8a8_device_status(reset=True) == 0

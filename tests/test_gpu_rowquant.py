@@ -1,0 +1,121 @@
+"""Parity of the per-token quantization kernels with the oracle, through the C ABI:
+int8 codes, fp32 scales and bf16 residual sums bit-exact, on shapes spanning one vector per
+thread up to the largest rows, ragged rows and zero rows."""
+import numpy as np
+import pytest
+import torch
+
+import int8_w8a8_quantized_smoothed_b200 as w8
+import oracle
+from int8_w8a8_quantized_smoothed_b200 import synth
+from helpers import (assert_rms_rows_match, bf16_out, dev, dev_bf16, f32_out, host, host_bf16,
+                     i8_out)
+
+pytestmark = pytest.mark.gpu
+
+ROW_SHAPES = [(1, 16), (3, 48), (16, 256), (37, 4096), (5, 8192), (64, 14336), (3, 28672),
+              (2, 32768), (300, 4096), (7, 4112)]
+
+
+def _sinv(K, seed):
+    g = synth.gamma(K, seed)  # positive values around 1
+    return (1.0 / np.abs(g)).astype(np.float32)
+
+
+@pytest.mark.parametrize("M,K", ROW_SHAPES)
+@pytest.mark.parametrize("smooth", [False, True])
+def test_quantize_rows_bit_exact(M, K, smooth):
+    x = synth.activation(M, K, seed=M * 7 + K)
+    sinv = _sinv(K, K) if smooth else None
+    q_ref, s_ref = oracle.quantize_rows(x, sinv)
+    q, cq = i8_out((M, K))
+    s, cs = f32_out((M,))
+    w8.w8a8_quantize_rows(dev_bf16(x), None if sinv is None else dev(sinv), q=q, s_tok=s)
+    torch.cuda.synchronize()
+    cq(); cs()
+    assert np.array_equal(host(s), s_ref)
+    assert np.array_equal(host(q), q_ref)
+
+
+def test_quantize_rows_zero_and_tie_rows():
+    K = 64
+    x = np.zeros((3, K), dtype=np.float32)
+    x[1, :8] = [2.5, 3.5, -2.5, -3.5, 0.5, -0.5, 1.5, 127.0]  # s = 1: exact .5 ties
+    x[2, 5] = -7.0
+    xb = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    q_ref, s_ref = oracle.quantize_rows(xb)
+    q, s = w8.w8a8_quantize_rows(dev_bf16(xb))
+    assert np.array_equal(host(s), s_ref) and np.array_equal(host(q), q_ref)
+    assert host(s)[0] == 0 and not host(q)[0].any()
+    assert list(host(q)[1, :8]) == [2, 4, -2, -4, 0, 0, 2, 127]
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 256), (33, 4096), (20, 8192), (3, 48), (129, 4096),
+                                 (2, 28672)])
+@pytest.mark.parametrize("with_residual", [False, True])
+def test_smooth_rmsnorm_quant_bit_exact(M, K, with_residual):
+    x = synth.activation(M, K, seed=3 * M + K)
+    gam = synth.gamma(K, seed=K + 1)
+    s_fac = _sinv(K, K + 2)  # any positive smoothing factors
+    gf, _ = oracle.fold_gamma(gam, s_fac)
+    res = synth.normal_bf16((M, K), seed=M + 5) if with_residual else None
+    eps = 1e-5
+    q, cq = i8_out((M, K))
+    s, cs = f32_out((M,))
+    if with_residual:
+        h, ch = bf16_out((M, K))
+        w8.w8a8_smooth_rmsnorm_quant(dev_bf16(x), dev(gf), eps, residual=dev_bf16(res), h_out=h,
+                                     q=q, s_tok=s)
+    else:
+        w8.w8a8_smooth_rmsnorm_quant(dev_bf16(x), dev(gf), eps, q=q, s_tok=s)
+    torch.cuda.synchronize()
+    cq(); cs()
+    ref, _ = assert_rms_rows_match(host(q), host(s), x, gf, eps, residual=res)
+    if with_residual:
+        ch()
+        assert np.array_equal(host_bf16(h), ref["h"])
+
+
+def test_smooth_rmsnorm_h_out_may_alias_residual():
+    M, K = 9, 512
+    x = synth.activation(M, K, 1)
+    res = synth.normal_bf16((M, K), 2)
+    gf = synth.gamma(K, 3)
+    ref = oracle.smooth_rmsnorm_quant(x, gf, 1e-5, residual=res)
+    r = dev_bf16(res)
+    q, s, h = w8.w8a8_smooth_rmsnorm_quant(dev_bf16(x), dev(gf), 1e-5, residual=r, h_out=r)
+    assert np.array_equal(host_bf16(h), ref["h"])
+    assert_rms_rows_match(host(q), host(s), x, gf, 1e-5, residual=res, ref=ref)
+
+
+@pytest.mark.parametrize("M,I", [(1, 16), (9, 256), (33, 14336), (4, 28672), (130, 4096),
+                                 (2, 14352)])
+def test_silu_mul_quant_bit_exact(M, I):
+    gu = synth.normal_bf16((M, 2 * I), seed=M + I, std=2.5)
+    if M > 1:  # a row reaching the exp overflow/underflow ranges
+        gu[1, :8] = synth.normal_bf16((1, 8), 1)[0]
+        vals = np.array([95.0, -95.0, 88.5, -88.5, 104.5, -104.5, 0.0, -0.0], np.float32)
+        gu[1, :8] = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy() \
+            .view(np.uint16)
+    q_ref, s_ref = oracle.silu_mul_quant(gu)
+    q, cq = i8_out((M, I))
+    s, cs = f32_out((M,))
+    w8.w8a8_silu_mul_quant(dev_bf16(gu), q=q, s_tok=s)
+    torch.cuda.synchronize()
+    cq(); cs()
+    assert np.array_equal(host(s), s_ref)
+    assert np.array_equal(host(q), q_ref)
+
+
+def test_weight_rtn_through_quantize_rows():
+    # offline weight prep: quantize_rows(W, s) is the per-output-channel RTN of diag(s)-smoothed W
+    N, K = 96, 4096
+    w = synth.weight(N, K, 9)
+    s_fac = (1.0 / _sinv(K, 10)).astype(np.float32)
+    wq_ref, sch_ref = oracle.rtn_weights(w, s_fac)
+    wq, sch = w8.w8a8_quantize_rows(dev_bf16(w), dev(s_fac))
+    assert np.array_equal(host(wq), wq_ref) and np.array_equal(host(sch), sch_ref)
+
+
+def test_device_status_clean():
+    assert w8.w8a8_device_status(reset=True) == 0
