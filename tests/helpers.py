@@ -26,14 +26,16 @@ def host(t: torch.Tensor) -> np.ndarray:
 
 def with_canary(shape, dtype, fill):
     """An output tensor of `shape` carved from a larger buffer pre-filled with `fill`; the
-    returned `check()` verifies every element beyond the tensor is still `fill`."""
+    returned `check()` verifies every element beyond the tensor still holds `fill`'s bit
+    pattern (compared as integers, so a NaN fill works too)."""
     n = int(np.prod(shape))
     buf = torch.full((n + 256,), fill, dtype=dtype, device="cuda")
     t = buf[:n].view(*shape)
+    ibits = {1: torch.int8, 2: torch.int16, 4: torch.int32, 8: torch.int64}[buf.element_size()]
+    ref = buf[n:].clone().view(ibits)
 
     def check():
-        tail = buf[n:]
-        assert bool((tail == fill).all()), "write past the end of an output"
+        assert torch.equal(buf[n:].view(ibits), ref), "write past the end of an output"
     return t, check
 
 
