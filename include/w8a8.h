@@ -158,6 +158,38 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
                                    int tile_n);
 
 /*
+ * Small-M GEMM for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers of this library
+ * that hold no device allocator of their own, or must not use one at the moment they call:
+ * a plugin or hook run inside another runtime's launch path, code working within a fixed,
+ * pre-planned memory budget, or code running while a stream is being captured. For them
+ * cudaMalloc would synchronize the device, fail, or break the budget, so they cannot
+ * provide the zero-filled workspace that w8a8_gemm_dequant's split-K kernel needs.
+ *
+ * Computes exactly what w8a8_gemm_dequant computes, always with the swap-AB split-K kernel
+ * (M <= 256), and allocates nothing. Its split-K scratch is a file-scope device array of
+ * W8A8_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library; every GPU on which the library is
+ * loaded holds that array until the process exits. The caller still owns and passes every
+ * input and output. Arguments and requirements are those of w8a8_gemm_dequant without
+ * acc_out and workspace.
+ *   - Returns W8A8_ERR_WORKSPACE when this shape's split-K scratch (M * N * 4 bytes plus 4
+ *     bytes per 128 output channels, when more than one K split is used) exceeds
+ *     W8A8_NOALLOC_SCRATCH_BYTES; W8A8_ERR_UNSUPPORTED_SHAPE for M > 256.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Each call clears the part of the array it uses (cudaMemsetAsync on `stream`) before
+ *     its kernel runs, so an earlier failed call leaves no stale state.
+ *   - All calls on a device share the one array and it keeps the last call's contents:
+ *     calls whose kernels can overlap on the GPU (different streams without ordering
+ *     between them) race on it and give wrong results. Serialize them.
+ */
+#define W8A8_NOALLOC_SCRATCH_BYTES (4u << 20)
+W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                                       const float *s_ch, int64_t M, int64_t N, int64_t K,
+                                       w8a8_bf16 *y, w8a8_stream_t stream);
+
+/*
  * Device status: synchronizes the current device, then returns W8A8_OK or
  * W8A8_ERR_TIMEOUT if any kernel of this library on it gave up a bounded wait (every
  * mbarrier and ticket wait in the kernels is limited, ~2 s) since the last reset.

@@ -19,7 +19,8 @@ __all__ = [
     "W8A8Error", "lib", "LIB_PATH",
     "w8a8_quantize_rows", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
-    "w8a8_gemm_workspace_size_ex", "w8a8_device_status", "w8a8_status_string", "w8a8_version",
+    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_device_status",
+    "w8a8_status_string", "w8a8_version",
     "Workspace",
 ]
 
@@ -40,6 +41,7 @@ SIGNATURES = [
     ("w8a8_gemm_dequant_ex", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _I, _I,
                                   _I, _P]),
     ("w8a8_gemm_workspace_size_ex", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
+    ("w8a8_gemm_dequant_noalloc", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("w8a8_device_status", _I, [_I]),
     ("w8a8_status_string", C.c_char_p, [_I]),
     ("w8a8_version", _I, []),
@@ -239,3 +241,25 @@ def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=No
 def w8a8_gemm_dequant(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None, stream=None):
     return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=y, acc_out=acc_out,
                                 workspace=workspace, stream=stream)
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20  # W8A8_NOALLOC_SCRATCH_BYTES in include/w8a8.h
+
+
+def w8a8_gemm_dequant_noalloc(xq, s_tok, wq, s_ch, y=None, stream=None):
+    """The small-M (M <= 256) GEMM + dequant without any device allocation by the library:
+    its split-K scratch is a fixed 4 MiB array inside the library, for callers that cannot
+    allocate (see include/w8a8.h). Only `y` is allocated here, and only if not given."""
+    _need(xq, "xq", torch.int8)
+    _need(wq, "wq", torch.int8)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2:
+        raise ValueError(f"xq [M,K] and wq [N,K] disagree on K: {K} vs {K2}")
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _need(s_ch, "s_ch", torch.float32, (N,))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N))
+    _check("w8a8_gemm_dequant_noalloc", lib().w8a8_gemm_dequant_noalloc(
+        _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _stream(stream)))
+    return y

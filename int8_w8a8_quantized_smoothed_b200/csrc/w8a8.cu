@@ -476,3 +476,76 @@ int w8a8_device_status(int reset)
 }
 
 } // extern "C"
+
+// ------------------------------------------------------------------ no-allocation GEMM
+
+namespace {
+
+// Split-K scratch of w8a8_gemm_dequant_noalloc: accumulators and tickets live here instead
+// of in a caller-provided workspace. Host code must not pass `g_noalloc_scratch` itself to a
+// kernel (on the host it names a host-side shadow, not device memory); it passes the device
+// address looked up by noalloc_scratch().
+__device__ __align__(256) unsigned char g_noalloc_scratch[W8A8_NOALLOC_SCRATCH_BYTES];
+
+void *g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on device `dev` (the current device), looked up once.
+int noalloc_scratch(int dev, void **out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return W8A8_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return W8A8_OK;
+}
+
+} // namespace
+
+extern "C" int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                                         const float *s_ch, int64_t M, int64_t N, int64_t K,
+                                         w8a8_bf16 *y, w8a8_stream_t stream)
+{
+    if (!xq || !s_tok || !wq || !s_ch || !y)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc)
+        return rc;
+    if (M > 256)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(s_ch) || !aligned16(y))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    GemmPlan p;
+    if ((rc = plan_gemm(M, N, K, 2, 0, 0, sms, &p)))
+        return rc;
+    if (p.ws_bytes > W8A8_NOALLOC_SCRATCH_BYTES)
+        return W8A8_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (p.ws_bytes > 0) {
+        if ((rc = noalloc_scratch(dev, &scratch)))
+            return rc;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (p.ws_bytes > 0 && cudaMemsetAsync(scratch, 0, p.ws_bytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    CUtensorMap tw, tx;
+    if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
+        return W8A8_ERR_CUDA;
+    switch (p.nt) {
+    case 16: return launch_decode<16, 6, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
+    case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
+    case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
+    case 128: return launch_decode<128, 3, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
+    default: return launch_decode<256, 4, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
+    }
+}
