@@ -134,8 +134,9 @@ W8A8_API size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * workspace/workspace_bytes: see w8a8_gemm_workspace_size (may be NULL/0 when it returns 0).
  * Requires M >= 1, N >= 8, N % 8 == 0, K >= 16, K % 16 == 0, K <= 133144 (so that
  * 127 * 127 * K fits in int32), M, N <= 2^31 - 1.
- * Small M (at most 256 tokens) runs a swap-AB split-K kernel that streams the weight;
- * larger M runs a persistent tile kernel. Both give identical results.
+ * Small M (at most 64 tokens by default, up to 256 on request) runs a persistent swap-AB
+ * stream-K kernel that streams the weight; larger M runs a persistent tile kernel. Both give
+ * identical results.
  */
 W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq,
                       const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
@@ -145,16 +146,15 @@ W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_
 /*
  * The same GEMM with the kernel chosen by the caller, for tests and tuning:
  * variant 0 = automatic (as w8a8_gemm_dequant), 1 = persistent tile kernel, 2 = swap-AB
- * split-K kernel (M <= 256 only). splits = 0 picks the split count automatically, otherwise
- * the K range is cut into at most `splits` parts (variant 2). tile_n = 0 automatic, else 128
- * or 256 (variant 1). The workspace needed is w8a8_gemm_workspace_size_ex() of the same
- * arguments.
+ * stream-K kernel (M <= 256 only). ctas (variant 2) = number of persistent CTAs sharing the
+ * weight stream, 0 = one per SM. tile_n (variant 1) = 0 automatic, else 128 or 256. The
+ * workspace needed is w8a8_gemm_workspace_size_ex() of the same arguments.
  */
 W8A8_API int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
                          const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
                          int32_t *acc_out, void *workspace, size_t workspace_bytes,
-                         int variant, int splits, int tile_n, w8a8_stream_t stream);
-W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int splits,
+                         int variant, int ctas, int tile_n, w8a8_stream_t stream);
+W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int ctas,
                                    int tile_n);
 
 /*
@@ -165,17 +165,19 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
  * a plugin or hook run inside another runtime's launch path, code working within a fixed,
  * pre-planned memory budget, or code running while a stream is being captured. For them
  * cudaMalloc would synchronize the device, fail, or break the budget, so they cannot
- * provide the zero-filled workspace that w8a8_gemm_dequant's split-K kernel needs.
+ * provide the zero-filled workspace that w8a8_gemm_dequant's stream-K kernel needs.
  *
- * Computes exactly what w8a8_gemm_dequant computes, always with the swap-AB split-K kernel
- * (M <= 256), and allocates nothing. Its split-K scratch is a file-scope device array of
- * W8A8_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library; every GPU on which the library is
+ * Computes exactly what w8a8_gemm_dequant computes, always with the swap-AB stream-K kernel
+ * (M <= 256), and allocates nothing. Its scratch is a file-scope device array of
+ * W8A8_NOALLOC_SCRATCH_BYTES (8 MiB) inside the library; every GPU on which the library is
  * loaded holds that array until the process exits. The caller still owns and passes every
  * input and output. Arguments and requirements are those of w8a8_gemm_dequant without
  * acc_out and workspace.
- *   - Returns W8A8_ERR_WORKSPACE when this shape's split-K scratch (M * N * 4 bytes plus 4
- *     bytes per 128 output channels, when more than one K split is used) exceeds
- *     W8A8_NOALLOC_SCRATCH_BYTES; W8A8_ERR_UNSUPPORTED_SHAPE for M > 256.
+ *   - Returns W8A8_ERR_WORKSPACE when this shape's scratch exceeds
+ *     W8A8_NOALLOC_SCRATCH_BYTES: M * 512 bytes of partial sums per CTA plus 4 bytes per CTA
+ *     (one CTA per SM, fewer when the weight has fewer 128 x 128 blocks), needed only when a
+ *     CTA's share of the weight stream ends inside a 128-channel block. So on a 148-SM B200
+ *     M <= 110 always fits. W8A8_ERR_UNSUPPORTED_SHAPE for M > 256.
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
  *   - Each call clears the part of the array it uses (cudaMemsetAsync on `stream`) before
@@ -184,7 +186,7 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
  *     calls whose kernels can overlap on the GPU (different streams without ordering
  *     between them) race on it and give wrong results. Serialize them.
  */
-#define W8A8_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define W8A8_NOALLOC_SCRATCH_BYTES (8u << 20)
 W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, const int8_t *wq,
                                        const float *s_ch, int64_t M, int64_t N, int64_t K,
                                        w8a8_bf16 *y, w8a8_stream_t stream);
@@ -192,7 +194,7 @@ W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, con
 /*
  * Device status: synchronizes the current device, then returns W8A8_OK or
  * W8A8_ERR_TIMEOUT if any kernel of this library on it gave up a bounded wait (every
- * mbarrier and ticket wait in the kernels is limited, ~2 s) since the last reset.
+ * mbarrier and cross-CTA flag wait in the kernels is limited, ~2 s) since the last reset.
  * reset != 0 clears the word. Returns W8A8_ERR_CUDA if synchronization fails.
  */
 W8A8_API int w8a8_device_status(int reset);

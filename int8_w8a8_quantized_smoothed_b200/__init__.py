@@ -176,8 +176,8 @@ def w8a8_gemm_workspace_size(M, N, K) -> int:
     return int(lib().w8a8_gemm_workspace_size(M, N, K))
 
 
-def w8a8_gemm_workspace_size_ex(M, N, K, variant=0, splits=0, tile_n=0) -> int:
-    return int(lib().w8a8_gemm_workspace_size_ex(M, N, K, variant, splits, tile_n))
+def w8a8_gemm_workspace_size_ex(M, N, K, variant=0, ctas=0, tile_n=0) -> int:
+    return int(lib().w8a8_gemm_workspace_size_ex(M, N, K, variant, ctas, tile_n))
 
 
 class Workspace:
@@ -209,9 +209,10 @@ def _workspace_for(device):
 
 
 def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None,
-                         variant=0, splits=0, tile_n=0, stream=None):
+                         variant=0, ctas=0, tile_n=0, stream=None):
     """y = bf16((float(xq @ wq.T) * s_tok[:, None]) * s_ch[None, :]) on the tensor cores.
-    variant 0 = automatic, 1 = persistent tile kernel, 2 = swap-AB split-K kernel."""
+    variant 0 = automatic, 1 = persistent tile kernel, 2 = swap-AB stream-K kernel
+    (ctas = persistent CTAs, 0 = one per SM)."""
     _need(xq, "xq", torch.int8)
     _need(wq, "wq", torch.int8)
     M, K = xq.shape
@@ -224,7 +225,7 @@ def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=No
     _need(y, "y", torch.bfloat16, (M, N))
     if acc_out is not None:
         _need(acc_out, "acc_out", torch.int32, (M, N))
-    need = w8a8_gemm_workspace_size_ex(M, N, K, variant, splits, tile_n)
+    need = w8a8_gemm_workspace_size_ex(M, N, K, variant, ctas, tile_n)
     if workspace is None:
         workspace = _workspace_for(xq.device)
     if isinstance(workspace, Workspace):
@@ -234,7 +235,7 @@ def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=No
                                    * workspace.element_size())
     _check("w8a8_gemm_dequant", lib().w8a8_gemm_dequant_ex(
         _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _ptr(acc_out),
-        _ptr(wbuf), wbytes, int(variant), int(splits), int(tile_n), _stream(stream)))
+        _ptr(wbuf), wbytes, int(variant), int(ctas), int(tile_n), _stream(stream)))
     return y
 
 
@@ -243,12 +244,12 @@ def w8a8_gemm_dequant(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None,
                                 workspace=workspace, stream=stream)
 
 
-NOALLOC_SCRATCH_BYTES = 4 << 20  # W8A8_NOALLOC_SCRATCH_BYTES in include/w8a8.h
+NOALLOC_SCRATCH_BYTES = 8 << 20  # W8A8_NOALLOC_SCRATCH_BYTES in include/w8a8.h
 
 
 def w8a8_gemm_dequant_noalloc(xq, s_tok, wq, s_ch, y=None, stream=None):
     """The small-M (M <= 256) GEMM + dequant without any device allocation by the library:
-    its split-K scratch is a fixed 4 MiB array inside the library, for callers that cannot
+    its stream-K scratch is a fixed 8 MiB array inside the library, for callers that cannot
     allocate (see include/w8a8.h). Only `y` is allocated here, and only if not given."""
     _need(xq, "xq", torch.int8)
     _need(wq, "wq", torch.int8)

@@ -13,9 +13,9 @@
 // prefill kernel: persistent over 128 x BN output tiles (BN = 128 or 256), two TMEM
 //   accumulators so the epilogue of tile t overlaps the MMAs of tile t+1.
 // decode kernel: swap-AB (D^T = W X^T: the weight fills the MMA's 128-row side, the <= 256
-//   tokens its N side) and split-K over the grid's y dimension; partial int32 sums meet in
-//   an int32 workspace through red.global.add (exact, order-free), and the last CTA of
-//   each 128-channel block (atomic ticket) dequantizes and re-zeroes the workspace.
+//   tokens its N side), persistent stream-K: each CTA streams an equal contiguous share of
+//   the (channel block, k-block) units, several k-blocks per pipeline stage; blocks split
+//   between CTAs are summed exactly in int32 by the block's owner (see below).
 #pragma once
 
 #include "ptx.cuh"
@@ -230,55 +230,101 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 }
 
-// ---------------------------------------------------------------- decode (swap-AB split-K)
+// ---------------------------------------------------------------- decode (swap-AB stream-K)
+//
+// Work units are (channel block t, k-block kb) pairs in tile-major order, U = NB * KB of
+// them. CTA g of G (one per SM, persistent) takes the contiguous range
+// [floor(g U / G), floor((g+1) U / G)), so every SM streams the same number of weight bytes.
+// A range is cut into segments at channel-block boundaries. A segment covering a whole block
+// is dequantized and stored directly. A block split between CTAs has one owner, the segment
+// holding k-block 0 (the last segment of its CTA, so it finishes last); every other segment
+// of that block (the first segment of a later CTA) stores its int32 partial in the CTA's own
+// workspace slot and raises the CTA's flag; the owner waits for the flags of the later CTAs
+// that share its block, adds their partials (exact int32), dequantizes, stores, and lowers
+// the flags again so the workspace is zero between calls.
 
-template <int NT, int STAGES> struct DecodeCfg {
-    static constexpr int kWBytes = kBM * kBK;  // 128 weight rows x 128 B
-    static constexpr int kXBytes = NT * kBK;   // NT token rows x 128 B
-    static constexpr int kStageBytes = kWBytes + kXBytes;
+template <int NT, int STAGES, int KPS> struct DecodeCfg {
+    static constexpr int kWBytes = kBM * kBK;           // one k-block of 128 weight rows
+    static constexpr int kXBytes = NT * kBK;            // one k-block of NT token rows
+    static constexpr int kStageBytes = KPS * (kWBytes + kXBytes);
     static constexpr int kBarOff = STAGES * kStageBytes;
-    static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 2) * 8 + 16 + 16 + 1024;
-    static constexpr int kTmemCols = NT < 32 ? 32 : NT;
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot, flag word
+    static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 32 + 1024;
+    static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
     static_assert(kXBytes % 1024 == 0, "token tile must keep stages 1024-byte aligned");
+    static_assert(kTmemCols <= 512, "two accumulators must fit TMEM");
 };
 
-template <int NT, int STAGES, int MINB>
-__global__ void __launch_bounds__(kGemmThreads, MINB)
+// CTA holding unit v under the even split of U units over G CTAs.
+__host__ __device__ __forceinline__ int64_t sk_owner_of(int64_t v, int64_t U, int64_t G)
+{
+    int64_t c = (v * G) / U;
+    while (c + 1 < G && ((c + 1) * U) / G <= v)
+        ++c;
+    while (c > 0 && (c * U) / G > v)
+        --c;
+    return c;
+}
+
+struct SkSegment {
+    int64_t t;   // channel block
+    int kb0, kb1; // k-block range [kb0, kb1)
+};
+
+// Segment iterator over [u, u1): next segment starting at u.
+__device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
+{
+    SkSegment sg;
+    sg.t = u / KB;
+    sg.kb0 = static_cast<int>(u - sg.t * KB);
+    const int64_t left = u1 - u;
+    sg.kb1 = static_cast<int>(min(static_cast<int64_t>(KB), sg.kb0 + left));
+    return sg;
+}
+
+template <int NT, int STAGES, int KPS>
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX, const float *__restrict__ s_tok,
-                       const float *__restrict__ s_ch, int M, int N, int K, int kb_per_split,
-                       int splits, uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
-                       int32_t *__restrict__ ws_acc, unsigned int *__restrict__ ws_ticket,
+                       const float *__restrict__ s_ch, int M, int N, int K,
+                       uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
+                       int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
                        unsigned long long limit_ns)
 {
-    using Cfg = DecodeCfg<NT, STAGES>;
+    using Cfg = DecodeCfg<NT, STAGES, KPS>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sW = sbase;
-    const uint32_t sX = sbase + STAGES * Cfg::kWBytes;
+    const uint32_t sW = sbase;                               // [STAGES][KPS][128 x 128 B]
+    const uint32_t sX = sbase + STAGES * KPS * Cfg::kWBytes; // [STAGES][KPS][NT x 128 B]
     const uint32_t bar_full = sbase + Cfg::kBarOff;
     const uint32_t bar_empty = bar_full + 8 * STAGES;
     const uint32_t bar_tfull = bar_empty + 8 * STAGES;
-    const uint32_t tslot = bar_tfull + 16;
-    uint32_t *tslot_ptr = reinterpret_cast<uint32_t *>(smem + Cfg::kBarOff + (2 * STAGES + 2) * 8);
-    volatile uint32_t *last_flag = tslot_ptr + 4;
+    const uint32_t bar_tempty = bar_tfull + 16;
+    const uint32_t tslot = bar_tempty + 16;
+    uint32_t *tslot_ptr = reinterpret_cast<uint32_t *>(smem + Cfg::kBarOff + (2 * STAGES + 4) * 8);
+    volatile uint32_t *sh_word = tslot_ptr + 4;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nb = blockIdx.x;
-    const int sp = blockIdx.y;
-    const int kblocks = (K + kBK - 1) / kBK;
-    const int kb0 = sp * kb_per_split;
-    const int kb1 = min(kblocks, kb0 + kb_per_split);
+    const int KB = (K + kBK - 1) / kBK;
+    const int64_t NB = (N + kBM - 1) / kBM;
+    const int64_t U = NB * KB;
+    const int64_t G = gridDim.x;
+    const int64_t g = blockIdx.x;
+    const int64_t u_begin = (g * U) / G;
+    const int64_t u_end = ((g + 1) * U) / G;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        mbar_init(bar_tfull, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 4);
+        }
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -299,17 +345,25 @@ __global__ void __launch_bounds__(kGemmThreads, MINB)
             const uint64_t pol_w = policy_evict_first(); // weights are streamed once
             uint32_t it = 0;
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                const uint32_t s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1u;
-                if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, limit_ns)) {
-                    ok = false;
-                    break;
+            for (int64_t u = u_begin; u < u_end && ok;) {
+                const SkSegment sg = sk_segment(u, u_end, KB);
+                for (int kb = sg.kb0; kb < sg.kb1; kb += KPS, ++it) {
+                    const int nk = min(KPS, sg.kb1 - kb);
+                    const uint32_t s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(bar_full + 8 * s, nk * (Cfg::kWBytes + Cfg::kXBytes));
+                    for (int j = 0; j < nk; ++j) {
+                        tma_load_2d_hint(sW + (s * KPS + j) * Cfg::kWBytes, &tmW, bar_full + 8 * s,
+                                         (kb + j) * kBK, static_cast<int32_t>(sg.t * kBM), pol_w);
+                        tma_load_2d(sX + (s * KPS + j) * Cfg::kXBytes, &tmX, bar_full + 8 * s,
+                                    (kb + j) * kBK, 0);
+                    }
                 }
-                mbar_expect_tx(bar_full + 8 * s, Cfg::kStageBytes);
-                tma_load_2d_hint(sW + s * Cfg::kWBytes, &tmW, bar_full + 8 * s, kb * kBK, nb * kBM,
-                                 pol_w);
-                tma_load_2d(sX + s * Cfg::kXBytes, &tmX, bar_full + 8 * s, kb * kBK, 0);
+                u += sg.kb1 - sg.kb0;
             }
             if (ok) {
                 for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
@@ -319,96 +373,158 @@ __global__ void __launch_bounds__(kGemmThreads, MINB)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_i8(kBM, NT);
-            uint32_t it = 0;
+            uint32_t it = 0, seg = 0;
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                const uint32_t s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1u;
-                if (!mbar_wait(bar_full + 8 * s, ph, limit_ns)) {
-                    ok = false;
+            for (int64_t u = u_begin; u < u_end && ok; ++seg) {
+                const SkSegment sg = sk_segment(u, u_end, KB);
+                const uint32_t buf = seg & 1u;
+                const uint32_t aph = (seg >> 1) & 1u;
+                if (!mbar_wait(bar_tempty + 8 * buf, aph ^ 1u, limit_ns))
                     break;
-                }
                 tc_fence_after();
-                const uint32_t w0 = sW + s * Cfg::kWBytes;
-                const uint32_t x0 = sX + s * Cfg::kXBytes;
+                const uint32_t d = tmem_base + buf * NT;
+                for (int kb = sg.kb0; kb < sg.kb1; kb += KPS, ++it) {
+                    const int nk = min(KPS, sg.kb1 - kb);
+                    const uint32_t s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(bar_full + 8 * s, ph, limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int j = 0; j < nk; ++j) {
+                        const uint32_t w0 = sW + (s * KPS + j) * Cfg::kWBytes;
+                        const uint32_t x0 = sX + (s * KPS + j) * Cfg::kXBytes;
 #pragma unroll
-                for (int k = 0; k < kBK / kUmmaK; ++k)
-                    umma_i8(tmem_base, sw128_kmajor_desc(w0 + k * kUmmaK),
-                            sw128_kmajor_desc(x0 + k * kUmmaK), idesc, (it > 0 || k > 0) ? 1u : 0u);
-                umma_commit(bar_empty + 8 * s);
+                        for (int k = 0; k < kBK / kUmmaK; ++k)
+                            umma_i8(d, sw128_kmajor_desc(w0 + k * kUmmaK),
+                                    sw128_kmajor_desc(x0 + k * kUmmaK), idesc,
+                                    (kb > sg.kb0 || j > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar_empty + 8 * s);
+                }
+                if (ok)
+                    umma_commit(bar_tfull + 8 * buf);
+                u += sg.kb1 - sg.kb0;
             }
-            if (ok)
-                umma_commit(bar_tfull);
         }
     } else {
+        // Epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = channels of the block.
         const int quarter = warp & 3;
         const int etid = threadIdx.x - 64; // 0..127
-        const int n = nb * kBM + quarter * 32 + lane;
-        const bool n_ok = n < N;
-        const float sc = n_ok ? __ldg(s_ch + n) : 0.0f;
-        const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-        const bool ok = mbar_wait(bar_tfull, 0, limit_ns);
-        if (ok)
-            tc_fence_after();
-        // Columns of the accumulator are tokens: column j holds token j.
+        const int r = quarter * 32 + lane; // channel within the block
         constexpr int kChunk = NT < 32 ? NT : 32;
-#pragma unroll 1
-        for (int c0 = 0; c0 < NT && ok; c0 += kChunk) {
-            uint32_t r[32];
-            if constexpr (kChunk == 32) {
-                tmem_ld_32x32b_x32(tbase + c0, r);
-            } else {
-                uint32_t r16[16];
-                tmem_ld_32x32b_x16(tbase + c0, r16);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    r[i] = r16[i];
+        uint32_t seg = 0;
+        bool ok = true;
+        for (int64_t u = u_begin; u < u_end && ok; ++seg) {
+            const SkSegment sg = sk_segment(u, u_end, KB);
+            u += sg.kb1 - sg.kb0;
+            const uint32_t buf = seg & 1u;
+            const uint32_t aph = (seg >> 1) & 1u;
+            const bool whole = (sg.kb0 == 0 && sg.kb1 == KB);
+            const bool owner = (sg.kb0 == 0 && !whole);
+            const int n = static_cast<int>(sg.t * kBM) + r;
+            const bool n_ok = n < N;
+            const float sc = n_ok ? __ldg(s_ch + n) : 0.0f;
+            // contributors to an owned block: the later CTAs whose ranges reach into it
+            int64_t g_last = g;
+            if (owner) {
+                g_last = sk_owner_of(sg.t * KB + KB - 1, U, G);
+                if (etid == 0) {
+                    bool all = true;
+                    for (int64_t c = g + 1; c <= g_last && all; ++c) {
+                        const volatile unsigned int *f = ws_flag + c;
+                        if (*f == 0u) {
+                            const uint64_t t0 = globaltimer_ns();
+                            while (*f == 0u) {
+                                if (globaltimer_ns() - t0 > limit_ns) {
+                                    flag_timeout();
+                                    all = false;
+                                    break;
+                                }
+                            }
+                        }
+                    }
+                    *sh_word = all ? 1u : 0u;
+                }
+                named_bar_sync(1, 128);
+                if (*sh_word == 0u)
+                    ok = false;
+                __threadfence();
             }
-            tmem_ld_wait();
-            if (n_ok) {
+            if (!mbar_wait(bar_tfull + 8 * buf, aph, limit_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + buf * NT + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < NT && c0 < M; c0 += kChunk) {
+                uint32_t a[32];
+                if constexpr (kChunk == 32) {
+                    tmem_ld_32x32b_x32(tbase + c0, a);
+                } else {
+                    uint32_t a16[16];
+                    tmem_ld_32x32b_x16(tbase + c0, a16);
 #pragma unroll
-                for (int j = 0; j < kChunk; ++j) {
-                    const int m = c0 + j;
-                    if (m < M) {
-                        const int32_t a = static_cast<int32_t>(r[j]);
-                        const int64_t off = static_cast<int64_t>(m) * N + n;
-                        if (splits == 1) {
-                            y[off] = static_cast<uint16_t>(bf16_bits(dequant_f32(a, __ldg(s_tok + m), sc)));
+                    for (int i = 0; i < 16; ++i)
+                        a[i] = a16[i];
+                }
+                tmem_ld_wait();
+                if (!whole && !owner) {
+                    // contributor: partial sums to this CTA's slot, [m][128] int32
+#pragma unroll
+                    for (int j = 0; j < kChunk; ++j) {
+                        const int m = c0 + j;
+                        if (m < M)
+                            __stcg(ws_part + (g * M + m) * kBM + r, static_cast<int32_t>(a[j]));
+                    }
+                    continue;
+                }
+                if (owner) {
+                    for (int64_t c = g + 1; c <= g_last; ++c) {
+#pragma unroll
+                        for (int j = 0; j < kChunk; ++j) {
+                            const int m = c0 + j;
+                            if (m < M) {
+                                int32_t *pp = ws_part + (c * M + m) * kBM + r;
+                                a[j] = static_cast<uint32_t>(static_cast<int32_t>(a[j]) + __ldcg(pp));
+                                __stcg(pp, 0); // the workspace is zero again after the call
+                            }
+                        }
+                    }
+                }
+                if (n_ok) {
+#pragma unroll
+                    for (int j = 0; j < kChunk; ++j) {
+                        const int m = c0 + j;
+                        if (m < M) {
+                            const int32_t v = static_cast<int32_t>(a[j]);
+                            const int64_t off = static_cast<int64_t>(m) * N + n;
+                            y[off] = static_cast<uint16_t>(bf16_bits(dequant_f32(v, __ldg(s_tok + m), sc)));
                             if (acc_out)
-                                acc_out[off] = a;
-                        } else {
-                            atomicAdd(ws_acc + off, a);
+                                acc_out[off] = v;
                         }
                     }
                 }
             }
-        }
-        if (splits > 1) {
-            __threadfence();
-            named_bar_sync(1, 128);
-            if (etid == 0) {
-                const unsigned int ticket = atomicAdd(ws_ticket + nb, 1u);
-                *last_flag = (ticket == static_cast<unsigned int>(splits - 1)) ? 1u : 0u;
-            }
-            named_bar_sync(1, 128);
-            if (*last_flag) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_tempty + 8 * buf);
+            if (!whole && !owner) {
+                // publish the partial: every thread's stores, then one flag write
                 __threadfence();
-                if (n_ok) {
-#pragma unroll 4
-                    for (int m = 0; m < M; ++m) {
-                        const int64_t off = static_cast<int64_t>(m) * N + n;
-                        const int32_t a = __ldcg(ws_acc + off);
-                        __stcg(ws_acc + off, 0);
-                        y[off] = static_cast<uint16_t>(bf16_bits(dequant_f32(a, __ldg(s_tok + m), sc)));
-                        if (acc_out)
-                            acc_out[off] = a;
-                    }
-                }
+                named_bar_sync(1, 128);
                 if (etid == 0)
-                    ws_ticket[nb] = 0u;
+                    atomicExch(ws_flag + g, 1u);
+            } else if (owner) {
+                named_bar_sync(1, 128);
+                if (etid == 0)
+                    for (int64_t c = g + 1; c <= g_last; ++c)
+                        atomicExch(ws_flag + c, 0u);
             }
         }
-        tc_fence_before();
     }
     __syncwarp();
     __syncthreads();

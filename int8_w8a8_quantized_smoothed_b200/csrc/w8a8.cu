@@ -167,13 +167,12 @@ void launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int 
 // ------------------------------------------------------------------ GEMM planning
 
 struct GemmPlan {
-    int variant = 0; // 1 prefill, 2 decode
-    int tile_n = 256;
-    int nt = 16;          // decode token tile
-    int splits = 1;       // decode split count
-    int kb_per_split = 0; // decode k-blocks per split
+    int variant = 0;   // 1 prefill, 2 decode
+    int tile_n = 256;  // prefill tile width
+    int nt = 16;       // decode token tile
+    int ctas = 1;      // decode persistent grid
     size_t ws_bytes = 0;
-    size_t ticket_off = 0;
+    size_t flag_off = 0;
 };
 
 int decode_nt(int64_t M)
@@ -181,17 +180,17 @@ int decode_nt(int64_t M)
     return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
 }
 
-int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int splits, int tile_n, int num_sms,
+int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
               GemmPlan *p)
 {
-    if (variant < 0 || variant > 2 || splits < 0 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
+    if (variant < 0 || variant > 2 || ctas < 0 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
         return W8A8_ERR_INVALID_ARG;
     if (variant == 0)
         variant = (M <= 64) ? 2 : 1;
     if (variant == 2 && M > 256)
         return W8A8_ERR_UNSUPPORTED_SHAPE;
     p->variant = variant;
-    const int64_t kblocks = (K + kBK - 1) / kBK;
+    const int64_t KB = (K + kBK - 1) / kBK;
     if (variant == 1) {
         if (tile_n == 0) {
             const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
@@ -202,26 +201,21 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int splits, int tile
         return W8A8_OK;
     }
     p->nt = decode_nt(M);
-    const int64_t nb = (N + kBM - 1) / kBM;
-    const int64_t per_sm = p->nt <= 128 ? 2 : 1;
-    int64_t sp = splits;
-    if (sp == 0) {
-        sp = (num_sms * per_sm) / nb;
-        if (sp < 1)
-            sp = 1;
-    }
-    if (sp > kblocks)
-        sp = kblocks;
-    if (sp > 65535)
-        sp = 65535;
-    const int64_t kb_per = (kblocks + sp - 1) / sp;
-    sp = (kblocks + kb_per - 1) / kb_per;
-    p->splits = static_cast<int>(sp);
-    p->kb_per_split = static_cast<int>(kb_per);
-    if (sp > 1) {
-        const size_t acc_bytes = static_cast<size_t>(M) * static_cast<size_t>(N) * 4u;
-        p->ticket_off = (acc_bytes + 255) & ~static_cast<size_t>(255);
-        p->ws_bytes = p->ticket_off + static_cast<size_t>(nb) * 4u;
+    const int64_t NB = (N + kBM - 1) / kBM;
+    const int64_t U = NB * KB;
+    // every CTA must be resident at once (owners wait on later CTAs): at most one per SM
+    int64_t G = (ctas == 0 || ctas > num_sms) ? num_sms : ctas;
+    if (G > U)
+        G = U;
+    p->ctas = static_cast<int>(G);
+    // a workspace is needed only if some CTA boundary falls inside a channel block
+    bool split = false;
+    for (int64_t g = 1; g < G && !split; ++g)
+        split = ((g * U) / G) % KB != 0;
+    if (split) {
+        const size_t part = static_cast<size_t>(G) * static_cast<size_t>(M) * kBM * 4u;
+        p->flag_off = (part + 255) & ~static_cast<size_t>(255);
+        p->ws_bytes = p->flag_off + static_cast<size_t>(G) * 4u;
     } else {
         p->ws_bytes = 0;
     }
@@ -255,26 +249,39 @@ int launch_prefill(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_
     return launch_status();
 }
 
-template <int NT, int STAGES, int MINB>
+template <int NT, int STAGES, int KPS>
 int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
                   const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
                   uint16_t *y, int32_t *acc, void *ws, int dev, cudaStream_t st)
 {
-    using Cfg = DecodeCfg<NT, STAGES>;
-    const void *fn = reinterpret_cast<const void *>(&gemm_decode_kernel<NT, STAGES, MINB>);
+    using Cfg = DecodeCfg<NT, STAGES, KPS>;
+    const void *fn = reinterpret_cast<const void *>(&gemm_decode_kernel<NT, STAGES, KPS>);
     int rc = ensure_smem(fn, dev, Cfg::kSmemBytes);
     if (rc)
         return rc;
-    const int64_t nb = (N + kBM - 1) / kBM;
-    dim3 grid(static_cast<unsigned>(nb), static_cast<unsigned>(p.splits));
-    int32_t *ws_acc = p.splits > 1 ? static_cast<int32_t *>(ws) : nullptr;
-    unsigned int *ws_ticket =
-        p.splits > 1 ? reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.ticket_off)
-                     : nullptr;
-    gemm_decode_kernel<NT, STAGES, MINB><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(
-        tw, tx, s_tok, s_ch, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-        p.kb_per_split, p.splits, y, acc, ws_acc, ws_ticket, kWaitLimitNs);
+    int32_t *ws_part = p.ws_bytes ? static_cast<int32_t *>(ws) : nullptr;
+    unsigned int *ws_flag =
+        p.ws_bytes ? reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.flag_off)
+                   : nullptr;
+    gemm_decode_kernel<NT, STAGES, KPS><<<p.ctas, kGemmThreads, Cfg::kSmemBytes, st>>>(
+        tw, tx, s_tok, s_ch, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
+        acc, ws_part, ws_flag, kWaitLimitNs);
     return launch_status();
+}
+
+// Decode launch by token tile: (stages, k-blocks per stage) keep ~200 KB of weight and
+// token bytes in flight per SM.
+int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
+                     const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
+                     uint16_t *y, int32_t *acc, void *ws, int dev, cudaStream_t st)
+{
+    switch (p.nt) {
+    case 16: return launch_decode<16, 3, 4>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    case 128: return launch_decode<128, 6, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    default: return launch_decode<256, 4, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    }
 }
 
 } // namespace
@@ -387,7 +394,7 @@ int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *
     return launch_status();
 }
 
-size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int splits,
+size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int ctas,
                                    int tile_n)
 {
     if (check_gemm_shape(M, N, K))
@@ -396,7 +403,7 @@ size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant,
     if (current_device(&dev, &sms))
         sms = 148;
     GemmPlan p;
-    if (plan_gemm(M, N, K, variant, splits, tile_n, sms, &p))
+    if (plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p))
         return 0;
     return p.ws_bytes;
 }
@@ -409,7 +416,7 @@ size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
 int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
                          const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
                          int32_t *acc_out, void *workspace, size_t workspace_bytes, int variant,
-                         int splits, int tile_n, w8a8_stream_t stream)
+                         int ctas, int tile_n, w8a8_stream_t stream)
 {
     if (!xq || !s_tok || !wq || !s_ch || !y)
         return W8A8_ERR_INVALID_ARG;
@@ -423,7 +430,7 @@ int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
     if ((rc = current_device(&dev, &sms)))
         return rc;
     GemmPlan p;
-    if ((rc = plan_gemm(M, N, K, variant, splits, tile_n, sms, &p)))
+    if ((rc = plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p)))
         return rc;
     if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
         return W8A8_ERR_WORKSPACE;
@@ -439,13 +446,7 @@ int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
     CUtensorMap tw, tx;
     if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
         return W8A8_ERR_CUDA;
-    switch (p.nt) {
-    case 16: return launch_decode<16, 6, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
-    case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
-    case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
-    case 128: return launch_decode<128, 3, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
-    default: return launch_decode<256, 4, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
-    }
+    return launch_decode_nt(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
 }
 
 int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, const float *s_ch,
@@ -541,11 +542,5 @@ extern "C" int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, c
     CUtensorMap tw, tx;
     if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
         return W8A8_ERR_CUDA;
-    switch (p.nt) {
-    case 16: return launch_decode<16, 6, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
-    case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
-    case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
-    case 128: return launch_decode<128, 3, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
-    default: return launch_decode<256, 4, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
-    }
+    return launch_decode_nt(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
 }

@@ -1,7 +1,7 @@
 """Parity of the tcgen05 INT8 GEMM + dequant kernels with the oracle, through the C ABI:
 int32 accumulators and bf16 outputs bit-exact (the bar is 1 bf16 ulp; the epilogue is built
 to the oracle's operation order, so 0 is expected and asserted, and the ulp distance is
-reported on failure). Both kernels (persistent tile / swap-AB split-K) are run on the same
+reported on failure). Both kernels (persistent tile / swap-AB stream-K) are run on the same
 shapes, including ragged M, N and K tails, several tiles, and extreme accumulators."""
 import numpy as np
 import pytest
@@ -23,12 +23,12 @@ def _inputs(M, N, K, seed):
     return xq, st, wq, sc
 
 
-def _run(xq, st, wq, sc, variant, splits=0, tile_n=0):
+def _run(xq, st, wq, sc, variant, ctas=0, tile_n=0):
     M, N = xq.shape[0], wq.shape[0]
     y, cy = bf16_out((M, N))
     acc, ca = with_canary((M, N), torch.int32, -7)
     w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), y=y, acc_out=acc,
-                            variant=variant, splits=splits, tile_n=tile_n)
+                            variant=variant, ctas=ctas, tile_n=tile_n)
     torch.cuda.synchronize()
     cy(); ca()
     return host_bf16(y), host(acc)
@@ -47,11 +47,13 @@ DECODE_SHAPES = [(1, 8, 16), (1, 512, 256), (16, 512, 256), (8, 1024, 4096), (3,
 
 
 @pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
-@pytest.mark.parametrize("splits", [0, 1, 3])
-def test_decode_kernel_bit_exact(M, N, K, splits):
+@pytest.mark.parametrize("ctas", [0, 1, 3, 7])
+def test_decode_kernel_bit_exact(M, N, K, ctas):
+    # ctas=1: one CTA walks every block whole; 3 and 7: blocks split between CTAs (owner +
+    # contributors); 0: one CTA per SM (the launch the benchmark times)
     xq, st, wq, sc = _inputs(M, N, K, seed=M + N + K)
     y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
-    y, acc = _run(xq, st, wq, sc, variant=2, splits=splits)
+    y, acc = _run(xq, st, wq, sc, variant=2, ctas=ctas)
     _compare(y, acc, y_ref, acc_ref)
 
 
@@ -95,7 +97,7 @@ def test_extreme_accumulators():
 
 
 def test_auto_variant_and_workspace_reuse():
-    # the split-K workspace must come back zero-filled: run twice through one workspace
+    # the stream-K workspace must come back zero-filled: run twice through one workspace
     for (M, N, K) in [(8, 6144, 4096), (64, 4096, 4096), (512, 1024, 1024)]:
         xq, st, wq, sc = _inputs(M, N, K, 11)
         y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
@@ -124,10 +126,10 @@ def test_zero_scales_give_zero():
 def test_workspace_too_small_is_reported():
     M, N, K = 8, 1024, 4096
     xq, st, wq, sc = _inputs(M, N, K, 1)
-    need = w8.w8a8_gemm_workspace_size_ex(M, N, K, 2, 4, 0)
+    need = w8.w8a8_gemm_workspace_size_ex(M, N, K, 2, 7, 0)
     assert need > 0
     small = torch.zeros(need - 4, dtype=torch.uint8, device="cuda")
     with pytest.raises(w8.W8A8Error, match="WORKSPACE"):
         w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), workspace=small, variant=2,
-                                splits=4)
+                                ctas=7)
     assert w8.w8a8_device_status(reset=True) == 0

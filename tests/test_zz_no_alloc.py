@@ -1,7 +1,7 @@
 """The no-allocation GEMM entry point (w8a8_gemm_dequant_noalloc), for callers that cannot
 allocate device memory (a plugin inside another runtime's launch path, a fixed memory
 budget, a stream under capture). It must give the same output as w8a8_gemm_dequant, call
-after call, using only its built-in 4 MiB scratch array.
+after call, using only its built-in 8 MiB scratch array.
 
 This file is collected last on purpose, and passes both alone in a fresh process and after
 the rest of the suite."""
@@ -26,8 +26,8 @@ def _bits(y):
     return y.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-# shapes whose automatic plan uses several K splits (so the scratch array is used), and one
-# that uses a single split (no scratch)
+# shapes whose stream-K plan splits 128-channel blocks between CTAs, so the scratch array is
+# used ((1, 512, 256) has 8 weight blocks of 128 x 128: 8 CTAs, one k-block each)
 SHAPES = [(8, 6144, 4096), (64, 4096, 14336), (1, 512, 256), (33, 1032, 4096),
           (256, 1024, 512), (64, 28672, 4096)]
 
@@ -52,7 +52,7 @@ def test_noalloc_matches_gemm_dequant_twice(M, N, K):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     dev = torch.device("cuda", 0)
-    M, N, K = 256, 8192, 4096  # split-K scratch 8 MiB > 4 MiB
+    M, N, K = 256, 8192, 4096  # scratch 148 CTAs x 256 x 512 B = 19 MB > 8 MiB
     assert w8.w8a8_gemm_workspace_size_ex(M, N, K, 2, 0, 0) > w8.NOALLOC_SCRATCH_BYTES
     xq = torch.zeros((M, K), dtype=torch.int8, device=dev)
     wq = torch.zeros((N, K), dtype=torch.int8, device=dev)
