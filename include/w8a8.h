@@ -115,8 +115,9 @@ W8A8_API int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I,
 /*
  * Bytes of device workspace w8a8_gemm_dequant needs for this shape (0 if none). The
  * workspace must be zero-filled before its first use; every call that returns W8A8_OK
- * leaves it zero-filled again, so one zeroed buffer serves any number of calls issued in
- * order on one stream. Calls that may run concurrently need separate workspaces.
+ * leaves it ready for the next one (its flag words zero again), so one buffer serves any
+ * number of calls issued in order on one stream. Calls that may run concurrently need
+ * separate workspaces.
  */
 W8A8_API size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
@@ -134,9 +135,10 @@ W8A8_API size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * workspace/workspace_bytes: see w8a8_gemm_workspace_size (may be NULL/0 when it returns 0).
  * Requires M >= 1, N >= 8, N % 8 == 0, K >= 16, K % 16 == 0, K <= 133144 (so that
  * 127 * 127 * K fits in int32), M, N <= 2^31 - 1.
- * Small M (at most 64 tokens by default, up to 256 on request) runs a persistent swap-AB
- * stream-K kernel that streams the weight; larger M runs a persistent tile kernel. Both give
- * identical results.
+ * Small M (at most 64 tokens by default, up to 256 on request) runs a swap-AB kernel that
+ * streams the weight: split-K over thread-block clusters (partials summed in distributed
+ * shared memory) when the weight has few 128-channel blocks, persistent stream-K over all SMs
+ * otherwise; larger M runs a persistent tile kernel. All give identical results.
  */
 W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq,
                       const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
@@ -146,9 +148,12 @@ W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_
 /*
  * The same GEMM with the kernel chosen by the caller, for tests and tuning:
  * variant 0 = automatic (as w8a8_gemm_dequant), 1 = persistent tile kernel, 2 = swap-AB
- * stream-K kernel (M <= 256 only). ctas (variant 2) = number of persistent CTAs sharing the
- * weight stream, 0 = one per SM. tile_n (variant 1) = 0 automatic, else 128 or 256. The
- * workspace needed is w8a8_gemm_workspace_size_ex() of the same arguments.
+ * stream-K kernel, 3 = swap-AB cluster split-K kernel (2 and 3: M <= 256 only). ctas:
+ * variant 2 = persistent CTAs sharing the weight stream (0 = one per SM, at most one per SM);
+ * variant 3 = cluster size, the number of K splits per 128-channel block (0 = automatic,
+ * at most 8, fewer if the clusters would not all fit on the GPU at once). tile_n (variant 1)
+ * = 0 automatic, else 128 or 256. The workspace needed is w8a8_gemm_workspace_size_ex() of
+ * the same arguments (only variant 2 uses one).
  */
 W8A8_API int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
                          const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
@@ -167,17 +172,18 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
  * cudaMalloc would synchronize the device, fail, or break the budget, so they cannot
  * provide the zero-filled workspace that w8a8_gemm_dequant's stream-K kernel needs.
  *
- * Computes exactly what w8a8_gemm_dequant computes, always with the swap-AB stream-K kernel
- * (M <= 256), and allocates nothing. Its scratch is a file-scope device array of
+ * Computes exactly what w8a8_gemm_dequant computes, always with its small-M swap-AB kernels
+ * (M <= 256), and allocates nothing. Only the stream-K kernel, used when the weight has many
+ * 128-channel blocks, needs scratch; it is a file-scope device array of
  * W8A8_NOALLOC_SCRATCH_BYTES (8 MiB) inside the library; every GPU on which the library is
  * loaded holds that array until the process exits. The caller still owns and passes every
  * input and output. Arguments and requirements are those of w8a8_gemm_dequant without
  * acc_out and workspace.
  *   - Returns W8A8_ERR_WORKSPACE when this shape's scratch exceeds
- *     W8A8_NOALLOC_SCRATCH_BYTES: M * 512 bytes of partial sums per CTA plus 4 bytes per CTA
- *     (one CTA per SM, fewer when the weight has fewer 128 x 128 blocks), needed only when a
- *     CTA's share of the weight stream ends inside a 128-channel block. So on a 148-SM B200
- *     M <= 110 always fits. W8A8_ERR_UNSUPPORTED_SHAPE for M > 256.
+ *     W8A8_NOALLOC_SCRATCH_BYTES: 4 KiB of flags plus 512 bytes per token (M rounded up to
+ *     a multiple of 4) of partial sums per CTA (one CTA per SM), needed only when a CTA's
+ *     share of the weight stream ends inside a 128-channel block. So on a 148-SM B200
+ *     M <= 108 always fits. W8A8_ERR_UNSUPPORTED_SHAPE for M > 256.
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
  *   - Each call clears the part of the array it uses (cudaMemsetAsync on `stream`) before
@@ -190,6 +196,23 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
 W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, const int8_t *wq,
                                        const float *s_ch, int64_t M, int64_t N, int64_t K,
                                        w8a8_bf16 *y, w8a8_stream_t stream);
+
+/*
+ * Kernel overlap mode, process-wide (default 1). Results are identical in every mode.
+ *   0: each kernel of this library starts after the previous work in its stream completes.
+ *   1: programmatic dependent launch: a kernel may launch and run its prologue (barrier
+ *      set-up, tensor-memory allocation, descriptor prefetch) while the previous kernel in
+ *      the stream is still running; it waits for that kernel to complete before it reads
+ *      any input or writes any output.
+ *   2: as 1, and the GEMMs also start streaming their int8 weights (wq) before that wait,
+ *      so a GEMM's weight traffic overlaps the tail of the kernels before it. Only valid
+ *      when no kernel enqueued on the stream since its last completed synchronization
+ *      writes wq -- e.g. weights prepared once and synchronized before serving.
+ * Returns the previous mode, or W8A8_ERR_INVALID_ARG for another value. Applies to launches
+ * made after the call (a captured CUDA graph keeps the mode it was captured with).
+ */
+W8A8_API int w8a8_set_overlap(int mode);
+W8A8_API int w8a8_get_overlap(void);
 
 /*
  * Device status: synchronizes the current device, then returns W8A8_OK or

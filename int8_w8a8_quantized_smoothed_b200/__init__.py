@@ -19,7 +19,8 @@ __all__ = [
     "W8A8Error", "lib", "LIB_PATH",
     "w8a8_quantize_rows", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
-    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_device_status",
+    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_set_overlap",
+    "w8a8_get_overlap", "w8a8_device_status",
     "w8a8_status_string", "w8a8_version",
     "Workspace",
 ]
@@ -42,6 +43,8 @@ SIGNATURES = [
                                   _I, _P]),
     ("w8a8_gemm_workspace_size_ex", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
     ("w8a8_gemm_dequant_noalloc", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    ("w8a8_set_overlap", _I, [_I]),
+    ("w8a8_get_overlap", _I, []),
     ("w8a8_device_status", _I, [_I]),
     ("w8a8_status_string", C.c_char_p, [_I]),
     ("w8a8_version", _I, []),
@@ -111,6 +114,20 @@ def w8a8_status_string(status: int) -> str:
 
 def w8a8_version() -> int:
     return lib().w8a8_version()
+
+
+def w8a8_set_overlap(mode: int) -> int:
+    """0 plain stream order, 1 dependent launch (default), 2 also prefetch static weights
+    before the dependency wait (weights must not be written by kernels still in flight).
+    Returns the previous mode."""
+    rc = lib().w8a8_set_overlap(int(mode))
+    if rc < 0:
+        raise W8A8Error("w8a8_set_overlap", rc)
+    return rc
+
+
+def w8a8_get_overlap() -> int:
+    return lib().w8a8_get_overlap()
 
 
 def w8a8_device_status(reset: bool = False) -> int:

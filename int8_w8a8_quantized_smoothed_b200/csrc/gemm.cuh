@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap tmB, const float *__restrict__ s_tok,
                         const float *__restrict__ s_ch, int M, int N, int K,
                         uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
-                        unsigned long long limit_ns)
+                        int prefetch_static, unsigned long long limit_ns)
 {
     using Cfg = PrefillCfg<BN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -107,9 +107,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tslot_ptr);
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
+            // With prefetch_static the weight (B) tiles of the first ring of stages are
+            // requested before waiting for the previous kernel: the caller guarantees no
+            // kernel still in flight writes the weights. Activations always come after.
+            uint32_t npre = 0;
+            if (prefetch_static) {
+                for (int tile = blockIdx.x; tile < tiles && npre < STAGES; tile += gridDim.x) {
+                    int mb, nb;
+                    tile_coords(tile, num_m, num_n, mb, nb);
+                    for (int kb = 0; kb < kblocks && npre < STAGES; ++kb, ++npre) {
+                        mbar_expect_tx(bar_full + 8 * npre, Cfg::kStageBytes);
+                        tma_load_2d(sB + npre * Cfg::kBBytes, &tmB, bar_full + 8 * npre, kb * kBK,
+                                    nb * BN);
+                    }
+                }
+            }
+            pdl_wait();
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
@@ -117,6 +135,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tile_coords(tile, num_m, num_n, mb, nb);
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const uint32_t s = it % STAGES;
+                    if (it < npre) { // weights already requested; add the activation tile
+                        tma_load_2d(sA + s * Cfg::kABytes, &tmA, bar_full + 8 * s, kb * kBK,
+                                    mb * kBM);
+                        continue;
+                    }
                     const uint32_t ph = (it / STAGES) & 1u;
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, limit_ns)) {
                         ok = false;
@@ -169,6 +192,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
+        pdl_wait(); // s_tok comes from the previous kernel; y may still be read by it
         const int quarter = warp & 3;
         uint32_t t = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++t) {
@@ -230,29 +254,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 }
 
-// ---------------------------------------------------------------- decode (swap-AB stream-K)
+// ---------------------------------------------------------------- decode (swap-AB)
 //
-// Work units are (channel block t, k-block kb) pairs in tile-major order, U = NB * KB of
-// them. CTA g of G (one per SM, persistent) takes the contiguous range
-// [floor(g U / G), floor((g+1) U / G)), so every SM streams the same number of weight bytes.
-// A range is cut into segments at channel-block boundaries. A segment covering a whole block
-// is dequantized and stored directly. A block split between CTAs has one owner, the segment
-// holding k-block 0 (the last segment of its CTA, so it finishes last); every other segment
-// of that block (the first segment of a later CTA) stores its int32 partial in the CTA's own
-// workspace slot and raises the CTA's flag; the owner waits for the flags of the later CTAs
-// that share its block, adds their partials (exact int32), dequantizes, stores, and lowers
-// the flags again so the workspace is zero between calls.
+// Work units are (channel block t, k-block kb) pairs in block-major order, U = NB * KB of
+// them; a CTA owns a contiguous unit range and walks it in segments (the part of its range
+// inside one channel block). Two schedules:
+//
+// CLUSTER (few channel blocks): grid (S, NB) with thread-block clusters of S CTAs along K;
+//   CTA r of block t takes k-blocks [r KB / S, (r+1) KB / S). The S partial accumulators meet
+//   in shared memory: each CTA writes its partial to its own (now idle) stage buffers, the
+//   cluster synchronizes, and CTA r sums rows [r 128 / S, (r+1) 128 / S) of all S partials
+//   through distributed shared memory, dequantizes and stores them. No global workspace.
+//
+// stream-K (many channel blocks): G persistent CTAs (one per SM) take equal contiguous
+//   ranges [g U / G, (g+1) U / G), so every SM streams the same weight bytes. A block split
+//   between CTAs has one owner, the segment holding k-block 0 (its CTA's last segment, so it
+//   finishes last); the other segments (first segments of later CTAs) store their int32
+//   partials in their CTA's workspace slot and raise the CTA's flag; the owner waits for the
+//   flags of the later CTAs sharing its block, adds their partials, dequantizes, stores and
+//   lowers the flags so the workspace is ready for the next call.
 
-template <int NT, int STAGES, int KPS> struct DecodeCfg {
-    static constexpr int kWBytes = kBM * kBK;           // one k-block of 128 weight rows
-    static constexpr int kXBytes = NT * kBK;            // one k-block of NT token rows
+template <int NT, int STAGES, int KPS, bool CLUSTER> struct DecodeCfg {
+    static constexpr int kWBytes = kBM * kBK;  // one k-block of 128 weight rows
+    static constexpr int kXBytes = NT * kBK;   // one k-block of NT token rows
     static constexpr int kStageBytes = KPS * (kWBytes + kXBytes);
-    static constexpr int kBarOff = STAGES * kStageBytes;
+    // stream-K stages its bf16 output tile [NT][128] for coalesced stores
+    static constexpr int kYBytes = CLUSTER ? 0 : NT * kBM * 2;
+    static constexpr int kYOff = STAGES * kStageBytes;
+    static constexpr int kStokOff = kYOff + kYBytes; // fp32 token scales [NT]
+    static constexpr int kBarOff = kStokOff + NT * 4;
     // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot, flag word
     static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 32 + 1024;
     static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
     static_assert(kXBytes % 1024 == 0, "token tile must keep stages 1024-byte aligned");
     static_assert(kTmemCols <= 512, "two accumulators must fit TMEM");
+    static_assert(!CLUSTER || NT * kBM * 4 <= STAGES * kStageBytes,
+                  "the cluster partial tile reuses the stage buffers");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 // CTA holding unit v under the even split of U units over G CTAs.
@@ -267,11 +305,11 @@ __host__ __device__ __forceinline__ int64_t sk_owner_of(int64_t v, int64_t U, in
 }
 
 struct SkSegment {
-    int64_t t;   // channel block
+    int64_t t;    // channel block
     int kb0, kb1; // k-block range [kb0, kb1)
 };
 
-// Segment iterator over [u, u1): next segment starting at u.
+// The segment of [u, u1) that starts at u.
 __device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
 {
     SkSegment sg;
@@ -282,22 +320,24 @@ __device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
     return sg;
 }
 
-template <int NT, int STAGES, int KPS>
+template <int NT, int STAGES, int KPS, bool CLUSTER>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX, const float *__restrict__ s_tok,
                        const float *__restrict__ s_ch, int M, int N, int K,
                        uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
                        int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
-                       unsigned long long limit_ns)
+                       int prefetch_static, unsigned long long limit_ns)
 {
-    using Cfg = DecodeCfg<NT, STAGES, KPS>;
+    using Cfg = DecodeCfg<NT, STAGES, KPS, CLUSTER>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sW = sbase;                               // [STAGES][KPS][128 x 128 B]
     const uint32_t sX = sbase + STAGES * KPS * Cfg::kWBytes; // [STAGES][KPS][NT x 128 B]
+    uint16_t *ysm = reinterpret_cast<uint16_t *>(smem + Cfg::kYOff);
+    float *sh_stok = reinterpret_cast<float *>(smem + Cfg::kStokOff);
     const uint32_t bar_full = sbase + Cfg::kBarOff;
     const uint32_t bar_empty = bar_full + 8 * STAGES;
     const uint32_t bar_tfull = bar_empty + 8 * STAGES;
@@ -313,8 +353,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int64_t U = NB * KB;
     const int64_t G = gridDim.x;
     const int64_t g = blockIdx.x;
-    const int64_t u_begin = (g * U) / G;
-    const int64_t u_end = ((g + 1) * U) / G;
+    int64_t u_begin, u_end;
+    if constexpr (CLUSTER) {
+        const int64_t t = blockIdx.y;
+        u_begin = t * KB + (g * KB) / G;
+        u_end = t * KB + ((g + 1) * KB) / G;
+    } else {
+        u_begin = (g * U) / G;
+        u_end = ((g + 1) * U) / G;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -339,10 +386,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tslot_ptr);
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first(); // weights are streamed once
+            // With prefetch_static the weight tiles of the first ring of stages are requested
+            // before waiting for the previous kernel (the caller guarantees no kernel still
+            // in flight writes the weights); token tiles always come after the wait.
+            uint32_t npre = 0;
+            if (prefetch_static) {
+                for (int64_t u = u_begin; u < u_end && npre < STAGES;) {
+                    const SkSegment sg = sk_segment(u, u_end, KB);
+                    for (int kb = sg.kb0; kb < sg.kb1 && npre < STAGES; kb += KPS, ++npre) {
+                        const int nk = min(KPS, sg.kb1 - kb);
+                        mbar_expect_tx(bar_full + 8 * npre, nk * (Cfg::kWBytes + Cfg::kXBytes));
+                        for (int j = 0; j < nk; ++j)
+                            tma_load_2d_hint(sW + (npre * KPS + j) * Cfg::kWBytes, &tmW,
+                                             bar_full + 8 * npre, (kb + j) * kBK,
+                                             static_cast<int32_t>(sg.t * kBM), pol_w);
+                    }
+                    u += sg.kb1 - sg.kb0;
+                }
+            }
+            pdl_wait();
             uint32_t it = 0;
             bool ok = true;
             for (int64_t u = u_begin; u < u_end && ok;) {
@@ -350,6 +418,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int kb = sg.kb0; kb < sg.kb1; kb += KPS, ++it) {
                     const int nk = min(KPS, sg.kb1 - kb);
                     const uint32_t s = it % STAGES;
+                    if (it < npre) { // weights already requested; add the token tiles
+                        for (int j = 0; j < nk; ++j)
+                            tma_load_2d(sX + (s * KPS + j) * Cfg::kXBytes, &tmX, bar_full + 8 * s,
+                                        (kb + j) * kBK, 0);
+                        continue;
+                    }
                     const uint32_t ph = (it / STAGES) & 1u;
                     if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, limit_ns)) {
                         ok = false;
@@ -409,11 +483,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
     } else {
-        // Epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = channels of the block.
+        // Epilogue warps: warp w reads TMEM lanes 32*(w%4)..+31 = channels of the block.
+        pdl_wait(); // s_tok and the workspace may still be in use by the previous kernel
         const int quarter = warp & 3;
         const int etid = threadIdx.x - 64; // 0..127
         const int r = quarter * 32 + lane; // channel within the block
-        constexpr int kChunk = NT < 32 ? NT : 32;
+        for (int i = etid; i < M; i += 128)
+            sh_stok[i] = __ldg(s_tok + i);
+        named_bar_sync(1, 128);
+        const int mt = M < NT ? M : NT; // tokens held in the accumulator
+        const int Mp = (M + 3) & ~3;    // tokens per partial row in the workspace
         uint32_t seg = 0;
         bool ok = true;
         for (int64_t u = u_begin; u < u_end && ok; ++seg) {
@@ -421,8 +500,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             u += sg.kb1 - sg.kb0;
             const uint32_t buf = seg & 1u;
             const uint32_t aph = (seg >> 1) & 1u;
-            const bool whole = (sg.kb0 == 0 && sg.kb1 == KB);
-            const bool owner = (sg.kb0 == 0 && !whole);
+            const bool whole = CLUSTER || (sg.kb0 == 0 && sg.kb1 == KB);
+            const bool owner = !CLUSTER && sg.kb0 == 0 && !whole;
+            const bool contrib = !CLUSTER && sg.kb0 > 0;
             const int n = static_cast<int>(sg.t * kBM) + r;
             const bool n_ok = n < N;
             const float sc = n_ok ? __ldg(s_ch + n) : 0.0f;
@@ -457,54 +537,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             tc_fence_after();
+            if constexpr (CLUSTER)
+                fence_proxy_async_smem(); // the partial tile reuses TMA-written smem
             const uint32_t tbase = tmem_base + buf * NT + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < NT && c0 < M; c0 += kChunk) {
-                uint32_t a[32];
-                if constexpr (kChunk == 32) {
-                    tmem_ld_32x32b_x32(tbase + c0, a);
-                } else {
-                    uint32_t a16[16];
-                    tmem_ld_32x32b_x16(tbase + c0, a16);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        a[i] = a16[i];
-                }
+            for (int c0 = 0; c0 < mt; c0 += 16) {
+                uint32_t a[16];
+                tmem_ld_32x32b_x16(tbase + c0, a);
                 tmem_ld_wait();
-                if (!whole && !owner) {
-                    // contributor: partial sums to this CTA's slot, [m][128] int32
+                if constexpr (CLUSTER) {
+                    // partial tile P[m][128] int32 in this CTA's stage buffers
+                    int32_t *P = reinterpret_cast<int32_t *>(smem);
 #pragma unroll
-                    for (int j = 0; j < kChunk; ++j) {
-                        const int m = c0 + j;
-                        if (m < M)
-                            __stcg(ws_part + (g * M + m) * kBM + r, static_cast<int32_t>(a[j]));
-                    }
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < mt)
+                            P[(c0 + j) * kBM + r] = static_cast<int32_t>(a[j]);
+                    continue;
+                }
+                if (contrib) {
+                    // this CTA's slot: [128 channels][Mp tokens] int32, 16-byte vectors
+                    int4 *dst = reinterpret_cast<int4 *>(ws_part + (g * kBM + r) * Mp + c0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (c0 + 4 * q < mt)
+                            __stcg(dst + q, make_int4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]));
                     continue;
                 }
                 if (owner) {
+#pragma unroll 2
                     for (int64_t c = g + 1; c <= g_last; ++c) {
+                        const int4 *src =
+                            reinterpret_cast<const int4 *>(ws_part + (c * kBM + r) * Mp + c0);
+                        int4 v[4];
 #pragma unroll
-                        for (int j = 0; j < kChunk; ++j) {
-                            const int m = c0 + j;
-                            if (m < M) {
-                                int32_t *pp = ws_part + (c * M + m) * kBM + r;
-                                a[j] = static_cast<uint32_t>(static_cast<int32_t>(a[j]) + __ldcg(pp));
-                                __stcg(pp, 0); // the workspace is zero again after the call
-                            }
+                        for (int q = 0; q < 4; ++q)
+                            v[q] = (c0 + 4 * q < mt) ? __ldcg(src + q) : make_int4(0, 0, 0, 0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            a[4 * q] += static_cast<uint32_t>(v[q].x);
+                            a[4 * q + 1] += static_cast<uint32_t>(v[q].y);
+                            a[4 * q + 2] += static_cast<uint32_t>(v[q].z);
+                            a[4 * q + 3] += static_cast<uint32_t>(v[q].w);
                         }
                     }
                 }
-                if (n_ok) {
+                // dequantize into the staged output tile [m][128] bf16
 #pragma unroll
-                    for (int j = 0; j < kChunk; ++j) {
-                        const int m = c0 + j;
-                        if (m < M) {
-                            const int32_t v = static_cast<int32_t>(a[j]);
-                            const int64_t off = static_cast<int64_t>(m) * N + n;
-                            y[off] = static_cast<uint16_t>(bf16_bits(dequant_f32(v, __ldg(s_tok + m), sc)));
-                            if (acc_out)
-                                acc_out[off] = v;
-                        }
+                for (int j = 0; j < 16; ++j) {
+                    const int m = c0 + j;
+                    if (m < mt) {
+                        const int32_t v = static_cast<int32_t>(a[j]);
+                        ysm[m * kBM + r] =
+                            static_cast<uint16_t>(bf16_bits(dequant_f32(v, sh_stok[m], sc)));
+                        if (acc_out && n_ok)
+                            acc_out[static_cast<int64_t>(m) * N + n] = v;
                     }
                 }
             }
@@ -512,21 +598,66 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar_tempty + 8 * buf);
-            if (!whole && !owner) {
-                // publish the partial: every thread's stores, then one flag write
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (etid == 0)
-                    atomicExch(ws_flag + g, 1u);
-            } else if (owner) {
-                named_bar_sync(1, 128);
-                if (etid == 0)
-                    for (int64_t c = g + 1; c <= g_last; ++c)
-                        atomicExch(ws_flag + c, 0u);
+            if constexpr (!CLUSTER) {
+                if (contrib) {
+                    // publish the partial: every thread's stores, then one flag write
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (etid == 0)
+                        atomicExch(ws_flag + g, 1u);
+                } else {
+                    // whole or owned block: copy the staged tile out, 16 bytes per thread
+                    named_bar_sync(1, 128);
+                    const int nvalid = min(kBM, N - static_cast<int>(sg.t * kBM));
+                    for (int v = etid; v < mt * 16; v += 128) {
+                        const int m = v >> 4, cv = v & 15;
+                        if (cv * 8 < nvalid)
+                            *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(m) * N +
+                                                       sg.t * kBM + cv * 8) =
+                                *reinterpret_cast<const uint4 *>(ysm + m * kBM + cv * 8);
+                    }
+                    named_bar_sync(1, 128);
+                    if (owner && etid == 0)
+                        for (int64_t c = g + 1; c <= g_last; ++c)
+                            atomicExch(ws_flag + c, 0u);
+                }
             }
         }
     }
     __syncwarp();
+    if constexpr (CLUSTER) {
+        // every thread of the cluster: partial tiles are complete in shared memory
+        cluster_sync();
+        if (warp >= 2) {
+            const int etid = threadIdx.x - 64;
+            const uint32_t S = static_cast<uint32_t>(gridDim.x);
+            const uint32_t rank = cluster_ctarank();
+            const int r0 = static_cast<int>((rank * kBM) / S);
+            const int r1 = static_cast<int>(((rank + 1) * kBM) / S);
+            const int w = r1 - r0;
+            const int64_t t = blockIdx.y;
+            const int mt = M < NT ? M : NT;
+            const uint32_t P = sbase; // partial tiles sit at the same offset in every CTA
+            for (int idx = etid; idx < mt * w; idx += 128) {
+                const int m = idx / w;
+                const int row = r0 + (idx - m * w);
+                const uint32_t la = P + static_cast<uint32_t>((m * kBM + row) * 4);
+                int32_t sum = 0;
+                for (uint32_t p = 0; p < S; ++p)
+                    sum += ld_dsmem_s32(map_peer_smem(la, p));
+                const int n = static_cast<int>(t * kBM) + row;
+                if (n < N) {
+                    const int64_t off = static_cast<int64_t>(m) * N + n;
+                    y[off] = static_cast<uint16_t>(
+                        bf16_bits(dequant_f32(sum, sh_stok[m], __ldg(s_ch + n))));
+                    if (acc_out)
+                        acc_out[off] = sum;
+                }
+            }
+        }
+        // nobody leaves while a peer may still read its shared memory
+        cluster_sync();
+    }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();

@@ -30,6 +30,22 @@ __device__ __forceinline__ void flag_timeout()
     atomicOr(&g_status_word, kStatusTimeout);
 }
 
+// ------------------------------------------------------------------------- dependent launch
+
+// Programmatic dependent launch: lets the next kernel in the stream launch (and run its
+// prologue) while this one is still running. Harmless when launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Blocks until every prerequisite grid has completed and its memory is visible. Every read
+// of data produced by an earlier kernel, and every global write, comes after this.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
@@ -242,6 +258,42 @@ __host__ __device__ constexpr uint32_t idesc_i8(int m, int n)
            | (1u << 10)                                   // B format: signed 8-bit
            | (static_cast<uint32_t>(n >> 3) << 17)        // N / 8
            | (static_cast<uint32_t>(m >> 4) << 24);       // M / 16
+}
+
+// ------------------------------------------------------------------------- clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster arrives (release) and waits (acquire).
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_peer_smem(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ int32_t ld_dsmem_s32(uint32_t addr)
+{
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Named barrier over `nthreads` threads (multiple of 32), id 1..15.

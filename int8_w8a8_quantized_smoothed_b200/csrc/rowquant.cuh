@@ -131,6 +131,9 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const uint16_t *__r
                                                              float *__restrict__ s_tok)
 {
     __shared__ float sh[33];
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // every input may come from the previous kernel
     const int64_t row = blockIdx.x;
     const int nvec = K >> 3;
     const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * K);
@@ -176,6 +179,9 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(
 {
     __shared__ double shd[33];
     __shared__ float shf[33];
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // every input may come from the previous kernel
     const int64_t row = blockIdx.x;
     const int nvec = K >> 3;
     const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * K);
@@ -273,6 +279,9 @@ __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const uint16_t *__
                                                               float *__restrict__ s_tok)
 {
     __shared__ float sh[33];
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // every input may come from the previous kernel
     const int64_t row = blockIdx.x;
     const int nvec = I >> 3;
     const uint4 *gr = reinterpret_cast<const uint4 *>(gu + row * 2 * static_cast<int64_t>(I));

@@ -5,8 +5,10 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 #include <set>
+#include <tuple>
 #include <utility>
 
 #include "gemm.cuh"
@@ -73,15 +75,19 @@ int current_device(int *dev, int *num_sms)
     return W8A8_OK;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device.
+// Once per kernel and device: raise the dynamic shared-memory limit, and ask for the
+// largest shared-memory carveout for every kernel of the library, so consecutive launches
+// of row kernels and GEMMs never reconfigure the L1/shared split between them.
 int ensure_smem(const void *kernel, int dev, int bytes)
 {
     std::lock_guard<std::mutex> lk(g_mu);
     auto key = std::make_pair(kernel, dev);
     if (g_smem_set.count(key))
         return W8A8_OK;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess) {
+    if ((bytes > 0 && cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           bytes) != cudaSuccess) ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
         cudaGetLastError();
         return W8A8_ERR_CUDA;
     }
@@ -89,9 +95,65 @@ int ensure_smem(const void *kernel, int dev, int bytes)
     return W8A8_OK;
 }
 
-int launch_status()
+// Overlap mode (w8a8_set_overlap): 0 plain stream order, 1 programmatic dependent launch,
+// 2 dependent launch + weight prefetch before the dependency wait.
+std::atomic<int> g_overlap{1};
+
+// Launches `kernel`, with programmatic stream serialization when the overlap mode asks for
+// it (the kernels call griddepcontrol.wait before touching dependent data either way).
+template <typename... KArgs, typename... Args>
+int launch_kernel_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, unsigned cluster_x, Args &&...args)
 {
-    return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (g_overlap.load(std::memory_order_relaxed) >= 1) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    return W8A8_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                  Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (g_overlap.load(std::memory_order_relaxed) >= 1) {
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    return W8A8_OK;
 }
 
 // 2-D int8 [rows, K] K-contiguous tensor, box = 128 bytes of K x box_rows, 128B swizzle,
@@ -139,58 +201,83 @@ int check_row_shape(int64_t M, int64_t K)
 }
 
 template <int NCH>
-void launch_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int K, int8_t *q,
-                          float *s, int threads, cudaStream_t st)
+int launch_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int K, int8_t *q,
+                         float *s, int threads, int dev, cudaStream_t st)
 {
-    quantize_rows_kernel<NCH><<<static_cast<unsigned>(M), threads, 0, st>>>(x, sinv, K, q, s);
+    if (int rc = ensure_smem(reinterpret_cast<const void *>(&quantize_rows_kernel<NCH>), dev, 0))
+        return rc;
+    return launch_kernel(quantize_rows_kernel<NCH>, dim3(static_cast<unsigned>(M)), dim3(threads), 0,
+                         st, x, sinv, K, q, s);
 }
 
 template <int NCH>
-void launch_rmsnorm(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
-                    int64_t M, int K, int8_t *q, float *s, int threads, cudaStream_t st)
+int launch_rmsnorm(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
+                   int64_t M, int K, int8_t *q, float *s, int threads, int dev, cudaStream_t st)
 {
-    if (r)
-        rmsnorm_quant_kernel<NCH, true><<<static_cast<unsigned>(M), threads, 0, st>>>(
-            x, r, h, g, eps, K, q, s);
-    else
-        rmsnorm_quant_kernel<NCH, false><<<static_cast<unsigned>(M), threads, 0, st>>>(
-            x, r, h, g, eps, K, q, s);
+    if (r) {
+        if (int rc = ensure_smem(
+                reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, true>), dev, 0))
+            return rc;
+        return launch_kernel(rmsnorm_quant_kernel<NCH, true>, dim3(static_cast<unsigned>(M)),
+                             dim3(threads), 0, st, x, r, h, g, eps, K, q, s);
+    } else {
+        if (int rc = ensure_smem(
+                reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, false>), dev, 0))
+            return rc;
+        return launch_kernel(rmsnorm_quant_kernel<NCH, false>, dim3(static_cast<unsigned>(M)),
+                             dim3(threads), 0, st, x, r, h, g, eps, K, q, s);
+    }
 }
 
 template <int NCH>
-void launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int threads,
-                 cudaStream_t st)
+int launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int threads, int dev,
+                cudaStream_t st)
 {
-    silu_mul_quant_kernel<NCH><<<static_cast<unsigned>(M), threads, 0, st>>>(gu, I, q, s);
+    if (int rc = ensure_smem(reinterpret_cast<const void *>(&silu_mul_quant_kernel<NCH>), dev, 0))
+        return rc;
+    return launch_kernel(silu_mul_quant_kernel<NCH>, dim3(static_cast<unsigned>(M)), dim3(threads),
+                         0, st, gu, I, q, s);
 }
 
 // ------------------------------------------------------------------ GEMM planning
 
 struct GemmPlan {
-    int variant = 0;   // 1 prefill, 2 decode
+    int variant = 0;   // 1 prefill tiles, 2 decode stream-K, 3 decode cluster split-K
     int tile_n = 256;  // prefill tile width
     int nt = 16;       // decode token tile
-    int ctas = 1;      // decode persistent grid
+    int ctas = 1;      // stream-K persistent grid, or cluster size
     size_t ws_bytes = 0;
     size_t flag_off = 0;
+    size_t part_off = 0;
 };
+
+// stream-K workspace: one flag word per CTA (at most kMaxCtas) in the first kFlagBytes
+constexpr int kMaxCtas = 1024;
+constexpr size_t kFlagBytes = kMaxCtas * 4;
 
 int decode_nt(int64_t M)
 {
     return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
 }
 
+constexpr int kMaxCluster = 8; // portable thread-block cluster size
+
 int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
               GemmPlan *p)
 {
-    if (variant < 0 || variant > 2 || ctas < 0 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
+    if (variant < 0 || variant > 3 || ctas < 0 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
         return W8A8_ERR_INVALID_ARG;
-    if (variant == 0)
-        variant = (M <= 64) ? 2 : 1;
-    if (variant == 2 && M > 256)
+    const int64_t KB = (K + kBK - 1) / kBK;
+    const int64_t NB = (N + kBM - 1) / kBM;
+    if (variant == 0) {
+        if (M > 64)
+            variant = 1;
+        else // few channel blocks: split K inside clusters; many: stream-K over all SMs
+            variant = (2 * NB <= num_sms && KB >= 2) ? 3 : 2;
+    }
+    if ((variant == 2 || variant == 3) && M > 256)
         return W8A8_ERR_UNSUPPORTED_SHAPE;
     p->variant = variant;
-    const int64_t KB = (K + kBK - 1) / kBK;
     if (variant == 1) {
         if (tile_n == 0) {
             const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
@@ -201,21 +288,34 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
         return W8A8_OK;
     }
     p->nt = decode_nt(M);
-    const int64_t NB = (N + kBM - 1) / kBM;
+    if (variant == 3) {
+        int64_t S = ctas > 0 ? ctas : num_sms / NB;
+        S = S < 1 ? 1 : S;
+        S = S > kMaxCluster ? kMaxCluster : S;
+        S = S > KB ? KB : S;
+        p->ctas = static_cast<int>(S);
+        p->ws_bytes = 0;
+        return W8A8_OK;
+    }
     const int64_t U = NB * KB;
     // every CTA must be resident at once (owners wait on later CTAs): at most one per SM
     int64_t G = (ctas == 0 || ctas > num_sms) ? num_sms : ctas;
     if (G > U)
         G = U;
+    if (G > kMaxCtas)
+        G = kMaxCtas;
     p->ctas = static_cast<int>(G);
     // a workspace is needed only if some CTA boundary falls inside a channel block
     bool split = false;
     for (int64_t g = 1; g < G && !split; ++g)
         split = ((g * U) / G) % KB != 0;
     if (split) {
-        const size_t part = static_cast<size_t>(G) * static_cast<size_t>(M) * kBM * 4u;
-        p->flag_off = (part + 255) & ~static_cast<size_t>(255);
-        p->ws_bytes = p->flag_off + static_cast<size_t>(G) * 4u;
+        // flag words first, at a fixed place whatever the shape (they are the only part that
+        // must be zero when a call starts); partial slots after them
+        const int64_t Mp = (M + 3) & ~static_cast<int64_t>(3);
+        p->flag_off = 0;
+        p->part_off = kFlagBytes;
+        p->ws_bytes = kFlagBytes + static_cast<size_t>(G) * kBM * static_cast<size_t>(Mp) * 4u;
     } else {
         p->ws_bytes = 0;
     }
@@ -243,10 +343,50 @@ int launch_prefill(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_
         return rc;
     const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    gemm_prefill_kernel<BN, STAGES><<<grid, kGemmThreads, Cfg::kSmemBytes, st>>>(
-        ta, tb, s_tok, s_ch, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y, acc,
-        kWaitLimitNs);
-    return launch_status();
+    const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
+    return launch_kernel(gemm_prefill_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads),
+                         Cfg::kSmemBytes, st, ta, tb, s_tok, s_ch, static_cast<int>(M),
+                         static_cast<int>(N), static_cast<int>(K), y, acc, prefetch,
+                         kWaitLimitNs);
+}
+
+// Largest cluster size <= want whose clusters can all be resident at once (one wave).
+template <typename Kern>
+int fit_cluster(Kern kernel, int want, int64_t clusters_needed, int smem, int dev)
+{
+    static std::mutex mu;
+    static std::set<std::tuple<const void *, int, int, int>> ok_set, bad_set;
+    for (int S = want; S > 1; --S) {
+        const auto key = std::make_tuple(reinterpret_cast<const void *>(kernel), S, dev,
+                                         static_cast<int>(clusters_needed));
+        {
+            std::lock_guard<std::mutex> lk(mu);
+            if (ok_set.count(key))
+                return S;
+            if (bad_set.count(key))
+                continue;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(S, static_cast<unsigned>(clusters_needed));
+        cfg.blockDim = dim3(kGemmThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        const bool fits = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess &&
+                          n >= clusters_needed;
+        cudaGetLastError();
+        std::lock_guard<std::mutex> lk(mu);
+        (fits ? ok_set : bad_set).insert(key);
+        if (fits)
+            return S;
+    }
+    return 1;
 }
 
 template <int NT, int STAGES, int KPS>
@@ -254,19 +394,32 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
                   const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
                   uint16_t *y, int32_t *acc, void *ws, int dev, cudaStream_t st)
 {
-    using Cfg = DecodeCfg<NT, STAGES, KPS>;
-    const void *fn = reinterpret_cast<const void *>(&gemm_decode_kernel<NT, STAGES, KPS>);
-    int rc = ensure_smem(fn, dev, Cfg::kSmemBytes);
-    if (rc)
+    const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
+    if (p.variant == 3) {
+        using Cfg = DecodeCfg<NT, STAGES, KPS, true>;
+        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true>;
+        if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
+            return rc;
+        const int64_t NB = (N + kBM - 1) / kBM;
+        const int S = fit_cluster(kernel, p.ctas, NB, Cfg::kSmemBytes, dev);
+        return launch_kernel_cluster(kernel, dim3(S, static_cast<unsigned>(NB)), dim3(kGemmThreads),
+                                     Cfg::kSmemBytes, st, static_cast<unsigned>(S), tw, tx, s_tok,
+                                     s_ch, static_cast<int>(M), static_cast<int>(N),
+                                     static_cast<int>(K), y, acc, static_cast<int32_t *>(nullptr),
+                                     static_cast<unsigned int *>(nullptr), prefetch, kWaitLimitNs);
+    }
+    using Cfg = DecodeCfg<NT, STAGES, KPS, false>;
+    auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false>;
+    if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
         return rc;
-    int32_t *ws_part = p.ws_bytes ? static_cast<int32_t *>(ws) : nullptr;
+    int32_t *ws_part =
+        p.ws_bytes ? reinterpret_cast<int32_t *>(static_cast<char *>(ws) + p.part_off) : nullptr;
     unsigned int *ws_flag =
         p.ws_bytes ? reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.flag_off)
                    : nullptr;
-    gemm_decode_kernel<NT, STAGES, KPS><<<p.ctas, kGemmThreads, Cfg::kSmemBytes, st>>>(
-        tw, tx, s_tok, s_ch, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
-        acc, ws_part, ws_flag, kWaitLimitNs);
-    return launch_status();
+    return launch_kernel(kernel, dim3(p.ctas), dim3(kGemmThreads), Cfg::kSmemBytes, st, tw, tx,
+                         s_tok, s_ch, static_cast<int>(M), static_cast<int>(N),
+                         static_cast<int>(K), y, acc, ws_part, ws_flag, prefetch, kWaitLimitNs);
 }
 
 // Decode launch by token tile: (stages, k-blocks per stage) keep ~200 KB of weight and
@@ -279,8 +432,8 @@ int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *
     case 16: return launch_decode<16, 3, 4>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
     case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
     case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
-    case 128: return launch_decode<128, 6, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
-    default: return launch_decode<256, 4, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    case 128: return launch_decode<128, 5, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    default: return launch_decode<256, 3, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
     }
 }
 
@@ -335,11 +488,10 @@ int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, i
     const RowLaunch L = row_launch(K);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (L.nch) {
-    case 1: launch_quantize_rows<1>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, st); break;
-    case 2: launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, st); break;
-    default: launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, st); break;
+    case 1: return launch_quantize_rows<1>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, st);
+    case 2: return launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, st);
+    default: return launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, st);
     }
-    return launch_status();
 }
 
 int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a8_bf16 *h_out,
@@ -364,11 +516,10 @@ int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a
     const RowLaunch L = row_launch(K);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (L.nch) {
-    case 1: launch_rmsnorm<1>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, st); break;
-    case 2: launch_rmsnorm<2>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, st); break;
-    default: launch_rmsnorm<4>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, st); break;
+    case 1: return launch_rmsnorm<1>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, st);
+    case 2: return launch_rmsnorm<2>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, st);
+    default: return launch_rmsnorm<4>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, st);
     }
-    return launch_status();
 }
 
 int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *q, float *s_tok,
@@ -387,11 +538,10 @@ int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *
     const RowLaunch L = row_launch(I);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (L.nch) {
-    case 1: launch_silu<1>(gate_up, M, (int)I, q, s_tok, L.threads, st); break;
-    case 2: launch_silu<2>(gate_up, M, (int)I, q, s_tok, L.threads, st); break;
-    default: launch_silu<4>(gate_up, M, (int)I, q, s_tok, L.threads, st); break;
+    case 1: return launch_silu<1>(gate_up, M, (int)I, q, s_tok, L.threads, dev, st);
+    case 2: return launch_silu<2>(gate_up, M, (int)I, q, s_tok, L.threads, dev, st);
+    default: return launch_silu<4>(gate_up, M, (int)I, q, s_tok, L.threads, dev, st);
     }
-    return launch_status();
 }
 
 size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int ctas,
@@ -455,6 +605,18 @@ int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, co
 {
     return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace,
                                 workspace_bytes, 0, 0, 0, stream);
+}
+
+int w8a8_set_overlap(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return W8A8_ERR_INVALID_ARG;
+    return g_overlap.exchange(mode);
+}
+
+int w8a8_get_overlap(void)
+{
+    return g_overlap.load();
 }
 
 int w8a8_device_status(int reset)
@@ -524,8 +686,10 @@ extern "C" int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, c
     int dev, sms;
     if ((rc = current_device(&dev, &sms)))
         return rc;
+    // the decode kernels, chosen as w8a8_gemm_dequant chooses them for small M
+    const int64_t NB = (N + kBM - 1) / kBM, KB = (K + kBK - 1) / kBK;
     GemmPlan p;
-    if ((rc = plan_gemm(M, N, K, 2, 0, 0, sms, &p)))
+    if ((rc = plan_gemm(M, N, K, (2 * NB <= sms && KB >= 2) ? 3 : 2, 0, 0, sms, &p)))
         return rc;
     if (p.ws_bytes > W8A8_NOALLOC_SCRATCH_BYTES)
         return W8A8_ERR_WORKSPACE;

@@ -10,7 +10,7 @@ import torch
 import int8_w8a8_quantized_smoothed_b200 as w8
 import oracle
 from int8_w8a8_quantized_smoothed_b200 import synth
-from helpers import bf16_out, bf16_ulp_distance, dev, host, host_bf16, with_canary
+from helpers import bf16_out, bf16_ulp_distance, dev, dev_bf16, host, host_bf16, with_canary
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +57,17 @@ def test_decode_kernel_bit_exact(M, N, K, ctas):
     _compare(y, acc, y_ref, acc_ref)
 
 
+@pytest.mark.parametrize("M,N,K", DECODE_SHAPES)
+@pytest.mark.parametrize("cluster", [0, 1, 2, 3, 5, 8])
+def test_decode_cluster_kernel_bit_exact(M, N, K, cluster):
+    # K split over a thread-block cluster of `cluster` CTAs per 128-channel block; partials
+    # summed in distributed shared memory (0: automatic size)
+    xq, st, wq, sc = _inputs(M, N, K, seed=2 * M + N + K)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    y, acc = _run(xq, st, wq, sc, variant=3, ctas=cluster)
+    _compare(y, acc, y_ref, acc_ref)
+
+
 PREFILL_SHAPES = [(1, 8, 16), (16, 512, 256), (128, 256, 128), (129, 264, 400), (200, 136, 208),
                   (300, 1024, 4096), (512, 2048, 1024), (257, 520, 14336), (1000, 3000, 64)]
 
@@ -91,14 +102,15 @@ def test_extreme_accumulators():
     sc = synth.scales(N, 2)
     y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
     assert acc_ref[0, 0] == 127 * 127 * K
-    for variant in (1, 2):
+    for variant in (1, 2, 3):
         y, acc = _run(xq, st, wq, sc, variant=variant)
         _compare(y, acc, y_ref, acc_ref)
 
 
 def test_auto_variant_and_workspace_reuse():
-    # the stream-K workspace must come back zero-filled: run twice through one workspace
-    for (M, N, K) in [(8, 6144, 4096), (64, 4096, 4096), (512, 1024, 1024)]:
+    # the stream-K workspace must come back ready for the next call (flags zero): run twice
+    # through one workspace, with the automatic choice and forced stream-K
+    for (M, N, K) in [(8, 6144, 4096), (64, 4096, 4096), (512, 1024, 1024), (8, 28672, 4096)]:
         xq, st, wq, sc = _inputs(M, N, K, 11)
         y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
         ws = w8.Workspace()
@@ -106,8 +118,11 @@ def test_auto_variant_and_workspace_reuse():
             y = w8.w8a8_gemm_dequant(dev(xq), dev(st), dev(wq), dev(sc), workspace=ws)
             torch.cuda.synchronize()
             assert np.array_equal(host_bf16(y), y_ref)
-        if ws.buf is not None:
-            assert int(ws.buf.count_nonzero()) == 0
+        for _ in range(2):
+            y = w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), workspace=ws,
+                                        variant=2 if M <= 256 else 1)
+            torch.cuda.synchronize()
+            assert np.array_equal(host_bf16(y), y_ref)
 
 
 def test_zero_scales_give_zero():
@@ -116,7 +131,7 @@ def test_zero_scales_give_zero():
     st[2] = 0.0
     sc[5] = 0.0
     y_ref, _ = oracle.gemm_dequant(xq, st, wq, sc)
-    for variant in (1, 2):
+    for variant in (1, 2, 3):
         y = w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), variant=variant)
         yh = host_bf16(y)
         assert np.array_equal(yh, y_ref)
@@ -132,4 +147,51 @@ def test_workspace_too_small_is_reported():
     with pytest.raises(w8.W8A8Error, match="WORKSPACE"):
         w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), workspace=small, variant=2,
                                 ctas=7)
+    assert w8.w8a8_device_status(reset=True) == 0
+
+
+def _chain(layers, ws):
+    """rmsnorm+quant -> GEMM -> SiLU*up+quant -> GEMM, per layer, with no host sync."""
+    outs = []
+    for L in layers:
+        q, s = w8.w8a8_smooth_rmsnorm_quant(L["x"], L["g"], 1e-5)
+        gu = w8.w8a8_gemm_dequant(q, s, *L["w1"], workspace=ws)
+        q2, s2 = w8.w8a8_silu_mul_quant(gu)
+        outs.append(w8.w8a8_gemm_dequant(q2, s2, *L["w2"], workspace=ws))
+    return outs
+
+
+@pytest.mark.parametrize("M", [1, 33, 300])
+def test_overlap_modes_give_identical_results(M):
+    # modes 0/1/2 only change when kernels may start; every output must be the same bits,
+    # eagerly and when the chain is replayed from a CUDA graph
+    H, I = 512, 1024
+    layers = []
+    for i in range(3):
+        layers.append(dict(
+            x=dev_bf16(synth.activation(M, H, 10 + i)),
+            g=dev(synth.gamma(H, 20 + i)),
+            w1=(dev(synth.int8_codes((2 * I, H), 30 + i)), dev(synth.scales(2 * I, 40 + i))),
+            w2=(dev(synth.int8_codes((H, I), 50 + i)), dev(synth.scales(H, 60 + i)))))
+    torch.cuda.synchronize()
+    ws = w8.Workspace()
+    prev = w8.w8a8_get_overlap()
+    try:
+        results = {}
+        for mode in (0, 1, 2):
+            w8.w8a8_set_overlap(mode)
+            eager = [host_bf16(t) for t in _chain(layers, ws)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                outs = _chain(layers, ws)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            results[mode] = (eager, [host_bf16(t) for t in outs])
+            del g
+        for mode in (0, 1, 2):
+            for a, b in zip(results[0][0] + results[0][1], results[mode][0] + results[mode][1]):
+                assert np.array_equal(a, b)
+    finally:
+        w8.w8a8_set_overlap(prev)
     assert w8.w8a8_device_status(reset=True) == 0

@@ -26,10 +26,10 @@ def _bits(y):
     return y.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-# shapes whose stream-K plan splits 128-channel blocks between CTAs, so the scratch array is
-# used ((1, 512, 256) has 8 weight blocks of 128 x 128: 8 CTAs, one k-block each)
-SHAPES = [(8, 6144, 4096), (64, 4096, 14336), (1, 512, 256), (33, 1032, 4096),
-          (256, 1024, 512), (64, 28672, 4096)]
+# weights with many 128-channel blocks run the stream-K kernel, whose partial sums go through
+# the scratch array; the others run the cluster split-K kernel and need no scratch
+SHAPES = [(64, 28672, 4096), (16, 20480, 1024), (100, 10240, 2048), (8, 6144, 4096),
+          (64, 4096, 14336), (1, 512, 256), (33, 1032, 4096)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -52,7 +52,7 @@ def test_noalloc_matches_gemm_dequant_twice(M, N, K):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     dev = torch.device("cuda", 0)
-    M, N, K = 256, 8192, 4096  # scratch 148 CTAs x 256 x 512 B = 19 MB > 8 MiB
+    M, N, K = 256, 20480, 1024  # stream-K scratch 148 CTAs x 256 x 512 B = 19 MB > 8 MiB
     assert w8.w8a8_gemm_workspace_size_ex(M, N, K, 2, 0, 0) > w8.NOALLOC_SCRATCH_BYTES
     xq = torch.zeros((M, K), dtype=torch.int8, device=dev)
     wq = torch.zeros((N, K), dtype=torch.int8, device=dev)
