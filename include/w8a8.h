@@ -198,6 +198,14 @@ W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, con
                                        w8a8_bf16 *y, w8a8_stream_t stream);
 
 /*
+ * Measurement aid, not part of the W8A8 path (the pages have no counterpart): launches `ctas`
+ * CTAs (0 = one per SM), each issuing `iters` back-to-back dense tcgen05.mma kind::i8 of
+ * shape 128 x n x 32 (n = 128 or 256) on shared-memory operands into tensor memory. Timing
+ * it gives the device's INT8 tensor-core rate, 2 * 128 * n * 32 * iters * ctas operations.
+ */
+W8A8_API int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream);
+
+/*
  * Kernel overlap mode, process-wide (default 1). Results are identical in every mode.
  *   0: each kernel of this library starts after the previous work in its stream completes.
  *   1: programmatic dependent launch: a kernel may launch and run its prologue (barrier

@@ -19,7 +19,7 @@ __all__ = [
     "W8A8Error", "lib", "LIB_PATH",
     "w8a8_quantize_rows", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
-    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_set_overlap",
+    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_probe_i8_mma", "w8a8_set_overlap",
     "w8a8_get_overlap", "w8a8_device_status",
     "w8a8_status_string", "w8a8_version",
     "Workspace",
@@ -43,6 +43,7 @@ SIGNATURES = [
                                   _I, _P]),
     ("w8a8_gemm_workspace_size_ex", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
     ("w8a8_gemm_dequant_noalloc", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    ("w8a8_probe_i8_mma", _I, [C.c_longlong, _I, _I, _P]),
     ("w8a8_set_overlap", _I, [_I]),
     ("w8a8_get_overlap", _I, []),
     ("w8a8_device_status", _I, [_I]),
@@ -114,6 +115,12 @@ def w8a8_status_string(status: int) -> str:
 
 def w8a8_version() -> int:
     return lib().w8a8_version()
+
+
+def w8a8_probe_i8_mma(iters: int, n: int = 256, ctas: int = 0, stream=None) -> None:
+    """Measurement aid: back-to-back dense INT8 tcgen05 MMAs on every SM (not the W8A8 path)."""
+    _check("w8a8_probe_i8_mma", lib().w8a8_probe_i8_mma(int(iters), int(n), int(ctas),
+                                                         _stream(stream)))
 
 
 def w8a8_set_overlap(mode: int) -> int:

@@ -23,6 +23,7 @@
 namespace w8a8 {
 
 constexpr int kGemmThreads = 192;
+constexpr int kMaxClusterSize = 8; // portable thread-block cluster size
 constexpr int kBM = 128;  // MMA M: TMEM lanes
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kUmmaK = 32; // K of one kind::i8 MMA
@@ -638,20 +639,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int64_t t = blockIdx.y;
             const int mt = M < NT ? M : NT;
             const uint32_t P = sbase; // partial tiles sit at the same offset in every CTA
-            for (int idx = etid; idx < mt * w; idx += 128) {
-                const int m = idx / w;
-                const int row = r0 + (idx - m * w);
-                const uint32_t la = P + static_cast<uint32_t>((m * kBM + row) * 4);
-                int32_t sum = 0;
-                for (uint32_t p = 0; p < S; ++p)
-                    sum += ld_dsmem_s32(map_peer_smem(la, p));
-                const int n = static_cast<int>(t * kBM) + row;
-                if (n < N) {
-                    const int64_t off = static_cast<int64_t>(m) * N + n;
-                    y[off] = static_cast<uint16_t>(
-                        bf16_bits(dequant_f32(sum, sh_stok[m], __ldg(s_ch + n))));
-                    if (acc_out)
-                        acc_out[off] = sum;
+            // the peers' copies of this CTA's partial-tile base
+            uint32_t peer[kMaxClusterSize];
+#pragma unroll
+            for (int p = 0; p < kMaxClusterSize; ++p)
+                peer[p] = map_peer_smem(P, p < static_cast<int>(S) ? p : 0);
+            const int total = mt * w;
+            // 4 elements per thread per pass, every DSMEM load issued before any sum
+            for (int base = etid; base < total; base += 4 * 128) {
+                int32_t part[4][kMaxClusterSize];
+                int mm[4], rr[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int idx = base + e * 128;
+                    mm[e] = idx / w;
+                    rr[e] = r0 + (idx - mm[e] * w);
+                    const uint32_t off = static_cast<uint32_t>((mm[e] * kBM + rr[e]) * 4);
+#pragma unroll
+                    for (int p = 0; p < kMaxClusterSize; ++p)
+                        part[e][p] = (idx < total && p < static_cast<int>(S))
+                                         ? ld_dsmem_s32(peer[p] + off)
+                                         : 0;
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int n = static_cast<int>(t * kBM) + rr[e];
+                    if (base + e * 128 < total && n < N) {
+                        int32_t sum = 0;
+#pragma unroll
+                        for (int p = 0; p < kMaxClusterSize; ++p)
+                            sum += part[e][p];
+                        const int64_t o = static_cast<int64_t>(mm[e]) * N + n;
+                        y[o] = static_cast<uint16_t>(
+                            bf16_bits(dequant_f32(sum, sh_stok[mm[e]], __ldg(s_ch + n))));
+                        if (acc_out)
+                            acc_out[o] = sum;
+                    }
                 }
             }
         }

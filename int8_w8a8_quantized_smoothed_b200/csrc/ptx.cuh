@@ -284,10 +284,12 @@ __device__ __forceinline__ uint32_t map_peer_smem(uint32_t saddr, uint32_t rank)
     return r;
 }
 
+// Kept in program order with the cluster barriers (volatile) but without a memory clobber,
+// so several of these loads can be in flight at once.
 __device__ __forceinline__ int32_t ld_dsmem_s32(uint32_t addr)
 {
     int32_t v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 

@@ -12,6 +12,7 @@
 #include <utility>
 
 #include "gemm.cuh"
+#include "probe.cuh"
 #include "rowquant.cuh"
 #include "w8a8.h"
 
@@ -260,7 +261,6 @@ int decode_nt(int64_t M)
     return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
 }
 
-constexpr int kMaxCluster = 8; // portable thread-block cluster size
 
 int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
               GemmPlan *p)
@@ -291,7 +291,7 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
     if (variant == 3) {
         int64_t S = ctas > 0 ? ctas : num_sms / NB;
         S = S < 1 ? 1 : S;
-        S = S > kMaxCluster ? kMaxCluster : S;
+        S = S > kMaxClusterSize ? kMaxClusterSize : S;
         S = S > KB ? KB : S;
         p->ctas = static_cast<int>(S);
         p->ws_bytes = 0;
@@ -605,6 +605,29 @@ int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, co
 {
     return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace,
                                 workspace_bytes, 0, 0, 0, stream);
+}
+
+int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream)
+{
+    if (iters < 1 || (n != 128 && n != 256) || ctas < 0)
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    const int grid = ctas == 0 ? sms : ctas;
+    const int smem = 128 * 128 + n * 128 + 64 + 1024;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (n == 256) {
+        if ((rc = ensure_smem(reinterpret_cast<const void *>(&mma_i8_probe_kernel<256>), dev, smem)))
+            return rc;
+        return launch_kernel(mma_i8_probe_kernel<256>, dim3(grid), dim3(128), smem, st, iters,
+                             kWaitLimitNs);
+    }
+    if ((rc = ensure_smem(reinterpret_cast<const void *>(&mma_i8_probe_kernel<128>), dev, smem)))
+        return rc;
+    return launch_kernel(mma_i8_probe_kernel<128>, dim3(grid), dim3(128), smem, st, iters,
+                         kWaitLimitNs);
 }
 
 int w8a8_set_overlap(int mode)
