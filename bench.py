@@ -559,7 +559,8 @@ def run_reference(args, world, rank):
 
 
 def run_case(args):
-    """`--case gemm:M:N:K[:variant]` or `rows:M:K`: one kernel launched repeatedly."""
+    """`--case gemm:M:N:K[:variant]`, `rms:M:K`, `rmsres:M:K`, `quant:M:K` or `silu:M:I`:
+    one kernel launched repeatedly (a CUDA graph of back-to-back launches)."""
     import int8_w8a8_quantized_smoothed_b200 as w8
     from int8_w8a8_quantized_smoothed_b200 import build as wbuild, synth
     wbuild.build()
@@ -582,28 +583,49 @@ def run_case(args):
                                     variant=variant)
         work = gemm_bytes(M, N, K)
     else:
-        M, K = int(parts[1]), int(parts[2])
-        x = synth.activation_device(M, K, 1, dev)
+        # row kernels: rms:M:K, rmsres:M:K, quant:M:K, silu:M:I; inputs rotate over enough
+        # copies to exceed L2
+        kind, M, K = parts[0], int(parts[1]), int(parts[2])
+        cols = 2 * K if kind == "silu" else K
+        copies = max(1, math.ceil(4 * 126e6 / (M * cols * 2)))
+        xs = [synth.activation_device(M, cols, 1 + c, dev) for c in range(copies)]
+        res = synth.activation_device(M, K, 99, dev)
+        h = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
         g = torch.ones(K, device=dev)
         q = torch.empty(M, K, dtype=torch.int8, device=dev)
         s = torch.empty(M, device=dev)
 
         def launch(i):
-            w8.w8a8_smooth_rmsnorm_quant(x, g, EPS, q=q, s_tok=s)
-        work = 3 * M * K + 4 * M + 4 * K
+            x = xs[i % copies]
+            if kind == "rms":
+                w8.w8a8_smooth_rmsnorm_quant(x, g, EPS, q=q, s_tok=s)
+            elif kind == "rmsres":
+                w8.w8a8_smooth_rmsnorm_quant(x, g, EPS, residual=res, h_out=h, q=q, s_tok=s)
+            elif kind == "quant":
+                w8.w8a8_quantize_rows(x, g, q=q, s_tok=s)
+            else:
+                w8.w8a8_silu_mul_quant(x, q=q, s_tok=s)
+        work = {"rms": 3 * M * K, "rmsres": 7 * M * K, "quant": 3 * M * K,
+                "silu": 5 * M * K}[kind] + 4 * M + 4 * K
     for i in range(args.warmup):
         launch(i)
     torch.cuda.synchronize()
+    # time a CUDA graph of `steps` launches, so launch gaps of short kernels do not count
+    cg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cg, capture_error_mode="thread_local"):
+        for i in range(args.steps):
+            launch(i)
+    cg.replay()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for i in range(args.steps):
-        launch(i)
+    cg.replay()
     e1.record()
     torch.cuda.synchronize()
     t = e0.elapsed_time(e1) / 1e3 / args.steps
     return {"case": args.case, "us_per_launch": round(t * 1e6, 3),
             "GBps_algorithmic": round(work / t / 1e9, 1),
-            "note": "eager launches: includes launch gaps when the kernel is short"}
+            "note": "CUDA graph of back-to-back launches"}
 
 
 def main(argv=None):

@@ -62,17 +62,67 @@ __device__ __forceinline__ double block_sum(double v, double *sh)
     return sh[32];
 }
 
-// q = clamp(round_half_even(y / s), -127, 127) with IEEE division; s == 0 gives 0.
-__device__ __forceinline__ int quant1(float y, float s)
+// Adding 1.5 * 2^23 to a binary32 v with |v| < 2^22 leaves v rounded to an integer
+// (round half to even, like rint) in the low bits of the sum: integer rounding on the FMA
+// pipe instead of a float-to-int conversion. For |v| <= 127 the sum's low byte is the int8.
+constexpr float kRoundMagic = 12582912.0f;
+constexpr int kRoundMagicBits = 0x4B400000;
+
+// Bits of RN(clamp(RN(y / s), -127, 127) + 1.5 * 2^23): the low byte is
+// clamp(round_half_even(y / s), -127, 127) as int8 (rounding and clamping commute here).
+__device__ __forceinline__ uint32_t quant_bits(float y, float s)
 {
-    const int v = __float2int_rn(__fdiv_rn(y, s));
-    return max(-127, min(127, v));
+    const float t = fminf(fmaxf(__fdiv_rn(y, s), -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(t, kRoundMagic));
 }
 
-__device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d)
+// Four codes from the low bytes of four quant_bits results.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {
-    return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-           ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// ---- packed binary32 pairs (sm_100 f32x2): each lane is an IEEE RN operation
+
+__device__ __forceinline__ unsigned long long f2_bits(float2 v)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 bits_f2(unsigned long long r)
+{
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(r);
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b)
+{
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+    return bits_f2(r);
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)),
+        "l"(f2_bits(c)));
+    return bits_f2(r);
+}
+
+__device__ __forceinline__ float2 splat2(float v)
+{
+    return make_float2(v, v);
 }
 
 // Quantizes the row held in registers (v[c][0..7] for vector c*blockDim + tid) given its
@@ -91,10 +141,10 @@ __device__ __forceinline__ void quantize_and_store(const float (&v)[NCH][8], flo
         if (vi < nvec) {
             uint2 out = make_uint2(0u, 0u);
             if (amax > 0.0f) {
-                out.x = pack_i8x4(quant1(v[c][0], s), quant1(v[c][1], s), quant1(v[c][2], s),
-                                  quant1(v[c][3], s));
-                out.y = pack_i8x4(quant1(v[c][4], s), quant1(v[c][5], s), quant1(v[c][6], s),
-                                  quant1(v[c][7], s));
+                out.x = pack_low_bytes(quant_bits(v[c][0], s), quant_bits(v[c][1], s),
+                                       quant_bits(v[c][2], s), quant_bits(v[c][3], s));
+                out.y = pack_low_bytes(quant_bits(v[c][4], s), quant_bits(v[c][5], s),
+                                       quant_bits(v[c][6], s), quant_bits(v[c][7], s));
             }
             reinterpret_cast<uint2 *>(qrow)[vi] = out;
         }
@@ -147,14 +197,12 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const uint16_t *__r
             if (sinv) {
                 const float4 a = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * vi);
                 const float4 b = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * vi + 1);
-                v[c][0] = __fmul_rn(v[c][0], a.x);
-                v[c][1] = __fmul_rn(v[c][1], a.y);
-                v[c][2] = __fmul_rn(v[c][2], a.z);
-                v[c][3] = __fmul_rn(v[c][3], a.w);
-                v[c][4] = __fmul_rn(v[c][4], b.x);
-                v[c][5] = __fmul_rn(v[c][5], b.y);
-                v[c][6] = __fmul_rn(v[c][6], b.z);
-                v[c][7] = __fmul_rn(v[c][7], b.w);
+                const float2 p0 = mul2(make_float2(v[c][0], v[c][1]), make_float2(a.x, a.y));
+                const float2 p1 = mul2(make_float2(v[c][2], v[c][3]), make_float2(a.z, a.w));
+                const float2 p2 = mul2(make_float2(v[c][4], v[c][5]), make_float2(b.x, b.y));
+                const float2 p3 = mul2(make_float2(v[c][6], v[c][7]), make_float2(b.z, b.w));
+                v[c][0] = p0.x; v[c][1] = p0.y; v[c][2] = p1.x; v[c][3] = p1.y;
+                v[c][4] = p2.x; v[c][5] = p2.y; v[c][6] = p3.x; v[c][7] = p3.y;
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -224,9 +272,12 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(
             const float4 b = __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi + 1);
             const float g[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                v[c][i] = __fmul_rn(__fmul_rn(v[c][i], rstd), g[i]);
-                amax = fmaxf(amax, fabsf(v[c][i]));
+            for (int i = 0; i < 8; i += 2) { // (h * rstd) * gamma', two lanes at a time
+                const float2 p = mul2(mul2(make_float2(v[c][i], v[c][i + 1]), splat2(rstd)),
+                                      make_float2(g[i], g[i + 1]));
+                v[c][i] = p.x;
+                v[c][i + 1] = p.y;
+                amax = fmaxf(amax, fmaxf(fabsf(p.x), fabsf(p.y)));
             }
         }
     }
@@ -236,41 +287,47 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(
 
 // ----------------------------------------------------------------- SiLU(gate)*up + quant
 
-// Binary32 exp fixed by the library's contract (header w8a8.h): Cody-Waite reduction with
-// a 16-bit head of ln 2, degree-7 Taylor polynomial by Horner in fused multiply-adds,
-// exact scaling by two powers of two.
-__device__ __forceinline__ float w8a8_exp(float x)
+// Binary32 exp fixed by the library's contract (header w8a8.h), two lanes at a time:
+// Cody-Waite reduction with a 16-bit head of ln 2, degree-7 Taylor polynomial by Horner in
+// fused multiply-adds, exact scaling by two powers of two; every step is the scalar
+// definition's IEEE operation, lane by lane.
+__device__ __forceinline__ float2 w8a8_exp2(float2 x)
 {
-    if (x != x)
-        return x;
-    if (x > 89.0f)
-        return __int_as_float(0x7f800000);
-    if (x < -104.0f)
-        return 0.0f;
     const float kInvLn2 = 1.44269502162933349609375f;           // RN(1 / ln 2)
     const float kLn2Hi = 0.693145751953125f;                    // ln 2, 16 significant bits
     const float kLn2Lo = 1.428606765330187045037746429443359375e-06f; // RN(ln 2 - kLn2Hi)
-    const float kf = rintf(__fmul_rn(x, kInvLn2));
-    const int k = static_cast<int>(kf);
-    float r = __fmaf_rn(-kf, kLn2Hi, x);
-    r = __fmaf_rn(-kf, kLn2Lo, r);
-    float p = 1.0f / 5040.0f;
-    p = __fmaf_rn(p, r, 1.0f / 720.0f);
-    p = __fmaf_rn(p, r, 1.0f / 120.0f);
-    p = __fmaf_rn(p, r, 1.0f / 24.0f);
-    p = __fmaf_rn(p, r, 1.0f / 6.0f);
-    p = __fmaf_rn(p, r, 0.5f);
-    p = __fmaf_rn(p, r, 1.0f);
-    p = __fmaf_rn(p, r, 1.0f);
-    const int k1 = k / 2;
-    const int k2 = k - k1;
-    return __fmul_rn(__fmul_rn(p, __int_as_float((k1 + 127) << 23)),
-                     __int_as_float((k2 + 127) << 23));
+    // k = rint(x / ln 2) (|x / ln 2| < 2^22 in range: magic-constant rounding is rint)
+    const float2 km = add2(mul2(x, splat2(kInvLn2)), splat2(kRoundMagic));
+    const float2 kf = add2(km, splat2(-kRoundMagic));
+    float2 r = fma2(kf, splat2(-kLn2Hi), x);
+    r = fma2(kf, splat2(-kLn2Lo), r);
+    float2 p = splat2(1.0f / 5040.0f);
+    p = fma2(p, r, splat2(1.0f / 720.0f));
+    p = fma2(p, r, splat2(1.0f / 120.0f));
+    p = fma2(p, r, splat2(1.0f / 24.0f));
+    p = fma2(p, r, splat2(1.0f / 6.0f));
+    p = fma2(p, r, splat2(0.5f));
+    p = fma2(p, r, splat2(1.0f));
+    p = fma2(p, r, splat2(1.0f));
+    const int ka = __float_as_int(km.x) - kRoundMagicBits;
+    const int kb = __float_as_int(km.y) - kRoundMagicBits;
+    const int ka1 = ka / 2, kb1 = kb / 2; // truncation toward zero
+    const float2 s1 = make_float2(__int_as_float((ka1 + 127) << 23), __int_as_float((kb1 + 127) << 23));
+    const float2 s2 = make_float2(__int_as_float((ka - ka1 + 127) << 23),
+                                  __int_as_float((kb - kb1 + 127) << 23));
+    float2 e = mul2(mul2(p, s1), s2);
+    // outside the reduction's range: NaN stays NaN, x > 89 gives +inf, x < -104 gives +0
+    const float inf = __int_as_float(0x7f800000);
+    e.x = (x.x != x.x) ? x.x : (x.x > 89.0f ? inf : (x.x < -104.0f ? 0.0f : e.x));
+    e.y = (x.y != x.y) ? x.y : (x.y > 89.0f ? inf : (x.y < -104.0f ? 0.0f : e.y));
+    return e;
 }
 
-__device__ __forceinline__ float silu_f32(float g)
+// a = silu(g) * u = (g / (1 + exp(-g))) * u for two lanes; the division stays IEEE scalar.
+__device__ __forceinline__ float2 silu_mul2(float2 g, float2 u)
 {
-    return __fdiv_rn(g, __fadd_rn(1.0f, w8a8_exp(-g)));
+    const float2 d = add2(splat2(1.0f), w8a8_exp2(make_float2(-g.x, -g.y)));
+    return mul2(make_float2(__fdiv_rn(g.x, d.x), __fdiv_rn(g.y, d.y)), u);
 }
 
 template <int NCH>
@@ -296,9 +353,11 @@ __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const uint16_t *__
             unpack8(ldg_nc_v4(gr + vi), g);
             unpack8(ldg_nc_v4(ur + vi), u);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                v[c][i] = __fmul_rn(silu_f32(g[i]), u[i]);
-                amax = fmaxf(amax, fabsf(v[c][i]));
+            for (int i = 0; i < 8; i += 2) {
+                const float2 a2 = silu_mul2(make_float2(g[i], g[i + 1]), make_float2(u[i], u[i + 1]));
+                v[c][i] = a2.x;
+                v[c][i + 1] = a2.y;
+                amax = fmaxf(amax, fmaxf(fabsf(a2.x), fabsf(a2.y)));
             }
         } else {
 #pragma unroll

@@ -119,3 +119,25 @@ def test_weight_rtn_through_quantize_rows():
 
 def test_device_status_clean():
     assert w8.w8a8_device_status(reset=True) == 0
+
+
+def test_quantize_near_half_integer_quotients():
+    # x holds j + 0.5 (j = 0..126) and 127, so with sinv near 1 every y / s lands within a few
+    # ulps of a half-integer: the product-with-reciprocal shortcut must defer to the exact
+    # quotient there, and ties must go to even
+    K = 256
+    base = np.concatenate([np.arange(127) + 0.5, [127.0], -(np.arange(127) + 0.5), [-127.0]])
+    rows = []
+    for i in range(64):
+        rows.append(np.roll(base, i))
+    xf = np.stack(rows).astype(np.float32)
+    xb = torch.from_numpy(xf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    rng = np.random.default_rng(0)
+    for trial in range(4):
+        sinv = (1.0 + (rng.integers(-8, 9, K) * 2.0 ** -23)).astype(np.float32)
+        if trial == 0:
+            sinv[:] = 1.0
+        q_ref, s_ref = oracle.quantize_rows(xb, sinv)
+        q, s = w8.w8a8_quantize_rows(dev_bf16(xb), dev(sinv))
+        assert np.array_equal(host(s), s_ref)
+        assert np.array_equal(host(q), q_ref)
