@@ -152,8 +152,9 @@ W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_
  * variant 2 = persistent CTAs sharing the weight stream (0 = one per SM, at most one per SM);
  * variant 3 = cluster size, the number of K splits per 128-channel block (0 = automatic,
  * at most 8, fewer if the clusters would not all fit on the GPU at once). tile_n (variant 1)
- * = 0 automatic, else 128 or 256. The workspace needed is w8a8_gemm_workspace_size_ex() of
- * the same arguments (only variant 2 uses one).
+ * = 0 automatic, 128 (128 x 128 output tiles), 256 (128 x 256) or 512 (256 x 256). The
+ * workspace needed is w8a8_gemm_workspace_size_ex() of the same arguments (only variant 2
+ * uses one).
  */
 W8A8_API int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
                          const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,

@@ -28,7 +28,27 @@ constexpr int kBM = 128;  // MMA M: TMEM lanes
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kUmmaK = 32; // K of one kind::i8 MMA
 
+// Producer tail of an mbarrier ring: waits until the consumer has released the last
+// min(issued, stages) stages, i.e. until the empty-barrier phase that each of the last
+// issued iterations j completes (parity (j / stages) & 1) has completed.
+__device__ __forceinline__ void drain_ring(uint32_t bar_empty, uint32_t issued, uint32_t stages,
+                                           unsigned long long limit_ns)
+{
+    for (uint32_t j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+        if (!mbar_wait(bar_empty + 8 * (j % stages), (j / stages) & 1u, limit_ns))
+            return;
+}
+
 // ---------------------------------------------------------------- prefill (persistent)
+//
+// gemm_prefill_kernel: one CTA per 128 x BN output tile (BN = 128 or 256), two TMEM
+// accumulators so the epilogue of tile t overlaps the MMAs of tile t+1.
+//
+// gemm_prefill_pair_kernel: a cluster of two CTAs per 256 x 256 tile with the 2-SM MMA
+// (cta_group::2). Each CTA loads only its 128-row halves of A and B, and the pair's tensor
+// cores share them, so per SM the shared-memory traffic (TMA writes plus operand reads) is
+// two thirds of a one-CTA 128 x 256 tile's for the same MACs: the one-CTA kernel is bound by
+// that traffic, not by DRAM or the tensor pipe.
 
 template <int BN, int STAGES> struct PrefillCfg {
     static constexpr int kABytes = kBM * kBK;
@@ -39,6 +59,7 @@ template <int BN, int STAGES> struct PrefillCfg {
     static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 16 + 1024;
     static constexpr int kTmemCols = 2 * BN;
     static_assert(kTmemCols <= 512, "two accumulators must fit TMEM");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 // Tile order: groups of kGroupM row-tiles, column-major inside a group, so CTAs running
@@ -54,6 +75,39 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
     const int local = tile - group * per_group;
     mb = first_m + local % gm;
     nb = local / gm;
+}
+
+// Dequantizes 32 accumulator columns of one output row and stores them as bf16 (16-byte
+// stores); also the raw int32 values when acc_out is given.
+__device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row, int n0, int N,
+                                                float st, const float *__restrict__ s_ch,
+                                                uint16_t *__restrict__ y,
+                                                int32_t *__restrict__ acc_out)
+{
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const int n = n0 + 8 * g;
+        if (n < N) {
+            const float4 c0 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
+            const float4 c1 = __ldg(reinterpret_cast<const float4 *>(s_ch + n) + 1);
+            const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                f[i] = dequant_f32(static_cast<int32_t>(r[8 * g + i]), st, sc[i]);
+            uint4 o;
+            o.x = pack_bf16x2(f[0], f[1]);
+            o.y = pack_bf16x2(f[2], f[3]);
+            o.z = pack_bf16x2(f[4], f[5]);
+            o.w = pack_bf16x2(f[6], f[7]);
+            *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(row) * N + n) = o;
+            if (acc_out) {
+                int4 *ap = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + n);
+                ap[0] = make_int4(r[8 * g + 0], r[8 * g + 1], r[8 * g + 2], r[8 * g + 3]);
+                ap[1] = make_int4(r[8 * g + 4], r[8 * g + 5], r[8 * g + 6], r[8 * g + 7]);
+            }
+        }
+    }
 }
 
 template <int BN, int STAGES>
@@ -102,14 +156,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (warp == 1) {
         tmem_alloc(tslot, Cfg::kTmemCols);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tslot_ptr);
-    if (threadIdx.x == 0)
-        pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -151,12 +202,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tma_load_2d(sB + s * Cfg::kBBytes, &tmB, bar_full + 8 * s, kb * kBK, nb * BN);
                 }
             }
-            // Wait until the loads still in the ring have landed before the CTA may exit.
-            if (ok) {
-                const uint32_t n_issued = it;
-                for (uint32_t j = (n_issued > STAGES ? n_issued - STAGES : 0); j < n_issued; ++j)
-                    mbar_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1u, limit_ns);
-            }
+            // Producer tail: wait until the MMA warp has released the last ring of stages,
+            // so no load and no tcgen05.commit arrival is still in flight when the CTA exits.
+            if (ok)
+                drain_ring(bar_empty, it, STAGES, limit_ns);
+            // every stage consumed: the next kernel in the stream may launch now
+            pdl_launch_dependents();
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -213,33 +264,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tbase + c * 32, r);
                 tmem_ld_wait();
-                const int n0 = nb * BN + c * 32;
-                if (row_ok) {
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int n = n0 + 8 * g;
-                        if (n < N) {
-                            const float4 c0 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
-                            const float4 c1 = __ldg(reinterpret_cast<const float4 *>(s_ch + n) + 1);
-                            const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                            float f[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                f[i] = dequant_f32(static_cast<int32_t>(r[8 * g + i]), st, sc[i]);
-                            uint4 o;
-                            o.x = pack_bf16x2(f[0], f[1]);
-                            o.y = pack_bf16x2(f[2], f[3]);
-                            o.z = pack_bf16x2(f[4], f[5]);
-                            o.w = pack_bf16x2(f[6], f[7]);
-                            *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(row) * N + n) = o;
-                            if (acc_out) {
-                                int4 *ap = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + n);
-                                ap[0] = make_int4(r[8 * g + 0], r[8 * g + 1], r[8 * g + 2], r[8 * g + 3]);
-                                ap[1] = make_int4(r[8 * g + 4], r[8 * g + 5], r[8 * g + 6], r[8 * g + 7]);
-                            }
-                        }
-                    }
-                }
+                if (row_ok)
+                    store_row_chunk(r, row, nb * BN + c * 32, N, st, s_ch, y, acc_out);
             }
             tc_fence_before();
             __syncwarp();
@@ -248,11 +274,215 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     }
     __syncwarp();
+    if (warp == 1)
+        tmem_relinquish(); // after the work, as the allocator's permit protocol expects
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
     }
+}
+
+// ---------------------------------------------------------------- prefill, CTA pairs
+
+template <int STAGES> struct PairCfg {
+    static constexpr int kHalf = 128;             // rows of A and of B per CTA
+    static constexpr int kABytes = kHalf * kBK;   // 16 KB
+    static constexpr int kBBytes = kHalf * kBK;   // 16 KB
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kBarOff = STAGES * kStageBytes;
+    static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 16 + 1024;
+    static constexpr int kTmemCols = 512;         // two 128 x 256 accumulators per CTA
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB,
+                             const float *__restrict__ s_tok, const float *__restrict__ s_ch,
+                             int M, int N, int K, uint16_t *__restrict__ y,
+                             int32_t *__restrict__ acc_out, int prefetch_static,
+                             unsigned long long limit_ns)
+{
+    using Cfg = PairCfg<STAGES>;
+    constexpr int TN = 256, TM = 256;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sA = sbase;
+    const uint32_t sB = sbase + STAGES * Cfg::kABytes;
+    const uint32_t bar_full = sbase + Cfg::kBarOff;     // used in the even CTA
+    const uint32_t bar_empty = bar_full + 8 * STAGES;   // both CTAs
+    const uint32_t bar_tfull = bar_empty + 8 * STAGES;  // both CTAs
+    const uint32_t bar_tempty = bar_tfull + 16;         // used in the even CTA
+    const uint32_t tslot = bar_tempty + 16;
+    uint32_t *tslot_ptr = reinterpret_cast<uint32_t *>(smem + Cfg::kBarOff + (2 * STAGES + 4) * 8);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank(); // 0: leader (issues the MMAs), 1: peer
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int num_m = (M + TM - 1) / TM;
+    const int num_n = (N + TN - 1) / TN;
+    const int tiles = num_m * num_n;
+    const int kblocks = (K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull + 8 * b, 1);
+            mbar_init(bar_tempty + 8 * b, 8); // 4 epilogue warps in each CTA of the pair
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    // Both CTAs' barriers are initialized before either uses the other's, and both CTAs are
+    // running before the pair allocates tensor memory together (allocating first, with the
+    // pair launched early behind the previous kernel, intermittently never returned).
+    cluster_sync();
+    if (warp == 1) {
+        tmem_alloc_pair(tslot, Cfg::kTmemCols);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tslot_ptr);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t full0 = map_peer_smem(bar_full, 0); // the leader's full barriers
+            uint32_t npre = 0;
+            if (prefetch_static) {
+                for (int tile = pair; tile < tiles && npre < STAGES; tile += npairs) {
+                    int mb, nb;
+                    tile_coords(tile, num_m, num_n, mb, nb);
+                    for (int kb = 0; kb < kblocks && npre < STAGES; ++kb, ++npre) {
+                        if (rank == 0)
+                            mbar_expect_tx(bar_full + 8 * npre, 2 * Cfg::kStageBytes);
+                        tma_load_2d_pair(sB + npre * Cfg::kBBytes, &tmB, full0 + 8 * npre,
+                                         kb * kBK, nb * TN + rank * Cfg::kHalf);
+                    }
+                }
+            }
+            pdl_wait();
+            uint32_t it = 0;
+            for (int tile = pair; tile < tiles; tile += npairs) {
+                int mb, nb;
+                tile_coords(tile, num_m, num_n, mb, nb);
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const uint32_t s = it % STAGES;
+                    if (it < npre) {
+                        tma_load_2d_pair(sA + s * Cfg::kABytes, &tmA, full0 + 8 * s, kb * kBK,
+                                         mb * TM + rank * Cfg::kHalf);
+                        continue;
+                    }
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0)
+                        mbar_expect_tx(bar_full + 8 * s, 2 * Cfg::kStageBytes);
+                    tma_load_2d_pair(sA + s * Cfg::kABytes, &tmA, full0 + 8 * s, kb * kBK,
+                                     mb * TM + rank * Cfg::kHalf);
+                    tma_load_2d_pair(sB + s * Cfg::kBBytes, &tmB, full0 + 8 * s, kb * kBK,
+                                     nb * TN + rank * Cfg::kHalf);
+                }
+                if (!ok) {
+                    it = 0; // leave the tail: a stage wait already ran out
+                    break;
+                }
+            }
+            // Producer tail (each CTA): the leader's multicast commits have released every
+            // stage of this CTA's ring before it may exit.
+            drain_ring(bar_empty, it, STAGES, limit_ns);
+            pdl_launch_dependents(); // the pair's main loop is done in this CTA
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_i8(TM, TN);
+            uint32_t it = 0, t = 0;
+            bool ok = true;
+            for (int tile = pair; tile < tiles && ok; tile += npairs, ++t) {
+                const uint32_t buf = t & 1u;
+                const uint32_t aph = (t >> 1) & 1u;
+                if (!mbar_wait(bar_tempty + 8 * buf, aph ^ 1u, limit_ns))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + buf * TN;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const uint32_t s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(bar_full + 8 * s, ph, limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = sA + s * Cfg::kABytes;
+                    const uint32_t b0 = sB + s * Cfg::kBBytes;
+#pragma unroll
+                    for (int k = 0; k < kBK / kUmmaK; ++k)
+                        umma_i8_pair(d, sw128_kmajor_desc(a0 + k * kUmmaK),
+                                     sw128_kmajor_desc(b0 + k * kUmmaK), idesc,
+                                     (kb > 0 || k > 0) ? 1u : 0u);
+                    umma_commit_pair(bar_empty + 8 * s, 0x3); // frees the stage in both CTAs
+                }
+                if (ok)
+                    umma_commit_pair(bar_tfull + 8 * buf, 0x3);
+            }
+        }
+    } else {
+        // epilogue warps 2..5: this CTA's 128 accumulator rows of the 256-row tile
+        pdl_wait();
+        const int quarter = warp & 3;
+        const uint32_t tempty0 = map_peer_smem(bar_tempty, 0);
+        uint32_t t = 0;
+        for (int tile = pair; tile < tiles; tile += npairs, ++t) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            const uint32_t buf = t & 1u;
+            const uint32_t aph = (t >> 1) & 1u;
+            if (!mbar_wait(bar_tfull + 8 * buf, aph, limit_ns))
+                break;
+            tc_fence_after();
+            const int row = mb * TM + static_cast<int>(rank) * Cfg::kHalf + quarter * 32 + lane;
+            const bool row_ok = row < M;
+            const float st = row_ok ? __ldg(s_tok + row) : 0.0f;
+            const uint32_t tbase = tmem_base + buf * TN + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < TN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tbase + c * 32, r);
+                tmem_ld_wait();
+                if (row_ok)
+                    store_row_chunk(r, row, nb * TN + c * 32, N, st, s_ch, y, acc_out);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(tempty0 + 8 * buf); // release the leader's accumulator
+        }
+    }
+    __syncwarp();
+    if (warp == 1)
+        tmem_relinquish_pair(); // after the work, as the allocator's permit protocol expects
+    // every MMA, commit and remote arrive of the pair is done before either CTA frees
+    // its tensor memory or leaves
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
 }
 
 // ---------------------------------------------------------------- decode (swap-AB)
@@ -381,14 +611,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (warp == 1) {
         tmem_alloc(tslot, Cfg::kTmemCols);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tslot_ptr);
-    if (threadIdx.x == 0)
-        pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -440,10 +667,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 u += sg.kb1 - sg.kb0;
             }
-            if (ok) {
-                for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    mbar_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1u, limit_ns);
-            }
+            // Producer tail: every stage released by the MMA warp before the CTA may exit.
+            if (ok)
+                drain_ring(bar_empty, it, STAGES, limit_ns);
+            // every stage consumed: the next kernel in the stream may launch now
+            pdl_launch_dependents();
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -681,6 +909,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // nobody leaves while a peer may still read its shared memory
         cluster_sync();
     }
+    if (warp == 1)
+        tmem_relinquish(); // after the work, as the allocator's permit protocol expects
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();

@@ -265,7 +265,8 @@ int decode_nt(int64_t M)
 int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
               GemmPlan *p)
 {
-    if (variant < 0 || variant > 3 || ctas < 0 || (tile_n != 0 && tile_n != 128 && tile_n != 256))
+    if (variant < 0 || variant > 3 || ctas < 0 ||
+        (tile_n != 0 && tile_n != 128 && tile_n != 256 && tile_n != 512))
         return W8A8_ERR_INVALID_ARG;
     const int64_t KB = (K + kBK - 1) / kBK;
     const int64_t NB = (N + kBM - 1) / kBM;
@@ -280,8 +281,24 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
     p->variant = variant;
     if (variant == 1) {
         if (tile_n == 0) {
-            const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
-            tile_n = tiles256 >= num_sms ? 256 : 128;
+            // Cost model: a tile is bound by its SMs' shared-memory traffic (TMA writes plus
+            // tensor-core operand reads) for its MACs. Relative tile times: 128x128 on one SM
+            // -> 2, 128x256 on one SM -> 3, 256x256 on a CTA pair -> 2 (each SM does 128x256
+            // MACs with two thirds of the traffic). A launch takes ceil(tiles / concurrent
+            // tiles) tile times.
+            const int64_t cand[3][4] = {{128, 128, 2, 1}, {128, 256, 3, 1}, {256, 256, 2, 2}};
+            int64_t best = -1, best_cost = 0;
+            for (int i = 0; i < 3; ++i) {
+                const int64_t tiles = ((M + cand[i][0] - 1) / cand[i][0]) *
+                                      ((N + cand[i][1] - 1) / cand[i][1]);
+                const int64_t slots = num_sms / cand[i][3];
+                const int64_t cost = ((tiles + slots - 1) / slots) * cand[i][2];
+                if (best < 0 || cost < best_cost) {
+                    best = i;
+                    best_cost = cost;
+                }
+            }
+            tile_n = best == 0 ? 128 : best == 1 ? 256 : 512;
         }
         p->tile_n = tile_n;
         p->ws_bytes = 0;
@@ -348,6 +365,58 @@ int launch_prefill(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_
                          Cfg::kSmemBytes, st, ta, tb, s_tok, s_ch, static_cast<int>(M),
                          static_cast<int>(N), static_cast<int>(K), y, acc, prefetch,
                          kWaitLimitNs);
+}
+
+// Resident pair clusters of the pair kernel on this device (cached per device).
+int pair_clusters(const void *kernel, int smem, int dev, int num_sms)
+{
+    static std::mutex mu;
+    static int cached[kMaxDevices] = {0};
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (cached[dev] > 0)
+            return cached[dev];
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n < 1)
+        n = num_sms / 2;
+    cudaGetLastError();
+    std::lock_guard<std::mutex> lk(mu);
+    cached[dev] = n;
+    return n;
+}
+
+template <int STAGES>
+int launch_prefill_pair(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
+                        const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y,
+                        int32_t *acc, int dev, int num_sms, cudaStream_t st)
+{
+    using Cfg = PairCfg<STAGES>;
+    auto kernel = gemm_prefill_pair_kernel<STAGES>;
+    int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes);
+    if (rc)
+        return rc;
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    int64_t pairs = pair_clusters(reinterpret_cast<const void *>(kernel), Cfg::kSmemBytes, dev,
+                                  num_sms);
+    if (pairs > tiles)
+        pairs = tiles;
+    const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
+    return launch_kernel_cluster(kernel, dim3(static_cast<unsigned>(2 * pairs)),
+                                 dim3(kGemmThreads), Cfg::kSmemBytes, st, 2u, ta, tb, s_tok, s_ch,
+                                 static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
+                                 acc, prefetch, kWaitLimitNs);
 }
 
 // Largest cluster size <= want whose clusters can all be resident at once (one wave).
@@ -586,9 +655,13 @@ int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
         return W8A8_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (p.variant == 1) {
+        // tile_n: 128 -> 128 x 128, 256 -> 128 x 256, 512 -> 256 x 256 by a CTA pair
+        const int bn = p.tile_n == 128 ? 128 : p.tile_n == 256 ? 256 : 128;
         CUtensorMap ta, tb;
-        if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, p.tile_n))
+        if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, bn))
             return W8A8_ERR_CUDA;
+        if (p.tile_n == 512)
+            return launch_prefill_pair<6>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
         if (p.tile_n == 256)
             return launch_prefill<256, 4>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
         return launch_prefill<128, 6>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);

@@ -73,8 +73,9 @@ PREFILL_SHAPES = [(1, 8, 16), (16, 512, 256), (128, 256, 128), (129, 264, 400), 
 
 
 @pytest.mark.parametrize("M,N,K", PREFILL_SHAPES)
-@pytest.mark.parametrize("tile_n", [128, 256])
+@pytest.mark.parametrize("tile_n", [128, 256, 512])
 def test_prefill_kernel_bit_exact(M, N, K, tile_n):
+    # tile_n 128 / 256: 128-row tiles, double-buffered accumulators; 512: 256 x 256 tiles
     xq, st, wq, sc = _inputs(M, N, K, seed=3 * M + N + K)
     y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
     y, acc = _run(xq, st, wq, sc, variant=1, tile_n=tile_n)
@@ -86,7 +87,7 @@ def test_persistent_kernel_many_tiles_per_cta():
     M, N, K = 2048, 4096, 256
     xq, st, wq, sc = _inputs(M, N, K, 5)
     y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
-    for tn in (128, 256):
+    for tn in (128, 256, 512):
         y, acc = _run(xq, st, wq, sc, variant=1, tile_n=tn)
         _compare(y, acc, y_ref, acc_ref)
 
