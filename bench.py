@@ -293,13 +293,28 @@ class Layer:
             w8.w8a8_gemm_dequant(self.q4, self.s4, *self.w["down"], y=self.down, workspace=ws)
 
 
-def measure_int8_peak(iters=20000, reps=3):
-    """Dense INT8 tensor-core rate of this device in TOPS: the best of `reps` launches of the
-    library's tcgen05 kind::i8 probe (128 x 256 x 32 MMAs back to back on every SM)."""
+def measure_int8_peak(iters=20000, reps=3, sustained_s=0.0):
+    """Dense INT8 tensor-core rate of this device in TOPS from the library's tcgen05 kind::i8
+    probe (128 x 256 x 32 MMAs back to back on every SM): the best of `reps` launches
+    (burst), or with sustained_s > 0 the average over launches back to back for that many
+    seconds (the rate under the power cap, for kernels timed inside a long step)."""
     import int8_w8a8_quantized_smoothed_b200 as w8
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    ops = 2 * 128 * 256 * 32 * iters * sms
     w8.w8a8_probe_i8_mma(1000)
     torch.cuda.synchronize()
+    if sustained_s > 0:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n, t0 = 0, time.perf_counter()
+        e0.record()
+        while time.perf_counter() - t0 < sustained_s:
+            for _ in range(10):
+                w8.w8a8_probe_i8_mma(iters)
+            n += 10
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        return ops * n / (e0.elapsed_time(e1) / 1e3) / 1e12
     best = 0.0
     for _ in range(reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -307,7 +322,7 @@ def measure_int8_peak(iters=20000, reps=3):
         w8.w8a8_probe_i8_mma(iters)
         e1.record()
         torch.cuda.synchronize()
-        best = max(best, 2 * 128 * 256 * 32 * iters * sms / (e0.elapsed_time(e1) / 1e3) / 1e12)
+        best = max(best, ops / (e0.elapsed_time(e1) / 1e3) / 1e12)
     return best
 
 
@@ -427,12 +442,18 @@ def run_ours(args, world, rank, local):
     t_roof_meas = max(ops / (int8_peak * 1e12), nbytes / (hbm_peak * 1e9))
     tensor_bound = ops / (int8_peak * 1e12) > g_bytes / (hbm_peak * 1e9)
     if tensor_bound:
-        roofline = {"kernel": "gemm_prefill_kernel (all GEMM launches of the step)",
+        # the GEMMs run inside a long step under the power cap: the sustained probe rate is
+        # the denominator; the burst rate and the nominal figure are reported beside it
+        int8_sus = measure_int8_peak(sustained_s=3.0)
+        roofline = {"kernel": "gemm_prefill_pair_kernel / gemm_prefill_kernel "
+                              "(all GEMM launches of the step)",
                     "bound": "tensor", "achieved": round(gemm_tops, 1),
-                    "peak": round(int8_peak, 1), "unit": "TFLOP/s",
-                    "frac": round(gemm_tops / int8_peak, 4),
-                    "peak_source": "measured: tcgen05 kind::i8 probe in this run (burst); "
-                                   f"nominal dense INT8 {INT8_NOMINAL_TOPS:.0f}",
+                    "peak": round(int8_sus, 1), "unit": "TFLOP/s",
+                    "frac": round(gemm_tops / int8_sus, 4),
+                    "peak_source": "measured: tcgen05 kind::i8 probe in this run, 3 s back to "
+                                   "back (sustained)",
+                    "peak_burst": round(int8_peak, 1),
+                    "frac_of_burst": round(gemm_tops / int8_peak, 4),
                     "frac_of_nominal": round(gemm_tops / INT8_NOMINAL_TOPS, 4),
                     "traffic": None}
     else:
