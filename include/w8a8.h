@@ -201,8 +201,9 @@ W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, con
 /*
  * Measurement aid, not part of the W8A8 path (the pages have no counterpart): launches `ctas`
  * CTAs (0 = one per SM), each issuing `iters` back-to-back dense tcgen05.mma kind::i8 of
- * shape 128 x n x 32 (n = 128 or 256) on shared-memory operands into tensor memory. Timing
- * it gives the device's INT8 tensor-core rate, 2 * 128 * n * 32 * iters * ctas operations.
+ * shape 128 x n x 32 (n = 16, 32, 64, 128 or 256) on shared-memory operands into tensor
+ * memory. Timing it gives the device's INT8 tensor-core rate at that shape,
+ * 2 * 128 * n * 32 * iters * ctas operations. W8A8_ERR_INVALID_ARG for any other n.
  */
 W8A8_API int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream);
 

@@ -55,8 +55,10 @@ template <int BN, int STAGES> struct PrefillCfg {
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kBarOff = STAGES * kStageBytes;
-    // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot
-    static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 16 + 1024;
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot; then each epilogue warp's
+    // channel scales of two tiles [4][2][BN]
+    static constexpr int kSchOff = (kBarOff + (2 * STAGES + 4) * 8 + 16 + 15) & ~15;
+    static constexpr int kSmemBytes = kSchOff + 4 * 2 * BN * 4 + 1024;
     static constexpr int kTmemCols = 2 * BN;
     static_assert(kTmemCols <= 512, "two accumulators must fit TMEM");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -78,9 +80,10 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
 }
 
 // Dequantizes 32 accumulator columns of one output row and stores them as bf16 (16-byte
-// stores); also the raw int32 values when acc_out is given.
+// stores); also the raw int32 values when acc_out is given. sc: the 32 channel scales of
+// these columns, in shared memory.
 __device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row, int n0, int N,
-                                                float st, const float *__restrict__ s_ch,
+                                                float st, const float *sc,
                                                 uint16_t *__restrict__ y,
                                                 int32_t *__restrict__ acc_out)
 {
@@ -88,13 +91,13 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row
     for (int g = 0; g < 4; ++g) {
         const int n = n0 + 8 * g;
         if (n < N) {
-            const float4 c0 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
-            const float4 c1 = __ldg(reinterpret_cast<const float4 *>(s_ch + n) + 1);
-            const float sc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const float4 c0 = reinterpret_cast<const float4 *>(sc)[2 * g];
+            const float4 c1 = reinterpret_cast<const float4 *>(sc)[2 * g + 1];
+            const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
             float f[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                f[i] = dequant_f32(static_cast<int32_t>(r[8 * g + i]), st, sc[i]);
+                f[i] = dequant_f32(static_cast<int32_t>(r[8 * g + i]), st, cs[i]);
             uint4 o;
             o.x = pack_bf16x2(f[0], f[1]);
             o.y = pack_bf16x2(f[2], f[3]);
@@ -109,6 +112,33 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row
         }
     }
 }
+
+// Scales of one output tile for the prefill epilogues, fetched one tile ahead by each
+// epilogue warp so that their global-memory latency overlaps the current tile's work: the BN
+// channel scales (BN / 32 per lane, published to the warp's own shared-memory copy) and the
+// token scale of the lane's own row. Warp-private, so no barrier beyond __syncwarp is needed.
+template <int BN> struct TileScales {
+    float sc[BN / 32];
+    float st;
+    __device__ __forceinline__ void fetch(const float *__restrict__ s_ch,
+                                          const float *__restrict__ s_tok, int n0, int N, int row,
+                                          int M, int lane)
+    {
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j) {
+            const int n = n0 + lane + 32 * j;
+            sc[j] = n < N ? __ldg(s_ch + n) : 0.0f;
+        }
+        st = row < M ? __ldg(s_tok + row) : 0.0f;
+    }
+    __device__ __forceinline__ void publish(float *sh, int lane) const
+    {
+#pragma unroll
+        for (int j = 0; j < BN / 32; ++j)
+            sh[lane + 32 * j] = sc[j];
+        __syncwarp();
+    }
+};
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -246,18 +276,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
         pdl_wait(); // s_tok comes from the previous kernel; y may still be read by it
         const int quarter = warp & 3;
+        float *sh_sch = reinterpret_cast<float *>(smem + Cfg::kSchOff) + (warp - 2) * 2 * BN;
+        TileScales<BN> nxt;
+        auto fetch = [&](int tile) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            nxt.fetch(s_ch, s_tok, nb * BN, N, mb * kBM + quarter * 32 + lane, M, lane);
+        };
+        if (static_cast<int>(blockIdx.x) < tiles)
+            fetch(blockIdx.x);
         uint32_t t = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++t) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
             const uint32_t buf = t & 1u;
             const uint32_t aph = (t >> 1) & 1u;
+            // this tile's scales to the warp's shared memory (the buffer of tile t-2 is free:
+            // the warp synchronized after it), the next tile's requested
+            nxt.publish(sh_sch + buf * BN, lane);
+            const float st = nxt.st;
+            if (tile + static_cast<int>(gridDim.x) < tiles)
+                fetch(tile + gridDim.x);
             if (!mbar_wait(bar_tfull + 8 * buf, aph, limit_ns))
                 break;
             tc_fence_after();
             const int row = mb * kBM + quarter * 32 + lane;
             const bool row_ok = row < M;
-            const float st = row_ok ? __ldg(s_tok + row) : 0.0f;
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
@@ -265,7 +309,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tmem_ld_32x32b_x32(tbase + c * 32, r);
                 tmem_ld_wait();
                 if (row_ok)
-                    store_row_chunk(r, row, nb * BN + c * 32, N, st, s_ch, y, acc_out);
+                    store_row_chunk(r, row, nb * BN + c * 32, N, st, sh_sch + buf * BN + c * 32,
+                                    y, acc_out);
             }
             tc_fence_before();
             __syncwarp();
@@ -291,7 +336,8 @@ template <int STAGES> struct PairCfg {
     static constexpr int kBBytes = kHalf * kBK;   // 16 KB
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kBarOff = STAGES * kStageBytes;
-    static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 16 + 1024;
+    static constexpr int kSchOff = (kBarOff + (2 * STAGES + 4) * 8 + 16 + 15) & ~15;
+    static constexpr int kSmemBytes = kSchOff + 4 * 2 * 256 * 4 + 1024; // + scales [4][2][256]
     static constexpr int kTmemCols = 512;         // two 128 x 256 accumulators per CTA
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
@@ -446,18 +492,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         pdl_wait();
         const int quarter = warp & 3;
         const uint32_t tempty0 = map_peer_smem(bar_tempty, 0);
+        const int row_in_tile = static_cast<int>(rank) * Cfg::kHalf + quarter * 32 + lane;
+        float *sh_sch = reinterpret_cast<float *>(smem + Cfg::kSchOff) + (warp - 2) * 2 * TN;
+        TileScales<TN> nxt;
+        auto fetch = [&](int tile) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            nxt.fetch(s_ch, s_tok, nb * TN, N, mb * TM + row_in_tile, M, lane);
+        };
+        if (pair < tiles)
+            fetch(pair);
         uint32_t t = 0;
         for (int tile = pair; tile < tiles; tile += npairs, ++t) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
             const uint32_t buf = t & 1u;
             const uint32_t aph = (t >> 1) & 1u;
+            // this tile's scales to the warp's shared memory, the next tile's requested
+            nxt.publish(sh_sch + buf * TN, lane);
+            const float st = nxt.st;
+            if (tile + npairs < tiles)
+                fetch(tile + npairs);
             if (!mbar_wait(bar_tfull + 8 * buf, aph, limit_ns))
                 break;
             tc_fence_after();
-            const int row = mb * TM + static_cast<int>(rank) * Cfg::kHalf + quarter * 32 + lane;
+            const int row = mb * TM + row_in_tile;
             const bool row_ok = row < M;
-            const float st = row_ok ? __ldg(s_tok + row) : 0.0f;
             const uint32_t tbase = tmem_base + buf * TN + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < TN / 32; ++c) {
@@ -465,7 +525,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tmem_ld_32x32b_x32(tbase + c * 32, r);
                 tmem_ld_wait();
                 if (row_ok)
-                    store_row_chunk(r, row, nb * TN + c * 32, N, st, s_ch, y, acc_out);
+                    store_row_chunk(r, row, nb * TN + c * 32, N, st, sh_sch + buf * TN + c * 32,
+                                    y, acc_out);
             }
             tc_fence_before();
             __syncwarp();
@@ -493,16 +554,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //
 // CLUSTER (few channel blocks): grid (S, NB) with thread-block clusters of S CTAs along K;
 //   CTA r of block t takes k-blocks [r KB / S, (r+1) KB / S). The S partial accumulators meet
-//   in shared memory: each CTA writes its partial to its own (now idle) stage buffers, the
-//   cluster synchronizes, and CTA r sums rows [r 128 / S, (r+1) 128 / S) of all S partials
-//   through distributed shared memory, dequantizes and stores them. No global workspace.
+//   in shared memory: each CTA writes its partial tile [token][128 channels] to its own (now
+//   idle) stage buffers; CTA r owns tokens [r M / S, (r+1) M / S) and every other CTA adds
+//   its rows for them into r's tile with one asynchronous bulk reduction (counted in bytes on
+//   r's barrier); r then dequantizes and stores its rows. No global workspace.
 //
 // stream-K (many channel blocks): G persistent CTAs (one per SM) take equal contiguous
 //   ranges [g U / G, (g+1) U / G), so every SM streams the same weight bytes. A block split
 //   between CTAs has one owner, the segment holding k-block 0 (its CTA's last segment, so it
 //   finishes last); the other segments (first segments of later CTAs) store their int32
 //   partials in their CTA's workspace slot and raise the CTA's flag; the owner waits for the
-//   flags of the later CTAs sharing its block, adds their partials, dequantizes, stores and
+//   flags of the later CTAs sharing its block (as soon as its own first segment is done, so
+//   the partial sums are fetched while its MMAs still run), adds their partials, dequantizes,
+//   stores and
 //   lowers the flags so the workspace is ready for the next call.
 
 template <int NT, int STAGES, int KPS, bool CLUSTER> struct DecodeCfg {
@@ -514,8 +578,10 @@ template <int NT, int STAGES, int KPS, bool CLUSTER> struct DecodeCfg {
     static constexpr int kYOff = STAGES * kStageBytes;
     static constexpr int kStokOff = kYOff + kYBytes; // fp32 token scales [NT]
     static constexpr int kBarOff = kStokOff + NT * 4;
-    // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot, flag word
-    static constexpr int kSmemBytes = kBarOff + (2 * STAGES + 4) * 8 + 32 + 1024;
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot, flag word, then the
+    // cluster reduction barrier
+    static constexpr int kRedBarOff = kBarOff + (2 * STAGES + 4) * 8 + 32;
+    static constexpr int kSmemBytes = kRedBarOff + 8 + 1024;
     static constexpr int kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
     static_assert(kXBytes % 1024 == 0, "token tile must keep stages 1024-byte aligned");
     static_assert(kTmemCols <= 512, "two accumulators must fit TMEM");
@@ -576,6 +642,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tslot = bar_tempty + 16;
     uint32_t *tslot_ptr = reinterpret_cast<uint32_t *>(smem + Cfg::kBarOff + (2 * STAGES + 4) * 8);
     volatile uint32_t *sh_word = tslot_ptr + 4;
+    const uint32_t bar_red = sbase + Cfg::kRedBarOff;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -603,6 +670,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(bar_tfull + 8 * b, 1);
             mbar_init(bar_tempty + 8 * b, 4);
         }
+        if constexpr (CLUSTER)
+            mbar_init(bar_red, 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -722,6 +791,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         named_bar_sync(1, 128);
         const int mt = M < NT ? M : NT; // tokens held in the accumulator
         const int Mp = (M + 3) & ~3;    // tokens per partial row in the workspace
+        // an owner's contributor sums, per token of its channel (small token tiles only)
+        constexpr int kPre = (!CLUSTER && NT <= 64) ? NT : 0;
+        int32_t pre[kPre > 0 ? kPre : 1];
+        // This CTA owns a block shared with later CTAs iff its range ends inside a block it
+        // starts; the later CTAs' shares of that block are their first segments.
+        int64_t own_t = -1, own_last = g;
+        if constexpr (!CLUSTER) {
+            const int64_t tl = (u_end - 1) / KB;
+            if (u_end > u_begin && tl * KB >= u_begin && u_end < (tl + 1) * KB) {
+                own_t = tl;
+                own_last = sk_owner_of(tl * KB + KB - 1, U, G);
+            }
+        }
+        // Waits for the contributors' flags and, for small token tiles, adds their partial
+        // sums into pre[]. Done as soon as this CTA's first segment is finished (the
+        // contributors' first segments finish at about the same time), so that the loads
+        // overlap the MMAs of this CTA's remaining segments.
+        auto fetch_contributions = [&]() -> bool {
+            if (etid == 0) {
+                bool all = true;
+                for (int64_t c = g + 1; c <= own_last && all; ++c) {
+                    if (ld_acquire_gpu(ws_flag + c) == 0u) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_gpu(ws_flag + c) == 0u) {
+                            if (globaltimer_ns() - t0 > limit_ns) {
+                                flag_timeout();
+                                all = false;
+                                break;
+                            }
+                        }
+                    }
+                }
+                *sh_word = all ? 1u : 0u;
+            }
+            named_bar_sync(1, 128);
+            const bool all_ok = *sh_word != 0u;
+            if constexpr (kPre > 0) {
+#pragma unroll
+                for (int j = 0; j < kPre; ++j)
+                    pre[j] = 0;
+                for (int64_t c = g + 1; c <= own_last; ++c) {
+                    const int4 *src = reinterpret_cast<const int4 *>(ws_part + (c * kBM + r) * Mp);
+#pragma unroll
+                    for (int q = 0; q < kPre / 4; ++q) {
+                        if (4 * q < mt) {
+                            const int4 v = __ldcg(src + q);
+                            pre[4 * q] += v.x;
+                            pre[4 * q + 1] += v.y;
+                            pre[4 * q + 2] += v.z;
+                            pre[4 * q + 3] += v.w;
+                        }
+                    }
+                }
+            }
+            return all_ok;
+        };
+        bool fetched = false;
         uint32_t seg = 0;
         bool ok = true;
         for (int64_t u = u_begin; u < u_end && ok; ++seg) {
@@ -729,38 +855,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             u += sg.kb1 - sg.kb0;
             const uint32_t buf = seg & 1u;
             const uint32_t aph = (seg >> 1) & 1u;
-            const bool whole = CLUSTER || (sg.kb0 == 0 && sg.kb1 == KB);
-            const bool owner = !CLUSTER && sg.kb0 == 0 && !whole;
+            // a segment is a whole block, the owned start of a split block, or a contribution
+            const bool owner = !CLUSTER && sg.t == own_t && sg.kb0 == 0;
             const bool contrib = !CLUSTER && sg.kb0 > 0;
             const int n = static_cast<int>(sg.t * kBM) + r;
             const bool n_ok = n < N;
             const float sc = n_ok ? __ldg(s_ch + n) : 0.0f;
-            // contributors to an owned block: the later CTAs whose ranges reach into it
-            int64_t g_last = g;
-            if (owner) {
-                g_last = sk_owner_of(sg.t * KB + KB - 1, U, G);
-                if (etid == 0) {
-                    bool all = true;
-                    for (int64_t c = g + 1; c <= g_last && all; ++c) {
-                        const volatile unsigned int *f = ws_flag + c;
-                        if (*f == 0u) {
-                            const uint64_t t0 = globaltimer_ns();
-                            while (*f == 0u) {
-                                if (globaltimer_ns() - t0 > limit_ns) {
-                                    flag_timeout();
-                                    all = false;
-                                    break;
-                                }
-                            }
-                        }
-                    }
-                    *sh_word = all ? 1u : 0u;
-                }
-                named_bar_sync(1, 128);
-                if (*sh_word == 0u)
+            if (own_t >= 0 && !fetched && (seg >= 1 || owner)) {
+                fetched = true;
+                if (!fetch_contributions())
                     ok = false;
-                __threadfence();
             }
+            // contributors to an owned block: CTAs g+1 .. g_last
+            const int64_t g_last = owner ? own_last : g;
             if (!mbar_wait(bar_tfull + 8 * buf, aph, limit_ns)) {
                 ok = false;
                 break;
@@ -769,8 +876,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if constexpr (CLUSTER)
                 fence_proxy_async_smem(); // the partial tile reuses TMA-written smem
             const uint32_t tbase = tmem_base + buf * NT + (static_cast<uint32_t>(quarter * 32) << 16);
-#pragma unroll 1
-            for (int c0 = 0; c0 < mt; c0 += 16) {
+            // 16 tokens of this thread's channel
+            auto chunk = [&](const int c0) {
                 uint32_t a[16];
                 tmem_ld_32x32b_x16(tbase + c0, a);
                 tmem_ld_wait();
@@ -781,7 +888,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int j = 0; j < 16; ++j)
                         if (c0 + j < mt)
                             P[(c0 + j) * kBM + r] = static_cast<int32_t>(a[j]);
-                    continue;
+                    return;
                 }
                 if (contrib) {
                     // this CTA's slot: [128 channels][Mp tokens] int32, 16-byte vectors
@@ -790,23 +897,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int q = 0; q < 4; ++q)
                         if (c0 + 4 * q < mt)
                             __stcg(dst + q, make_int4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]));
-                    continue;
+                    return;
                 }
                 if (owner) {
+                    if constexpr (kPre > 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            a[j] += static_cast<uint32_t>(pre[c0 + j]);
+                    } else {
 #pragma unroll 2
-                    for (int64_t c = g + 1; c <= g_last; ++c) {
-                        const int4 *src =
-                            reinterpret_cast<const int4 *>(ws_part + (c * kBM + r) * Mp + c0);
-                        int4 v[4];
+                        for (int64_t c = g + 1; c <= g_last; ++c) {
+                            const int4 *src =
+                                reinterpret_cast<const int4 *>(ws_part + (c * kBM + r) * Mp + c0);
+                            int4 v[4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            v[q] = (c0 + 4 * q < mt) ? __ldcg(src + q) : make_int4(0, 0, 0, 0);
+                            for (int q = 0; q < 4; ++q)
+                                v[q] = (c0 + 4 * q < mt) ? __ldcg(src + q) : make_int4(0, 0, 0, 0);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            a[4 * q] += static_cast<uint32_t>(v[q].x);
-                            a[4 * q + 1] += static_cast<uint32_t>(v[q].y);
-                            a[4 * q + 2] += static_cast<uint32_t>(v[q].z);
-                            a[4 * q + 3] += static_cast<uint32_t>(v[q].w);
+                            for (int q = 0; q < 4; ++q) {
+                                a[4 * q] += static_cast<uint32_t>(v[q].x);
+                                a[4 * q + 1] += static_cast<uint32_t>(v[q].y);
+                                a[4 * q + 2] += static_cast<uint32_t>(v[q].z);
+                                a[4 * q + 3] += static_cast<uint32_t>(v[q].w);
+                            }
                         }
                     }
                 }
@@ -822,6 +935,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             acc_out[static_cast<int64_t>(m) * N + n] = v;
                     }
                 }
+            };
+            if constexpr (kPre > 0) {
+#pragma unroll
+                for (int c0 = 0; c0 < NT; c0 += 16)
+                    if (c0 < mt)
+                        chunk(c0);
+            } else {
+#pragma unroll 1
+                for (int c0 = 0; c0 < mt; c0 += 16)
+                    chunk(c0);
             }
             tc_fence_before();
             __syncwarp();
@@ -829,11 +952,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 mbar_arrive(bar_tempty + 8 * buf);
             if constexpr (!CLUSTER) {
                 if (contrib) {
-                    // publish the partial: every thread's stores, then one flag write
-                    __threadfence();
+                    // publish the partial: every thread's stores, a CTA barrier, then one
+                    // release of the flag
                     named_bar_sync(1, 128);
-                    if (etid == 0)
-                        atomicExch(ws_flag + g, 1u);
+                    if (etid == 0) {
+                        fence_acq_rel_gpu();
+                        st_relaxed_gpu(ws_flag + g, 1u);
+                    }
                 } else {
                     // whole or owned block: copy the staged tile out, 16 bytes per thread
                     named_bar_sync(1, 128);
@@ -846,67 +971,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 *reinterpret_cast<const uint4 *>(ysm + m * kBM + cv * 8);
                     }
                     named_bar_sync(1, 128);
-                    if (owner && etid == 0)
+                    if (owner && etid == 0) // ready for the next call
                         for (int64_t c = g + 1; c <= g_last; ++c)
-                            atomicExch(ws_flag + c, 0u);
+                            st_relaxed_gpu(ws_flag + c, 0u);
                 }
             }
         }
     }
     __syncwarp();
     if constexpr (CLUSTER) {
-        // every thread of the cluster: partial tiles are complete in shared memory
-        cluster_sync();
-        if (warp >= 2) {
+        // Split-K sum in distributed shared memory. CTA q of the cluster owns the tokens
+        // [q mt / S, (q+1) mt / S) of the block; every other CTA adds its partial rows for
+        // those tokens into q's tile with one bulk reduction, counted in bytes on q's
+        // barrier; q then dequantizes its rows.
+        const uint32_t S = gridDim.x;
+        const uint32_t rank = cluster_ctarank();
+        const uint32_t mt = static_cast<uint32_t>(M < NT ? M : NT);
+        const uint32_t m0 = (rank * mt) / S, m1 = ((rank + 1) * mt) / S;
+        constexpr uint32_t kRowBytes = kBM * 4;
+        if (threadIdx.x == 64)
+            mbar_expect_tx(bar_red, (m1 - m0) * kRowBytes * (S - 1));
+        fence_proxy_async_smem(); // this thread's partial-tile writes, before the bulk reads
+        cluster_sync();           // every tile complete, every reduction barrier armed
+        if (threadIdx.x == 64) {
+            for (uint32_t q = 0; q < S; ++q) {
+                const uint32_t a0 = (q * mt) / S, a1 = ((q + 1) * mt) / S;
+                if (q != rank && a1 > a0)
+                    bulk_reduce_add_s32_peer(map_peer_smem(sbase + a0 * kRowBytes, q),
+                                             sbase + a0 * kRowBytes, (a1 - a0) * kRowBytes,
+                                             map_peer_smem(bar_red, q));
+            }
+        }
+        if (warp >= 2 && mbar_wait(bar_red, 0, limit_ns)) {
             const int etid = threadIdx.x - 64;
-            const uint32_t S = static_cast<uint32_t>(gridDim.x);
-            const uint32_t rank = cluster_ctarank();
-            const int r0 = static_cast<int>((rank * kBM) / S);
-            const int r1 = static_cast<int>(((rank + 1) * kBM) / S);
-            const int w = r1 - r0;
             const int64_t t = blockIdx.y;
-            const int mt = M < NT ? M : NT;
-            const uint32_t P = sbase; // partial tiles sit at the same offset in every CTA
-            // the peers' copies of this CTA's partial-tile base
-            uint32_t peer[kMaxClusterSize];
-#pragma unroll
-            for (int p = 0; p < kMaxClusterSize; ++p)
-                peer[p] = map_peer_smem(P, p < static_cast<int>(S) ? p : 0);
-            const int total = mt * w;
-            // 4 elements per thread per pass, every DSMEM load issued before any sum
-            for (int base = etid; base < total; base += 4 * 128) {
-                int32_t part[4][kMaxClusterSize];
-                int mm[4], rr[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int idx = base + e * 128;
-                    mm[e] = idx / w;
-                    rr[e] = r0 + (idx - mm[e] * w);
-                    const uint32_t off = static_cast<uint32_t>((mm[e] * kBM + rr[e]) * 4);
-#pragma unroll
-                    for (int p = 0; p < kMaxClusterSize; ++p)
-                        part[e][p] = (idx < total && p < static_cast<int>(S))
-                                         ? ld_dsmem_s32(peer[p] + off)
-                                         : 0;
-                }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int n = static_cast<int>(t * kBM) + rr[e];
-                    if (base + e * 128 < total && n < N) {
-                        int32_t sum = 0;
-#pragma unroll
-                        for (int p = 0; p < kMaxClusterSize; ++p)
-                            sum += part[e][p];
-                        const int64_t o = static_cast<int64_t>(mm[e]) * N + n;
-                        y[o] = static_cast<uint16_t>(
-                            bf16_bits(dequant_f32(sum, sh_stok[mm[e]], __ldg(s_ch + n))));
-                        if (acc_out)
-                            acc_out[o] = sum;
-                    }
+            const int32_t *P = reinterpret_cast<const int32_t *>(smem);
+            // 4 channels per thread per row: 16-byte tile reads, 8-byte output stores
+            const int nv = static_cast<int>(m1 - m0) * (kBM / 4);
+            for (int v = etid; v < nv; v += 128) {
+                const int m = static_cast<int>(m0) + v / (kBM / 4);
+                const int c = (v % (kBM / 4)) * 4;
+                const int n = static_cast<int>(t * kBM) + c;
+                if (n < N) { // N % 8 == 0: the 4 channels are all valid or all past N
+                    const int4 s4 = *reinterpret_cast<const int4 *>(P + m * kBM + c);
+                    const float4 c4 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
+                    const float st = sh_stok[m];
+                    uint2 o;
+                    o.x = bf16_bits(dequant_f32(s4.x, st, c4.x)) |
+                          (bf16_bits(dequant_f32(s4.y, st, c4.y)) << 16);
+                    o.y = bf16_bits(dequant_f32(s4.z, st, c4.z)) |
+                          (bf16_bits(dequant_f32(s4.w, st, c4.w)) << 16);
+                    const int64_t off = static_cast<int64_t>(m) * N + n;
+                    *reinterpret_cast<uint2 *>(y + off) = o;
+                    if (acc_out)
+                        *reinterpret_cast<int4 *>(acc_out + off) = s4;
                 }
             }
         }
-        // nobody leaves while a peer may still read its shared memory
+        // nobody leaves, or reuses its tile, while a peer's reduction may still read it
         cluster_sync();
     }
     if (warp == 1)

@@ -26,8 +26,9 @@ __global__ void __launch_bounds__(128, 1) mma_i8_probe_kernel(long long iters,
         mbar_init(bar, 1);
         fence_mbar_init();
     }
+    constexpr uint32_t kCols = N < 32 ? 32 : N; // allocation: a power of two >= 32
     if (threadIdx.x < 32) {
-        tmem_alloc(smem_u32(tslot_ptr), N);
+        tmem_alloc(smem_u32(tslot_ptr), kCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(128, 1) mma_i8_probe_kernel(long long iters,
     __syncthreads();
     if (threadIdx.x < 32) {
         tc_fence_after();
-        tmem_dealloc(tmem, N);
+        tmem_dealloc(tmem, kCols);
     }
 }
 

@@ -30,6 +30,27 @@ __device__ __forceinline__ void flag_timeout()
     atomicOr(&g_status_word, kStatusTimeout);
 }
 
+// ------------------------------------------------------------------------- flags in global memory
+
+// Release pattern for a flag published by one thread on behalf of its CTA: every thread's
+// stores, a CTA barrier, then this fence and the relaxed flag store on one thread.
+__device__ __forceinline__ void fence_acq_rel_gpu()
+{
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned int *p, unsigned int v)
+{
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p)
+{
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------------- dependent launch
 
 // Programmatic dependent launch: lets the next kernel in the stream launch (and run its
@@ -349,13 +370,18 @@ __device__ __forceinline__ uint32_t map_peer_smem(uint32_t saddr, uint32_t rank)
     return r;
 }
 
-// Kept in program order with the cluster barriers (volatile) but without a memory clobber,
-// so several of these loads can be in flight at once.
-__device__ __forceinline__ int32_t ld_dsmem_s32(uint32_t addr)
+// Asynchronous bulk reduction of `bytes` (multiple of 16, both addresses 16-byte aligned) of
+// int32 from this CTA's shared memory into a peer CTA's shared memory: dst[i] += src[i].
+// Completion is counted in bytes on the peer's mbarrier (`bar_cluster`, a shared::cluster
+// address in the destination CTA); the source must stay unchanged until that barrier's phase
+// has completed.
+__device__ __forceinline__ void bulk_reduce_add_s32_peer(uint32_t dst_cluster, uint32_t src,
+                                                         uint32_t bytes, uint32_t bar_cluster)
 {
-    int32_t v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
+    asm volatile("cp.reduce.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes"
+                 ".add.s32 [%0], [%1], %2, [%3];"
+                 ::"r"(dst_cluster), "r"(src), "r"(bytes), "r"(bar_cluster)
+                 : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem()

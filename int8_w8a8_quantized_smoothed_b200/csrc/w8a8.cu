@@ -508,6 +508,22 @@ int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *
 
 } // namespace
 
+namespace {
+
+template <int N>
+int launch_probe(long long iters, int grid, int dev, cudaStream_t st)
+{
+    const int smem = 128 * 128 + N * 128 + 64 + 1024;
+    const void *fn = reinterpret_cast<const void *>(&mma_i8_probe_kernel<N>);
+    int rc = ensure_smem(fn, dev, smem);
+    if (rc)
+        return rc;
+    return launch_kernel(mma_i8_probe_kernel<N>, dim3(grid), dim3(128), smem, st, iters,
+                         kWaitLimitNs);
+}
+
+} // namespace
+
 extern "C" {
 
 int w8a8_version(void)
@@ -682,25 +698,22 @@ int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, co
 
 int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream)
 {
-    if (iters < 1 || (n != 128 && n != 256) || ctas < 0)
+    if (iters < 1 || ctas < 0)
         return W8A8_ERR_INVALID_ARG;
     int dev, sms;
     int rc = current_device(&dev, &sms);
     if (rc)
         return rc;
     const int grid = ctas == 0 ? sms : ctas;
-    const int smem = 128 * 128 + n * 128 + 64 + 1024;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (n == 256) {
-        if ((rc = ensure_smem(reinterpret_cast<const void *>(&mma_i8_probe_kernel<256>), dev, smem)))
-            return rc;
-        return launch_kernel(mma_i8_probe_kernel<256>, dim3(grid), dim3(128), smem, st, iters,
-                             kWaitLimitNs);
+    switch (n) {
+    case 16: return launch_probe<16>(iters, grid, dev, st);
+    case 32: return launch_probe<32>(iters, grid, dev, st);
+    case 64: return launch_probe<64>(iters, grid, dev, st);
+    case 128: return launch_probe<128>(iters, grid, dev, st);
+    case 256: return launch_probe<256>(iters, grid, dev, st);
+    default: return W8A8_ERR_INVALID_ARG;
     }
-    if ((rc = ensure_smem(reinterpret_cast<const void *>(&mma_i8_probe_kernel<128>), dev, smem)))
-        return rc;
-    return launch_kernel(mma_i8_probe_kernel<128>, dim3(grid), dim3(128), smem, st, iters,
-                         kWaitLimitNs);
 }
 
 int w8a8_set_overlap(int mode)
