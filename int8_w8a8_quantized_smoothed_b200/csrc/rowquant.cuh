@@ -1,7 +1,9 @@
 // Per-token quantization kernels (HBM-bound): quantize_rows, smoothed RMSNorm + quant and
-// SiLU(gate)*up + quant. One CTA per row; each thread keeps NCH vectors of 8 values in
-// registers, so the row is read from HBM once and written once. Loads and stores are
-// 16-byte (bf16 x 8) / 8-byte (int8 x 8) and coalesced: vector v = c*blockDim + tid.
+// SiLU(gate)*up + quant. A CTA handles one row at a time and keeps it in registers (NCH
+// vectors of 8 values per thread), so the row is read from HBM once and written once. The
+// grid is persistent (at most as many CTAs as are resident on the device, looping over
+// rows). Loads and stores are 16-byte (bf16 x 8) / 8-byte (int8 x 8) and coalesced: vector
+// v = c*blockDim + tid.
 #pragma once
 
 #include "ptx.cuh"
@@ -24,8 +26,12 @@ __device__ __forceinline__ double warp_sum(double v)
     return v;
 }
 
-// Block-wide max of non-negative floats; `sh` holds >= 33 floats. Exact (max is
-// order-free). All threads receive the result.
+// Block-wide reductions with one barrier: each warp reduces its values and publishes the
+// result in sh[warp]; after the barrier every warp reduces all the warps' results itself
+// (in the same fixed order, so every thread gets the same value). A buffer may be written
+// again only after a later barrier that every thread reaches after reading it.
+
+// Max of non-negative floats (exact: max is order-free); sh holds >= 32 floats.
 __device__ __forceinline__ float block_max(float v, float *sh)
 {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -34,16 +40,11 @@ __device__ __forceinline__ float block_max(float v, float *sh)
     if (l == 0)
         sh[w] = v;
     __syncthreads();
-    if (w == 0) {
-        float t = (l < nw) ? sh[l] : 0.0f;
-        t = warp_max(t);
-        if (l == 0)
-            sh[32] = t;
-    }
-    __syncthreads();
-    return sh[32];
+    return warp_max(l < nw ? sh[l] : 0.0f);
 }
 
+// Sum in binary64 (any order: the caller accepts either neighbour where it matters); sh
+// holds >= 32 doubles.
 __device__ __forceinline__ double block_sum(double v, double *sh)
 {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -52,14 +53,7 @@ __device__ __forceinline__ double block_sum(double v, double *sh)
     if (l == 0)
         sh[w] = v;
     __syncthreads();
-    if (w == 0) {
-        double t = (l < nw) ? sh[l] : 0.0;
-        t = warp_sum(t);
-        if (l == 0)
-            sh[32] = t;
-    }
-    __syncthreads();
-    return sh[32];
+    return warp_sum(l < nw ? sh[l] : 0.0);
 }
 
 // Adding 1.5 * 2^23 to a binary32 v with |v| < 2^22 leaves v rounded to an integer
@@ -125,22 +119,50 @@ __device__ __forceinline__ float2 splat2(float v)
     return make_float2(v, v);
 }
 
-// Quantizes the row held in registers (v[c][0..7] for vector c*blockDim + tid) given its
-// absmax, writes q and the scale.
+// Codes of two values given the row's scale s and r = RN(1 / s) (s >= 2^-100), as the bits
+// whose low bytes are the int8 codes (see quant_bits). t = RN(y r) is within 2^-15 of
+// RN(y / s) (both within 127 * 2^-23 + 2^-18 of y / s), so when t is more than 2^-14 away
+// from every half-integer, rint(t) = rint(RN(y / s)) and |rint(t)| <= 127 needs no clamp;
+// otherwise (probability about 2^-13 per value) the exact quotient decides.
+__device__ __forceinline__ void quant_bits2(float y0, float y1, float s, float r, uint32_t &b0,
+                                            uint32_t &b1)
+{
+    const float2 t = mul2(make_float2(y0, y1), splat2(r));
+    const float2 m = add2(t, splat2(kRoundMagic));      // rint(t) + 1.5 * 2^23
+    const float2 n = add2(m, splat2(-kRoundMagic));     // rint(t)
+    const float2 d = add2(t, make_float2(-n.x, -n.y));  // t - rint(t), exact
+    constexpr float kNearHalf = 0.5f - 6.103515625e-05f; // 0.5 - 2^-14
+    b0 = fabsf(d.x) < kNearHalf ? __float_as_uint(m.x) : quant_bits(y0, s);
+    b1 = fabsf(d.y) < kNearHalf ? __float_as_uint(m.y) : quant_bits(y1, s);
+}
+
+// Quantizes the part of a row held in registers (v[c][0..7] for vector v0 + c*blockDim + tid,
+// vectors below v1) given the row's absmax, writes its codes; the CTA's thread 0 writes the
+// scale when s_out is given.
 template <int NCH>
-__device__ __forceinline__ void quantize_and_store(const float (&v)[NCH][8], float amax,
-                                                   int nvec, int8_t *__restrict__ qrow,
+__device__ __forceinline__ void quantize_and_store(const float (&v)[NCH][8], float amax, int v0,
+                                                   int v1, int8_t *__restrict__ qrow,
                                                    float *__restrict__ s_out)
 {
     const float s = __fdiv_rn(amax, 127.0f);
-    if (threadIdx.x == 0)
+    if (s_out && threadIdx.x == 0)
         *s_out = s;
+    // the product path needs a finite reciprocal; tiny scales take the exact quotient
+    const bool by_product = s >= 7.888609052210118e-31f; // 2^-100
+    const float r = by_product ? __frcp_rn(s) : 0.0f;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
-        const int vi = c * blockDim.x + threadIdx.x;
-        if (vi < nvec) {
+        const int vi = v0 + c * blockDim.x + threadIdx.x;
+        if (vi < v1) {
             uint2 out = make_uint2(0u, 0u);
-            if (amax > 0.0f) {
+            if (by_product) {
+                uint32_t b[8];
+#pragma unroll
+                for (int i = 0; i < 8; i += 2)
+                    quant_bits2(v[c][i], v[c][i + 1], s, r, b[i], b[i + 1]);
+                out.x = pack_low_bytes(b[0], b[1], b[2], b[3]);
+                out.y = pack_low_bytes(b[4], b[5], b[6], b[7]);
+            } else if (amax > 0.0f) {
                 out.x = pack_low_bytes(quant_bits(v[c][0], s), quant_bits(v[c][1], s),
                                        quant_bits(v[c][2], s), quant_bits(v[c][3], s));
                 out.y = pack_low_bytes(quant_bits(v[c][4], s), quant_bits(v[c][5], s),
@@ -172,117 +194,167 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
     return r;
 }
 
-// ----------------------------------------------------------------- quantize_rows
-
+// Raw 16-byte vectors of one row for this thread (zero past the row's end).
 template <int NCH>
-__global__ void __launch_bounds__(1024) quantize_rows_kernel(const uint16_t *__restrict__ x,
-                                                             const float *__restrict__ sinv,
-                                                             int K, int8_t *__restrict__ q,
-                                                             float *__restrict__ s_tok)
+__device__ __forceinline__ void load_row(const uint4 *__restrict__ xr, int nvec, uint4 (&raw)[NCH])
 {
-    __shared__ float sh[33];
-    if (threadIdx.x == 0)
-        pdl_launch_dependents();
-    pdl_wait(); // every input may come from the previous kernel
-    const int64_t row = blockIdx.x;
-    const int nvec = K >> 3;
-    const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * K);
-    float v[NCH][8];
-    float amax = 0.0f;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
         const int vi = c * blockDim.x + threadIdx.x;
-        if (vi < nvec) {
-            unpack8(ldg_nc_v4(xr + vi), v[c]);
-            if (sinv) {
-                const float4 a = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * vi);
-                const float4 b = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * vi + 1);
-                const float2 p0 = mul2(make_float2(v[c][0], v[c][1]), make_float2(a.x, a.y));
-                const float2 p1 = mul2(make_float2(v[c][2], v[c][3]), make_float2(a.z, a.w));
-                const float2 p2 = mul2(make_float2(v[c][4], v[c][5]), make_float2(b.x, b.y));
-                const float2 p3 = mul2(make_float2(v[c][6], v[c][7]), make_float2(b.z, b.w));
-                v[c][0] = p0.x; v[c][1] = p0.y; v[c][2] = p1.x; v[c][3] = p1.y;
-                v[c][4] = p2.x; v[c][5] = p2.y; v[c][6] = p3.x; v[c][7] = p3.y;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                amax = fmaxf(amax, fabsf(v[c][i]));
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[c][i] = 0.0f;
-        }
+        raw[c] = vi < nvec ? ldg_nc_v4(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
     }
-    amax = block_max(amax, sh);
-    quantize_and_store<NCH>(v, amax, nvec, q + row * K, s_tok + row);
+}
+
+// ----------------------------------------------------------------- quantize_rows
+//
+// Rows of up to 4096 values run with at most 256 threads (NCH <= 2); those kernels are
+// compiled for several resident CTAs per SM (at most 40 registers for quantize_rows and
+// SiLU, 64 for RMSNorm, which keeps gamma' in registers), since with so little work per
+// thread the arithmetic and the reductions' latency, not HBM, set their pace.
+
+template <int NCH>
+__global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quantize_rows_kernel(const uint16_t *__restrict__ x,
+                                                             const float *__restrict__ sinv,
+                                                             int K, int M,
+                                                             int8_t *__restrict__ q,
+                                                             float *__restrict__ s_tok)
+{
+    __shared__ float sh[2][32]; // by row parity: one barrier per row
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // every input may come from the previous kernel
+    const int nvec = K >> 3;
+    int64_t row = blockIdx.x;
+    for (uint32_t it = 0; row < M; row += gridDim.x, ++it) {
+        uint4 raw[NCH];
+        load_row<NCH>(reinterpret_cast<const uint4 *>(x + row * K), nvec, raw);
+        float v[NCH][8];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+            unpack8(raw[c], v[c]);
+        float amax = 0.0f;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int vi = c * blockDim.x + threadIdx.x;
+            if (vi < nvec) {
+                if (sinv) {
+                    const float4 a = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * vi);
+                    const float4 b = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * vi + 1);
+                    const float2 p0 = mul2(make_float2(v[c][0], v[c][1]), make_float2(a.x, a.y));
+                    const float2 p1 = mul2(make_float2(v[c][2], v[c][3]), make_float2(a.z, a.w));
+                    const float2 p2 = mul2(make_float2(v[c][4], v[c][5]), make_float2(b.x, b.y));
+                    const float2 p3 = mul2(make_float2(v[c][6], v[c][7]), make_float2(b.z, b.w));
+                    v[c][0] = p0.x; v[c][1] = p0.y; v[c][2] = p1.x; v[c][3] = p1.y;
+                    v[c][4] = p2.x; v[c][5] = p2.y; v[c][6] = p3.x; v[c][7] = p3.y;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    amax = fmaxf(amax, fabsf(v[c][i]));
+            }
+        }
+        amax = block_max(amax, sh[it & 1u]);
+        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * K, s_tok + row);
+    }
 }
 
 // ----------------------------------------------------------------- smoothed RMSNorm + quant
 
 template <int NCH, bool RES>
-__global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(
+__global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsnorm_quant_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ res, uint16_t *__restrict__ h_out,
-    const float *__restrict__ gamma, float eps, int K, int8_t *__restrict__ q,
+    const float *__restrict__ gamma, float eps, int K, int M, int8_t *__restrict__ q,
     float *__restrict__ s_tok)
 {
-    __shared__ double shd[33];
-    __shared__ float shf[33];
+    // the sum's and the max's buffers alternate, so each is rewritten only after the other's
+    // barrier: two barriers per row
+    __shared__ double shd[32];
+    __shared__ float shf[32];
     if (threadIdx.x == 0)
         pdl_launch_dependents();
     pdl_wait(); // every input may come from the previous kernel
-    const int64_t row = blockIdx.x;
     const int nvec = K >> 3;
-    const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * K);
-    float v[NCH][8];
-    double ss = 0.0;
+    // gamma' of this thread's vectors, the same for every row: for short rows read once,
+    // together with the first row (its latency then overlaps the row's), and kept in
+    // registers; for long rows re-read per row
+    constexpr bool kKeepGamma = NCH <= 2;
+    float gk[kKeepGamma ? NCH : 1][8];
+    if constexpr (kKeepGamma) {
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        const int vi = c * blockDim.x + threadIdx.x;
-        if (vi < nvec) {
-            unpack8(ldg_nc_v4(xr + vi), v[c]);
-            if (RES) {
+        for (int c = 0; c < NCH; ++c) {
+            const int vi = c * blockDim.x + threadIdx.x;
+            const float4 a = vi < nvec ? __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 b = vi < nvec ? __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi + 1)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            gk[c][0] = a.x; gk[c][1] = a.y; gk[c][2] = a.z; gk[c][3] = a.w;
+            gk[c][4] = b.x; gk[c][5] = b.y; gk[c][6] = b.z; gk[c][7] = b.w;
+        }
+    }
+    int64_t row = blockIdx.x;
+    for (; row < M; row += gridDim.x) {
+        uint4 rx[NCH], rr[RES ? NCH : 1];
+        load_row<NCH>(reinterpret_cast<const uint4 *>(x + row * K), nvec, rx);
+        if constexpr (RES)
+            load_row<NCH>(reinterpret_cast<const uint4 *>(res + row * K), nvec, rr);
+        float v[NCH][8];
+        double ss = 0.0;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            unpack8(rx[c], v[c]);
+            if constexpr (RES) {
+                const int vi = c * blockDim.x + threadIdx.x;
                 float r[8];
-                unpack8(ldg_nc_v4(reinterpret_cast<const uint4 *>(res + row * K) + vi), r);
+                unpack8(rr[c], r);
                 uint4 hb;
                 hb.x = pack_bf16x2(__fadd_rn(v[c][0], r[0]), __fadd_rn(v[c][1], r[1]));
                 hb.y = pack_bf16x2(__fadd_rn(v[c][2], r[2]), __fadd_rn(v[c][3], r[3]));
                 hb.z = pack_bf16x2(__fadd_rn(v[c][4], r[4]), __fadd_rn(v[c][5], r[5]));
                 hb.w = pack_bf16x2(__fadd_rn(v[c][6], r[6]), __fadd_rn(v[c][7], r[7]));
-                reinterpret_cast<uint4 *>(h_out + row * K)[vi] = hb;
+                if (vi < nvec)
+                    reinterpret_cast<uint4 *>(h_out + row * K)[vi] = hb;
                 unpack8(hb, v[c]);
             }
+        }
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
 #pragma unroll
             for (int i = 0; i < 8; ++i) // each square of a bf16 value is exact in binary32
                 ss = __dadd_rn(ss, static_cast<double>(__fmul_rn(v[c][i], v[c][i])));
-        } else {
+        const double sum = block_sum(ss, shd);
+        // sum / K: a power-of-two K divides exactly by scaling
+        const double mean = (K & (K - 1)) == 0 ? __dmul_rn(sum, 1.0 / static_cast<double>(K))
+                                               : __ddiv_rn(sum, static_cast<double>(K));
+        const float ms = __double2float_rn(mean);
+        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+        float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[c][i] = 0.0f;
-        }
-    }
-    const double sum = block_sum(ss, shd);
-    const float ms = __double2float_rn(__ddiv_rn(sum, static_cast<double>(K)));
-    const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
-    float amax = 0.0f;
+        for (int c = 0; c < NCH; ++c) {
+            const int vi = c * blockDim.x + threadIdx.x;
+            if (vi < nvec) {
+                float g[8];
+                if constexpr (kKeepGamma) {
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        const int vi = c * blockDim.x + threadIdx.x;
-        if (vi < nvec) {
-            const float4 a = __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi);
-            const float4 b = __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi + 1);
-            const float g[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    for (int i = 0; i < 8; ++i)
+                        g[i] = gk[c][i];
+                } else {
+                    const float4 a = __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi);
+                    const float4 b = __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi + 1);
+                    g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w;
+                    g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
+                }
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) { // (h * rstd) * gamma', two lanes at a time
-                const float2 p = mul2(mul2(make_float2(v[c][i], v[c][i + 1]), splat2(rstd)),
-                                      make_float2(g[i], g[i + 1]));
-                v[c][i] = p.x;
-                v[c][i + 1] = p.y;
-                amax = fmaxf(amax, fmaxf(fabsf(p.x), fabsf(p.y)));
+                for (int i = 0; i < 8; i += 2) { // (h * rstd) * gamma', two lanes at a time
+                    const float2 p = mul2(mul2(make_float2(v[c][i], v[c][i + 1]), splat2(rstd)),
+                                          make_float2(g[i], g[i + 1]));
+                    v[c][i] = p.x;
+                    v[c][i + 1] = p.y;
+                    amax = fmaxf(amax, fmaxf(fabsf(p.x), fabsf(p.y)));
+                }
             }
         }
+        amax = block_max(amax, shf);
+        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * K, s_tok + row);
     }
-    amax = block_max(amax, shf);
-    quantize_and_store<NCH>(v, amax, nvec, q + row * K, s_tok + row);
 }
 
 // ----------------------------------------------------------------- SiLU(gate)*up + quant
@@ -311,6 +383,12 @@ __device__ __forceinline__ float2 w8a8_exp2(float2 x)
     p = fma2(p, r, splat2(1.0f));
     const int ka = __float_as_int(km.x) - kRoundMagicBits;
     const int kb = __float_as_int(km.y) - kRoundMagicBits;
+    if (fabsf(x.x) <= 80.0f && fabsf(x.y) <= 80.0f) {
+        // |k| <= 115 and p in [0.7, 1.5): every partial product of the two power-of-two
+        // scalings is a normal number, so both are exact and equal adding k to p's exponent
+        return make_float2(__uint_as_float(__float_as_uint(p.x) + (static_cast<uint32_t>(ka) << 23)),
+                           __uint_as_float(__float_as_uint(p.y) + (static_cast<uint32_t>(kb) << 23)));
+    }
     const int ka1 = ka / 2, kb1 = kb / 2; // truncation toward zero
     const float2 s1 = make_float2(__int_as_float((ka1 + 127) << 23), __int_as_float((kb1 + 127) << 23));
     const float2 s2 = make_float2(__int_as_float((ka - ka1 + 127) << 23),
@@ -331,42 +409,48 @@ __device__ __forceinline__ float2 silu_mul2(float2 g, float2 u)
 }
 
 template <int NCH>
-__global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const uint16_t *__restrict__ gu,
-                                                              int I, int8_t *__restrict__ q,
+__global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) silu_mul_quant_kernel(const uint16_t *__restrict__ gu,
+                                                              int I, int M,
+                                                              int8_t *__restrict__ q,
                                                               float *__restrict__ s_tok)
 {
-    __shared__ float sh[33];
+    __shared__ float sh[2][32]; // by row parity: one barrier per row
     if (threadIdx.x == 0)
         pdl_launch_dependents();
     pdl_wait(); // every input may come from the previous kernel
-    const int64_t row = blockIdx.x;
     const int nvec = I >> 3;
-    const uint4 *gr = reinterpret_cast<const uint4 *>(gu + row * 2 * static_cast<int64_t>(I));
-    const uint4 *ur = gr + nvec;
-    float v[NCH][8];
-    float amax = 0.0f;
+    int64_t row = blockIdx.x;
+    for (uint32_t it = 0; row < M; row += gridDim.x, ++it) {
+        uint4 cg[NCH], cu[NCH];
+        const uint4 *gr = reinterpret_cast<const uint4 *>(gu + row * 2 * static_cast<int64_t>(I));
+        load_row<NCH>(gr, nvec, cg);
+        load_row<NCH>(gr + nvec, nvec, cu);
+        float v[NCH][8];
+        float amax = 0.0f;
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        const int vi = c * blockDim.x + threadIdx.x;
-        if (vi < nvec) {
-            float g[8], u[8];
-            unpack8(ldg_nc_v4(gr + vi), g);
-            unpack8(ldg_nc_v4(ur + vi), u);
+        for (int c = 0; c < NCH; ++c) {
+            const int vi = c * blockDim.x + threadIdx.x;
+            if (vi < nvec) {
+                float g[8], u[8];
+                unpack8(cg[c], g);
+                unpack8(cu[c], u);
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                const float2 a2 = silu_mul2(make_float2(g[i], g[i + 1]), make_float2(u[i], u[i + 1]));
-                v[c][i] = a2.x;
-                v[c][i + 1] = a2.y;
-                amax = fmaxf(amax, fmaxf(fabsf(a2.x), fabsf(a2.y)));
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 a2 = silu_mul2(make_float2(g[i], g[i + 1]),
+                                                make_float2(u[i], u[i + 1]));
+                    v[c][i] = a2.x;
+                    v[c][i + 1] = a2.y;
+                    amax = fmaxf(amax, fmaxf(fabsf(a2.x), fabsf(a2.y)));
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    v[c][i] = 0.0f;
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[c][i] = 0.0f;
         }
+        amax = block_max(amax, sh[it & 1u]);
+        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * I, s_tok + row);
     }
-    amax = block_max(amax, sh);
-    quantize_and_store<NCH>(v, amax, nvec, q + row * I, s_tok + row);
 }
 
 } // namespace w8a8

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <set>
 #include <tuple>
@@ -201,43 +202,75 @@ int check_row_shape(int64_t M, int64_t K)
     return W8A8_OK;
 }
 
+// Persistent row grid: at most as many CTAs as are resident on the device at once (cached
+// per kernel, block size and device), never more than there are rows.
+unsigned row_grid(const void *kernel, int threads, int64_t M, int dev, int sms)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, int, int>, int> cache;
+    int occ = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto key = std::make_tuple(kernel, threads, dev);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            occ = it->second;
+        } else {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                occ = 1;
+            }
+            occ = occ < 1 ? 1 : occ;
+            cache[key] = occ;
+        }
+    }
+    const int64_t g = static_cast<int64_t>(sms) * occ;
+    return static_cast<unsigned>(M < g ? M : g);
+}
+
 template <int NCH>
 int launch_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int K, int8_t *q,
-                         float *s, int threads, int dev, cudaStream_t st)
+                         float *s, int threads, int dev, int sms, cudaStream_t st)
 {
-    if (int rc = ensure_smem(reinterpret_cast<const void *>(&quantize_rows_kernel<NCH>), dev, 0))
+    const void *fn = reinterpret_cast<const void *>(&quantize_rows_kernel<NCH>);
+    if (int rc = ensure_smem(fn, dev, 0))
         return rc;
-    return launch_kernel(quantize_rows_kernel<NCH>, dim3(static_cast<unsigned>(M)), dim3(threads), 0,
-                         st, x, sinv, K, q, s);
+    return launch_kernel(quantize_rows_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
+                         dim3(threads), 0, st, x, sinv, K, static_cast<int>(M), q, s);
+}
+
+template <int NCH, bool RES>
+int launch_rmsnorm_t(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
+                     int64_t M, int K, int8_t *q, float *s, int threads, int dev, int sms,
+                     cudaStream_t st)
+{
+    const void *fn = reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, RES>);
+    if (int rc = ensure_smem(fn, dev, 0))
+        return rc;
+    return launch_kernel(rmsnorm_quant_kernel<NCH, RES>, dim3(row_grid(fn, threads, M, dev, sms)),
+                         dim3(threads), 0, st, x, r, h, g, eps, K, static_cast<int>(M), q, s);
 }
 
 template <int NCH>
 int launch_rmsnorm(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
-                   int64_t M, int K, int8_t *q, float *s, int threads, int dev, cudaStream_t st)
+                   int64_t M, int K, int8_t *q, float *s, int threads, int dev, int sms,
+                   cudaStream_t st)
 {
-    if (r) {
-        if (int rc = ensure_smem(
-                reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, true>), dev, 0))
-            return rc;
-        return launch_kernel(rmsnorm_quant_kernel<NCH, true>, dim3(static_cast<unsigned>(M)),
-                             dim3(threads), 0, st, x, r, h, g, eps, K, q, s);
-    } else {
-        if (int rc = ensure_smem(
-                reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, false>), dev, 0))
-            return rc;
-        return launch_kernel(rmsnorm_quant_kernel<NCH, false>, dim3(static_cast<unsigned>(M)),
-                             dim3(threads), 0, st, x, r, h, g, eps, K, q, s);
-    }
+    if (r)
+        return launch_rmsnorm_t<NCH, true>(x, r, h, g, eps, M, K, q, s, threads, dev, sms, st);
+    return launch_rmsnorm_t<NCH, false>(x, r, h, g, eps, M, K, q, s, threads, dev, sms, st);
 }
 
 template <int NCH>
 int launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int threads, int dev,
-                cudaStream_t st)
+                int sms, cudaStream_t st)
 {
-    if (int rc = ensure_smem(reinterpret_cast<const void *>(&silu_mul_quant_kernel<NCH>), dev, 0))
+    const void *fn = reinterpret_cast<const void *>(&silu_mul_quant_kernel<NCH>);
+    if (int rc = ensure_smem(fn, dev, 0))
         return rc;
-    return launch_kernel(silu_mul_quant_kernel<NCH>, dim3(static_cast<unsigned>(M)), dim3(threads),
-                         0, st, gu, I, q, s);
+    return launch_kernel(silu_mul_quant_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
+                         dim3(threads), 0, st, gu, I, static_cast<int>(M), q, s);
 }
 
 // ------------------------------------------------------------------ GEMM planning
@@ -573,9 +606,9 @@ int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, i
     const RowLaunch L = row_launch(K);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (L.nch) {
-    case 1: return launch_quantize_rows<1>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, st);
-    case 2: return launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, st);
-    default: return launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, st);
+    case 1: return launch_quantize_rows<1>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    case 2: return launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    default: return launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
     }
 }
 
@@ -601,9 +634,9 @@ int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a
     const RowLaunch L = row_launch(K);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (L.nch) {
-    case 1: return launch_rmsnorm<1>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, st);
-    case 2: return launch_rmsnorm<2>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, st);
-    default: return launch_rmsnorm<4>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, st);
+    case 1: return launch_rmsnorm<1>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    case 2: return launch_rmsnorm<2>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    default: return launch_rmsnorm<4>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
     }
 }
 
@@ -620,12 +653,12 @@ int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *
     int dev, sms;
     if ((rc = current_device(&dev, &sms)))
         return rc;
-    const RowLaunch L = row_launch(I);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const RowLaunch L = row_launch(I);
     switch (L.nch) {
-    case 1: return launch_silu<1>(gate_up, M, (int)I, q, s_tok, L.threads, dev, st);
-    case 2: return launch_silu<2>(gate_up, M, (int)I, q, s_tok, L.threads, dev, st);
-    default: return launch_silu<4>(gate_up, M, (int)I, q, s_tok, L.threads, dev, st);
+    case 1: return launch_silu<1>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
+    case 2: return launch_silu<2>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
+    default: return launch_silu<4>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
     }
 }
 

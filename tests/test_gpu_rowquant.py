@@ -141,3 +141,58 @@ def test_quantize_near_half_integer_quotients():
         q, s = w8.w8a8_quantize_rows(dev_bf16(xb), dev(sinv))
         assert np.array_equal(host(s), s_ref)
         assert np.array_equal(host(q), q_ref)
+
+
+# Row counts above the persistent grid (resident CTAs on the device), so that every CTA
+# loops over several rows and, for blocks of up to 512 threads, prefetches the next row.
+@pytest.mark.parametrize("M,K", [(5000, 256), (1500, 4096), (700, 28672)])
+def test_quantize_rows_persistent_loop(M, K):
+    x = synth.activation(M, K, seed=M + K + 17)
+    sinv = _sinv(K, K + 3)
+    q_ref, s_ref = oracle.quantize_rows(x, sinv)
+    q, s = w8.w8a8_quantize_rows(dev_bf16(x), dev(sinv))
+    assert np.array_equal(host(s), s_ref)
+    assert np.array_equal(host(q), q_ref)
+
+
+@pytest.mark.parametrize("M,K", [(5000, 256), (1500, 4096), (600, 8192), (300, 28672)])
+@pytest.mark.parametrize("with_residual", [False, True])
+def test_smooth_rmsnorm_quant_persistent_loop(M, K, with_residual):
+    x = synth.activation(M, K, seed=2 * M + K)
+    gf = synth.gamma(K, seed=K + 7)
+    res = synth.normal_bf16((M, K), seed=M + 9) if with_residual else None
+    if with_residual:
+        q, s, h = w8.w8a8_smooth_rmsnorm_quant(dev_bf16(x), dev(gf), 1e-5, residual=dev_bf16(res),
+                                               h_out=torch.empty(M, K, dtype=torch.bfloat16,
+                                                                 device="cuda"))
+    else:
+        q, s = w8.w8a8_smooth_rmsnorm_quant(dev_bf16(x), dev(gf), 1e-5)
+    ref, _ = assert_rms_rows_match(host(q), host(s), x, gf, 1e-5, residual=res)
+    if with_residual:
+        assert np.array_equal(host_bf16(h), ref["h"])
+
+
+@pytest.mark.parametrize("M,I", [(5000, 128), (700, 14336), (300, 28672)])
+def test_silu_mul_quant_persistent_loop(M, I):
+    gu = synth.normal_bf16((M, 2 * I), seed=M + I + 5, std=2.5)
+    q_ref, s_ref = oracle.silu_mul_quant(gu)
+    q, s = w8.w8a8_silu_mul_quant(dev_bf16(gu))
+    assert np.array_equal(host(s), s_ref)
+    assert np.array_equal(host(q), q_ref)
+
+
+def test_quantize_tiny_scales_take_exact_quotient():
+    # rows whose absmax is so small that the scale is below 2^-100 (the reciprocal would
+    # leave the binary32 range) are quantized through the exact quotient
+    K = 256
+    rng = np.random.default_rng(5)
+    rows = []
+    for mag in (1e-38, 3e-35, 1e-30, 1e-28, 1.0):
+        rows.append(rng.standard_normal(K) * mag)
+    xf = np.stack(rows).astype(np.float32)
+    xb = torch.from_numpy(xf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    q_ref, s_ref = oracle.quantize_rows(xb)
+    q, s = w8.w8a8_quantize_rows(dev_bf16(xb))
+    assert np.array_equal(host(s), s_ref)
+    assert np.array_equal(host(q), q_ref)
+    assert (s_ref[:3] < 2.0 ** -100).all() and s_ref[3] > 2.0 ** -100
