@@ -48,6 +48,11 @@ WORKLOADS = {
     "set70b": dict(arch=LLAMA70B, Ms=[16, 4096], desc="Llama-3.1-70B-shaped linear set"),
 }
 
+# DRAM bytes (read + write, ncu dram__bytes_read.sum + dram__bytes_write.sum) per GEMM launch,
+# averaged over the GEMM launches of one step of the workload, as captured with the current
+# GEMM kernels; None where no capture exists. Re-capture whenever a GEMM kernel changes.
+NCU_GEMM_TRAFFIC = {"decode8b": 55.16e6, "prefill8b": 239.1e6}
+
 # Measured peaks (driver-written); fallbacks are the pool's earlier measurements.
 FALLBACK_HBM_GBS = 6650.0
 INT8_NOMINAL_TOPS = 4500.0
@@ -494,8 +499,11 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(arch)
-    if args.traffic is not None:
-        result["roofline"]["traffic"] = args.traffic
+    traffic = args.traffic if args.traffic is not None else NCU_GEMM_TRAFFIC.get(args.workload)
+    if traffic is not None:
+        result["roofline"]["traffic"] = traffic
+        result["roofline"]["traffic_per"] = "GEMM launch (ncu DRAM read + write bytes)"
+        result["roofline"]["algorithmic_bytes_per_launch"] = round(g_bytes / (4 * len(layers)))
     del g_step, g_gemm, g_rows, g_e2e
     return result
 
