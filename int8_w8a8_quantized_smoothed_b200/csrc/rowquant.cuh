@@ -119,21 +119,31 @@ __device__ __forceinline__ float2 splat2(float v)
     return make_float2(v, v);
 }
 
-// Codes of two values given the row's scale s and r = RN(1 / s) (s >= 2^-100), as the bits
-// whose low bytes are the int8 codes (see quant_bits). t = RN(y r) is within 2^-15 of
+// Codes of eight values given the row's scale s and r = RN(1 / s) (s >= 2^-100), as the
+// bits whose low bytes are the int8 codes (see quant_bits). t = RN(y r) is within 2^-15 of
 // RN(y / s) (both within 127 * 2^-23 + 2^-18 of y / s), so when t is more than 2^-14 away
-// from every half-integer, rint(t) = rint(RN(y / s)) and |rint(t)| <= 127 needs no clamp;
-// otherwise (probability about 2^-13 per value) the exact quotient decides.
-__device__ __forceinline__ void quant_bits2(float y0, float y1, float s, float r, uint32_t &b0,
-                                            uint32_t &b1)
+// from every half-integer, rint(t) = rint(RN(y / s)) and |rint(t)| <= 127 needs no clamp.
+// When any of the eight is that close (probability about 2^-10 per vector), the exact
+// quotient decides all eight (one branch per vector keeps the common path branch-free).
+__device__ __forceinline__ void quant_bits8(const float (&y)[8], float s, float r, uint32_t (&b)[8])
 {
-    const float2 t = mul2(make_float2(y0, y1), splat2(r));
-    const float2 m = add2(t, splat2(kRoundMagic));      // rint(t) + 1.5 * 2^23
-    const float2 n = add2(m, splat2(-kRoundMagic));     // rint(t)
-    const float2 d = add2(t, make_float2(-n.x, -n.y));  // t - rint(t), exact
     constexpr float kNearHalf = 0.5f - 6.103515625e-05f; // 0.5 - 2^-14
-    b0 = fabsf(d.x) < kNearHalf ? __float_as_uint(m.x) : quant_bits(y0, s);
-    b1 = fabsf(d.y) < kNearHalf ? __float_as_uint(m.y) : quant_bits(y1, s);
+    bool near = false;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float2 t = mul2(make_float2(y[i], y[i + 1]), splat2(r));
+        const float2 m = add2(t, splat2(kRoundMagic));     // rint(t) + 1.5 * 2^23
+        const float2 n = add2(m, splat2(-kRoundMagic));    // rint(t)
+        const float2 d = add2(t, make_float2(-n.x, -n.y)); // t - rint(t), exact
+        near |= !(fabsf(d.x) < kNearHalf) | !(fabsf(d.y) < kNearHalf);
+        b[i] = __float_as_uint(m.x);
+        b[i + 1] = __float_as_uint(m.y);
+    }
+    if (near) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            b[i] = quant_bits(y[i], s);
+    }
 }
 
 // Quantizes the part of a row held in registers (v[c][0..7] for vector v0 + c*blockDim + tid,
@@ -157,9 +167,7 @@ __device__ __forceinline__ void quantize_and_store(const float (&v)[NCH][8], flo
             uint2 out = make_uint2(0u, 0u);
             if (by_product) {
                 uint32_t b[8];
-#pragma unroll
-                for (int i = 0; i < 8; i += 2)
-                    quant_bits2(v[c][i], v[c][i + 1], s, r, b[i], b[i + 1]);
+                quant_bits8(v[c], s, r, b);
                 out.x = pack_low_bytes(b[0], b[1], b[2], b[3]);
                 out.y = pack_low_bytes(b[4], b[5], b[6], b[7]);
             } else if (amax > 0.0f) {
@@ -362,8 +370,8 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsno
 // Binary32 exp fixed by the library's contract (header w8a8.h), two lanes at a time:
 // Cody-Waite reduction with a 16-bit head of ln 2, degree-7 Taylor polynomial by Horner in
 // fused multiply-adds, exact scaling by two powers of two; every step is the scalar
-// definition's IEEE operation, lane by lane.
-__device__ __forceinline__ float2 w8a8_exp2(float2 x)
+// definition's IEEE operation, lane by lane. exp_poly2 returns the polynomial p and k.
+__device__ __forceinline__ float2 exp_poly2(float2 x, int &ka, int &kb)
 {
     const float kInvLn2 = 1.44269502162933349609375f;           // RN(1 / ln 2)
     const float kLn2Hi = 0.693145751953125f;                    // ln 2, 16 significant bits
@@ -381,31 +389,55 @@ __device__ __forceinline__ float2 w8a8_exp2(float2 x)
     p = fma2(p, r, splat2(0.5f));
     p = fma2(p, r, splat2(1.0f));
     p = fma2(p, r, splat2(1.0f));
-    const int ka = __float_as_int(km.x) - kRoundMagicBits;
-    const int kb = __float_as_int(km.y) - kRoundMagicBits;
-    if (fabsf(x.x) <= 80.0f && fabsf(x.y) <= 80.0f) {
-        // |k| <= 115 and p in [0.7, 1.5): every partial product of the two power-of-two
-        // scalings is a normal number, so both are exact and equal adding k to p's exponent
-        return make_float2(__uint_as_float(__float_as_uint(p.x) + (static_cast<uint32_t>(ka) << 23)),
-                           __uint_as_float(__float_as_uint(p.y) + (static_cast<uint32_t>(kb) << 23)));
-    }
-    const int ka1 = ka / 2, kb1 = kb / 2; // truncation toward zero
-    const float2 s1 = make_float2(__int_as_float((ka1 + 127) << 23), __int_as_float((kb1 + 127) << 23));
-    const float2 s2 = make_float2(__int_as_float((ka - ka1 + 127) << 23),
-                                  __int_as_float((kb - kb1 + 127) << 23));
-    float2 e = mul2(mul2(p, s1), s2);
-    // outside the reduction's range: NaN stays NaN, x > 89 gives +inf, x < -104 gives +0
-    const float inf = __int_as_float(0x7f800000);
-    e.x = (x.x != x.x) ? x.x : (x.x > 89.0f ? inf : (x.x < -104.0f ? 0.0f : e.x));
-    e.y = (x.y != x.y) ? x.y : (x.y > 89.0f ? inf : (x.y < -104.0f ? 0.0f : e.y));
-    return e;
+    ka = __float_as_int(km.x) - kRoundMagicBits;
+    kb = __float_as_int(km.y) - kRoundMagicBits;
+    return p;
 }
 
-// a = silu(g) * u = (g / (1 + exp(-g))) * u for two lanes; the division stays IEEE scalar.
-__device__ __forceinline__ float2 silu_mul2(float2 g, float2 u)
+// p * 2^k1 * 2^k2 (k1 = k / 2 truncated, k2 = k - k1), and the range rules: NaN stays NaN,
+// x > 89 gives +inf, x < -104 gives +0.
+__device__ __forceinline__ float exp_scale_full(float p, int k, float x)
 {
-    const float2 d = add2(splat2(1.0f), w8a8_exp2(make_float2(-g.x, -g.y)));
-    return mul2(make_float2(__fdiv_rn(g.x, d.x), __fdiv_rn(g.y, d.y)), u);
+    const int k1 = k / 2; // truncation toward zero
+    const float e = __fmul_rn(__fmul_rn(p, __int_as_float((k1 + 127) << 23)),
+                              __int_as_float((k - k1 + 127) << 23));
+    const float inf = __int_as_float(0x7f800000);
+    return (x != x) ? x : (x > 89.0f ? inf : (x < -104.0f ? 0.0f : e));
+}
+
+// a = silu(g) * u = (g / (1 + exp(-g))) * u for the eight values of one vector; the
+// divisions stay IEEE scalar. When every |g| <= 80 (one test per vector), |k| <= 115 and
+// p in [0.7, 1.5) make every partial product of the two power-of-two scalings a normal
+// number, so both are exact and equal adding k to p's exponent.
+__device__ __forceinline__ void silu_mul8(const float (&g)[8], const float (&u)[8], float (&a)[8])
+{
+    float e[8];
+    int k[8];
+    bool in_range = true;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float2 p = exp_poly2(make_float2(-g[i], -g[i + 1]), k[i], k[i + 1]);
+        e[i] = p.x;
+        e[i + 1] = p.y;
+        in_range &= (fabsf(g[i]) <= 80.0f) & (fabsf(g[i + 1]) <= 80.0f);
+    }
+    if (in_range) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            e[i] = __uint_as_float(__float_as_uint(e[i]) + (static_cast<uint32_t>(k[i]) << 23));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            e[i] = exp_scale_full(e[i], k[i], -g[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float2 d = add2(splat2(1.0f), make_float2(e[i], e[i + 1]));
+        const float2 q = make_float2(__fdiv_rn(g[i], d.x), __fdiv_rn(g[i + 1], d.y));
+        const float2 r = mul2(q, make_float2(u[i], u[i + 1]));
+        a[i] = r.x;
+        a[i + 1] = r.y;
+    }
 }
 
 template <int NCH>
@@ -434,14 +466,10 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) silu_
                 float g[8], u[8];
                 unpack8(cg[c], g);
                 unpack8(cu[c], u);
+                silu_mul8(g, u, v[c]);
 #pragma unroll
-                for (int i = 0; i < 8; i += 2) {
-                    const float2 a2 = silu_mul2(make_float2(g[i], g[i + 1]),
-                                                make_float2(u[i], u[i + 1]));
-                    v[c][i] = a2.x;
-                    v[c][i + 1] = a2.y;
-                    amax = fmaxf(amax, fmaxf(fabsf(a2.x), fabsf(a2.y)));
-                }
+                for (int i = 0; i < 8; ++i)
+                    amax = fmaxf(amax, fabsf(v[c][i]));
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
