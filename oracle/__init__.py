@@ -34,6 +34,9 @@ def lib():
         L.oracle_f32_to_bf16.argtypes = [C.c_float]
         L.oracle_quantize_row_f32.argtypes = [P, I64, P, P]
         L.oracle_quantize_rows.argtypes = [P, P, I64, I64, P, P, C.c_int]
+        L.oracle_minmax_scale.restype = C.c_float
+        L.oracle_minmax_scale.argtypes = [P, I64]
+        L.oracle_quantize_rows_static.argtypes = [P, P, C.c_float, I64, I64, P, C.c_int]
         L.oracle_smooth_rmsnorm_quant.argtypes = [P, P, P, P, C.c_float, I64, I64, P, P, P, P,
                                                   P, P, C.c_int]
         L.oracle_exp.restype = C.c_float
@@ -117,6 +120,24 @@ def quantize_rows(x_bf16, sinv=None, nthreads=NTHREADS):
     s = np.empty(M, dtype=np.float32)
     lib().oracle_quantize_rows(_p(x), _p(sinv), M, K, _p(q), _p(s), nthreads)
     return q, s
+
+
+def minmax_scale(values_f32):
+    """Symmetric min-max calibration scale S = max(|min|, |max|) / 127 of a tensor."""
+    v = _c(values_f32, np.float32).ravel()
+    return np.float32(lib().oracle_minmax_scale(_p(v), v.size))
+
+
+def quantize_rows_static(x_bf16, scale, sinv=None, nthreads=NTHREADS):
+    """Static per-tensor quantization with a fixed scale -> q int8 [M, K]."""
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    sinv = _c(sinv, np.float32)
+    q = np.empty((M, K), dtype=np.int8)
+    rc = lib().oracle_quantize_rows_static(_p(x), _p(sinv), float(scale), M, K, _p(q), nthreads)
+    if rc != 0:
+        raise ValueError("scale must be > 0")
+    return q
 
 
 def smooth_rmsnorm_quant(x_bf16, gamma, eps, residual=None, ms_override=None,

@@ -171,6 +171,67 @@ int oracle_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int64_
     return 0;
 }
 
+/* ------------------------------------------------- static per-tensor quantization */
+
+/*
+ * Symmetric min-max calibration of one tensor [P3 "1. Min-Max Calibration"]: the observed
+ * range [min, max] of the calibration values maps onto [-127, 127] with
+ * S = max(|min|, |max|) / 127 (binary32 division). Returns 0 for an empty or all-zero set.
+ */
+float oracle_minmax_scale(const float *v, int64_t n)
+{
+    if (n <= 0)
+        return 0.0f;
+    float lo = v[0], hi = v[0];
+    for (int64_t j = 1; j < n; ++j) {
+        if (v[j] < lo)
+            lo = v[j];
+        if (v[j] > hi)
+            hi = v[j];
+    }
+    float a = fabsf(lo) > fabsf(hi) ? fabsf(lo) : fabsf(hi);
+    return a / 127.0f;
+}
+
+struct qstatic_ctx {
+    const uint16_t *x;
+    const float *sinv;
+    float S;
+    int64_t K;
+    int8_t *q;
+};
+
+static void qstatic_row(void *vctx, int64_t m)
+{
+    struct qstatic_ctx *c = (struct qstatic_ctx *)vctx;
+    for (int64_t j = 0; j < c->K; ++j) {
+        float y = oracle_bf16_to_f32(c->x[m * c->K + j]);
+        if (c->sinv)
+            y = y * c->sinv[j];
+        float t = rintf(y / c->S); /* ties to even */
+        if (t > 127.0f)
+            t = 127.0f;
+        if (t < -127.0f)
+            t = -127.0f;
+        c->q[m * c->K + j] = (int8_t)t;
+    }
+}
+
+/*
+ * Static per-tensor activation quantization [P3 "1. Min-Max Calibration"]: one scale S > 0,
+ * fixed offline by calibration, for every token; q = clamp(round_half_even(y / S), -127,
+ * 127) with y = x (or x * sinv[j]). Values beyond the calibrated range saturate at +-127.
+ */
+int oracle_quantize_rows_static(const uint16_t *x, const float *sinv, float S, int64_t M,
+                                int64_t K, int8_t *q, int nthreads)
+{
+    if (!(S > 0.0f))
+        return -1;
+    struct qstatic_ctx c = {x, sinv, S, K, q};
+    parallel_rows(qstatic_row, &c, M, nthreads);
+    return 0;
+}
+
 /* --------------------------------------------------------- smoothed RMSNorm + quant */
 
 struct rms_ctx {

@@ -412,3 +412,55 @@ def test_rtn_weights_are_rowwise_quant_of_smoothed_weight():
     for n in range(16):
         exact = Fraction(float(np.abs(ws[n]).max())) / 127
         assert abs(Fraction(float(s_ch[n])) - exact) <= Fraction(ulp32(s_ch[n])) / 2
+
+
+# ----------------------------------------------------------------- static per-tensor scale
+
+
+def _bf16_bits(xf):
+    return torch.from_numpy(np.asarray(xf, np.float32)).to(torch.bfloat16).view(torch.int16) \
+        .numpy().view(np.uint16)
+
+
+def test_static_minmax_calibration_worked_example(golden):
+    # the page's calibration set: S = max(|min|, |max|) / 127 and the most negative value
+    # codes to -127 with that fixed scale
+    g = golden("p3_minmax_scale.txt")
+    S = oracle.minmax_scale(np.array(g["values"], np.float32))
+    ref = Fraction(max(abs(g["min_val"][0]), abs(g["max_val"][0]))) / 127
+    assert float(S) == round_fraction_to_f32(ref)
+    q = oracle.quantize_rows_static(_bf16_bits([g["values"]]), S)
+    assert q[0, 0] == g["code_of_min"][0]
+    assert q.max() <= 127 and q.min() >= -127
+
+
+def test_static_reduces_to_dynamic_with_the_rows_own_scale():
+    # with S equal to a row's own dynamic scale, static quantization is per-token dynamic
+    # quantization of that row (including its smoothing)
+    x = synth.activation(6, 512, seed=3)
+    sinv = (1.0 / synth.gamma(512, 4)).astype(np.float32)
+    q_dyn, s_dyn = oracle.quantize_rows(x, sinv)
+    for m in range(6):
+        q_st = oracle.quantize_rows_static(x[m:m + 1], s_dyn[m], sinv)
+        assert np.array_equal(q_st[0], q_dyn[m])
+
+
+def test_static_exact_multiples_ties_and_saturation():
+    # S = 2^-4: y = k S is exact, (k + 1/2) S is an exact tie (half to even), and values
+    # past 127 S saturate
+    S = np.float32(0.0625)
+    k = np.arange(-140, 141)
+    y = np.concatenate([k * 0.0625, (np.arange(-20, 20) + 0.5) * 0.0625]).astype(np.float32)
+    q = oracle.quantize_rows_static(_bf16_bits([y]), S)[0]
+    expect_k = np.clip(k, -127, 127)
+    # j + 1/2 lies between j and j + 1: the even one of the two
+    expect_h = np.array([j if j % 2 == 0 else j + 1 for j in range(-20, 20)])
+    assert np.array_equal(q[:len(k)], expect_k)
+    assert np.array_equal(q[len(k):], expect_h)
+
+
+def test_static_rejects_nonpositive_scale():
+    x = _bf16_bits([[1.0, 2.0]])
+    for bad in (0.0, -1.0):
+        with pytest.raises(ValueError):
+            oracle.quantize_rows_static(x, bad)
