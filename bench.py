@@ -588,7 +588,8 @@ def run_reference(args, world, rank):
 
 
 def run_case(args):
-    """`--case gemm:M:N:K[:variant]`, `rms:M:K`, `rmsres:M:K`, `quant:M:K` or `silu:M:I`:
+    """`--case gemm:M:N:K[:variant]`, `rms:M:K`, `rmsres:M:K`, `quant:M:K`, `static:M:K` or
+    `silu:M:I`:
     one kernel launched repeatedly (a CUDA graph of back-to-back launches)."""
     import int8_w8a8_quantized_smoothed_b200 as w8
     from int8_w8a8_quantized_smoothed_b200 import build as wbuild, synth
@@ -632,9 +633,11 @@ def run_case(args):
                 w8.w8a8_smooth_rmsnorm_quant(x, g, EPS, residual=res, h_out=h, q=q, s_tok=s)
             elif kind == "quant":
                 w8.w8a8_quantize_rows(x, g, q=q, s_tok=s)
+            elif kind == "static":
+                w8.w8a8_quantize_rows_static(x, 0.05, g, q=q, s_tok=s)
             else:
                 w8.w8a8_silu_mul_quant(x, q=q, s_tok=s)
-        work = {"rms": 3 * M * K, "rmsres": 7 * M * K, "quant": 3 * M * K,
+        work = {"rms": 3 * M * K, "rmsres": 7 * M * K, "quant": 3 * M * K, "static": 3 * M * K,
                 "silu": 5 * M * K}[kind] + 4 * M + 4 * K
     for i in range(args.warmup):
         launch(i)

@@ -77,6 +77,21 @@ W8A8_API int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int
                        int8_t *q, float *s_tok, w8a8_stream_t stream);
 
 /*
+ * Static per-tensor symmetric quantization of activations [PTQ "1. Min-Max Calibration"]:
+ * one scale for every token, fixed offline from a calibration batch as
+ * scale = max(|min|, |max|) / 127, so no per-token range is measured at run time:
+ *   y[m,j]   = float(x[m,j]) * smooth_inv[j]          (or float(x[m,j]) if smooth_inv == NULL)
+ *   q[m,j]   = clamp(round_half_even(y[m,j] / scale), -127, 127)   (values beyond the
+ *              calibrated range saturate at +-127)
+ *   s_tok[m] = scale  (when s_tok is not NULL, so w8a8_gemm_dequant can consume it as is)
+ * scale: finite and > 0, else W8A8_ERR_INVALID_ARG. Layout, alignment and shape rules as
+ * for w8a8_quantize_rows; s_tok may be NULL.
+ */
+W8A8_API int w8a8_quantize_rows_static(const w8a8_bf16 *x, const float *smooth_inv, float scale,
+                                       int64_t M, int64_t K, int8_t *q, float *s_tok,
+                                       w8a8_stream_t stream);
+
+/*
  * Smoothed RMSNorm fused with per-token quantization [W8A8 "How SmoothQuant prevents
  * outliers in activation tensors": RMSNorm divides by the RMS, then multiplies by gamma;
  * SmoothQuant divides gamma by s]:

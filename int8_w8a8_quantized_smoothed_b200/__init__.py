@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "W8A8Error", "lib", "LIB_PATH",
-    "w8a8_quantize_rows", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
+    "w8a8_quantize_rows", "w8a8_quantize_rows_static", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
     "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_probe_i8_mma", "w8a8_set_overlap",
     "w8a8_get_overlap", "w8a8_device_status",
@@ -35,6 +35,7 @@ STATUS = {0: "W8A8_OK", -1: "W8A8_ERR_INVALID_ARG", -2: "W8A8_ERR_ALIGNMENT",
 _P, _I64, _I, _F, _SZ = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
 SIGNATURES = [
     ("w8a8_quantize_rows", _I, [_P, _P, _I64, _I64, _P, _P, _P]),
+    ("w8a8_quantize_rows_static", _I, [_P, _P, _F, _I64, _I64, _P, _P, _P]),
     ("w8a8_smooth_rmsnorm_quant", _I, [_P, _P, _P, _P, _F, _I64, _I64, _P, _P, _P]),
     ("w8a8_silu_mul_quant", _I, [_P, _I64, _I64, _P, _P, _P]),
     ("w8a8_gemm_workspace_size", _SZ, [_I64, _I64, _I64]),
@@ -154,6 +155,22 @@ def w8a8_quantize_rows(x, smooth_inv=None, q=None, s_tok=None, stream=None):
     _need(s_tok, "s_tok", torch.float32, (M,))
     _check("w8a8_quantize_rows", lib().w8a8_quantize_rows(
         _ptr(x), _ptr(smooth_inv), M, K, _ptr(q), _ptr(s_tok), _stream(stream)))
+    return q, s_tok
+
+
+def w8a8_quantize_rows_static(x, scale, smooth_inv=None, q=None, s_tok=None, stream=None):
+    """Static per-tensor int8 quantization of bf16 x [M, K] with a fixed calibrated scale;
+    s_tok (filled with the scale) is returned too so that the GEMM can consume it."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    if smooth_inv is not None:
+        _need(smooth_inv, "smooth_inv", torch.float32, (K,))
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _need(q, "q", torch.int8, (M, K))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_quantize_rows_static", lib().w8a8_quantize_rows_static(
+        _ptr(x), _ptr(smooth_inv), float(scale), M, K, _ptr(q), _ptr(s_tok), _stream(stream)))
     return q, s_tok
 
 

@@ -125,13 +125,18 @@ __device__ __forceinline__ float2 splat2(float v)
 // from every half-integer, rint(t) = rint(RN(y / s)) and |rint(t)| <= 127 needs no clamp.
 // When any of the eight is that close (probability about 2^-10 per vector), the exact
 // quotient decides all eight (one branch per vector keeps the common path branch-free).
+// SAT: values may lie beyond +-127 s (a fixed scale); t is clamped to [-127, 127] first,
+// which commutes with the rounding because the bounds are integers.
+template <bool SAT = false>
 __device__ __forceinline__ void quant_bits8(const float (&y)[8], float s, float r, uint32_t (&b)[8])
 {
     constexpr float kNearHalf = 0.5f - 6.103515625e-05f; // 0.5 - 2^-14
     bool near = false;
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-        const float2 t = mul2(make_float2(y[i], y[i + 1]), splat2(r));
+        float2 t = mul2(make_float2(y[i], y[i + 1]), splat2(r));
+        if constexpr (SAT)
+            t = make_float2(fminf(fmaxf(t.x, -127.0f), 127.0f), fminf(fmaxf(t.y, -127.0f), 127.0f));
         const float2 m = add2(t, splat2(kRoundMagic));     // rint(t) + 1.5 * 2^23
         const float2 n = add2(m, splat2(-kRoundMagic));    // rint(t)
         const float2 d = add2(t, make_float2(-n.x, -n.y)); // t - rint(t), exact
@@ -263,6 +268,81 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quant
         amax = block_max(amax, sh[it & 1u]);
         quantize_and_store<NCH>(v, amax, 0, nvec, q + row * K, s_tok + row);
     }
+}
+
+// ----------------------------------------------------------------- static per-tensor scale
+//
+// One scale S for every token, fixed offline by min-max calibration: no reduction, so the
+// kernel is a grid-stride pass over the 8-value vectors of all rows (HBM-bound). Values
+// beyond the calibrated range saturate at +-127.
+
+__global__ void __launch_bounds__(256) quantize_rows_static_kernel(
+    const uint16_t *__restrict__ x, const float *__restrict__ sinv, float S, int K,
+    int64_t nvec_total, int M, int8_t *__restrict__ q, float *__restrict__ s_tok)
+{
+    constexpr int kU = 4; // vectors per thread per pass, all loads issued before any use
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // every input may come from the previous kernel
+    const int nvec = K >> 3;
+    const bool by_product = S >= 7.888609052210118e-31f; // 2^-100: finite reciprocal
+    const float r = by_product ? __frcp_rn(S) : 0.0f;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    // each CTA walks one contiguous range of vectors (DRAM locality), kU * blockDim.x
+    // vectors per pass, consecutive threads on consecutive vectors
+    const int64_t per_cta = (nvec_total + gridDim.x - 1) / gridDim.x;
+    const int64_t begin = static_cast<int64_t>(blockIdx.x) * per_cta;
+    const int64_t end = begin + per_cta < nvec_total ? begin + per_cta : nvec_total;
+    const int step = static_cast<int>(blockDim.x) % nvec; // column advance per vector step
+    int c0 = static_cast<int>((begin + threadIdx.x) % nvec);
+    for (int64_t v0 = begin + threadIdx.x; v0 < end; v0 += kU * blockDim.x) {
+        uint4 raw[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t v = v0 + u * static_cast<int64_t>(blockDim.x);
+            raw[u] = v < end ? ldg_nc_v4(xv + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        int c = c0;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t v = v0 + u * static_cast<int64_t>(blockDim.x);
+            if (v >= end)
+                break;
+            float y[8];
+            unpack8(raw[u], y);
+            if (sinv) {
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * c);
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(sinv) + 2 * c + 1);
+                const float w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 p = mul2(make_float2(y[i], y[i + 1]), make_float2(w[i], w[i + 1]));
+                    y[i] = p.x;
+                    y[i + 1] = p.y;
+                }
+            }
+            uint32_t bits[8];
+            if (by_product) {
+                quant_bits8<true>(y, S, r, bits);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    bits[i] = quant_bits(y[i], S);
+            }
+            reinterpret_cast<uint2 *>(q)[v] =
+                make_uint2(pack_low_bytes(bits[0], bits[1], bits[2], bits[3]),
+                           pack_low_bytes(bits[4], bits[5], bits[6], bits[7]));
+            c += step;
+            if (c >= nvec)
+                c -= nvec;
+        }
+        c0 = c; // after kU steps (or the end)
+    }
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    if (s_tok)
+        for (int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; m < M;
+             m += stride)
+            s_tok[m] = S;
 }
 
 // ----------------------------------------------------------------- smoothed RMSNorm + quant

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <map>
 #include <mutex>
@@ -610,6 +611,35 @@ int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, i
     case 2: return launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
     default: return launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
     }
+}
+
+int w8a8_quantize_rows_static(const w8a8_bf16 *x, const float *smooth_inv, float scale,
+                              int64_t M, int64_t K, int8_t *q, float *s_tok,
+                              w8a8_stream_t stream)
+{
+    if (!x || !q)
+        return W8A8_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || !(scale <= 3.4028234663852886e38f))
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, K);
+    if (rc)
+        return rc;
+    if (!aligned16(x) || !aligned16(q) || (smooth_inv && !aligned16(smooth_inv)))
+        return W8A8_ERR_ALIGNMENT;
+    if (static_cast<const void *>(x) == static_cast<const void *>(q))
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    const void *fn = reinterpret_cast<const void *>(&quantize_rows_static_kernel);
+    if ((rc = ensure_smem(fn, dev, 0)))
+        return rc;
+    const int64_t nvec_total = M * (K / 8);
+    const int64_t want = (nvec_total + 255) / 256;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+    return launch_kernel(quantize_rows_static_kernel, dim3(grid), dim3(256), 0,
+                         reinterpret_cast<cudaStream_t>(stream), x, smooth_inv, scale,
+                         static_cast<int>(K), nvec_total, static_cast<int>(M), q, s_tok);
 }
 
 int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a8_bf16 *h_out,

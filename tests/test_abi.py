@@ -72,6 +72,14 @@ def test_host_validation_without_device(L):
     assert L.w8a8_smooth_rmsnorm_quant(_p(A), None, None, _p(A), C.c_float(-1.0), 4, 64,
                                        _p(A), _p(A), None) == -1
     assert L.w8a8_silu_mul_quant(_p(A), 4, 40, _p(A), _p(A), None) == -3
+    # static scale: must be finite and positive; same shape / alignment rules
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert L.w8a8_quantize_rows_static(_p(A), None, C.c_float(bad), 4, 64, _p(A + 4096),
+                                           None, None) == -1
+    assert L.w8a8_quantize_rows_static(_p(A), None, C.c_float(0.1), 4, 24, _p(A + 4096), None,
+                                       None) == -3
+    assert L.w8a8_quantize_rows_static(_p(A), _p(A + 4), C.c_float(0.1), 4, 64, _p(A + 4096),
+                                       None, None) == -2
     # GEMM: N % 8, K % 16, K limit, alignment
     args = [_p(A), _p(A), _p(A), _p(A)]
     assert L.w8a8_gemm_dequant(*args, 4, 12, 64, _p(A), None, None, 0, None) == -3

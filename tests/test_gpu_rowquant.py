@@ -196,3 +196,38 @@ def test_quantize_tiny_scales_take_exact_quotient():
     assert np.array_equal(host(s), s_ref)
     assert np.array_equal(host(q), q_ref)
     assert (s_ref[:3] < 2.0 ** -100).all() and s_ref[3] > 2.0 ** -100
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (37, 4096), (300, 4112), (3000, 4096), (5, 28672)])
+@pytest.mark.parametrize("smooth", [False, True])
+def test_quantize_rows_static_bit_exact(M, K, smooth):
+    # the scale is calibrated on a different batch, so some values of x lie beyond it and
+    # saturate; the near-half-integer and exact-quotient paths are exercised by the data
+    x = synth.activation(M, K, seed=M + 3 * K)
+    cal = synth.activation(64, K, seed=K + 11)
+    sinv = _sinv(K, K + 5) if smooth else None
+    calf = oracle.bf16_to_f32(cal) * (sinv if smooth else 1.0)
+    S = oracle.minmax_scale(calf.astype(np.float32)) * np.float32(0.5)
+    q_ref = oracle.quantize_rows_static(x, S, sinv)
+    q, s = w8.w8a8_quantize_rows_static(dev_bf16(x), float(S), None if sinv is None else dev(sinv))
+    assert np.array_equal(host(q), q_ref)
+    assert (host(s) == S).all()
+    if M * K >= 4096:
+        assert (np.abs(q_ref) == 127).any()  # saturation happened
+
+
+def test_quantize_rows_static_tiny_and_equal_to_dynamic():
+    # a scale below 2^-100 takes the exact quotient; with a row's own dynamic scale the codes
+    # are the dynamic codes
+    K = 256
+    x = synth.activation(4, K, 21)
+    q_dyn, s_dyn = oracle.quantize_rows(x)
+    for m in range(4):
+        q, _ = w8.w8a8_quantize_rows_static(dev_bf16(x[m:m + 1]), float(s_dyn[m]))
+        assert np.array_equal(host(q)[0], q_dyn[m])
+    tiny = (synth.activation(2, K, 22).view(np.uint16) & 0x807F) | 0x0080  # |x| ~ 2^-126
+    S = np.float32(2.0 ** -132)  # subnormal: |x| / S in [64, 128), the largest saturate
+    q, _ = w8.w8a8_quantize_rows_static(dev_bf16(tiny), float(S))
+    q_ref = oracle.quantize_rows_static(tiny, S)
+    assert np.array_equal(host(q), q_ref)
+    assert (np.abs(q_ref) >= 64).all() and (np.abs(q_ref) == 127).any()
