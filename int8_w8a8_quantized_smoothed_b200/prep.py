@@ -67,3 +67,15 @@ def prepare_linear(w: torch.Tensor, a_max, alpha: float):
     wq, s_ch = quantize_weight(w, s_dev)
     return dict(s=s, s_inv=s_inv, wq=wq, s_ch=s_ch, s_dev=s_dev,
                 s_inv_dev=torch.from_numpy(s_inv).to(w.device))
+
+
+def static_activation_scale(x_cal: torch.Tensor, smooth_inv=None) -> float:
+    """Static per-tensor activation scale from a calibration batch [PTQ page, "1. Min-Max
+    Calibration"]: S = max(|min|, |max|) / 127 over the (smoothed) calibration values, in
+    binary32, for ``w8a8_quantize_rows_static``. The maximum is exact; the division is one
+    IEEE binary32 operation."""
+    y = x_cal.float()
+    if smooth_inv is not None:
+        y = y * smooth_inv.float()
+    a = y.abs().amax().reshape(1)
+    return float((a / torch.tensor([127.0], dtype=torch.float32, device=a.device)).item())

@@ -231,3 +231,12 @@ def test_quantize_rows_static_tiny_and_equal_to_dynamic():
     q_ref = oracle.quantize_rows_static(tiny, S)
     assert np.array_equal(host(q), q_ref)
     assert (np.abs(q_ref) >= 64).all() and (np.abs(q_ref) == 127).any()
+
+
+def test_static_scale_calibration_matches_oracle():
+    from int8_w8a8_quantized_smoothed_b200 import prep
+    cal = synth.activation(128, 4096, 31)
+    sinv = _sinv(4096, 32)
+    S = prep.static_activation_scale(dev_bf16(cal), dev(sinv))
+    ref = oracle.minmax_scale((oracle.bf16_to_f32(cal) * sinv).astype(np.float32))
+    assert np.float32(S) == ref
