@@ -214,6 +214,30 @@ W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, con
                                        w8a8_bf16 *y, w8a8_stream_t stream);
 
 /*
+ * The gate|up projection of a Llama MLP fused with SiLU(gate)*up [SiLU*up is not on the
+ * pages; it is the decoder block's MLP]: the INT8 GEMM of w8a8_gemm_dequant whose epilogue
+ * forms a = silu(g) * u instead of storing the [M, 2I] gate|up output, followed by the
+ * per-token quantization of a. Results are bit for bit those of w8a8_gemm_dequant followed by
+ * w8a8_silu_mul_quant on the plain weight:
+ *   g, u     = the bf16 outputs of w8a8_gemm_dequant for gate channel j and up channel j
+ *   a[m,j]   = (g / (1 + exp(-g))) * u in binary32 (exp as in w8a8_silu_mul_quant)
+ *   s_out[m] = max_j |a[m,j]| / 127,  q[m,j] = clamp(round_half_even(a[m,j] / s_out[m]), +-127)
+ * xq, s_tok: as for w8a8_gemm_dequant (M tokens, K inputs). wq_il: int8 [2I, K], the gate|up
+ * weight with its rows interleaved in blocks of 64: rows 128b .. 128b+63 are gate rows
+ * 64b .. 64b+63 and rows 128b+64 .. 128b+127 are up rows 64b .. 64b+63 (b < I/64); s_ch_il:
+ * fp32 [2I], the channel scales in the same order. I % 64 == 0.
+ * a: fp32 [M, I] (written, then read by the quantization; 16-byte aligned). q: int8 [M, I],
+ * s_out: fp32 [M]. workspace: w8a8_gemm_silu_quant_workspace_size(M, I, K) bytes, 16-byte
+ * aligned, zero-filled before its first use; each call leaves it zero again. Other
+ * requirements and errors as for w8a8_gemm_dequant (acc_out is not available here).
+ */
+W8A8_API size_t w8a8_gemm_silu_quant_workspace_size(int64_t M, int64_t I, int64_t K);
+W8A8_API int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_il,
+                                  const float *s_ch_il, int64_t M, int64_t I, int64_t K,
+                                  float *a, int8_t *q, float *s_out, void *workspace,
+                                  size_t workspace_bytes, w8a8_stream_t stream);
+
+/*
  * Measurement aid, not part of the W8A8 path (the pages have no counterpart): launches `ctas`
  * CTAs (0 = one per SM), each issuing `iters` back-to-back dense tcgen05.mma kind::i8 of
  * shape 128 x n x 32 (n = 16, 32, 64, 128 or 256) on shared-memory operands into tensor

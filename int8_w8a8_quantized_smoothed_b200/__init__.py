@@ -19,7 +19,8 @@ __all__ = [
     "W8A8Error", "lib", "LIB_PATH",
     "w8a8_quantize_rows", "w8a8_quantize_rows_static", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
-    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_probe_i8_mma", "w8a8_set_overlap",
+    "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_gemm_silu_quant",
+    "w8a8_gemm_silu_quant_workspace_size", "w8a8_probe_i8_mma", "w8a8_set_overlap",
     "w8a8_get_overlap", "w8a8_device_status",
     "w8a8_status_string", "w8a8_version",
     "Workspace",
@@ -44,6 +45,8 @@ SIGNATURES = [
                                   _I, _P]),
     ("w8a8_gemm_workspace_size_ex", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
     ("w8a8_gemm_dequant_noalloc", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    ("w8a8_gemm_silu_quant_workspace_size", _SZ, [_I64, _I64, _I64]),
+    ("w8a8_gemm_silu_quant", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     ("w8a8_probe_i8_mma", _I, [C.c_longlong, _I, _I, _P]),
     ("w8a8_set_overlap", _I, [_I]),
     ("w8a8_get_overlap", _I, []),
@@ -283,6 +286,46 @@ def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=No
 def w8a8_gemm_dequant(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None, stream=None):
     return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=y, acc_out=acc_out,
                                 workspace=workspace, stream=stream)
+
+
+def w8a8_gemm_silu_quant_workspace_size(M: int, I: int, K: int) -> int:
+    return int(lib().w8a8_gemm_silu_quant_workspace_size(M, I, K))
+
+
+def w8a8_gemm_silu_quant(xq, s_tok, wq_il, s_ch_il, a=None, q=None, s_out=None,
+                         workspace=None, stream=None):
+    """The gate|up GEMM with the SiLU(gate)*up epilogue, then per-token quantization of a:
+    the same q, s as w8a8_gemm_dequant + w8a8_silu_mul_quant on the plain weight. wq_il,
+    s_ch_il: the gate|up weight and scales with rows interleaved in blocks of 64 (see
+    prep.interleave_gate_up). Returns (q, s_out, a)."""
+    _need(xq, "xq", torch.int8)
+    _need(wq_il, "wq_il", torch.int8)
+    M, K = xq.shape
+    N, K2 = wq_il.shape
+    if K != K2 or N % 2:
+        raise ValueError(f"xq [M,K] and wq_il [2I,K] disagree: {tuple(xq.shape)} {tuple(wq_il.shape)}")
+    I = N // 2
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _need(s_ch_il, "s_ch_il", torch.float32, (N,))
+    e = dict(device=xq.device)
+    a = torch.empty((M, I), dtype=torch.float32, **e) if a is None else a
+    q = torch.empty((M, I), dtype=torch.int8, **e) if q is None else q
+    s_out = torch.empty(M, dtype=torch.float32, **e) if s_out is None else s_out
+    _need(a, "a", torch.float32, (M, I))
+    _need(q, "q", torch.int8, (M, I))
+    _need(s_out, "s_out", torch.float32, (M,))
+    need = w8a8_gemm_silu_quant_workspace_size(M, I, K)
+    if workspace is None:
+        workspace = _workspace_for(xq.device)
+    if isinstance(workspace, Workspace):
+        wbuf, wbytes = workspace.get(need)
+    else:
+        wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
+                                   * workspace.element_size())
+    _check("w8a8_gemm_silu_quant", lib().w8a8_gemm_silu_quant(
+        _ptr(xq), _ptr(s_tok), _ptr(wq_il), _ptr(s_ch_il), M, I, K, _ptr(a), _ptr(q),
+        _ptr(s_out), _ptr(wbuf), wbytes, _stream(stream)))
+    return q, s_out, a
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # W8A8_NOALLOC_SCRATCH_BYTES in include/w8a8.h

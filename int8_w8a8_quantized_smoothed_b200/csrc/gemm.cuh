@@ -16,9 +16,18 @@
 //   tokens its N side), persistent stream-K: each CTA streams an equal contiguous share of
 //   the (channel block, k-block) units, several k-blocks per pipeline stage; blocks split
 //   between CTAs are summed exactly in int32 by the block's owner (see below).
+//
+// Fused SiLU(gate)*up epilogue (template flag SILU), for the gate|up projection of a Llama
+// MLP: the weight's rows are interleaved in blocks of 64 (gate channels 64b..64b+63, then up
+// channels 64b..64b+63), so every 128-row group of weight rows holds the gate and up rows of
+// the same 64 output channels. The epilogue rounds both dequantized values to bf16 (exactly
+// what the plain epilogue stores), forms a = silu(g) * u in binary32 as the SiLU*up row
+// kernel does, stores a, and raises a per-token maximum |a| (atomicMax on its bits) that a
+// following quantization pass turns into the per-token scale.
 #pragma once
 
 #include "ptx.cuh"
+#include "rowquant.cuh"
 
 namespace w8a8 {
 
@@ -27,6 +36,50 @@ constexpr int kMaxClusterSize = 8; // portable thread-block cluster size
 constexpr int kBM = 128;  // MMA M: TMEM lanes
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kUmmaK = 32; // K of one kind::i8 MMA
+
+// Outputs of the fused SiLU*up epilogue: a [M, I] binary32 and per-token max |a| words.
+struct SiluOut {
+    float *a;
+    unsigned int *amax;
+    int I;
+};
+
+__device__ __forceinline__ float bf16_round(float f)
+{
+    return __uint_as_float(bf16_bits(f) << 16);
+}
+
+// One thread's row: 32 gate columns (rg, channel scales scg) and the 32 up columns of the
+// same output channels (ru, scu) -> a = silu(bf16(g)) * bf16(u), stored at dst (32 floats,
+// 16-byte stores); returns max |a|.
+__device__ __forceinline__ float silu_row_chunk(const uint32_t (&rg)[32], const uint32_t (&ru)[32],
+                                                float st, const float *scg, const float *scu,
+                                                float *__restrict__ dst)
+{
+    float mx = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float g[8], u[8], a[8];
+        const float4 g0 = reinterpret_cast<const float4 *>(scg)[2 * e];
+        const float4 g1 = reinterpret_cast<const float4 *>(scg)[2 * e + 1];
+        const float4 u0 = reinterpret_cast<const float4 *>(scu)[2 * e];
+        const float4 u1 = reinterpret_cast<const float4 *>(scu)[2 * e + 1];
+        const float cg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float cu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            g[i] = bf16_round(dequant_f32(static_cast<int32_t>(rg[8 * e + i]), st, cg[i]));
+            u[i] = bf16_round(dequant_f32(static_cast<int32_t>(ru[8 * e + i]), st, cu[i]));
+        }
+        silu_mul8(g, u, a);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            mx = fmaxf(mx, fabsf(a[i]));
+        reinterpret_cast<float4 *>(dst)[2 * e] = make_float4(a[0], a[1], a[2], a[3]);
+        reinterpret_cast<float4 *>(dst)[2 * e + 1] = make_float4(a[4], a[5], a[6], a[7]);
+    }
+    return mx;
+}
 
 // Producer tail of an mbarrier ring: waits until the consumer has released the last
 // min(issued, stages) stages, i.e. until the empty-barrier phase that each of the last
@@ -140,12 +193,12 @@ template <int BN> struct TileScales {
     }
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SILU = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const float *__restrict__ s_tok,
                         const float *__restrict__ s_ch, int M, int N, int K,
-                        uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
+                        uint16_t *__restrict__ y, int32_t *__restrict__ acc_out, SiluOut so,
                         int prefetch_static, unsigned long long limit_ns)
 {
     using Cfg = PrefillCfg<BN, STAGES>;
@@ -303,14 +356,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int row = mb * kBM + quarter * 32 + lane;
             const bool row_ok = row < M;
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quarter * 32) << 16);
+            if constexpr (SILU) {
+                // gate chunk cg and up chunk cg + 2 hold the same 32 output channels
+                float rowmax = 0.0f;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tbase + c * 32, r);
-                tmem_ld_wait();
+                for (int p = 0; p < BN / 64; ++p) {
+                    const int cg = (p >> 1) * 4 + (p & 1);
+                    const int ch0 = nb * (BN / 2) + (p >> 1) * 64 + (p & 1) * 32;
+                    uint32_t rg[32], ru[32];
+                    tmem_ld_32x32b_x32(tbase + cg * 32, rg);
+                    tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
+                    tmem_ld_wait();
+                    if (row_ok && ch0 < so.I)
+                        rowmax = fmaxf(rowmax, silu_row_chunk(
+                                                   rg, ru, st, sh_sch + buf * BN + cg * 32,
+                                                   sh_sch + buf * BN + (cg + 2) * 32,
+                                                   so.a + static_cast<int64_t>(row) * so.I + ch0));
+                }
                 if (row_ok)
-                    store_row_chunk(r, row, nb * BN + c * 32, N, st, sh_sch + buf * BN + c * 32,
-                                    y, acc_out);
+                    atomicMax(so.amax + row, __float_as_uint(rowmax));
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, r);
+                    tmem_ld_wait();
+                    if (row_ok)
+                        store_row_chunk(r, row, nb * BN + c * 32, N, st,
+                                        sh_sch + buf * BN + c * 32, y, acc_out);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -342,13 +416,13 @@ template <int STAGES> struct PairCfg {
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
-template <int STAGES>
+template <int STAGES, bool SILU = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
                              const float *__restrict__ s_tok, const float *__restrict__ s_ch,
                              int M, int N, int K, uint16_t *__restrict__ y,
-                             int32_t *__restrict__ acc_out, int prefetch_static,
+                             int32_t *__restrict__ acc_out, SiluOut so, int prefetch_static,
                              unsigned long long limit_ns)
 {
     using Cfg = PairCfg<STAGES>;
@@ -519,14 +593,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int row = mb * TM + row_in_tile;
             const bool row_ok = row < M;
             const uint32_t tbase = tmem_base + buf * TN + (static_cast<uint32_t>(quarter * 32) << 16);
+            if constexpr (SILU) {
+                float rowmax = 0.0f;
 #pragma unroll 1
-            for (int c = 0; c < TN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tbase + c * 32, r);
-                tmem_ld_wait();
+                for (int p = 0; p < TN / 64; ++p) {
+                    const int cg = (p >> 1) * 4 + (p & 1);
+                    const int ch0 = nb * (TN / 2) + (p >> 1) * 64 + (p & 1) * 32;
+                    uint32_t rg[32], ru[32];
+                    tmem_ld_32x32b_x32(tbase + cg * 32, rg);
+                    tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
+                    tmem_ld_wait();
+                    if (row_ok && ch0 < so.I)
+                        rowmax = fmaxf(rowmax, silu_row_chunk(
+                                                   rg, ru, st, sh_sch + buf * TN + cg * 32,
+                                                   sh_sch + buf * TN + (cg + 2) * 32,
+                                                   so.a + static_cast<int64_t>(row) * so.I + ch0));
+                }
                 if (row_ok)
-                    store_row_chunk(r, row, nb * TN + c * 32, N, st, sh_sch + buf * TN + c * 32,
-                                    y, acc_out);
+                    atomicMax(so.amax + row, __float_as_uint(rowmax));
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < TN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, r);
+                    tmem_ld_wait();
+                    if (row_ok)
+                        store_row_chunk(r, row, nb * TN + c * 32, N, st,
+                                        sh_sch + buf * TN + c * 32, y, acc_out);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -617,14 +711,49 @@ __device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
     return sg;
 }
 
-template <int NT, int STAGES, int KPS, bool CLUSTER>
+// The SiLU*up form of the final step of a block (see SiluOut): the block's 128 weight rows
+// are gate rows 0..63 and up rows 64..127 of output channels [64 t, 64 t + 64); v8 = (token,
+// group of 8 channels) vectors, 8 per token, consecutive lanes on one token's 8 groups so that
+// the token's maximum is reduced over 8 lanes. gate(m, j) / up(m, j) give the bf16-rounded
+// values; tokens m0 .. m0 + mt - 1; every thread of the warp calls this the same number of
+// times (shuffles).
+template <typename GateUp>
+__device__ __forceinline__ void silu_block_rows(int m0, int mt, int t, int etid, const SiluOut &so,
+                                                GateUp gate_up)
+{
+    const int lane = etid & 31;
+    for (int base = 0; base < mt * 8; base += 128) {
+        const int v = base + etid;
+        const bool act = v < mt * 8;
+        const int m = m0 + (v >> 3), j0 = (v & 7) * 8;
+        float mx = 0.0f;
+        if (act) {
+            float g[8], u[8], a[8];
+            gate_up(m, j0, g, u);
+            silu_mul8(g, u, a);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mx = fmaxf(mx, fabsf(a[i]));
+            float *dst = so.a + static_cast<int64_t>(m) * so.I + static_cast<int64_t>(t) * 64 + j0;
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(a[0], a[1], a[2], a[3]);
+            reinterpret_cast<float4 *>(dst)[1] = make_float4(a[4], a[5], a[6], a[7]);
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (act && (lane & 7) == 0)
+            atomicMax(so.amax + m, __float_as_uint(mx));
+    }
+}
+
+template <int NT, int STAGES, int KPS, bool CLUSTER, bool SILU = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX, const float *__restrict__ s_tok,
                        const float *__restrict__ s_ch, int M, int N, int K,
                        uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
                        int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
-                       int prefetch_static, unsigned long long limit_ns)
+                       SiluOut so, int prefetch_static, unsigned long long limit_ns)
 {
     using Cfg = DecodeCfg<NT, STAGES, KPS, CLUSTER>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -962,13 +1091,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 } else {
                     // whole or owned block: copy the staged tile out, 16 bytes per thread
                     named_bar_sync(1, 128);
-                    const int nvalid = min(kBM, N - static_cast<int>(sg.t * kBM));
-                    for (int v = etid; v < mt * 16; v += 128) {
-                        const int m = v >> 4, cv = v & 15;
-                        if (cv * 8 < nvalid)
-                            *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(m) * N +
-                                                       sg.t * kBM + cv * 8) =
-                                *reinterpret_cast<const uint4 *>(ysm + m * kBM + cv * 8);
+                    if constexpr (SILU) {
+                        silu_block_rows(0, mt, static_cast<int>(sg.t), etid, so,
+                                        [&](int m, int j0, float (&g)[8], float (&u)[8]) {
+                                            unpack8(*reinterpret_cast<const uint4 *>(ysm + m * kBM + j0), g);
+                                            unpack8(*reinterpret_cast<const uint4 *>(ysm + m * kBM + 64 + j0), u);
+                                        });
+                    } else {
+                        const int nvalid = min(kBM, N - static_cast<int>(sg.t * kBM));
+                        for (int v = etid; v < mt * 16; v += 128) {
+                            const int m = v >> 4, cv = v & 15;
+                            if (cv * 8 < nvalid)
+                                *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(m) * N +
+                                                           sg.t * kBM + cv * 8) =
+                                    *reinterpret_cast<const uint4 *>(ysm + m * kBM + cv * 8);
+                        }
                     }
                     named_bar_sync(1, 128);
                     if (owner && etid == 0) // ready for the next call
@@ -1002,7 +1139,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                              map_peer_smem(bar_red, q));
             }
         }
-        if (warp >= 2 && mbar_wait(bar_red, 0, limit_ns)) {
+        if constexpr (SILU) {
+            // warp-uniform: the token maxima are reduced with shuffles
+            if (warp >= 2 && __all_sync(0xffffffffu, mbar_wait(bar_red, 0, limit_ns))) {
+                const int etid = threadIdx.x - 64;
+                const int t = static_cast<int>(blockIdx.y);
+                const int32_t *P = reinterpret_cast<const int32_t *>(smem);
+                // this CTA's tokens only: rows m0 .. m1 - 1 of the summed tile
+                silu_block_rows(static_cast<int>(m0), static_cast<int>(m1 - m0), t, etid, so,
+                                [&](int m, int j0, float (&g)[8], float (&u)[8]) {
+                                    const float st = sh_stok[m];
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i) {
+                                        const int ng = t * kBM + j0 + i, nu = ng + 64;
+                                        g[i] = bf16_round(dequant_f32(P[m * kBM + j0 + i], st, __ldg(s_ch + ng)));
+                                        u[i] = bf16_round(dequant_f32(P[m * kBM + 64 + j0 + i], st, __ldg(s_ch + nu)));
+                                    }
+                                });
+            }
+        } else if (warp >= 2 && mbar_wait(bar_red, 0, limit_ns)) {
             const int etid = threadIdx.x - 64;
             const int64_t t = blockIdx.y;
             const int32_t *P = reinterpret_cast<const int32_t *>(smem);

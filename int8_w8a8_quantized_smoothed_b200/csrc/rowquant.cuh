@@ -561,4 +561,45 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) silu_
     }
 }
 
+// ----------------------------------------------------------------- quantization with a known absmax
+//
+// Second half of the fused SiLU*up path: a (binary32 [M, I], written by the GEMM epilogue)
+// is quantized per token with s = amax[m] / 127, amax[m] being the token's max |a| that the
+// epilogue raised with atomicMax on its bits. Each word is cleared after use, so the words
+// are zero again for the next call.
+
+template <int NCH>
+__global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quantize_f32_rows_kernel(
+    const float *__restrict__ a, unsigned int *__restrict__ amax_words, int I, int M,
+    int8_t *__restrict__ q, float *__restrict__ s_tok)
+{
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // a and the maxima come from the previous kernel
+    const int nvec = I >> 3;
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const float amax = __uint_as_float(__ldcg(amax_words + row));
+        const float4 *ar = reinterpret_cast<const float4 *>(a + row * I);
+        float v[NCH][8];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int vi = c * blockDim.x + threadIdx.x;
+            if (vi < nvec) {
+                const float4 lo = __ldcs(ar + 2 * vi);
+                const float4 hi = __ldcs(ar + 2 * vi + 1);
+                v[c][0] = lo.x; v[c][1] = lo.y; v[c][2] = lo.z; v[c][3] = lo.w;
+                v[c][4] = hi.x; v[c][5] = hi.y; v[c][6] = hi.z; v[c][7] = hi.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    v[c][i] = 0.0f;
+            }
+        }
+        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * I, s_tok + row);
+        __syncthreads(); // every thread has read the word
+        if (threadIdx.x == 0)
+            amax_words[row] = 0u;
+    }
+}
+
 } // namespace w8a8

@@ -274,6 +274,22 @@ int launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int t
                          dim3(threads), 0, st, gu, I, static_cast<int>(M), q, s);
 }
 
+template <int NCH>
+int launch_quantize_f32(const float *a, unsigned int *amax, int64_t M, int I, int8_t *q,
+                        float *s, int threads, int dev, int sms, cudaStream_t st)
+{
+    const void *fn = reinterpret_cast<const void *>(&quantize_f32_rows_kernel<NCH>);
+    if (int rc = ensure_smem(fn, dev, 0))
+        return rc;
+    return launch_kernel(quantize_f32_rows_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
+                         dim3(threads), 0, st, a, amax, I, static_cast<int>(M), q, s);
+}
+
+size_t align16_size(size_t b)
+{
+    return (b + 15) & ~static_cast<size_t>(15);
+}
+
 // ------------------------------------------------------------------ GEMM planning
 
 struct GemmPlan {
@@ -382,22 +398,22 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K)
     return W8A8_OK;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SILU>
 int launch_prefill(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
                    const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
-                   int dev, int num_sms, cudaStream_t st)
+                   const SiluOut &so, int dev, int num_sms, cudaStream_t st)
 {
     using Cfg = PrefillCfg<BN, STAGES>;
-    const void *fn = reinterpret_cast<const void *>(&gemm_prefill_kernel<BN, STAGES>);
+    const void *fn = reinterpret_cast<const void *>(&gemm_prefill_kernel<BN, STAGES, SILU>);
     int rc = ensure_smem(fn, dev, Cfg::kSmemBytes);
     if (rc)
         return rc;
     const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
-    return launch_kernel(gemm_prefill_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads),
+    return launch_kernel(gemm_prefill_kernel<BN, STAGES, SILU>, dim3(grid), dim3(kGemmThreads),
                          Cfg::kSmemBytes, st, ta, tb, s_tok, s_ch, static_cast<int>(M),
-                         static_cast<int>(N), static_cast<int>(K), y, acc, prefetch,
+                         static_cast<int>(N), static_cast<int>(K), y, acc, so, prefetch,
                          kWaitLimitNs);
 }
 
@@ -431,13 +447,13 @@ int pair_clusters(const void *kernel, int smem, int dev, int num_sms)
     return n;
 }
 
-template <int STAGES>
+template <int STAGES, bool SILU>
 int launch_prefill_pair(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
                         const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y,
-                        int32_t *acc, int dev, int num_sms, cudaStream_t st)
+                        int32_t *acc, const SiluOut &so, int dev, int num_sms, cudaStream_t st)
 {
     using Cfg = PairCfg<STAGES>;
-    auto kernel = gemm_prefill_pair_kernel<STAGES>;
+    auto kernel = gemm_prefill_pair_kernel<STAGES, SILU>;
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes);
     if (rc)
         return rc;
@@ -450,7 +466,7 @@ int launch_prefill_pair(const CUtensorMap &ta, const CUtensorMap &tb, const floa
     return launch_kernel_cluster(kernel, dim3(static_cast<unsigned>(2 * pairs)),
                                  dim3(kGemmThreads), Cfg::kSmemBytes, st, 2u, ta, tb, s_tok, s_ch,
                                  static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
-                                 acc, prefetch, kWaitLimitNs);
+                                 acc, so, prefetch, kWaitLimitNs);
 }
 
 // Largest cluster size <= want whose clusters can all be resident at once (one wave).
@@ -492,15 +508,15 @@ int fit_cluster(Kern kernel, int want, int64_t clusters_needed, int smem, int de
     return 1;
 }
 
-template <int NT, int STAGES, int KPS>
+template <int NT, int STAGES, int KPS, bool SILU>
 int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
                   const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
-                  uint16_t *y, int32_t *acc, void *ws, int dev, cudaStream_t st)
+                  uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev, cudaStream_t st)
 {
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
     if (p.variant == 3) {
         using Cfg = DecodeCfg<NT, STAGES, KPS, true>;
-        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true>;
+        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU>;
         if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
             return rc;
         const int64_t NB = (N + kBM - 1) / kBM;
@@ -509,10 +525,11 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
                                      Cfg::kSmemBytes, st, static_cast<unsigned>(S), tw, tx, s_tok,
                                      s_ch, static_cast<int>(M), static_cast<int>(N),
                                      static_cast<int>(K), y, acc, static_cast<int32_t *>(nullptr),
-                                     static_cast<unsigned int *>(nullptr), prefetch, kWaitLimitNs);
+                                     static_cast<unsigned int *>(nullptr), so, prefetch,
+                                     kWaitLimitNs);
     }
     using Cfg = DecodeCfg<NT, STAGES, KPS, false>;
-    auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false>;
+    auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false, SILU>;
     if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
         return rc;
     int32_t *ws_part =
@@ -522,22 +539,59 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
                    : nullptr;
     return launch_kernel(kernel, dim3(p.ctas), dim3(kGemmThreads), Cfg::kSmemBytes, st, tw, tx,
                          s_tok, s_ch, static_cast<int>(M), static_cast<int>(N),
-                         static_cast<int>(K), y, acc, ws_part, ws_flag, prefetch, kWaitLimitNs);
+                         static_cast<int>(K), y, acc, ws_part, ws_flag, so, prefetch,
+                         kWaitLimitNs);
 }
 
 // Decode launch by token tile: (stages, k-blocks per stage) keep ~200 KB of weight and
 // token bytes in flight per SM.
+template <bool SILU>
 int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
                      const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
-                     uint16_t *y, int32_t *acc, void *ws, int dev, cudaStream_t st)
+                     uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev,
+                     cudaStream_t st)
 {
     switch (p.nt) {
-    case 16: return launch_decode<16, 3, 4>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
-    case 32: return launch_decode<32, 5, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
-    case 64: return launch_decode<64, 4, 2>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
-    case 128: return launch_decode<128, 5, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
-    default: return launch_decode<256, 3, 1>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, dev, st);
+    case 16: return launch_decode<16, 3, 4, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 32: return launch_decode<32, 5, 2, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 64: return launch_decode<64, 4, 2, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 128: return launch_decode<128, 5, 1, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    default: return launch_decode<256, 3, 1, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
     }
+}
+
+// The GEMM launch for a plan: plain dequant epilogue (so == nullptr) or the fused SiLU*up
+// epilogue.
+int gemm_run(const int8_t *xq, const float *s_tok, const int8_t *wq, const float *s_ch,
+             int64_t M, int64_t N, int64_t K, uint16_t *y, int32_t *acc_out, void *workspace,
+             const GemmPlan &p, const SiluOut *so, int dev, int sms, cudaStream_t st)
+{
+    const SiluOut none{nullptr, nullptr, 0};
+    if (p.variant == 1) {
+        // tile_n: 128 -> 128 x 128, 256 -> 128 x 256, 512 -> 256 x 256 by a CTA pair
+        const int bn = p.tile_n == 128 ? 128 : p.tile_n == 256 ? 256 : 128;
+        CUtensorMap ta, tb;
+        if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, bn))
+            return W8A8_ERR_CUDA;
+        if (so) {
+            if (p.tile_n == 512)
+                return launch_prefill_pair<6, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, dev, sms, st);
+            if (p.tile_n == 256)
+                return launch_prefill<256, 4, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, dev, sms, st);
+            return launch_prefill<128, 6, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, dev, sms, st);
+        }
+        if (p.tile_n == 512)
+            return launch_prefill_pair<6, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, dev, sms, st);
+        if (p.tile_n == 256)
+            return launch_prefill<256, 4, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, dev, sms, st);
+        return launch_prefill<128, 6, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, dev, sms, st);
+    }
+    CUtensorMap tw, tx;
+    if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
+        return W8A8_ERR_CUDA;
+    if (so)
+        return launch_decode_nt<true>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, *so, dev, st);
+    return launch_decode_nt<false>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, none, dev, st);
 }
 
 } // namespace
@@ -692,6 +746,57 @@ int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *
     }
 }
 
+size_t w8a8_gemm_silu_quant_workspace_size(int64_t M, int64_t I, int64_t K)
+{
+    if (I < 64 || I % 64 != 0 || check_row_shape(M, I) || check_gemm_shape(M, 2 * I, K))
+        return 0;
+    int dev, sms = 148;
+    if (current_device(&dev, &sms))
+        sms = 148;
+    GemmPlan p;
+    if (plan_gemm(M, 2 * I, K, 0, 0, 0, sms, &p))
+        return 0;
+    return align16_size(p.ws_bytes) + align16_size(static_cast<size_t>(M) * 4u);
+}
+
+int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_il,
+                         const float *s_ch_il, int64_t M, int64_t I, int64_t K, float *a,
+                         int8_t *q, float *s_out, void *workspace, size_t workspace_bytes,
+                         w8a8_stream_t stream)
+{
+    if (!xq || !s_tok || !wq_il || !s_ch_il || !a || !q || !s_out)
+        return W8A8_ERR_INVALID_ARG;
+    if (I < 64 || I % 64 != 0)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    int rc = check_gemm_shape(M, 2 * I, K);
+    if (rc || (rc = check_row_shape(M, I)))
+        return rc;
+    if (!aligned16(xq) || !aligned16(wq_il) || !aligned16(s_ch_il) || !aligned16(a) ||
+        !aligned16(q) || (workspace && !aligned16(workspace)))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    GemmPlan p;
+    if ((rc = plan_gemm(M, 2 * I, K, 0, 0, 0, sms, &p)))
+        return rc;
+    const size_t amax_off = align16_size(p.ws_bytes);
+    if (!workspace || workspace_bytes < amax_off + align16_size(static_cast<size_t>(M) * 4u))
+        return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const SiluOut so{a, reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + amax_off),
+                     static_cast<int>(I)};
+    if ((rc = gemm_run(xq, s_tok, wq_il, s_ch_il, M, 2 * I, K, nullptr, nullptr, workspace, p,
+                       &so, dev, sms, st)))
+        return rc;
+    const RowLaunch L = row_launch(I);
+    switch (L.nch) {
+    case 1: return launch_quantize_f32<1>(a, so.amax, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    case 2: return launch_quantize_f32<2>(a, so.amax, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    default: return launch_quantize_f32<4>(a, so.amax, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    }
+}
+
 size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, int ctas,
                                    int tile_n)
 {
@@ -733,22 +838,8 @@ int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
     if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
         return W8A8_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (p.variant == 1) {
-        // tile_n: 128 -> 128 x 128, 256 -> 128 x 256, 512 -> 256 x 256 by a CTA pair
-        const int bn = p.tile_n == 128 ? 128 : p.tile_n == 256 ? 256 : 128;
-        CUtensorMap ta, tb;
-        if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, bn))
-            return W8A8_ERR_CUDA;
-        if (p.tile_n == 512)
-            return launch_prefill_pair<6>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
-        if (p.tile_n == 256)
-            return launch_prefill<256, 4>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
-        return launch_prefill<128, 6>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, dev, sms, st);
-    }
-    CUtensorMap tw, tx;
-    if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
-        return W8A8_ERR_CUDA;
-    return launch_decode_nt(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, dev, st);
+    return gemm_run(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace, p, nullptr, dev, sms,
+                    st);
 }
 
 int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, const float *s_ch,
@@ -878,5 +969,6 @@ extern "C" int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, c
     CUtensorMap tw, tx;
     if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
         return W8A8_ERR_CUDA;
-    return launch_decode_nt(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch, dev, st);
+    return launch_decode_nt<false>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch,
+                                   SiluOut{nullptr, nullptr, 0}, dev, st);
 }

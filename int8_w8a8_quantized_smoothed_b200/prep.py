@@ -79,3 +79,17 @@ def static_activation_scale(x_cal: torch.Tensor, smooth_inv=None) -> float:
         y = y * smooth_inv.float()
     a = y.abs().amax().reshape(1)
     return float((a / torch.tensor([127.0], dtype=torch.float32, device=a.device)).item())
+
+
+def interleave_gate_up(wq: torch.Tensor, s_ch: torch.Tensor):
+    """Row order of the gate|up weight [2I, K] (gate rows 0..I-1, up rows I..2I-1) for
+    ``w8a8_gemm_silu_quant``: blocks of 64 gate rows followed by the 64 up rows of the same
+    channels, so that each 128-row group holds both halves of 64 output channels. A pure
+    permutation of rows (and of their scales)."""
+    N, K = wq.shape
+    I = N // 2
+    if N % 2 or I % 64:
+        raise ValueError("the gate|up weight needs 2I rows with I % 64 == 0")
+    w = wq.view(2, I // 64, 64, K).permute(1, 0, 2, 3).reshape(N, K).contiguous()
+    s = s_ch.view(2, I // 64, 64).permute(1, 0, 2).reshape(N).contiguous()
+    return w, s

@@ -44,6 +44,7 @@ def lib():
         L.oracle_silu.restype = C.c_float
         L.oracle_silu.argtypes = [C.c_float]
         L.oracle_silu_mul_quant.argtypes = [P, I64, I64, P, P, C.c_int]
+        L.oracle_silu_mul.argtypes = [P, I64, I64, P, C.c_int]
         L.oracle_dequant.restype = C.c_uint16
         L.oracle_dequant.argtypes = [C.c_int32, C.c_float, C.c_float]
         L.oracle_gemm_dequant.argtypes = [P, P, P, P, I64, I64, I64, P, P, C.c_int]
@@ -157,6 +158,15 @@ def smooth_rmsnorm_quant(x_bf16, gamma, eps, residual=None, ms_override=None,
     lib().oracle_smooth_rmsnorm_quant(_p(x), _p(r), _p(h), _p(g), float(eps), M, K, _p(q),
                                       _p(s), _p(ms), _p(amb), _p(mo), _p(y), nthreads)
     return dict(q=q, s=s, h=h, ms=ms, ambiguous=amb.astype(bool), y=y)
+
+
+def silu_mul(gate_up_bf16, nthreads=NTHREADS):
+    """a = silu(gate) * up (binary32 [M, I]) of a [M, 2I] gate|up bf16 tensor."""
+    gu = _c(gate_up_bf16, np.uint16)
+    M, I2 = gu.shape
+    a = np.empty((M, I2 // 2), dtype=np.float32)
+    lib().oracle_silu_mul(_p(gu), M, I2 // 2, _p(a), nthreads)
+    return a
 
 
 def silu_mul_quant(gate_up_bf16, nthreads=NTHREADS):

@@ -371,20 +371,23 @@ struct silu_ctx {
     int64_t I;
     int8_t *q;
     float *s;
+    float *a_out;
 };
 
 static void silu_row(void *vctx, int64_t m)
 {
     struct silu_ctx *c = (struct silu_ctx *)vctx;
     const int64_t I = c->I;
-    float *a = (float *)malloc((size_t)I * sizeof(float));
+    float *a = c->a_out ? c->a_out + m * I : (float *)malloc((size_t)I * sizeof(float));
     for (int64_t j = 0; j < I; ++j) {
         float g = oracle_bf16_to_f32(c->gu[m * 2 * I + j]);     /* gate half */
         float u = oracle_bf16_to_f32(c->gu[m * 2 * I + I + j]); /* up half */
         a[j] = oracle_silu(g) * u;
     }
-    oracle_quantize_row_f32(a, I, c->q + m * I, c->s + m);
-    free(a);
+    if (c->q)
+        oracle_quantize_row_f32(a, I, c->q + m * I, c->s + m);
+    if (!c->a_out)
+        free(a);
 }
 
 /*
@@ -395,7 +398,16 @@ static void silu_row(void *vctx, int64_t m)
 int oracle_silu_mul_quant(const uint16_t *gate_up, int64_t M, int64_t I, int8_t *q, float *s,
                           int nthreads)
 {
-    struct silu_ctx c = {gate_up, I, q, s};
+    struct silu_ctx c = {gate_up, I, q, s, NULL};
+    parallel_rows(silu_row, &c, M, nthreads);
+    return 0;
+}
+
+/* The activation alone: a = silu(gate) * up in binary32, [M, I] (what oracle_silu_mul_quant
+ * quantizes). */
+int oracle_silu_mul(const uint16_t *gate_up, int64_t M, int64_t I, float *a, int nthreads)
+{
+    struct silu_ctx c = {gate_up, I, NULL, NULL, a};
     parallel_rows(silu_row, &c, M, nthreads);
     return 0;
 }

@@ -1,0 +1,68 @@
+"""Parity of the fused gate|up GEMM + SiLU(gate)*up + per-token quantization
+(w8a8_gemm_silu_quant) with the oracle's unfused chain: the gate|up GEMM with dequant to bf16,
+then SiLU*up and per-token quantization. a (binary32), the int8 codes and the scales are
+compared bit for bit, on decode shapes (cluster split-K and stream-K kernels) and prefill
+shapes (one-CTA and CTA-pair tile kernels)."""
+import numpy as np
+import pytest
+import torch
+
+import int8_w8a8_quantized_smoothed_b200 as w8
+import oracle
+from int8_w8a8_quantized_smoothed_b200 import prep, synth
+from helpers import dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(M, I, K, seed):
+    xq = synth.int8_codes((M, K), seed)
+    wq = synth.int8_codes((2 * I, K), seed + 1)
+    st = synth.scales(M, seed + 2, 1e-3, 0.5)
+    sc = synth.scales(2 * I, seed + 3, 1e-4, 2e-2)
+    return xq, st, wq, sc
+
+
+def _reference(xq, st, wq, sc):
+    y = oracle.gemm_dequant(xq, st, wq, sc)[0]
+    a = oracle.silu_mul(y)
+    q, s = oracle.silu_mul_quant(y)
+    return a, q, s
+
+
+SHAPES = [(1, 1024, 512), (8, 1024, 4096), (33, 2048, 1024), (64, 2048, 4096), (3, 128, 4112),
+          (8, 5120, 1024), (64, 5120, 512), (100, 5120, 256),
+          (300, 1024, 1024), (129, 512, 400), (1000, 4096, 256)]
+
+
+@pytest.mark.parametrize("M,I,K", SHAPES)
+def test_fused_gate_up_silu_quant_bit_exact(M, I, K):
+    xq, st, wq, sc = _inputs(M, I, K, seed=M + I + K)
+    a_ref, q_ref, s_ref = _reference(xq, st, wq, sc)
+    wq_il, sc_il = prep.interleave_gate_up(dev(wq), dev(sc))
+    ws = w8.Workspace()
+    for _ in range(2):  # the second call checks that the workspace came back zeroed
+        q, s, a = w8.w8a8_gemm_silu_quant(dev(xq), dev(st), wq_il, sc_il, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(a).view(np.uint32), a_ref.view(np.uint32))
+        assert np.array_equal(host(s), s_ref)
+        assert np.array_equal(host(q), q_ref)
+
+
+def test_fused_equals_unfused_gpu_chain():
+    M, I, K = 16, 14336, 4096
+    xq, st, wq, sc = _inputs(M, I, K, 7)
+    y = w8.w8a8_gemm_dequant(dev(xq), dev(st), dev(wq), dev(sc))
+    q0, s0 = w8.w8a8_silu_mul_quant(y)
+    wq_il, sc_il = prep.interleave_gate_up(dev(wq), dev(sc))
+    q1, s1, _ = w8.w8a8_gemm_silu_quant(dev(xq), dev(st), wq_il, sc_il)
+    assert torch.equal(q0, q1) and torch.equal(s0, s1)
+
+
+def test_interleave_is_a_row_permutation():
+    I, K = 192, 32
+    wq = torch.arange(2 * I, dtype=torch.int32).repeat_interleave(K).view(2 * I, K)
+    w, s = prep.interleave_gate_up(wq, torch.arange(2 * I, dtype=torch.float32))
+    order = [*range(0, 64), *range(I, I + 64), *range(64, 128), *range(I + 64, I + 128),
+             *range(128, 192), *range(I + 128, I + 192)]
+    assert w[:, 0].tolist() == order and s.tolist() == [float(v) for v in order]

@@ -464,3 +464,18 @@ def test_static_rejects_nonpositive_scale():
     for bad in (0.0, -1.0):
         with pytest.raises(ValueError):
             oracle.quantize_rows_static(x, bad)
+
+
+def test_silu_mul_is_what_silu_mul_quant_quantizes():
+    gu = synth.normal_bf16((5, 2 * 96), seed=8, std=2.5)
+    a = oracle.silu_mul(gu)
+    g = oracle.bf16_to_f32(gu[:, :96])
+    u = oracle.bf16_to_f32(gu[:, 96:])
+    # element by element: the scalar SiLU (pinned above) times up, one binary32 product
+    for m in range(5):
+        for j in range(0, 96, 7):
+            assert a[m, j] == np.float32(np.float32(oracle.silu(float(g[m, j]))) * u[m, j])
+    q, s = oracle.silu_mul_quant(gu)
+    for m in range(5):
+        q1, s1 = oracle.quantize_row_f32(a[m])
+        assert s1 == s[m] and np.array_equal(q1, q[m])
