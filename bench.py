@@ -234,6 +234,7 @@ class Layer:
         a_o = prep.column_absmax(a_cal)
         a_gu = prep.column_absmax(prep.rmsnorm_calibration(h_cal, g2, EPS))
         self.w = {}
+        self.fused = True
         for i, (name, (N, K)) in enumerate(P.items()):
             wb = synth.weight_device(N, K, seed + 10 + i, device)
             if name == "qkv":
@@ -250,6 +251,8 @@ class Layer:
                 p = dict(wq=wq, s_ch=sch)
             self.w[name] = (p["wq"], p["s_ch"])
             del wb
+        # the gate|up weight in the row order of the fused SiLU*up epilogue
+        self.w_gu_il = prep.interleave_gate_up(*self.w["gate_up"])
         torch.cuda.synchronize()
         # inputs (device) and their pinned host copies for the end-to-end measurement
         self.x = synth.activation_device(M, H, seed + 20, device)
@@ -267,6 +270,7 @@ class Layer:
         self.q3 = torch.empty(M, H, dtype=torch.int8, **e)
         self.s3 = torch.empty(M, dtype=torch.float32, **e)
         self.gu = torch.empty(M, 2 * I, dtype=torch.bfloat16, **e)
+        self.a = torch.empty(M, I, dtype=torch.float32, **e)  # SiLU*up of the fused path
         self.q4 = torch.empty(M, I, dtype=torch.int8, **e)
         self.s4 = torch.empty(M, dtype=torch.float32, **e)
         self.down = torch.empty(M, H, dtype=torch.bfloat16, **e)
@@ -277,8 +281,9 @@ class Layer:
         w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
         w8.w8a8_quantize_rows(self.attn, self.sinv_o, q=self.q2, s_tok=self.s2)
 
-    def chain(self, ws, gemms=True, rows=True):
+    def chain(self, ws, gemms=True, rows=True, fused=None):
         import int8_w8a8_quantized_smoothed_b200 as w8
+        fused = self.fused if fused is None else fused
         if rows:
             w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
         if gemms:
@@ -290,10 +295,17 @@ class Layer:
         if rows:
             w8.w8a8_smooth_rmsnorm_quant(self.o, self.g2f, EPS, residual=self.x, h_out=self.h,
                                          q=self.q3, s_tok=self.s3)
-        if gemms:
-            w8.w8a8_gemm_dequant(self.q3, self.s3, *self.w["gate_up"], y=self.gu, workspace=ws)
-        if rows:
-            w8.w8a8_silu_mul_quant(self.gu, q=self.q4, s_tok=self.s4)
+        if fused:
+            # gate|up GEMM with the SiLU*up epilogue, then its per-token quantization pass
+            if gemms:
+                w8.w8a8_gemm_silu_quant(self.q3, self.s3, *self.w_gu_il, a=self.a, q=self.q4,
+                                        s_out=self.s4, workspace=ws)
+        else:
+            if gemms:
+                w8.w8a8_gemm_dequant(self.q3, self.s3, *self.w["gate_up"], y=self.gu,
+                                     workspace=ws)
+            if rows:
+                w8.w8a8_silu_mul_quant(self.gu, q=self.q4, s_tok=self.s4)
         if gemms:
             w8.w8a8_gemm_dequant(self.q4, self.s4, *self.w["down"], y=self.down, workspace=ws)
 
@@ -374,9 +386,13 @@ def run_ours(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     arch = wl["arch"]
     layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev) for i, M in enumerate(wl["Ms"])]
+    for L in layers:
+        L.fused = not args.unfused
     ws = w8.Workspace(dev)
-    max_ws = max(w8.w8a8_gemm_workspace_size(L.M, N, K) for L in layers
-                 for (N, K) in projections(arch).values())
+    max_ws = max([w8.w8a8_gemm_workspace_size(L.M, N, K) for L in layers
+                  for (N, K) in projections(arch).values()] +
+                 [w8.w8a8_gemm_silu_quant_workspace_size(L.M, arch["I"], arch["H"])
+                  for L in layers])
     ws.get(max_ws)
     # the weights are prepared and synchronized: from here on no kernel writes them, so the
     # GEMMs may stream them ahead of the dependency wait (overlap mode 2)
@@ -387,7 +403,11 @@ def run_ours(args, world, rank, local):
         for L in layers:
             L.chain(ws)
 
-    def step_gemms():
+    def step_gemms():  # the GEMM kernels alone, plain dequant epilogues
+        for L in layers:
+            L.chain(ws, rows=False, fused=False)
+
+    def step_gemms_fused():  # the step's GEMM-type launches incl. the SiLU*up quant pass
         for L in layers:
             L.chain(ws, rows=False)
 
@@ -406,6 +426,7 @@ def run_ours(args, world, rank, local):
     ops = sum(layer_work(arch, L.M)[0] for L in layers)
     nbytes = sum(layer_work(arch, L.M)[1] for L in layers)
     g_bytes = sum(layer_work(arch, L.M)[3] for L in layers)
+
     launches_per_step = 8 * len(layers)
     h2d = sum(L.x.numel() * 2 + L.attn.numel() * 2 for L in layers)
     d2h = sum(L.down.numel() * 2 for L in layers)
@@ -435,6 +456,11 @@ def run_ours(args, world, rank, local):
     gsecs = time_graph(g_gemm, args.steps, args.warmup) / args.steps
     g_rows = capture(step_rows)
     rsecs = time_graph(g_rows, args.steps, args.warmup) / args.steps
+    gfsecs = None
+    if not args.unfused:
+        g_gemm_f = capture(step_gemms_fused)
+        gfsecs = time_graph(g_gemm_f, args.steps, args.warmup) / args.steps
+        del g_gemm_f
     g_e2e = capture(step_e2e)
     esecs = time_graph(g_e2e, args.steps, args.warmup) / args.steps
     e_value, _ = combine(nbytes, esecs, world)
@@ -462,7 +488,8 @@ def run_ours(args, world, rank, local):
                     "frac_of_nominal": round(gemm_tops / INT8_NOMINAL_TOPS, 4),
                     "traffic": None}
     else:
-        roofline = {"kernel": "gemm_decode_kernel (all GEMM launches of the step)",
+        roofline = {"kernel": "gemm_decode_kernel (all GEMM launches of the step, plain "
+                              "dequant epilogues, timed alone as a graph)",
                     "bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": hbm_peak,
                     "unit": "GB/s", "frac": round(gemm_gbs / hbm_peak, 4),
                     "peak_source": f"{peak_src} copy bandwidth (burst)", "traffic": None}
@@ -480,7 +507,9 @@ def run_ours(args, world, rank, local):
                          f"{sum(L.w[n][0].numel() for L in layers for n in L.w) / 1e6:.0f} MB "
                          "of int8 weights (> 126 MB L2)",
                    "timing": "CUDA graph of one step replayed K times, CUDA events",
-                   "overlap": args.overlap},
+                   "overlap": args.overlap,
+                   "silu_mul_quant": ("separate launch" if args.unfused else
+                                      "fused into the gate|up GEMM epilogue + quantization pass")},
         "tops": round(ops / t_max / 1e12, 3),
         "roofline_step": {"t_roof_us": round(t_roof * 1e6, 2),
                           "t_us": round(t_max * 1e6, 2), "frac": round(t_roof / t_max, 4),
@@ -489,7 +518,12 @@ def run_ours(args, world, rank, local):
         "int8_peak_tops_measured": round(int8_peak, 1),
         "roofline": roofline,
         "breakdown_us": {"step": round(t_max * 1e6, 2), "gemms": round(gsecs * 1e6, 2),
-                         "row_kernels": round(rsecs * 1e6, 2)},
+                         "row_kernels": round(rsecs * 1e6, 2),
+                         **({"gemms_with_fused_silu_and_quant_pass": round(gfsecs * 1e6, 2)}
+                            if gfsecs is not None else {}),
+                         "note": "gemms: plain epilogues; row_kernels: the step's row "
+                                 "launches" + ("" if args.unfused else
+                                               " (SiLU*up is fused into the gate|up GEMM)")},
         "e2e": {"value": round(e_value / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(esecs * 1e3, 5),
@@ -671,6 +705,9 @@ def main(argv=None):
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if measured")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="gate|up GEMM and SiLU*up+quant as separate launches instead of the "
+                         "fused SiLU*up epilogue")
     ap.add_argument("--overlap", type=int, choices=[0, 1, 2], default=2,
                     help="kernel overlap mode (w8a8_set_overlap); 2 = dependent launch with "
                          "static-weight prefetch")
