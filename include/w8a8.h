@@ -271,6 +271,15 @@ W8A8_API int w8a8_get_overlap(void);
  */
 W8A8_API int w8a8_device_status(int reset);
 
+/*
+ * Self-test of the failure path (no counterpart on the pages): launches one small kernel
+ * whose two waits -- on an mbarrier and on a global flag that nothing ever sets -- each give
+ * up after limit_ns nanoseconds (1e3 <= limit_ns <= 2e9, else W8A8_ERR_INVALID_ARG). The
+ * kernel then raises the device status word and returns, so the next w8a8_device_status()
+ * reports W8A8_ERR_TIMEOUT while the context stays usable. No fault, trap or hang is involved.
+ */
+W8A8_API int w8a8_selftest_wait_timeout(unsigned long long limit_ns, w8a8_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 W8A8_API const char *w8a8_status_string(int status);
 

@@ -20,7 +20,7 @@ __all__ = [
     "w8a8_quantize_rows", "w8a8_quantize_rows_static", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
     "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_gemm_silu_quant",
-    "w8a8_gemm_silu_quant_workspace_size", "w8a8_probe_i8_mma", "w8a8_set_overlap",
+    "w8a8_gemm_silu_quant_workspace_size", "w8a8_probe_i8_mma", "w8a8_selftest_wait_timeout", "w8a8_set_overlap",
     "w8a8_get_overlap", "w8a8_device_status",
     "w8a8_status_string", "w8a8_version",
     "Workspace",
@@ -48,6 +48,7 @@ SIGNATURES = [
     ("w8a8_gemm_silu_quant_workspace_size", _SZ, [_I64, _I64, _I64]),
     ("w8a8_gemm_silu_quant", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     ("w8a8_probe_i8_mma", _I, [C.c_longlong, _I, _I, _P]),
+    ("w8a8_selftest_wait_timeout", _I, [C.c_ulonglong, _P]),
     ("w8a8_set_overlap", _I, [_I]),
     ("w8a8_get_overlap", _I, []),
     ("w8a8_device_status", _I, [_I]),
@@ -119,6 +120,13 @@ def w8a8_status_string(status: int) -> str:
 
 def w8a8_version() -> int:
     return lib().w8a8_version()
+
+
+def w8a8_selftest_wait_timeout(limit_ns: int = 5_000_000, stream=None) -> None:
+    """Launch the failure-path self-test: two waits that nothing satisfies give up after
+    limit_ns; the next w8a8_device_status() reports W8A8_ERR_TIMEOUT."""
+    _check("w8a8_selftest_wait_timeout",
+           lib().w8a8_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def w8a8_probe_i8_mma(iters: int, n: int = 256, ctas: int = 0, stream=None) -> None:

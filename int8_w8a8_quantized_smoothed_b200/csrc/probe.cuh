@@ -1,3 +1,5 @@
+// Measurement and self-test aids (not part of the W8A8 path).
+//
 // Tensor-core throughput probe: measures the dense INT8 rate of tcgen05.mma kind::i8 on this
 // device, the denominator of the GEMM roofline. One CTA per SM; one thread issues `iters`
 // back-to-back 128 x N x 32 MMAs on zero-filled shared-memory operands into a TMEM
@@ -49,6 +51,34 @@ __global__ void __launch_bounds__(128, 1) mma_i8_probe_kernel(long long iters,
     if (threadIdx.x < 32) {
         tc_fence_after();
         tmem_dealloc(tmem, kCols);
+    }
+}
+
+// Failure-path self-test: one CTA whose waits can never be satisfied -- thread 0 on an
+// mbarrier nobody arrives at, thread 32 on a flag word nobody sets -- each bounded by
+// limit_ns, so both give up, raise the device status word and return. Shows that a wait that
+// runs out ends the kernel cleanly and leaves the context usable.
+__device__ unsigned int g_never_set_flag;
+
+__global__ void __launch_bounds__(64, 1) wait_timeout_selftest_kernel(unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        mbar_wait(smem_u32(&bar), 0, limit_ns); // flags the timeout itself
+    if (threadIdx.x == 32) {
+        const volatile unsigned int *f = &g_never_set_flag;
+        const uint64_t t0 = globaltimer_ns();
+        while (*f == 0u) {
+            if (globaltimer_ns() - t0 > limit_ns) {
+                flag_timeout();
+                break;
+            }
+        }
     }
 }
 

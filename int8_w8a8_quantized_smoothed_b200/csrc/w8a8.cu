@@ -882,6 +882,20 @@ int w8a8_get_overlap(void)
     return g_overlap.load();
 }
 
+int w8a8_selftest_wait_timeout(unsigned long long limit_ns, w8a8_stream_t stream)
+{
+    if (limit_ns < 1000ull || limit_ns > 2000000000ull)
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    wait_timeout_selftest_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+    if (cudaGetLastError() != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    return W8A8_OK;
+}
+
 int w8a8_device_status(int reset)
 {
     int dev, sms;

@@ -240,3 +240,18 @@ def test_static_scale_calibration_matches_oracle():
     S = prep.static_activation_scale(dev_bf16(cal), dev(sinv))
     ref = oracle.minmax_scale((oracle.bf16_to_f32(cal) * sinv).astype(np.float32))
     assert np.float32(S) == ref
+
+
+def test_wait_timeout_reports_status_and_context_stays_usable():
+    # a wait that nothing satisfies gives up after its limit, raises the status word and the
+    # kernel returns; afterwards the context runs kernels normally
+    assert w8.w8a8_device_status(reset=True) == 0
+    w8.w8a8_selftest_wait_timeout(2_000_000)  # 2 ms
+    assert w8.w8a8_device_status(reset=True) == -6  # W8A8_ERR_TIMEOUT
+    assert w8.w8a8_device_status(reset=False) == 0
+    x = synth.activation(4, 256, 3)
+    q_ref, s_ref = oracle.quantize_rows(x)
+    q, s = w8.w8a8_quantize_rows(dev_bf16(x))
+    assert np.array_equal(host(q), q_ref) and np.array_equal(host(s), s_ref)
+    with pytest.raises(w8.W8A8Error):
+        w8.w8a8_selftest_wait_timeout(10)  # below the allowed range
