@@ -163,7 +163,8 @@ W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_
 /*
  * The same GEMM with the kernel chosen by the caller, for tests and tuning:
  * variant 0 = automatic (as w8a8_gemm_dequant), 1 = persistent tile kernel, 2 = swap-AB
- * stream-K kernel, 3 = swap-AB cluster split-K kernel (2 and 3: M <= 256 only). ctas:
+ * stream-K kernel, 3 = swap-AB cluster split-K kernel (2 and 3: M <= 1024; beyond 256 tokens
+ * the tokens are taken 256 at a time, each channel block once per such tile). ctas:
  * variant 2 = persistent CTAs sharing the weight stream (0 = one per SM, at most one per SM);
  * variant 3 = cluster size, the number of K splits per 128-channel block (0 = automatic,
  * at most 8, fewer if the clusters would not all fit on the GPU at once). tile_n (variant 1)

@@ -663,6 +663,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   stores and
 //   lowers the flags so the workspace is ready for the next call.
 
+// Token tiles per launch of the swap-AB kernel: M <= kDecodeMaxTiles * NT. Each channel block
+// is computed once per token tile (tile tt holds tokens tt NT .. tt NT + NT - 1); a block's
+// consecutive units walk its token tiles first, so the weight rows re-read for the second
+// tile come from L2.
+constexpr int kDecodeMaxTiles = 4;
+
 template <int NT, int STAGES, int KPS, bool CLUSTER> struct DecodeCfg {
     static constexpr int kWBytes = kBM * kBK;  // one k-block of 128 weight rows
     static constexpr int kXBytes = NT * kBK;   // one k-block of NT token rows
@@ -670,8 +676,8 @@ template <int NT, int STAGES, int KPS, bool CLUSTER> struct DecodeCfg {
     // stream-K stages its bf16 output tile [NT][128] for coalesced stores
     static constexpr int kYBytes = CLUSTER ? 0 : NT * kBM * 2;
     static constexpr int kYOff = STAGES * kStageBytes;
-    static constexpr int kStokOff = kYOff + kYBytes; // fp32 token scales [NT]
-    static constexpr int kBarOff = kStokOff + NT * 4;
+    static constexpr int kStokOff = kYOff + kYBytes; // fp32 token scales [tiles * NT]
+    static constexpr int kBarOff = kStokOff + kDecodeMaxTiles * NT * 4;
     // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot, flag word, then the
     // cluster reduction barrier
     static constexpr int kRedBarOff = kBarOff + (2 * STAGES + 4) * 8 + 32;
@@ -696,7 +702,7 @@ __host__ __device__ __forceinline__ int64_t sk_owner_of(int64_t v, int64_t U, in
 }
 
 struct SkSegment {
-    int64_t t;    // channel block
+    int64_t t;    // block: channel block t / tiles, token tile t % tiles
     int kb0, kb1; // k-block range [kb0, kb1)
 };
 
@@ -776,7 +782,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int KB = (K + kBK - 1) / kBK;
-    const int64_t NB = (N + kBM - 1) / kBM;
+    const int TT = (M + NT - 1) / NT;                  // token tiles
+    const int64_t NB = ((N + kBM - 1) / kBM) * TT;     // blocks: (channel block, token tile)
     const int64_t U = NB * KB;
     const int64_t G = gridDim.x;
     const int64_t g = blockIdx.x;
@@ -831,7 +838,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         for (int j = 0; j < nk; ++j)
                             tma_load_2d_hint(sW + (npre * KPS + j) * Cfg::kWBytes, &tmW,
                                              bar_full + 8 * npre, (kb + j) * kBK,
-                                             static_cast<int32_t>(sg.t * kBM), pol_w);
+                                             static_cast<int32_t>((sg.t / TT) * kBM), pol_w);
                     }
                     u += sg.kb1 - sg.kb0;
                 }
@@ -844,10 +851,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int kb = sg.kb0; kb < sg.kb1; kb += KPS, ++it) {
                     const int nk = min(KPS, sg.kb1 - kb);
                     const uint32_t s = it % STAGES;
+                    const int32_t xrow = static_cast<int32_t>((sg.t % TT) * NT);
                     if (it < npre) { // weights already requested; add the token tiles
                         for (int j = 0; j < nk; ++j)
                             tma_load_2d(sX + (s * KPS + j) * Cfg::kXBytes, &tmX, bar_full + 8 * s,
-                                        (kb + j) * kBK, 0);
+                                        (kb + j) * kBK, xrow);
                         continue;
                     }
                     const uint32_t ph = (it / STAGES) & 1u;
@@ -858,9 +866,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     mbar_expect_tx(bar_full + 8 * s, nk * (Cfg::kWBytes + Cfg::kXBytes));
                     for (int j = 0; j < nk; ++j) {
                         tma_load_2d_hint(sW + (s * KPS + j) * Cfg::kWBytes, &tmW, bar_full + 8 * s,
-                                         (kb + j) * kBK, static_cast<int32_t>(sg.t * kBM), pol_w);
+                                         (kb + j) * kBK, static_cast<int32_t>((sg.t / TT) * kBM),
+                                         pol_w);
                         tma_load_2d(sX + (s * KPS + j) * Cfg::kXBytes, &tmX, bar_full + 8 * s,
-                                    (kb + j) * kBK, 0);
+                                    (kb + j) * kBK, xrow);
                     }
                 }
                 u += sg.kb1 - sg.kb0;
@@ -918,8 +927,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int i = etid; i < M; i += 128)
             sh_stok[i] = __ldg(s_tok + i);
         named_bar_sync(1, 128);
-        const int mt = M < NT ? M : NT; // tokens held in the accumulator
-        const int Mp = (M + 3) & ~3;    // tokens per partial row in the workspace
+        // tokens of block b's tile held in the accumulator (tile b % TT)
+        auto tile_tokens = [&](int64_t b) {
+            const int rest = M - static_cast<int>(b % TT) * NT;
+            return rest < NT ? rest : NT;
+        };
+        const int Mp = ((M < NT ? M : NT) + 3) & ~3; // tokens per partial row in the workspace
         // an owner's contributor sums, per token of its channel (small token tiles only)
         constexpr int kPre = (!CLUSTER && NT <= 64) ? NT : 0;
         int32_t pre[kPre > 0 ? kPre : 1];
@@ -957,6 +970,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             named_bar_sync(1, 128);
             const bool all_ok = *sh_word != 0u;
             if constexpr (kPre > 0) {
+                const int mt = tile_tokens(own_t);
 #pragma unroll
                 for (int j = 0; j < kPre; ++j)
                     pre[j] = 0;
@@ -987,7 +1001,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // a segment is a whole block, the owned start of a split block, or a contribution
             const bool owner = !CLUSTER && sg.t == own_t && sg.kb0 == 0;
             const bool contrib = !CLUSTER && sg.kb0 > 0;
-            const int n = static_cast<int>(sg.t * kBM) + r;
+            const int64_t tch = sg.t / TT;                 // channel block
+            const int mbase = static_cast<int>(sg.t % TT) * NT; // first token of the tile
+            const int mt = tile_tokens(sg.t);
+            const int n = static_cast<int>(tch * kBM) + r;
             const bool n_ok = n < N;
             const float sc = n_ok ? __ldg(s_ch + n) : 0.0f;
             if (own_t >= 0 && !fetched && (seg >= 1 || owner)) {
@@ -1058,10 +1075,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int m = c0 + j;
                     if (m < mt) {
                         const int32_t v = static_cast<int32_t>(a[j]);
-                        ysm[m * kBM + r] =
-                            static_cast<uint16_t>(bf16_bits(dequant_f32(v, sh_stok[m], sc)));
+                        ysm[m * kBM + r] = static_cast<uint16_t>(
+                            bf16_bits(dequant_f32(v, sh_stok[mbase + m], sc)));
                         if (acc_out && n_ok)
-                            acc_out[static_cast<int64_t>(m) * N + n] = v;
+                            acc_out[static_cast<int64_t>(mbase + m) * N + n] = v;
                     }
                 }
             };
@@ -1092,18 +1109,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     // whole or owned block: copy the staged tile out, 16 bytes per thread
                     named_bar_sync(1, 128);
                     if constexpr (SILU) {
-                        silu_block_rows(0, mt, static_cast<int>(sg.t), etid, so,
+                        silu_block_rows(mbase, mt, static_cast<int>(tch), etid, so,
                                         [&](int m, int j0, float (&g)[8], float (&u)[8]) {
-                                            unpack8(*reinterpret_cast<const uint4 *>(ysm + m * kBM + j0), g);
-                                            unpack8(*reinterpret_cast<const uint4 *>(ysm + m * kBM + 64 + j0), u);
+                                            const uint16_t *row = ysm + (m - mbase) * kBM;
+                                            unpack8(*reinterpret_cast<const uint4 *>(row + j0), g);
+                                            unpack8(*reinterpret_cast<const uint4 *>(row + 64 + j0), u);
                                         });
                     } else {
-                        const int nvalid = min(kBM, N - static_cast<int>(sg.t * kBM));
+                        const int nvalid = min(kBM, N - static_cast<int>(tch * kBM));
                         for (int v = etid; v < mt * 16; v += 128) {
                             const int m = v >> 4, cv = v & 15;
                             if (cv * 8 < nvalid)
-                                *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(m) * N +
-                                                           sg.t * kBM + cv * 8) =
+                                *reinterpret_cast<uint4 *>(y + static_cast<int64_t>(mbase + m) * N +
+                                                           tch * kBM + cv * 8) =
                                     *reinterpret_cast<const uint4 *>(ysm + m * kBM + cv * 8);
                         }
                     }
@@ -1123,7 +1141,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // barrier; q then dequantizes its rows.
         const uint32_t S = gridDim.x;
         const uint32_t rank = cluster_ctarank();
-        const uint32_t mt = static_cast<uint32_t>(M < NT ? M : NT);
+        const int64_t blk = blockIdx.y;
+        const int tch = static_cast<int>(blk / TT);             // channel block
+        const int mbase = static_cast<int>(blk % TT) * NT;      // first token of the tile
+        const uint32_t mt = static_cast<uint32_t>(M - mbase < NT ? M - mbase : NT);
         const uint32_t m0 = (rank * mt) / S, m1 = ((rank + 1) * mt) / S;
         constexpr uint32_t kRowBytes = kBM * 4;
         if (threadIdx.x == 64)
@@ -1143,32 +1164,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // warp-uniform: the token maxima are reduced with shuffles
             if (warp >= 2 && __all_sync(0xffffffffu, mbar_wait(bar_red, 0, limit_ns))) {
                 const int etid = threadIdx.x - 64;
-                const int t = static_cast<int>(blockIdx.y);
                 const int32_t *P = reinterpret_cast<const int32_t *>(smem);
                 // this CTA's tokens only: rows m0 .. m1 - 1 of the summed tile
-                silu_block_rows(static_cast<int>(m0), static_cast<int>(m1 - m0), t, etid, so,
-                                [&](int m, int j0, float (&g)[8], float (&u)[8]) {
+                silu_block_rows(mbase + static_cast<int>(m0), static_cast<int>(m1 - m0), tch,
+                                etid, so, [&](int m, int j0, float (&g)[8], float (&u)[8]) {
                                     const float st = sh_stok[m];
+                                    const int32_t *row = P + (m - mbase) * kBM;
 #pragma unroll
                                     for (int i = 0; i < 8; ++i) {
-                                        const int ng = t * kBM + j0 + i, nu = ng + 64;
-                                        g[i] = bf16_round(dequant_f32(P[m * kBM + j0 + i], st, __ldg(s_ch + ng)));
-                                        u[i] = bf16_round(dequant_f32(P[m * kBM + 64 + j0 + i], st, __ldg(s_ch + nu)));
+                                        const int ng = tch * kBM + j0 + i, nu = ng + 64;
+                                        g[i] = bf16_round(dequant_f32(row[j0 + i], st, __ldg(s_ch + ng)));
+                                        u[i] = bf16_round(dequant_f32(row[64 + j0 + i], st, __ldg(s_ch + nu)));
                                     }
                                 });
             }
         } else if (warp >= 2 && mbar_wait(bar_red, 0, limit_ns)) {
             const int etid = threadIdx.x - 64;
-            const int64_t t = blockIdx.y;
             const int32_t *P = reinterpret_cast<const int32_t *>(smem);
             // 4 channels per thread per row: 16-byte tile reads, 8-byte output stores
             const int nv = static_cast<int>(m1 - m0) * (kBM / 4);
             for (int v = etid; v < nv; v += 128) {
-                const int m = static_cast<int>(m0) + v / (kBM / 4);
+                const int ml = static_cast<int>(m0) + v / (kBM / 4); // token within the tile
+                const int m = mbase + ml;
                 const int c = (v % (kBM / 4)) * 4;
-                const int n = static_cast<int>(t * kBM) + c;
+                const int n = tch * kBM + c;
                 if (n < N) { // N % 8 == 0: the 4 channels are all valid or all past N
-                    const int4 s4 = *reinterpret_cast<const int4 *>(P + m * kBM + c);
+                    const int4 s4 = *reinterpret_cast<const int4 *>(P + ml * kBM + c);
                     const float4 c4 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
                     const float st = sh_stok[m];
                     uint2 o;

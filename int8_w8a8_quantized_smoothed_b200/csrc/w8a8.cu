@@ -326,7 +326,7 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
         else // few channel blocks: split K inside clusters; many: stream-K over all SMs
             variant = (2 * NB <= num_sms && KB >= 2) ? 3 : 2;
     }
-    if ((variant == 2 || variant == 3) && M > 256)
+    if ((variant == 2 || variant == 3) && M > kDecodeMaxTiles * 256)
         return W8A8_ERR_UNSUPPORTED_SHAPE;
     p->variant = variant;
     if (variant == 1) {
@@ -355,8 +355,9 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
         return W8A8_OK;
     }
     p->nt = decode_nt(M);
+    const int64_t TT = (M + p->nt - 1) / p->nt; // token tiles (M > 256: tiles of 256)
     if (variant == 3) {
-        int64_t S = ctas > 0 ? ctas : num_sms / NB;
+        int64_t S = ctas > 0 ? ctas : num_sms / (NB * TT);
         S = S < 1 ? 1 : S;
         S = S > kMaxClusterSize ? kMaxClusterSize : S;
         S = S > KB ? KB : S;
@@ -364,7 +365,7 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
         p->ws_bytes = 0;
         return W8A8_OK;
     }
-    const int64_t U = NB * KB;
+    const int64_t U = NB * TT * KB;
     // every CTA must be resident at once (owners wait on later CTAs): at most one per SM
     int64_t G = (ctas == 0 || ctas > num_sms) ? num_sms : ctas;
     if (G > U)
@@ -379,7 +380,7 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
     if (split) {
         // flag words first, at a fixed place whatever the shape (they are the only part that
         // must be zero when a call starts); partial slots after them
-        const int64_t Mp = (M + 3) & ~static_cast<int64_t>(3);
+        const int64_t Mp = ((M < p->nt ? M : p->nt) + 3) & ~static_cast<int64_t>(3);
         p->flag_off = 0;
         p->part_off = kFlagBytes;
         p->ws_bytes = kFlagBytes + static_cast<size_t>(G) * kBM * static_cast<size_t>(Mp) * 4u;
@@ -519,7 +520,7 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
         auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU>;
         if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
             return rc;
-        const int64_t NB = (N + kBM - 1) / kBM;
+        const int64_t NB = ((N + kBM - 1) / kBM) * ((M + NT - 1) / NT); // x token tiles
         const int S = fit_cluster(kernel, p.ctas, NB, Cfg::kSmemBytes, dev);
         return launch_kernel_cluster(kernel, dim3(S, static_cast<unsigned>(NB)), dim3(kGemmThreads),
                                      Cfg::kSmemBytes, st, static_cast<unsigned>(S), tw, tx, s_tok,

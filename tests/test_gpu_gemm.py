@@ -68,6 +68,19 @@ def test_decode_cluster_kernel_bit_exact(M, N, K, cluster):
     _compare(y, acc, y_ref, acc_ref)
 
 
+# beyond 256 tokens the swap-AB kernels take the tokens in tiles of 256 (ragged last tile)
+MULTI_TILE_SHAPES = [(300, 512, 1024), (512, 384, 4096), (777, 1024, 512), (1024, 256, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", MULTI_TILE_SHAPES)
+@pytest.mark.parametrize("variant,ctas", [(2, 0), (2, 5), (3, 0), (3, 3)])
+def test_decode_kernels_multi_token_tile_bit_exact(M, N, K, variant, ctas):
+    xq, st, wq, sc = _inputs(M, N, K, seed=5 * M + N + K)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    y, acc = _run(xq, st, wq, sc, variant=variant, ctas=ctas)
+    _compare(y, acc, y_ref, acc_ref)
+
+
 PREFILL_SHAPES = [(1, 8, 16), (16, 512, 256), (128, 256, 128), (129, 264, 400), (200, 136, 208),
                   (300, 1024, 4096), (512, 2048, 1024), (257, 520, 14336), (1000, 3000, 64)]
 
