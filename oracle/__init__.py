@@ -34,6 +34,14 @@ def lib():
         L.oracle_f32_to_bf16.argtypes = [C.c_float]
         L.oracle_quantize_row_f32.argtypes = [P, I64, P, P]
         L.oracle_quantize_rows.argtypes = [P, P, I64, I64, P, P, C.c_int]
+        L.oracle_e4m3_to_f32.restype = C.c_float
+        L.oracle_e4m3_to_f32.argtypes = [C.c_uint8]
+        L.oracle_f32_to_e4m3.restype = C.c_uint8
+        L.oracle_f32_to_e4m3.argtypes = [C.c_float]
+        L.oracle_quantize_row_f32_fp8.argtypes = [P, I64, P, P]
+        L.oracle_quantize_rows_fp8.argtypes = [P, P, I64, I64, P, P, C.c_int]
+        L.oracle_quantize_rows_f32_fp8.argtypes = [P, I64, I64, P, P, C.c_int]
+        L.oracle_gemm_fp8.argtypes = [P, P, P, P, I64, I64, I64, P, P, P]
         L.oracle_minmax_scale.restype = C.c_float
         L.oracle_minmax_scale.argtypes = [P, I64]
         L.oracle_quantize_rows_static.argtypes = [P, P, C.c_float, I64, I64, P, C.c_int]
@@ -121,6 +129,80 @@ def quantize_rows(x_bf16, sinv=None, nthreads=NTHREADS):
     s = np.empty(M, dtype=np.float32)
     lib().oracle_quantize_rows(_p(x), _p(sinv), M, K, _p(q), _p(s), nthreads)
     return q, s
+
+
+def e4m3_to_f32(b: int) -> float:
+    return lib().oracle_e4m3_to_f32(int(b))
+
+
+def f32_to_e4m3(v: float) -> int:
+    return int(lib().oracle_f32_to_e4m3(float(v)))
+
+
+def quantize_row_f32_fp8(y):
+    y = _c(y, np.float32)
+    q = np.empty(y.shape[-1], dtype=np.uint8)
+    s = np.zeros(1, dtype=np.float32)
+    lib().oracle_quantize_row_f32_fp8(_p(y), y.shape[-1], _p(q), _p(s))
+    return q, s[0]
+
+
+def quantize_rows_fp8(x_bf16, sinv=None, nthreads=NTHREADS):
+    """Per-token FP8 (E4M3) quantization -> (codes uint8 [M, K], scales float32 [M])."""
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    sinv = _c(sinv, np.float32)
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty(M, dtype=np.float32)
+    lib().oracle_quantize_rows_fp8(_p(x), _p(sinv), M, K, _p(q), _p(s), nthreads)
+    return q, s
+
+
+def quantize_rows_f32_fp8(y, nthreads=NTHREADS):
+    """Per-row FP8 quantization of fp32 rows -> (codes uint8 [M, K], scales float32 [M])."""
+    y = _c(y, np.float32)
+    M, K = y.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty(M, dtype=np.float32)
+    lib().oracle_quantize_rows_f32_fp8(_p(y), M, K, _p(q), _p(s), nthreads)
+    return q, s
+
+
+def smooth_rmsnorm_quant_fp8(x_bf16, gamma, eps, residual=None, ms_override=None,
+                             nthreads=NTHREADS):
+    """The smoothed RMSNorm of ``smooth_rmsnorm_quant`` with FP8 per-token quantization."""
+    r = smooth_rmsnorm_quant(x_bf16, gamma, eps, residual=residual, ms_override=ms_override,
+                             want_y=True, quantize=False, nthreads=nthreads)
+    r["q"], r["s"] = quantize_rows_f32_fp8(r["y"], nthreads)
+    return r
+
+
+def silu_mul_quant_fp8(gate_up_bf16, nthreads=NTHREADS):
+    """silu(gate) * up with FP8 per-token quantization -> (codes, scales)."""
+    return quantize_rows_f32_fp8(silu_mul(gate_up_bf16, nthreads), nthreads)
+
+
+def rtn_weights_fp8(w_bf16, s=None, nthreads=NTHREADS):
+    """FP8 round-to-nearest weights: rows (output channels) of W * diag(s) quantized to E4M3
+    with per-channel scales absmax / 448 -> (codes uint8 [N, K], s_ch float32 [N])."""
+    w = _c(w_bf16, np.uint16)
+    v = smooth_weight(w, s) if s is not None else bf16_to_f32(w)
+    return quantize_rows_f32_fp8(v, nthreads)
+
+
+def gemm_fp8(xq, s_tok, wq, s_ch):
+    """FP8 GEMM reference -> (y bf16 bits [M, N], exact acc float64, sum |products| float64)."""
+    xq = _c(xq, np.uint8)
+    wq = _c(wq, np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    st = _c(s_tok, np.float32)
+    sc = _c(s_ch, np.float32)
+    acc = np.empty((M, N), dtype=np.float64)
+    absacc = np.empty((M, N), dtype=np.float64)
+    y = np.empty((M, N), dtype=np.uint16)
+    lib().oracle_gemm_fp8(_p(xq), _p(st), _p(wq), _p(sc), M, N, K, _p(acc), _p(absacc), _p(y))
+    return y, acc, absacc
 
 
 def minmax_scale(values_f32):

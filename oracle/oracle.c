@@ -25,7 +25,13 @@
  *        "1. Min-Max Calibration" -- S = max(|min|,|max|)/127, range [-127, 127].
  *   [P4] "W8A8 ... accuracy and serving results" (Red Hat developer article), section
  *        "Inter-token latency (ITL)" -- per layer: measure the range, compute a scale,
- *        convert to INT8, multiply, convert back to BF16.
+ *        convert to INT8, multiply, convert back to BF16; "When W8A8 INT8 quantization is a
+ *        good fit" and "What to explore next" -- W8A8 FP8 as the variant for Hopper and
+ *        Blackwell GPUs.
+ *   [P5] "05 Quantization AWQ GPTQ FP8", section "Ladder" -- FP8 as the near-lossless
+ *        8-bit step. Neither page fixes the FP8 encoding; the FP8 functions take the OCP
+ *        E4M3 format with per-token / per-channel scales absmax / 448 (the largest E4M3
+ *        value), the analogue of the INT8 scales absmax / 127.
  */
 #include <math.h>
 #include <pthread.h>
@@ -229,6 +235,161 @@ int oracle_quantize_rows_static(const uint16_t *x, const float *sinv, float S, i
         return -1;
     struct qstatic_ctx c = {x, sinv, S, K, q};
     parallel_rows(qstatic_row, &c, M, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------ FP8 (E4M3) variant */
+
+/*
+ * OCP 8-bit floating point E4M3 (the "FN" form: no infinities, S.1111.111 is NaN): sign, 4
+ * exponent bits (bias 7), 3 fraction bits. Normal values 2^(e-7) (1 + f/8), e = 1..15;
+ * subnormals 2^-6 (f/8); largest finite 448. Encoding rounds to nearest, ties to even, and
+ * saturates to +-448 (the conversion used for W8A8 FP8 codes).
+ */
+float oracle_e4m3_to_f32(uint8_t b)
+{
+    const int sign = b >> 7, e = (b >> 3) & 15, f = b & 7;
+    if (e == 15 && f == 7)
+        return NAN;
+    const double v = e == 0 ? ldexp((double)f, -9) : ldexp(8.0 + f, e - 10);
+    return (float)(sign ? -v : v);
+}
+
+uint8_t oracle_f32_to_e4m3(float v)
+{
+    if (v != v)
+        return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a >= 448.0)
+        return sign | 0x7E; /* saturate */
+    if (a == 0.0)
+        return sign;
+    /* quantum of the binade of a (subnormal binade below 2^-6), then round the significand
+     * a / quantum to the nearest integer, ties to even */
+    int E;
+    frexp(a, &E);          /* a = m 2^E, m in [0.5, 1): binade exponent E - 1 */
+    int be = E - 1;
+    if (be < -6)
+        be = -6;
+    const double q = ldexp(1.0, be - 3);
+    const double n = rint(a / q); /* a / q is exact; rint: ties to even */
+    const double r = n * q;
+    if (r >= 448.0)
+        return sign | 0x7E;
+    if (r < ldexp(1.0, -6)) /* subnormal (or rounded up to the smallest normal below) */
+        return sign | (uint8_t)(r / ldexp(1.0, -9));
+    int E2;
+    frexp(r, &E2);
+    const int e = (E2 - 1) + 7;
+    const int f = (int)(r / ldexp(1.0, E2 - 1) * 8.0) - 8;
+    return sign | (uint8_t)((e << 3) | f);
+}
+
+/* Per-token FP8 quantization of one fp32 row: s = amax / 448, q_j = e4m3(y_j / s) (binary32
+ * division, then the rounding above); an all-zero row gets s = 0 and q = 0. */
+void oracle_quantize_row_f32_fp8(const float *y, int64_t K, uint8_t *q, float *s_out)
+{
+    float amax = 0.0f;
+    for (int64_t j = 0; j < K; ++j)
+        if (fabsf(y[j]) > amax)
+            amax = fabsf(y[j]);
+    if (amax == 0.0f) {
+        *s_out = 0.0f;
+        memset(q, 0, (size_t)K);
+        return;
+    }
+    const float s = amax / 448.0f;
+    *s_out = s;
+    for (int64_t j = 0; j < K; ++j)
+        q[j] = oracle_f32_to_e4m3(y[j] / s);
+}
+
+struct qrows8_ctx {
+    const uint16_t *x;
+    const float *sinv;
+    int64_t K;
+    uint8_t *q;
+    float *s;
+};
+
+static void qrows8_row(void *vctx, int64_t m)
+{
+    struct qrows8_ctx *c = (struct qrows8_ctx *)vctx;
+    float *y = (float *)malloc((size_t)c->K * sizeof(float));
+    for (int64_t j = 0; j < c->K; ++j) {
+        y[j] = oracle_bf16_to_f32(c->x[m * c->K + j]);
+        if (c->sinv)
+            y[j] = y[j] * c->sinv[j];
+    }
+    oracle_quantize_row_f32_fp8(y, c->K, c->q + m * c->K, c->s + m);
+    free(y);
+}
+
+/* Per-token FP8 quantization of bf16 activations [M, K] (optionally times sinv). */
+int oracle_quantize_rows_fp8(const uint16_t *x, const float *sinv, int64_t M, int64_t K,
+                             uint8_t *q, float *s, int nthreads)
+{
+    struct qrows8_ctx c = {x, sinv, K, q, s};
+    parallel_rows(qrows8_row, &c, M, nthreads);
+    return 0;
+}
+
+struct qf8_ctx {
+    const float *y;
+    int64_t K;
+    uint8_t *q;
+    float *s;
+};
+
+static void qf8_row(void *vctx, int64_t m)
+{
+    struct qf8_ctx *c = (struct qf8_ctx *)vctx;
+    oracle_quantize_row_f32_fp8(c->y + m * c->K, c->K, c->q + m * c->K, c->s + m);
+}
+
+/* Per-row FP8 quantization of fp32 rows [M, K] (normalized activations, SiLU*up, or
+ * smoothed weights, whose rows are output channels). */
+int oracle_quantize_rows_f32_fp8(const float *y, int64_t M, int64_t K, uint8_t *q, float *s,
+                                 int nthreads)
+{
+    struct qf8_ctx c = {y, K, q, s};
+    parallel_rows(qf8_row, &c, M, nthreads);
+    return 0;
+}
+
+/*
+ * FP8 GEMM reference: acc[m,n] = sum_k e4m3(xq[m,k]) e4m3(wq[n,k]) computed exactly (each
+ * product is exact in binary64 and the sum stays exact for K <= 2^15: the terms are
+ * multiples of 2^-18 below 2^18), also sum_k |products| (the scale of the rounding error of
+ * any binary32 accumulation), and y = bf16_RN((float(acc) s_tok) s_ch).
+ */
+int oracle_gemm_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const float *s_ch,
+                    int64_t M, int64_t N, int64_t K, double *acc, double *absacc, uint16_t *y)
+{
+    float *xd = (float *)malloc((size_t)(M * K) * sizeof(float));
+    float *wd = (float *)malloc((size_t)(N * K) * sizeof(float));
+    for (int64_t i = 0; i < M * K; ++i)
+        xd[i] = oracle_e4m3_to_f32(xq[i]);
+    for (int64_t i = 0; i < N * K; ++i)
+        wd[i] = oracle_e4m3_to_f32(wq[i]);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double a = 0.0, b = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double p = (double)xd[m * K + k] * (double)wd[n * K + k];
+                a += p;
+                b += fabs(p);
+            }
+            acc[m * N + n] = a;
+            absacc[m * N + n] = b;
+            float f = (float)a;
+            f = f * s_tok[m];
+            f = f * s_ch[n];
+            y[m * N + n] = oracle_f32_to_bf16(f);
+        }
+    free(xd);
+    free(wd);
     return 0;
 }
 
