@@ -218,10 +218,10 @@ class ClockSampler:
 class Layer:
     """One decoder block's linear path at M tokens: prepared weights, inputs, outputs."""
 
-    def __init__(self, arch, M, seed, device):
+    def __init__(self, arch, M, seed, device, fp8=False):
         import int8_w8a8_quantized_smoothed_b200 as w8
         from int8_w8a8_quantized_smoothed_b200 import prep, synth
-        self.M, self.arch = M, arch
+        self.M, self.arch, self.fp8 = M, arch, fp8
         H, I = arch["H"], arch["I"]
         P = projections(arch)
         g1 = synth.gamma_device(H, seed + 1, device)
@@ -248,11 +248,14 @@ class Layer:
                 self.g2f = torch.from_numpy(prep.fold(g2.cpu().numpy(), p["s"])[0]).to(device)
             else:  # down: its input is SiLU*up, no norm to fold into
                 wq, sch = w8.w8a8_quantize_rows(wb)
-                p = dict(wq=wq, s_ch=sch)
-            self.w[name] = (p["wq"], p["s_ch"])
-            del wb
+                p = dict(wq=wq, s_ch=sch, s_dev=None)
+            if fp8:  # E4M3 codes of the same smoothed weight, scales absmax / 448
+                self.w[name] = w8.w8a8_quantize_rows_fp8(wb, p["s_dev"])
+            else:
+                self.w[name] = (p["wq"], p["s_ch"])
+            del wb, p
         # the gate|up weight in the row order of the fused SiLU*up epilogue
-        self.w_gu_il = prep.interleave_gate_up(*self.w["gate_up"])
+        self.w_gu_il = None if fp8 else prep.interleave_gate_up(*self.w["gate_up"])
         torch.cuda.synchronize()
         # inputs (device) and their pinned host copies for the end-to-end measurement
         self.x = synth.activation_device(M, H, seed + 20, device)
@@ -260,18 +263,19 @@ class Layer:
         self.x_host = self.x.cpu().pin_memory()
         self.attn_host = self.attn.cpu().pin_memory()
         e = dict(device=device)
-        self.q1 = torch.empty(M, H, dtype=torch.int8, **e)
+        qt = w8.FP8 if fp8 else torch.int8
+        self.q1 = torch.empty(M, H, dtype=qt, **e)
         self.s1 = torch.empty(M, dtype=torch.float32, **e)
         self.qkv = torch.empty(M, P["qkv"][0], dtype=torch.bfloat16, **e)
-        self.q2 = torch.empty(M, H, dtype=torch.int8, **e)
+        self.q2 = torch.empty(M, H, dtype=qt, **e)
         self.s2 = torch.empty(M, dtype=torch.float32, **e)
         self.o = torch.empty(M, H, dtype=torch.bfloat16, **e)
         self.h = torch.empty(M, H, dtype=torch.bfloat16, **e)
-        self.q3 = torch.empty(M, H, dtype=torch.int8, **e)
+        self.q3 = torch.empty(M, H, dtype=qt, **e)
         self.s3 = torch.empty(M, dtype=torch.float32, **e)
         self.gu = torch.empty(M, 2 * I, dtype=torch.bfloat16, **e)
         self.a = torch.empty(M, I, dtype=torch.float32, **e)  # SiLU*up of the fused path
-        self.q4 = torch.empty(M, I, dtype=torch.int8, **e)
+        self.q4 = torch.empty(M, I, dtype=qt, **e)
         self.s4 = torch.empty(M, dtype=torch.float32, **e)
         self.down = torch.empty(M, H, dtype=torch.bfloat16, **e)
         self.down_host = torch.empty(M, H, dtype=torch.bfloat16).pin_memory()
@@ -283,6 +287,8 @@ class Layer:
 
     def chain(self, ws, gemms=True, rows=True, fused=None):
         import int8_w8a8_quantized_smoothed_b200 as w8
+        if self.fp8:
+            return self.chain_fp8(ws, gemms, rows)
         fused = self.fused if fused is None else fused
         if rows:
             w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
@@ -308,6 +314,30 @@ class Layer:
                 w8.w8a8_silu_mul_quant(self.gu, q=self.q4, s_tok=self.s4)
         if gemms:
             w8.w8a8_gemm_dequant(self.q4, self.s4, *self.w["down"], y=self.down, workspace=ws)
+
+
+    def chain_fp8(self, ws, gemms=True, rows=True):
+        """The same block with E4M3 codes: FP8 row kernels and FP8 GEMMs (SiLU*up unfused)."""
+        import int8_w8a8_quantized_smoothed_b200 as w8
+        if rows:
+            w8.w8a8_smooth_rmsnorm_quant_fp8(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
+        if gemms:
+            w8.w8a8_gemm_dequant_fp8(self.q1, self.s1, *self.w["qkv"], y=self.qkv, workspace=ws)
+        if rows:
+            w8.w8a8_quantize_rows_fp8(self.attn, self.sinv_o, q=self.q2, s_tok=self.s2)
+        if gemms:
+            w8.w8a8_gemm_dequant_fp8(self.q2, self.s2, *self.w["o"], y=self.o, workspace=ws)
+        if rows:
+            w8.w8a8_smooth_rmsnorm_quant_fp8(self.o, self.g2f, EPS, residual=self.x,
+                                             h_out=self.h, q=self.q3, s_tok=self.s3)
+        if gemms:
+            w8.w8a8_gemm_dequant_fp8(self.q3, self.s3, *self.w["gate_up"], y=self.gu,
+                                     workspace=ws)
+        if rows:
+            w8.w8a8_silu_mul_quant_fp8(self.gu, q=self.q4, s_tok=self.s4)
+        if gemms:
+            w8.w8a8_gemm_dequant_fp8(self.q4, self.s4, *self.w["down"], y=self.down,
+                                     workspace=ws)
 
 
 def measure_int8_peak(iters=20000, reps=3, sustained_s=0.0):
@@ -385,11 +415,15 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     wl = WORKLOADS[args.workload]
     arch = wl["arch"]
-    layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev) for i, M in enumerate(wl["Ms"])]
+    layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev, fp8=args.fp8)
+              for i, M in enumerate(wl["Ms"])]
+    unfused = args.unfused or args.fp8  # the SiLU*up epilogue is INT8 only
     for L in layers:
-        L.fused = not args.unfused
+        L.fused = not unfused
     ws = w8.Workspace(dev)
     max_ws = max([w8.w8a8_gemm_workspace_size(L.M, N, K) for L in layers
+                  for (N, K) in projections(arch).values()] +
+                 [w8.w8a8_gemm_fp8_workspace_size(L.M, N, K) for L in layers
                   for (N, K) in projections(arch).values()] +
                  [w8.w8a8_gemm_silu_quant_workspace_size(L.M, arch["I"], arch["H"])
                   for L in layers])
@@ -475,7 +509,7 @@ def run_ours(args, world, rank, local):
     g_rows = capture(step_rows)
     rsecs = time_graph(g_rows, args.steps, args.warmup) / args.steps
     gfsecs = None
-    if not args.unfused:
+    if not unfused:
         g_gemm_f = capture(step_gemms_fused)
         gfsecs = time_graph(g_gemm_f, args.steps, args.warmup) / args.steps
         del g_gemm_f
@@ -506,8 +540,9 @@ def run_ours(args, world, rank, local):
                     "frac_of_nominal": round(gemm_tops / INT8_NOMINAL_TOPS, 4),
                     "traffic": None}
     else:
-        roofline = {"kernel": "gemm_decode_kernel (all GEMM launches of the step, plain "
-                              "dequant epilogues, timed alone as a graph)",
+        roofline = {"kernel": "gemm_decode_kernel" + ("<F8>" if args.fp8 else "") +
+                              " (all GEMM launches of the step, plain dequant epilogues, timed "
+                              "alone as a graph)",
                     "bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": hbm_peak,
                     "unit": "GB/s", "frac": round(gemm_gbs / hbm_peak, 4),
                     "peak_source": f"{peak_src} copy bandwidth (burst)", "traffic": None}
@@ -516,7 +551,9 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value / 1e9, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8xi8->i32, fp32 scales, bf16 io", "data": "synthetic",
+        "vs_baseline": None,
+        "dtype": ("e4m3xe4m3->f32, fp32 scales, bf16 io" if args.fp8 else
+                  "i8xi8->i32, fp32 scales, bf16 io"), "data": "synthetic",
         "config": {"workload": f"{wl['desc']}, M in {wl['Ms']}: one decoder block's linear "
                                f"path per M on its own layer's weights",
                    "tokens": wl["Ms"], "hidden": arch["H"], "intermediate": arch["I"],
@@ -526,8 +563,10 @@ def run_ours(args, world, rank, local):
                          "of int8 weights (> 126 MB L2)",
                    "timing": "CUDA graph of one step replayed K times, CUDA events",
                    "overlap": args.overlap,
-                   "silu_mul_quant": ("separate launch" if args.unfused else
-                                      "fused into the gate|up GEMM epilogue + quantization pass")},
+                   "silu_mul_quant": ("separate launch" if unfused else
+                                      "fused into the gate|up GEMM epilogue + quantization pass"),
+                   "codes": "FP8 E4M3 (scale absmax / 448)" if args.fp8 else
+                            "INT8 (scale absmax / 127)"},
         "tops": round(ops / t_max / 1e12, 3),
         "roofline_step": {"t_roof_us": round(t_roof * 1e6, 2),
                           "t_us": round(t_max * 1e6, 2), "frac": round(t_roof / t_max, 4),
@@ -540,7 +579,7 @@ def run_ours(args, world, rank, local):
                          **({"gemms_with_fused_silu_and_quant_pass": round(gfsecs * 1e6, 2)}
                             if gfsecs is not None else {}),
                          "note": "gemms: plain epilogues; row_kernels: the step's row "
-                                 "launches" + ("" if args.unfused else
+                                 "launches" + ("" if unfused else
                                                " (SiLU*up is fused into the gate|up GEMM)")},
         "e2e": {"value": round(e_value / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -550,9 +589,10 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(t_wall0, time.perf_counter()),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
         result["cpu_baseline"] = cpu_baseline(arch)
-    traffic = args.traffic if args.traffic is not None else NCU_GEMM_TRAFFIC.get(args.workload)
+    traffic = args.traffic if args.traffic is not None else (
+        None if args.fp8 else NCU_GEMM_TRAFFIC.get(args.workload))
     if traffic is not None:
         result["roofline"]["traffic"] = traffic
         result["roofline"]["traffic_per"] = "GEMM launch (ncu DRAM read + write bytes)"
@@ -641,7 +681,7 @@ def run_reference(args, world, rank):
 
 
 def run_case(args):
-    """`--case gemm:M:N:K[:variant]`, `rms:M:K`, `rmsres:M:K`, `quant:M:K`, `static:M:K` or
+    """`--case gemm:M:N:K[:variant]` (INT8), `gemm8:M:N:K[:variant]` (FP8), `rms:M:K`, `rmsres:M:K`, `quant:M:K`, `static:M:K` or
     `silu:M:I`:
     one kernel launched repeatedly (a CUDA graph of back-to-back launches)."""
     import int8_w8a8_quantized_smoothed_b200 as w8
@@ -649,22 +689,30 @@ def run_case(args):
     wbuild.build()
     parts = args.case.split(":")
     dev = torch.device("cuda", 0)
-    if parts[0] == "gemm":
+    if parts[0] in ("gemm", "gemm8"):
         M, N, K = (int(v) for v in parts[1:4])
         variant = int(parts[4]) if len(parts) > 4 else 0
+        fp8 = parts[0] == "gemm8"
         copies = max(1, math.ceil(4 * 126e6 / (N * K)))  # rotate weights through > 4x L2
-        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+
+        def codes(shape):
+            if not fp8:
+                return torch.randint(-127, 128, shape, dtype=torch.int8, device=dev)
+            c = torch.randint(0, 256, shape, dtype=torch.uint8, device=dev)
+            c[(c & 0x7F) == 0x7F] = 0x30  # no NaN codes
+            return c.view(w8.FP8)
+        xq = codes((M, K))
         st = torch.rand(M, device=dev) * 1e-2
-        ws_ = [torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev)
-               for _ in range(copies)]
+        ws_ = [codes((N, K)) for _ in range(copies)]
         sc = torch.rand(N, device=dev) * 1e-3
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         wsp = w8.Workspace(dev)
+        gemm = w8.w8a8_gemm_dequant_fp8 if fp8 else w8.w8a8_gemm_dequant_ex
 
         def launch(i):
-            w8.w8a8_gemm_dequant_ex(xq, st, ws_[i % copies], sc, y=y, workspace=wsp,
-                                    variant=variant)
+            gemm(xq, st, ws_[i % copies], sc, y=y, workspace=wsp, variant=variant)
         work = gemm_bytes(M, N, K)
+        flops = 2 * M * N * K
     else:
         # row kernels: rms:M:K, rmsres:M:K, quant:M:K, silu:M:I; inputs rotate over enough
         # copies to exceed L2
@@ -708,9 +756,12 @@ def run_case(args):
     e1.record()
     torch.cuda.synchronize()
     t = e0.elapsed_time(e1) / 1e3 / args.steps
-    return {"case": args.case, "us_per_launch": round(t * 1e6, 3),
-            "GBps_algorithmic": round(work / t / 1e9, 1),
-            "note": "CUDA graph of back-to-back launches"}
+    out = {"case": args.case, "us_per_launch": round(t * 1e6, 3),
+           "GBps_algorithmic": round(work / t / 1e9, 1),
+           "note": "CUDA graph of back-to-back launches"}
+    if parts[0] in ("gemm", "gemm8"):
+        out["TOPS"] = round(flops / t / 1e12, 1)
+    return out
 
 
 def main(argv=None):
@@ -727,6 +778,8 @@ def main(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="gate|up GEMM and SiLU*up+quant as separate launches instead of the "
                          "fused SiLU*up epilogue")
+    ap.add_argument("--fp8", action="store_true",
+                    help="the FP8 (E4M3) variant of the path: FP8 row kernels and GEMMs")
     ap.add_argument("--overlap", type=int, choices=[0, 1, 2], default=2,
                     help="kernel overlap mode (w8a8_set_overlap); 2 = dependent launch with "
                          "static-weight prefetch")

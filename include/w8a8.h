@@ -9,6 +9,7 @@
  *   [W8A8]  "INT8 W8A8 quantization of Llama 3.1 8B with SmoothQuant and GPTQ" (arc-codex)
  *   [PTQ]   "INT8 Post-Training Quantization for LLM Inference on NVIDIA GPUs" (devtechtools)
  *   [SERVE] "W8A8 Llama 3.1 8B: accuracy and serving results" (Red Hat developers)
+ *   [INFENG] "05 Quantization AWQ GPTQ FP8" (inference-engineering notes)
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller; row-major, contiguous.
@@ -228,15 +229,62 @@ W8A8_API int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, con
  * 64b .. 64b+63 and rows 128b+64 .. 128b+127 are up rows 64b .. 64b+63 (b < I/64); s_ch_il:
  * fp32 [2I], the channel scales in the same order. I % 64 == 0.
  * a: fp32 [M, I] (written, then read by the quantization; 16-byte aligned). q: int8 [M, I],
- * s_out: fp32 [M]. workspace: w8a8_gemm_silu_quant_workspace_size(M, I, K) bytes, 16-byte
- * aligned, zero-filled before its first use; each call leaves it zero again. Other
- * requirements and errors as for w8a8_gemm_dequant (acc_out is not available here).
+ * s_out: fp32 [M]. workspace: w8a8_gemm_silu_quant_workspace_size(M, I, K) bytes (0 when the
+ * GEMM's plan needs none), 16-byte aligned: the GEMM's own workspace, with the rules of
+ * w8a8_gemm_workspace_size, so one zero-filled buffer serves calls of this entry point and of
+ * w8a8_gemm_dequant alike, issued in order on one stream. Other requirements and errors as
+ * for w8a8_gemm_dequant (acc_out is not available here).
  */
 W8A8_API size_t w8a8_gemm_silu_quant_workspace_size(int64_t M, int64_t I, int64_t K);
 W8A8_API int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_il,
                                   const float *s_ch_il, int64_t M, int64_t I, int64_t K,
                                   float *a, int8_t *q, float *s_out, void *workspace,
                                   size_t workspace_bytes, w8a8_stream_t stream);
+
+/*
+ * ---------------------------------------------------------------- FP8 (E4M3) variant
+ *
+ * W8A8 with 8-bit floating-point codes instead of int8, the variant for Hopper and Blackwell
+ * GPUs [SERVE "When W8A8 INT8 quantization is a good fit", "What to explore next"; INFENG
+ * "Ladder"]. The pages do not fix the encoding; this library uses
+ * OCP E4M3 (sign, 4 exponent bits with bias 7, 3 fraction bits; no infinities; largest
+ * finite 448; S.1111.111 is NaN) and:
+ *   e4m3(v)  = v rounded to nearest E4M3 value, ties to even, saturated to +-448
+ *   s        = amax / 448 (binary32), code = e4m3(RN(y / s)); an all-zero row: s = 0, codes +0
+ * Codes travel as uint8 bit patterns. Each entry point below is its INT8 namesake with those
+ * codes and that scale; arguments, layouts, alignment, shape rules and errors are the same.
+ */
+W8A8_API int w8a8_quantize_rows_fp8(const w8a8_bf16 *x, const float *smooth_inv, int64_t M,
+                                    int64_t K, uint8_t *q, float *s_tok, w8a8_stream_t stream);
+W8A8_API int w8a8_smooth_rmsnorm_quant_fp8(const w8a8_bf16 *x, const w8a8_bf16 *residual,
+                                           w8a8_bf16 *h_out, const float *gamma_smoothed,
+                                           float eps, int64_t M, int64_t K, uint8_t *q,
+                                           float *s_tok, w8a8_stream_t stream);
+W8A8_API int w8a8_silu_mul_quant_fp8(const w8a8_bf16 *gate_up, int64_t M, int64_t I, uint8_t *q,
+                                     float *s_tok, w8a8_stream_t stream);
+
+/*
+ * FP8 tensor-core GEMM (tcgen05.mma kind::f8f6f4, E4M3 x E4M3) with the dequantization
+ * epilogue:
+ *   acc[m,n] = sum_k e4m3(xq[m,k]) * e4m3(wq[n,k])   accumulated in binary32 by the tensor
+ *              cores (each product is exact; the order and the rounding of the additions are
+ *              the hardware's, so acc differs from the exact sum by at most a few units of
+ *              2^-24 times sum_k |products|; split-K partial sums are added in binary32)
+ *   y[m,n]   = bf16( (acc[m,n] * s_tok[m]) * s_ch[n] )  (binary32 RN, then RN to bf16)
+ * xq: uint8 E4M3 codes [M,K]; wq: uint8 E4M3 codes [N,K] (per-output-channel scales s_ch =
+ * max_k |w[n,k]| / 448); acc_out: fp32 [M,N] or NULL (the accumulators, as a check mode).
+ * variant, ctas, tile_n, workspace and all other rules as for w8a8_gemm_dequant_ex (the
+ * cluster split-K kernel, variant 3, adds the binary32 partials of a cluster in rank order,
+ * read from the CTAs' shared memory); the workspace size is w8a8_gemm_fp8_workspace_size() of
+ * the same arguments.
+ */
+W8A8_API size_t w8a8_gemm_fp8_workspace_size(int64_t M, int64_t N, int64_t K, int variant,
+                                             int ctas, int tile_n);
+W8A8_API int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq,
+                                   const float *s_ch, int64_t M, int64_t N, int64_t K,
+                                   w8a8_bf16 *y, float *acc_out, void *workspace,
+                                   size_t workspace_bytes, int variant, int ctas, int tile_n,
+                                   w8a8_stream_t stream);
 
 /*
  * Measurement aid, not part of the W8A8 path (the pages have no counterpart): launches `ctas`

@@ -23,7 +23,9 @@ __all__ = [
     "w8a8_gemm_silu_quant_workspace_size", "w8a8_probe_i8_mma", "w8a8_selftest_wait_timeout", "w8a8_set_overlap",
     "w8a8_get_overlap", "w8a8_device_status",
     "w8a8_status_string", "w8a8_version",
-    "Workspace",
+    "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
+    "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size",
+    "Workspace", "FP8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw8a8.so")
@@ -54,7 +56,16 @@ SIGNATURES = [
     ("w8a8_device_status", _I, [_I]),
     ("w8a8_status_string", C.c_char_p, [_I]),
     ("w8a8_version", _I, []),
+    ("w8a8_quantize_rows_fp8", _I, [_P, _P, _I64, _I64, _P, _P, _P]),
+    ("w8a8_smooth_rmsnorm_quant_fp8", _I, [_P, _P, _P, _P, _F, _I64, _I64, _P, _P, _P]),
+    ("w8a8_silu_mul_quant_fp8", _I, [_P, _I64, _I64, _P, _P, _P]),
+    ("w8a8_gemm_fp8_workspace_size", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
+    ("w8a8_gemm_dequant_fp8", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _I, _I,
+                                   _I, _P]),
 ]
+
+# FP8 codes are OCP E4M3 bit patterns, carried in torch.float8_e4m3fn tensors
+FP8 = torch.float8_e4m3fn
 
 _lib = None
 _lock = threading.Lock()
@@ -224,6 +235,63 @@ def w8a8_silu_mul_quant(gate_up, q=None, s_tok=None, stream=None):
     return q, s_tok
 
 
+def w8a8_quantize_rows_fp8(x, smooth_inv=None, q=None, s_tok=None, stream=None):
+    """Per-token FP8 (E4M3, scale amax / 448) quantization of bf16 x [M, K]."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    if smooth_inv is not None:
+        _need(smooth_inv, "smooth_inv", torch.float32, (K,))
+    q = torch.empty((M, K), dtype=FP8, device=x.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _need(q, "q", FP8, (M, K))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_quantize_rows_fp8", lib().w8a8_quantize_rows_fp8(
+        _ptr(x), _ptr(smooth_inv), M, K, _ptr(q), _ptr(s_tok), _stream(stream)))
+    return q, s_tok
+
+
+def w8a8_smooth_rmsnorm_quant_fp8(x, gamma_smoothed, eps, residual=None, h_out=None, q=None,
+                                  s_tok=None, stream=None):
+    """w8a8_smooth_rmsnorm_quant with FP8 (E4M3) codes."""
+    _need(x, "x", torch.bfloat16)
+    M, K = x.shape
+    _need(gamma_smoothed, "gamma_smoothed", torch.float32, (K,))
+    if residual is not None:
+        _need(residual, "residual", torch.bfloat16, (M, K))
+        h_out = torch.empty_like(x) if h_out is None else h_out
+        _need(h_out, "h_out", torch.bfloat16, (M, K))
+    q = torch.empty((M, K), dtype=FP8, device=x.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=x.device) if s_tok is None else s_tok
+    _need(q, "q", FP8, (M, K))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_smooth_rmsnorm_quant_fp8", lib().w8a8_smooth_rmsnorm_quant_fp8(
+        _ptr(x), _ptr(residual), _ptr(h_out), _ptr(gamma_smoothed), float(eps), M, K, _ptr(q),
+        _ptr(s_tok), _stream(stream)))
+    if residual is not None:
+        return q, s_tok, h_out
+    return q, s_tok
+
+
+def w8a8_silu_mul_quant_fp8(gate_up, q=None, s_tok=None, stream=None):
+    """w8a8_silu_mul_quant with FP8 (E4M3) codes."""
+    _need(gate_up, "gate_up", torch.bfloat16)
+    M, I2 = gate_up.shape
+    if I2 % 2:
+        raise ValueError("gate_up must have an even number of columns")
+    I = I2 // 2
+    q = torch.empty((M, I), dtype=FP8, device=gate_up.device) if q is None else q
+    s_tok = torch.empty(M, dtype=torch.float32, device=gate_up.device) if s_tok is None else s_tok
+    _need(q, "q", FP8, (M, I))
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _check("w8a8_silu_mul_quant_fp8", lib().w8a8_silu_mul_quant_fp8(
+        _ptr(gate_up), M, I, _ptr(q), _ptr(s_tok), _stream(stream)))
+    return q, s_tok
+
+
+def w8a8_gemm_fp8_workspace_size(M, N, K, variant=0, ctas=0, tile_n=0) -> int:
+    return int(lib().w8a8_gemm_fp8_workspace_size(M, N, K, variant, ctas, tile_n))
+
+
 def w8a8_gemm_workspace_size(M, N, K) -> int:
     return int(lib().w8a8_gemm_workspace_size(M, N, K))
 
@@ -286,6 +354,37 @@ def w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=No
         wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
                                    * workspace.element_size())
     _check("w8a8_gemm_dequant", lib().w8a8_gemm_dequant_ex(
+        _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _ptr(acc_out),
+        _ptr(wbuf), wbytes, int(variant), int(ctas), int(tile_n), _stream(stream)))
+    return y
+
+
+def w8a8_gemm_dequant_fp8(xq, s_tok, wq, s_ch, y=None, acc_out=None, workspace=None,
+                          variant=0, ctas=0, tile_n=0, stream=None):
+    """FP8 GEMM: y = bf16((acc * s_tok[:, None]) * s_ch[None, :]) with acc the binary32
+    tensor-core sum of E4M3 products (xq [M, K], wq [N, K] as torch.float8_e4m3fn).
+    variant 0 = automatic, 1 = persistent tile kernel, 2 = swap-AB stream-K kernel."""
+    _need(xq, "xq", FP8)
+    _need(wq, "wq", FP8)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2:
+        raise ValueError(f"xq [M,K] and wq [N,K] disagree on K: {K} vs {K2}")
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _need(s_ch, "s_ch", torch.float32, (N,))
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N))
+    if acc_out is not None:
+        _need(acc_out, "acc_out", torch.float32, (M, N))
+    need = w8a8_gemm_fp8_workspace_size(M, N, K, variant, ctas, tile_n)
+    if workspace is None:
+        workspace = _workspace_for(xq.device)
+    if isinstance(workspace, Workspace):
+        wbuf, wbytes = workspace.get(need)
+    else:
+        wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
+                                   * workspace.element_size())
+    _check("w8a8_gemm_dequant_fp8", lib().w8a8_gemm_dequant_fp8(
         _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _ptr(acc_out),
         _ptr(wbuf), wbytes, int(variant), int(ctas), int(tile_n), _stream(stream)))
     return y

@@ -1,5 +1,7 @@
 // INT8 x INT8 -> INT32 GEMM on the 5th-generation tensor cores (tcgen05.mma kind::i8) with
-// the dequantization epilogue y = bf16((float(acc) * s_tok[m]) * s_ch[n]) fused.
+// the dequantization epilogue y = bf16((float(acc) * s_tok[m]) * s_ch[n]) fused; with the
+// template flag F8 the same kernels run the FP8 variant, E4M3 x E4M3 -> binary32
+// (kind::f8f6f4), the epilogue then scaling the binary32 accumulator.
 //
 // Both kernels are warp-specialized, 192 threads:
 //   warp 0      TMA producer: one thread streams K-slices (128 bytes wide, 128B-swizzled)
@@ -22,8 +24,7 @@
 // channels 64b..64b+63), so every 128-row group of weight rows holds the gate and up rows of
 // the same 64 output channels. The epilogue rounds both dequantized values to bf16 (exactly
 // what the plain epilogue stores), forms a = silu(g) * u in binary32 as the SiLU*up row
-// kernel does, stores a, and raises a per-token maximum |a| (atomicMax on its bits) that a
-// following quantization pass turns into the per-token scale.
+// kernel does, and stores a; a following row pass takes each token's max |a| and quantizes.
 #pragma once
 
 #include "ptx.cuh"
@@ -37,10 +38,9 @@ constexpr int kBM = 128;  // MMA M: TMEM lanes
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kUmmaK = 32; // K of one kind::i8 MMA
 
-// Outputs of the fused SiLU*up epilogue: a [M, I] binary32 and per-token max |a| words.
+// Output of the fused SiLU*up epilogue: a [M, I] binary32.
 struct SiluOut {
     float *a;
-    unsigned int *amax;
     int I;
 };
 
@@ -51,12 +51,11 @@ __device__ __forceinline__ float bf16_round(float f)
 
 // One thread's row: 32 gate columns (rg, channel scales scg) and the 32 up columns of the
 // same output channels (ru, scu) -> a = silu(bf16(g)) * bf16(u), stored at dst (32 floats,
-// 16-byte stores); returns max |a|.
-__device__ __forceinline__ float silu_row_chunk(const uint32_t (&rg)[32], const uint32_t (&ru)[32],
+// 16-byte stores).
+__device__ __forceinline__ void silu_row_chunk(const uint32_t (&rg)[32], const uint32_t (&ru)[32],
                                                 float st, const float *scg, const float *scu,
                                                 float *__restrict__ dst)
 {
-    float mx = 0.0f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         float g[8], u[8], a[8];
@@ -72,13 +71,9 @@ __device__ __forceinline__ float silu_row_chunk(const uint32_t (&rg)[32], const 
             u[i] = bf16_round(dequant_f32(static_cast<int32_t>(ru[8 * e + i]), st, cu[i]));
         }
         silu_mul8(g, u, a);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            mx = fmaxf(mx, fabsf(a[i]));
         reinterpret_cast<float4 *>(dst)[2 * e] = make_float4(a[0], a[1], a[2], a[3]);
         reinterpret_cast<float4 *>(dst)[2 * e + 1] = make_float4(a[4], a[5], a[6], a[7]);
     }
-    return mx;
 }
 
 // Producer tail of an mbarrier ring: waits until the consumer has released the last
@@ -133,8 +128,9 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
 }
 
 // Dequantizes 32 accumulator columns of one output row and stores them as bf16 (16-byte
-// stores); also the raw int32 values when acc_out is given. sc: the 32 channel scales of
+// stores); also the raw accumulator words when acc_out is given. sc: the 32 channel scales of
 // these columns, in shared memory.
+template <bool F8>
 __device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row, int n0, int N,
                                                 float st, const float *sc,
                                                 uint16_t *__restrict__ y,
@@ -150,7 +146,7 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row
             float f[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                f[i] = dequant_f32(static_cast<int32_t>(r[8 * g + i]), st, cs[i]);
+                f[i] = dequant_acc<F8>(r[8 * g + i], st, cs[i]);
             uint4 o;
             o.x = pack_bf16x2(f[0], f[1]);
             o.y = pack_bf16x2(f[2], f[3]);
@@ -193,7 +189,7 @@ template <int BN> struct TileScales {
     }
 };
 
-template <int BN, int STAGES, bool SILU = false>
+template <int BN, int STAGES, bool SILU = false, bool F8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const float *__restrict__ s_tok,
@@ -201,6 +197,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         uint16_t *__restrict__ y, int32_t *__restrict__ acc_out, SiluOut so,
                         int prefetch_static, unsigned long long limit_ns)
 {
+    static_assert(!(SILU && F8), "the fused SiLU epilogue is INT8 only");
     using Cfg = PrefillCfg<BN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -294,7 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kBM, BN);
+            constexpr uint32_t idesc = idesc_8bit<F8>(kBM, BN);
             uint32_t it = 0, t = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++t) {
@@ -316,8 +313,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t b0 = sB + s * Cfg::kBBytes;
 #pragma unroll
                     for (int k = 0; k < kBK / kUmmaK; ++k)
-                        umma_i8(d, sw128_kmajor_desc(a0 + k * kUmmaK),
-                                sw128_kmajor_desc(b0 + k * kUmmaK), idesc,
+                        umma_8bit<F8>(d, sw128_kmajor_desc(a0 + k * kUmmaK),
+                                      sw128_kmajor_desc(b0 + k * kUmmaK), idesc,
                                 (kb > 0 || k > 0) ? 1u : 0u);
                     umma_commit(bar_empty + 8 * s);
                 }
@@ -358,7 +355,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quarter * 32) << 16);
             if constexpr (SILU) {
                 // gate chunk cg and up chunk cg + 2 hold the same 32 output channels
-                float rowmax = 0.0f;
 #pragma unroll 1
                 for (int p = 0; p < BN / 64; ++p) {
                     const int cg = (p >> 1) * 4 + (p & 1);
@@ -368,13 +364,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
                     tmem_ld_wait();
                     if (row_ok && ch0 < so.I)
-                        rowmax = fmaxf(rowmax, silu_row_chunk(
-                                                   rg, ru, st, sh_sch + buf * BN + cg * 32,
-                                                   sh_sch + buf * BN + (cg + 2) * 32,
-                                                   so.a + static_cast<int64_t>(row) * so.I + ch0));
+                        silu_row_chunk(rg, ru, st, sh_sch + buf * BN + cg * 32,
+                                       sh_sch + buf * BN + (cg + 2) * 32,
+                                       so.a + static_cast<int64_t>(row) * so.I + ch0);
                 }
-                if (row_ok)
-                    atomicMax(so.amax + row, __float_as_uint(rowmax));
             } else {
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
@@ -382,7 +375,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_32x32b_x32(tbase + c * 32, r);
                     tmem_ld_wait();
                     if (row_ok)
-                        store_row_chunk(r, row, nb * BN + c * 32, N, st,
+                        store_row_chunk<F8>(r, row, nb * BN + c * 32, N, st,
                                         sh_sch + buf * BN + c * 32, y, acc_out);
                 }
             }
@@ -416,7 +409,7 @@ template <int STAGES> struct PairCfg {
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
-template <int STAGES, bool SILU = false>
+template <int STAGES, bool SILU = false, bool F8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
@@ -425,6 +418,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              int32_t *__restrict__ acc_out, SiluOut so, int prefetch_static,
                              unsigned long long limit_ns)
 {
+    static_assert(!(SILU && F8), "the fused SiLU epilogue is INT8 only");
     using Cfg = PairCfg<STAGES>;
     constexpr int TN = 256, TM = 256;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -530,7 +524,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_i8(TM, TN);
+            constexpr uint32_t idesc = idesc_8bit<F8>(TM, TN);
             uint32_t it = 0, t = 0;
             bool ok = true;
             for (int tile = pair; tile < tiles && ok; tile += npairs, ++t) {
@@ -552,8 +546,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t b0 = sB + s * Cfg::kBBytes;
 #pragma unroll
                     for (int k = 0; k < kBK / kUmmaK; ++k)
-                        umma_i8_pair(d, sw128_kmajor_desc(a0 + k * kUmmaK),
-                                     sw128_kmajor_desc(b0 + k * kUmmaK), idesc,
+                        umma_8bit_pair<F8>(d, sw128_kmajor_desc(a0 + k * kUmmaK),
+                                           sw128_kmajor_desc(b0 + k * kUmmaK), idesc,
                                      (kb > 0 || k > 0) ? 1u : 0u);
                     umma_commit_pair(bar_empty + 8 * s, 0x3); // frees the stage in both CTAs
                 }
@@ -594,7 +588,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const bool row_ok = row < M;
             const uint32_t tbase = tmem_base + buf * TN + (static_cast<uint32_t>(quarter * 32) << 16);
             if constexpr (SILU) {
-                float rowmax = 0.0f;
 #pragma unroll 1
                 for (int p = 0; p < TN / 64; ++p) {
                     const int cg = (p >> 1) * 4 + (p & 1);
@@ -604,13 +597,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
                     tmem_ld_wait();
                     if (row_ok && ch0 < so.I)
-                        rowmax = fmaxf(rowmax, silu_row_chunk(
-                                                   rg, ru, st, sh_sch + buf * TN + cg * 32,
-                                                   sh_sch + buf * TN + (cg + 2) * 32,
-                                                   so.a + static_cast<int64_t>(row) * so.I + ch0));
+                        silu_row_chunk(rg, ru, st, sh_sch + buf * TN + cg * 32,
+                                       sh_sch + buf * TN + (cg + 2) * 32,
+                                       so.a + static_cast<int64_t>(row) * so.I + ch0);
                 }
-                if (row_ok)
-                    atomicMax(so.amax + row, __float_as_uint(rowmax));
             } else {
 #pragma unroll 1
                 for (int c = 0; c < TN / 32; ++c) {
@@ -618,7 +608,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_32x32b_x32(tbase + c * 32, r);
                     tmem_ld_wait();
                     if (row_ok)
-                        store_row_chunk(r, row, nb * TN + c * 32, N, st,
+                        store_row_chunk<F8>(r, row, nb * TN + c * 32, N, st,
                                         sh_sch + buf * TN + c * 32, y, acc_out);
                 }
             }
@@ -719,40 +709,24 @@ __device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
 
 // The SiLU*up form of the final step of a block (see SiluOut): the block's 128 weight rows
 // are gate rows 0..63 and up rows 64..127 of output channels [64 t, 64 t + 64); v8 = (token,
-// group of 8 channels) vectors, 8 per token, consecutive lanes on one token's 8 groups so that
-// the token's maximum is reduced over 8 lanes. gate(m, j) / up(m, j) give the bf16-rounded
-// values; tokens m0 .. m0 + mt - 1; every thread of the warp calls this the same number of
-// times (shuffles).
+// group of 8 channels) vectors, 8 per token. gate_up(m, j0, g, u) gives the bf16-rounded gate
+// and up values of channels j0 .. j0 + 7 of token m; tokens m0 .. m0 + mt - 1.
 template <typename GateUp>
 __device__ __forceinline__ void silu_block_rows(int m0, int mt, int t, int etid, const SiluOut &so,
                                                 GateUp gate_up)
 {
-    const int lane = etid & 31;
-    for (int base = 0; base < mt * 8; base += 128) {
-        const int v = base + etid;
-        const bool act = v < mt * 8;
+    for (int v = etid; v < mt * 8; v += 128) {
         const int m = m0 + (v >> 3), j0 = (v & 7) * 8;
-        float mx = 0.0f;
-        if (act) {
-            float g[8], u[8], a[8];
-            gate_up(m, j0, g, u);
-            silu_mul8(g, u, a);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                mx = fmaxf(mx, fabsf(a[i]));
-            float *dst = so.a + static_cast<int64_t>(m) * so.I + static_cast<int64_t>(t) * 64 + j0;
-            reinterpret_cast<float4 *>(dst)[0] = make_float4(a[0], a[1], a[2], a[3]);
-            reinterpret_cast<float4 *>(dst)[1] = make_float4(a[4], a[5], a[6], a[7]);
-        }
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1)
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (act && (lane & 7) == 0)
-            atomicMax(so.amax + m, __float_as_uint(mx));
+        float g[8], u[8], a[8];
+        gate_up(m, j0, g, u);
+        silu_mul8(g, u, a);
+        float *dst = so.a + static_cast<int64_t>(m) * so.I + static_cast<int64_t>(t) * 64 + j0;
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(a[0], a[1], a[2], a[3]);
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(a[4], a[5], a[6], a[7]);
     }
 }
 
-template <int NT, int STAGES, int KPS, bool CLUSTER, bool SILU = false>
+template <int NT, int STAGES, int KPS, bool CLUSTER, bool SILU = false, bool F8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX, const float *__restrict__ s_tok,
@@ -761,6 +735,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                        int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
                        SiluOut so, int prefetch_static, unsigned long long limit_ns)
 {
+    static_assert(!(SILU && F8), "the fused SiLU epilogue is INT8 only");
     using Cfg = DecodeCfg<NT, STAGES, KPS, CLUSTER>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -882,7 +857,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kBM, NT);
+            constexpr uint32_t idesc = idesc_8bit<F8>(kBM, NT);
             uint32_t it = 0, seg = 0;
             bool ok = true;
             for (int64_t u = u_begin; u < u_end && ok; ++seg) {
@@ -907,8 +882,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint32_t x0 = sX + (s * KPS + j) * Cfg::kXBytes;
 #pragma unroll
                         for (int k = 0; k < kBK / kUmmaK; ++k)
-                            umma_i8(d, sw128_kmajor_desc(w0 + k * kUmmaK),
-                                    sw128_kmajor_desc(x0 + k * kUmmaK), idesc,
+                            umma_8bit<F8>(d, sw128_kmajor_desc(w0 + k * kUmmaK),
+                                          sw128_kmajor_desc(x0 + k * kUmmaK), idesc,
                                     (kb > sg.kb0 || j > 0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(bar_empty + 8 * s);
@@ -935,7 +910,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int Mp = ((M < NT ? M : NT) + 3) & ~3; // tokens per partial row in the workspace
         // an owner's contributor sums, per token of its channel (small token tiles only)
         constexpr int kPre = (!CLUSTER && NT <= 64) ? NT : 0;
-        int32_t pre[kPre > 0 ? kPre : 1];
+        uint32_t pre[kPre > 0 ? kPre : 1];
         // This CTA owns a block shared with later CTAs iff its range ends inside a block it
         // starts; the later CTAs' shares of that block are their first segments.
         int64_t own_t = -1, own_last = g;
@@ -973,17 +948,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int mt = tile_tokens(own_t);
 #pragma unroll
                 for (int j = 0; j < kPre; ++j)
-                    pre[j] = 0;
+                    pre[j] = 0u; // +0 in both accumulator types
                 for (int64_t c = g + 1; c <= own_last; ++c) {
                     const int4 *src = reinterpret_cast<const int4 *>(ws_part + (c * kBM + r) * Mp);
 #pragma unroll
                     for (int q = 0; q < kPre / 4; ++q) {
                         if (4 * q < mt) {
                             const int4 v = __ldcg(src + q);
-                            pre[4 * q] += v.x;
-                            pre[4 * q + 1] += v.y;
-                            pre[4 * q + 2] += v.z;
-                            pre[4 * q + 3] += v.w;
+                            pre[4 * q] = acc_add<F8>(pre[4 * q], v.x);
+                            pre[4 * q + 1] = acc_add<F8>(pre[4 * q + 1], v.y);
+                            pre[4 * q + 2] = acc_add<F8>(pre[4 * q + 2], v.z);
+                            pre[4 * q + 3] = acc_add<F8>(pre[4 * q + 3], v.w);
                         }
                     }
                 }
@@ -1049,7 +1024,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if constexpr (kPre > 0) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            a[j] += static_cast<uint32_t>(pre[c0 + j]);
+                            a[j] = acc_add<F8>(a[j], pre[c0 + j]);
                     } else {
 #pragma unroll 2
                         for (int64_t c = g + 1; c <= g_last; ++c) {
@@ -1061,10 +1036,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 v[q] = (c0 + 4 * q < mt) ? __ldcg(src + q) : make_int4(0, 0, 0, 0);
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
-                                a[4 * q] += static_cast<uint32_t>(v[q].x);
-                                a[4 * q + 1] += static_cast<uint32_t>(v[q].y);
-                                a[4 * q + 2] += static_cast<uint32_t>(v[q].z);
-                                a[4 * q + 3] += static_cast<uint32_t>(v[q].w);
+                                a[4 * q] = acc_add<F8>(a[4 * q], v[q].x);
+                                a[4 * q + 1] = acc_add<F8>(a[4 * q + 1], v[q].y);
+                                a[4 * q + 2] = acc_add<F8>(a[4 * q + 2], v[q].z);
+                                a[4 * q + 3] = acc_add<F8>(a[4 * q + 3], v[q].w);
                             }
                         }
                     }
@@ -1074,11 +1049,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int j = 0; j < 16; ++j) {
                     const int m = c0 + j;
                     if (m < mt) {
-                        const int32_t v = static_cast<int32_t>(a[j]);
                         ysm[m * kBM + r] = static_cast<uint16_t>(
-                            bf16_bits(dequant_f32(v, sh_stok[mbase + m], sc)));
+                            bf16_bits(dequant_acc<F8>(a[j], sh_stok[mbase + m], sc)));
                         if (acc_out && n_ok)
-                            acc_out[static_cast<int64_t>(mbase + m) * N + n] = v;
+                            acc_out[static_cast<int64_t>(mbase + m) * N + n] =
+                                static_cast<int32_t>(a[j]);
                     }
                 }
             };
@@ -1134,7 +1109,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     }
     __syncwarp();
-    if constexpr (CLUSTER) {
+    if constexpr (CLUSTER && F8) {
+        // Split-K sum in distributed shared memory, binary32 partials (the bulk reduction
+        // into peer shared memory has integer forms only): after the cluster barrier, CTA q
+        // reads the rows of its tokens [q mt / S, (q+1) mt / S) from every CTA's tile, in
+        // rank order (so the sum does not depend on which CTA owns the rows), adds them,
+        // dequantizes and stores.
+        const uint32_t S = gridDim.x;
+        const uint32_t rank = cluster_ctarank();
+        const int64_t blk = blockIdx.y;
+        const int tch = static_cast<int>(blk / TT);             // channel block
+        const int mbase = static_cast<int>(blk % TT) * NT;      // first token of the tile
+        const uint32_t mt = static_cast<uint32_t>(M - mbase < NT ? M - mbase : NT);
+        const uint32_t m0 = (rank * mt) / S, m1 = ((rank + 1) * mt) / S;
+        cluster_sync(); // every CTA's partial tile complete and visible to the cluster
+        if (warp >= 2) {
+            const int etid = threadIdx.x - 64;
+            const int nv = static_cast<int>(m1 - m0) * (kBM / 4);
+            for (int v = etid; v < nv; v += 128) {
+                const int ml = static_cast<int>(m0) + v / (kBM / 4); // token within the tile
+                const int m = mbase + ml;
+                const int c = (v % (kBM / 4)) * 4;
+                const int n = tch * kBM + c;
+                if (n < N) { // N % 8 == 0: the 4 channels are all valid or all past N
+                    const uint32_t off = sbase + static_cast<uint32_t>(ml * kBM + c) * 4u;
+                    uint4 s4 = ld_dsmem_v4(map_peer_smem(off, 0));
+                    for (uint32_t q = 1; q < S; ++q) {
+                        const uint4 p4 = ld_dsmem_v4(map_peer_smem(off, q));
+                        s4.x = acc_add<true>(s4.x, p4.x);
+                        s4.y = acc_add<true>(s4.y, p4.y);
+                        s4.z = acc_add<true>(s4.z, p4.z);
+                        s4.w = acc_add<true>(s4.w, p4.w);
+                    }
+                    const float4 c4 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
+                    const float st = sh_stok[m];
+                    uint2 o;
+                    o.x = bf16_bits(dequant_acc<true>(s4.x, st, c4.x)) |
+                          (bf16_bits(dequant_acc<true>(s4.y, st, c4.y)) << 16);
+                    o.y = bf16_bits(dequant_acc<true>(s4.z, st, c4.z)) |
+                          (bf16_bits(dequant_acc<true>(s4.w, st, c4.w)) << 16);
+                    const int64_t goff = static_cast<int64_t>(m) * N + n;
+                    *reinterpret_cast<uint2 *>(y + goff) = o;
+                    if (acc_out)
+                        *reinterpret_cast<uint4 *>(acc_out + goff) = s4;
+                }
+            }
+        }
+        // nobody leaves, or reuses its tile, while a peer may still read it
+        cluster_sync();
+    } else if constexpr (CLUSTER) {
         // Split-K sum in distributed shared memory. CTA q of the cluster owns the tokens
         // [q mt / S, (q+1) mt / S) of the block; every other CTA adds its partial rows for
         // those tokens into q's tile with one bulk reduction, counted in bytes on q's
@@ -1161,8 +1184,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         if constexpr (SILU) {
-            // warp-uniform: the token maxima are reduced with shuffles
-            if (warp >= 2 && __all_sync(0xffffffffu, mbar_wait(bar_red, 0, limit_ns))) {
+            if (warp >= 2 && mbar_wait(bar_red, 0, limit_ns)) {
                 const int etid = threadIdx.x - 64;
                 const int32_t *P = reinterpret_cast<const int32_t *>(smem);
                 // this CTA's tokens only: rows m0 .. m1 - 1 of the summed tile

@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for sm_100a: mbarrier, TMA tile loads, tcgen05 (TMEM alloc,
-// MMA kind::i8, commit, ld) and the bounded waits every kernel of this library uses.
+// MMA kind::i8 and kind::f8f6f4, commit, ld) and the bounded waits every kernel of this library uses.
 #pragma once
 
 #include <cuda.h>
@@ -247,6 +247,52 @@ __device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
+// The FP8 forms: E4M3 x E4M3 -> binary32 accumulator (kind::f8f6f4), same operand layout
+// (one byte per element, K = 32 per instruction).
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 8-bit MMA of either element type: F8 = E4M3 with binary32 accumulators, else int8 with
+// int32 accumulators.
+template <bool F8>
+__device__ __forceinline__ void umma_8bit(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    if constexpr (F8)
+        umma_e4m3(d_tmem, a_desc, b_desc, idesc, accumulate);
+    else
+        umma_i8(d_tmem, a_desc, b_desc, idesc, accumulate);
+}
+
+template <bool F8>
+__device__ __forceinline__ void umma_8bit_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate)
+{
+    if constexpr (F8)
+        umma_e4m3_pair(d_tmem, a_desc, b_desc, idesc, accumulate);
+    else
+        umma_i8_pair(d_tmem, a_desc, b_desc, idesc, accumulate);
+}
+
 // Arrive on the barrier at offset `bar` in every CTA of `cta_mask` once the pair's MMAs
 // issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask)
@@ -346,6 +392,22 @@ __host__ __device__ constexpr uint32_t idesc_i8(int m, int n)
            | (static_cast<uint32_t>(m >> 4) << 24);       // M / 16
 }
 
+// Instruction descriptor of tcgen05.mma kind::f8f6f4 with E4M3 A and B (format code 0) and a
+// binary32 D, both operands K-major, shape M x N as for idesc_i8.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n)
+{
+    return (1u << 4)                                      // D format: F32
+           | (0u << 7)                                    // A format: E4M3
+           | (0u << 10)                                   // B format: E4M3
+           | (static_cast<uint32_t>(n >> 3) << 17)        // N / 8
+           | (static_cast<uint32_t>(m >> 4) << 24);       // M / 16
+}
+
+template <bool F8> __host__ __device__ constexpr uint32_t idesc_8bit(int m, int n)
+{
+    return F8 ? idesc_e4m3(m, n) : idesc_i8(m, n);
+}
+
 // ------------------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank()
@@ -367,6 +429,17 @@ __device__ __forceinline__ uint32_t map_peer_smem(uint32_t saddr, uint32_t rank)
 {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// 16 bytes from distributed shared memory (an address from map_peer_smem, 16-byte aligned).
+__device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t addr)
+{
+    uint4 r;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(addr)
+                 : "memory");
     return r;
 }
 
@@ -421,6 +494,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 __device__ __forceinline__ float dequant_f32(int32_t acc, float s_tok, float s_ch)
 {
     return __fmul_rn(__fmul_rn(__int2float_rn(acc), s_tok), s_ch);
+}
+
+// Sum of two accumulator words (int32 for INT8, binary32 bits for FP8).
+template <bool F8> __device__ __forceinline__ uint32_t acc_add(uint32_t a, uint32_t b)
+{
+    if constexpr (F8)
+        return __float_as_uint(__fadd_rn(__uint_as_float(a), __uint_as_float(b)));
+    else
+        return a + b;
+}
+
+// Dequantization of one accumulator word: y = (acc * s_tok) * s_ch in binary32 (the INT8
+// accumulator converted to binary32 first, round to nearest even).
+template <bool F8> __device__ __forceinline__ float dequant_acc(uint32_t w, float s_tok, float s_ch)
+{
+    if constexpr (F8)
+        return __fmul_rn(__fmul_rn(__uint_as_float(w), s_tok), s_ch);
+    else
+        return dequant_f32(static_cast<int32_t>(w), s_tok, s_ch);
 }
 
 } // namespace w8a8

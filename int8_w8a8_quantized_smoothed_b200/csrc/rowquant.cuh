@@ -151,15 +151,73 @@ __device__ __forceinline__ void quant_bits8(const float (&y)[8], float s, float 
     }
 }
 
+// ---- FP8 (OCP E4M3) codes
+//
+// E4M3: sign, 4 exponent bits (bias 7), 3 fraction bits, no infinities; largest finite 448.
+// A value's code is RN-even of it to E4M3 with saturation to +-448 (cvt.rn.satfinite), and
+// the per-token scale is s = amax / 448, so code = e4m3(RN(y / s)).
+
+// Codes of two binary32 values, lo in the low byte of the result.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+constexpr float kBracketLo = 0x1.ffffep-1f; // 1 - 2^-20
+constexpr float kBracketHi = 0x1.00001p+0f; // 1 + 2^-20
+
+// Codes of eight values (two 32-bit words, value i in byte i) given s, rl = RN(r (1 - 2^-20))
+// and rh = RN(r (1 + 2^-20)) with r = RN(1 / s), s >= 2^-100. Each of RN(y rl), RN(y rh)
+// carries at most three binary32 roundings (relative 3 * 2^-24 together) on top of the
+// +-2^-20 offset, so they bracket RN(y / s) strictly in magnitude, and rounding to E4M3 is
+// monotone: when both ends give the same code, so does the exact quotient. Otherwise (an
+// E4M3 rounding midpoint within about 2^-20 relative of y / s: probability about 2^-12 per
+// vector) the IEEE quotients decide all eight. Results in the binary32 subnormal range
+// (|y / s| < 2^-126) are all far below the smallest E4M3 step, so every form gives +-0 with
+// the sign of y.
+__device__ __forceinline__ uint2 quant_e4m3_8(const float (&y)[8], float s, float rl, float rh)
+{
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = mul2(make_float2(y[2 * i], y[2 * i + 1]), splat2(rl));
+        const float2 b = mul2(make_float2(y[2 * i], y[2 * i + 1]), splat2(rh));
+        lo[i] = e4m3x2(a.x, a.y);
+        hi[i] = e4m3x2(b.x, b.y);
+    }
+    uint2 out = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+    const uint2 chk = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+    if (out.x != chk.x || out.y != chk.y) {
+        uint32_t e[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            e[i] = e4m3x2(__fdiv_rn(y[2 * i], s), __fdiv_rn(y[2 * i + 1], s));
+        out = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+    }
+    return out;
+}
+
+// Codes by the IEEE quotient alone (tiny scales, whose reciprocal may not be finite).
+__device__ __forceinline__ uint2 quant_e4m3_8_exact(const float (&y)[8], float s)
+{
+    uint32_t e[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        e[i] = e4m3x2(__fdiv_rn(y[2 * i], s), __fdiv_rn(y[2 * i + 1], s));
+    return make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+}
+
 // Quantizes the part of a row held in registers (v[c][0..7] for vector v0 + c*blockDim + tid,
 // vectors below v1) given the row's absmax, writes its codes; the CTA's thread 0 writes the
-// scale when s_out is given.
-template <int NCH>
+// scale when s_out is given. F8: E4M3 codes with s = amax / 448, else int8 with s = amax / 127.
+template <int NCH, bool F8 = false>
 __device__ __forceinline__ void quantize_and_store(const float (&v)[NCH][8], float amax, int v0,
                                                    int v1, int8_t *__restrict__ qrow,
                                                    float *__restrict__ s_out)
 {
-    const float s = __fdiv_rn(amax, 127.0f);
+    const float s = __fdiv_rn(amax, F8 ? 448.0f : 127.0f);
     if (s_out && threadIdx.x == 0)
         *s_out = s;
     // the product path needs a finite reciprocal; tiny scales take the exact quotient
@@ -169,8 +227,13 @@ __device__ __forceinline__ void quantize_and_store(const float (&v)[NCH][8], flo
     for (int c = 0; c < NCH; ++c) {
         const int vi = v0 + c * blockDim.x + threadIdx.x;
         if (vi < v1) {
-            uint2 out = make_uint2(0u, 0u);
-            if (by_product) {
+            uint2 out = make_uint2(0u, 0u); // an all-zero row: s = 0, every code +0
+            if constexpr (F8) {
+                if (by_product)
+                    out = quant_e4m3_8(v[c], s, __fmul_rn(r, kBracketLo), __fmul_rn(r, kBracketHi));
+                else if (amax > 0.0f)
+                    out = quant_e4m3_8_exact(v[c], s);
+            } else if (by_product) {
                 uint32_t b[8];
                 quant_bits8(v[c], s, r, b);
                 out.x = pack_low_bytes(b[0], b[1], b[2], b[3]);
@@ -225,7 +288,7 @@ __device__ __forceinline__ void load_row(const uint4 *__restrict__ xr, int nvec,
 // SiLU, 64 for RMSNorm, which keeps gamma' in registers), since with so little work per
 // thread the arithmetic and the reductions' latency, not HBM, set their pace.
 
-template <int NCH>
+template <int NCH, bool F8 = false>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quantize_rows_kernel(const uint16_t *__restrict__ x,
                                                              const float *__restrict__ sinv,
                                                              int K, int M,
@@ -266,7 +329,7 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quant
             }
         }
         amax = block_max(amax, sh[it & 1u]);
-        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * K, s_tok + row);
+        quantize_and_store<NCH, F8>(v, amax, 0, nvec, q + row * K, s_tok + row);
     }
 }
 
@@ -347,7 +410,7 @@ __global__ void __launch_bounds__(256) quantize_rows_static_kernel(
 
 // ----------------------------------------------------------------- smoothed RMSNorm + quant
 
-template <int NCH, bool RES>
+template <int NCH, bool RES, bool F8 = false>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsnorm_quant_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ res, uint16_t *__restrict__ h_out,
     const float *__restrict__ gamma, float eps, int K, int M, int8_t *__restrict__ q,
@@ -441,7 +504,7 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsno
             }
         }
         amax = block_max(amax, shf);
-        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * K, s_tok + row);
+        quantize_and_store<NCH, F8>(v, amax, 0, nvec, q + row * K, s_tok + row);
     }
 }
 
@@ -520,7 +583,7 @@ __device__ __forceinline__ void silu_mul8(const float (&g)[8], const float (&u)[
     }
 }
 
-template <int NCH>
+template <int NCH, bool F8 = false>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) silu_mul_quant_kernel(const uint16_t *__restrict__ gu,
                                                               int I, int M,
                                                               int8_t *__restrict__ q,
@@ -557,30 +620,30 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) silu_
             }
         }
         amax = block_max(amax, sh[it & 1u]);
-        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * I, s_tok + row);
+        quantize_and_store<NCH, F8>(v, amax, 0, nvec, q + row * I, s_tok + row);
     }
 }
 
-// ----------------------------------------------------------------- quantization with a known absmax
+// ----------------------------------------------------------------- quantization of fp32 rows
 //
 // Second half of the fused SiLU*up path: a (binary32 [M, I], written by the GEMM epilogue)
-// is quantized per token with s = amax[m] / 127, amax[m] being the token's max |a| that the
-// epilogue raised with atomicMax on its bits. Each word is cleared after use, so the words
-// are zero again for the next call.
+// is quantized per token with s = max_j |a[m, j]| / 127, exactly as the SiLU*up row kernel
+// quantizes the same values.
 
 template <int NCH>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quantize_f32_rows_kernel(
-    const float *__restrict__ a, unsigned int *__restrict__ amax_words, int I, int M,
-    int8_t *__restrict__ q, float *__restrict__ s_tok)
+    const float *__restrict__ a, int I, int M, int8_t *__restrict__ q, float *__restrict__ s_tok)
 {
+    __shared__ float sh[2][32]; // by row parity: one barrier per row
     if (threadIdx.x == 0)
         pdl_launch_dependents();
-    pdl_wait(); // a and the maxima come from the previous kernel
+    pdl_wait(); // a comes from the previous kernel
     const int nvec = I >> 3;
-    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
-        const float amax = __uint_as_float(__ldcg(amax_words + row));
+    int64_t row = blockIdx.x;
+    for (uint32_t it = 0; row < M; row += gridDim.x, ++it) {
         const float4 *ar = reinterpret_cast<const float4 *>(a + row * I);
         float v[NCH][8];
+        float amax = 0.0f;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
             const int vi = c * blockDim.x + threadIdx.x;
@@ -595,10 +658,13 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quant
                     v[c][i] = 0.0f;
             }
         }
+#pragma unroll
+        for (int c = 0; c < NCH; ++c)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                amax = fmaxf(amax, fabsf(v[c][i]));
+        amax = block_max(amax, sh[it & 1u]);
         quantize_and_store<NCH>(v, amax, 0, nvec, q + row * I, s_tok + row);
-        __syncthreads(); // every thread has read the word
-        if (threadIdx.x == 0)
-            amax_words[row] = 0u;
     }
 }
 

@@ -230,64 +230,59 @@ unsigned row_grid(const void *kernel, int threads, int64_t M, int dev, int sms)
     return static_cast<unsigned>(M < g ? M : g);
 }
 
-template <int NCH>
+template <int NCH, bool F8>
 int launch_quantize_rows(const uint16_t *x, const float *sinv, int64_t M, int K, int8_t *q,
                          float *s, int threads, int dev, int sms, cudaStream_t st)
 {
-    const void *fn = reinterpret_cast<const void *>(&quantize_rows_kernel<NCH>);
+    const void *fn = reinterpret_cast<const void *>(&quantize_rows_kernel<NCH, F8>);
     if (int rc = ensure_smem(fn, dev, 0))
         return rc;
-    return launch_kernel(quantize_rows_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
+    return launch_kernel(quantize_rows_kernel<NCH, F8>, dim3(row_grid(fn, threads, M, dev, sms)),
                          dim3(threads), 0, st, x, sinv, K, static_cast<int>(M), q, s);
 }
 
-template <int NCH, bool RES>
+template <int NCH, bool RES, bool F8>
 int launch_rmsnorm_t(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
                      int64_t M, int K, int8_t *q, float *s, int threads, int dev, int sms,
                      cudaStream_t st)
 {
-    const void *fn = reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, RES>);
+    const void *fn = reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, RES, F8>);
     if (int rc = ensure_smem(fn, dev, 0))
         return rc;
-    return launch_kernel(rmsnorm_quant_kernel<NCH, RES>, dim3(row_grid(fn, threads, M, dev, sms)),
+    return launch_kernel(rmsnorm_quant_kernel<NCH, RES, F8>, dim3(row_grid(fn, threads, M, dev, sms)),
                          dim3(threads), 0, st, x, r, h, g, eps, K, static_cast<int>(M), q, s);
 }
 
-template <int NCH>
+template <int NCH, bool F8>
 int launch_rmsnorm(const uint16_t *x, const uint16_t *r, uint16_t *h, const float *g, float eps,
                    int64_t M, int K, int8_t *q, float *s, int threads, int dev, int sms,
                    cudaStream_t st)
 {
     if (r)
-        return launch_rmsnorm_t<NCH, true>(x, r, h, g, eps, M, K, q, s, threads, dev, sms, st);
-    return launch_rmsnorm_t<NCH, false>(x, r, h, g, eps, M, K, q, s, threads, dev, sms, st);
+        return launch_rmsnorm_t<NCH, true, F8>(x, r, h, g, eps, M, K, q, s, threads, dev, sms, st);
+    return launch_rmsnorm_t<NCH, false, F8>(x, r, h, g, eps, M, K, q, s, threads, dev, sms, st);
 }
 
-template <int NCH>
+template <int NCH, bool F8>
 int launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int threads, int dev,
                 int sms, cudaStream_t st)
 {
-    const void *fn = reinterpret_cast<const void *>(&silu_mul_quant_kernel<NCH>);
+    const void *fn = reinterpret_cast<const void *>(&silu_mul_quant_kernel<NCH, F8>);
     if (int rc = ensure_smem(fn, dev, 0))
         return rc;
-    return launch_kernel(silu_mul_quant_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
+    return launch_kernel(silu_mul_quant_kernel<NCH, F8>, dim3(row_grid(fn, threads, M, dev, sms)),
                          dim3(threads), 0, st, gu, I, static_cast<int>(M), q, s);
 }
 
 template <int NCH>
-int launch_quantize_f32(const float *a, unsigned int *amax, int64_t M, int I, int8_t *q,
-                        float *s, int threads, int dev, int sms, cudaStream_t st)
+int launch_quantize_f32(const float *a, int64_t M, int I, int8_t *q, float *s, int threads,
+                        int dev, int sms, cudaStream_t st)
 {
     const void *fn = reinterpret_cast<const void *>(&quantize_f32_rows_kernel<NCH>);
     if (int rc = ensure_smem(fn, dev, 0))
         return rc;
     return launch_kernel(quantize_f32_rows_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
-                         dim3(threads), 0, st, a, amax, I, static_cast<int>(M), q, s);
-}
-
-size_t align16_size(size_t b)
-{
-    return (b + 15) & ~static_cast<size_t>(15);
+                         dim3(threads), 0, st, a, I, static_cast<int>(M), q, s);
 }
 
 // ------------------------------------------------------------------ GEMM planning
@@ -313,7 +308,7 @@ int decode_nt(int64_t M)
 
 
 int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
-              GemmPlan *p)
+              GemmPlan *p, bool f8 = false)
 {
     if (variant < 0 || variant > 3 || ctas < 0 ||
         (tile_n != 0 && tile_n != 128 && tile_n != 256 && tile_n != 512))
@@ -399,20 +394,20 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K)
     return W8A8_OK;
 }
 
-template <int BN, int STAGES, bool SILU>
+template <int BN, int STAGES, bool SILU, bool F8 = false>
 int launch_prefill(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
                    const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
                    const SiluOut &so, int dev, int num_sms, cudaStream_t st)
 {
     using Cfg = PrefillCfg<BN, STAGES>;
-    const void *fn = reinterpret_cast<const void *>(&gemm_prefill_kernel<BN, STAGES, SILU>);
+    const void *fn = reinterpret_cast<const void *>(&gemm_prefill_kernel<BN, STAGES, SILU, F8>);
     int rc = ensure_smem(fn, dev, Cfg::kSmemBytes);
     if (rc)
         return rc;
     const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
-    return launch_kernel(gemm_prefill_kernel<BN, STAGES, SILU>, dim3(grid), dim3(kGemmThreads),
+    return launch_kernel(gemm_prefill_kernel<BN, STAGES, SILU, F8>, dim3(grid), dim3(kGemmThreads),
                          Cfg::kSmemBytes, st, ta, tb, s_tok, s_ch, static_cast<int>(M),
                          static_cast<int>(N), static_cast<int>(K), y, acc, so, prefetch,
                          kWaitLimitNs);
@@ -448,13 +443,13 @@ int pair_clusters(const void *kernel, int smem, int dev, int num_sms)
     return n;
 }
 
-template <int STAGES, bool SILU>
+template <int STAGES, bool SILU, bool F8 = false>
 int launch_prefill_pair(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
                         const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y,
                         int32_t *acc, const SiluOut &so, int dev, int num_sms, cudaStream_t st)
 {
     using Cfg = PairCfg<STAGES>;
-    auto kernel = gemm_prefill_pair_kernel<STAGES, SILU>;
+    auto kernel = gemm_prefill_pair_kernel<STAGES, SILU, F8>;
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes);
     if (rc)
         return rc;
@@ -509,7 +504,7 @@ int fit_cluster(Kern kernel, int want, int64_t clusters_needed, int smem, int de
     return 1;
 }
 
-template <int NT, int STAGES, int KPS, bool SILU>
+template <int NT, int STAGES, int KPS, bool SILU, bool F8 = false>
 int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
                   const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
                   uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev, cudaStream_t st)
@@ -517,7 +512,7 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
     if (p.variant == 3) {
         using Cfg = DecodeCfg<NT, STAGES, KPS, true>;
-        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU>;
+        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU, F8>;
         if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
             return rc;
         const int64_t NB = ((N + kBM - 1) / kBM) * ((M + NT - 1) / NT); // x token tiles
@@ -530,7 +525,7 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
                                      kWaitLimitNs);
     }
     using Cfg = DecodeCfg<NT, STAGES, KPS, false>;
-    auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false, SILU>;
+    auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false, SILU, F8>;
     if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
         return rc;
     int32_t *ws_part =
@@ -546,19 +541,43 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
 
 // Decode launch by token tile: (stages, k-blocks per stage) keep ~200 KB of weight and
 // token bytes in flight per SM.
-template <bool SILU>
+template <bool SILU, bool F8 = false>
 int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
                      const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
                      uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev,
                      cudaStream_t st)
 {
     switch (p.nt) {
-    case 16: return launch_decode<16, 3, 4, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
-    case 32: return launch_decode<32, 5, 2, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
-    case 64: return launch_decode<64, 4, 2, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
-    case 128: return launch_decode<128, 5, 1, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
-    default: return launch_decode<256, 3, 1, SILU>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 16: return launch_decode<16, 3, 4, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 32: return launch_decode<32, 5, 2, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 64: return launch_decode<64, 4, 2, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    case 128: return launch_decode<128, 5, 1, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    default: return launch_decode<256, 3, 1, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
     }
+}
+
+// The FP8 GEMM launch for a plan (plain dequant epilogue, variants 1 and 2).
+int gemm_run_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const float *s_ch,
+                 int64_t M, int64_t N, int64_t K, uint16_t *y, float *acc_out, void *workspace,
+                 const GemmPlan &p, int dev, int sms, cudaStream_t st)
+{
+    const SiluOut none{nullptr, 0};
+    int32_t *acc = reinterpret_cast<int32_t *>(acc_out); // raw binary32 words
+    if (p.variant == 1) {
+        const int bn = p.tile_n == 128 ? 128 : p.tile_n == 256 ? 256 : 128;
+        CUtensorMap ta, tb;
+        if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, bn))
+            return W8A8_ERR_CUDA;
+        if (p.tile_n == 512)
+            return launch_prefill_pair<6, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
+        if (p.tile_n == 256)
+            return launch_prefill<256, 4, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
+        return launch_prefill<128, 6, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
+    }
+    CUtensorMap tw, tx;
+    if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
+        return W8A8_ERR_CUDA;
+    return launch_decode_nt<false, true>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, workspace, none, dev, st);
 }
 
 // The GEMM launch for a plan: plain dequant epilogue (so == nullptr) or the fused SiLU*up
@@ -567,7 +586,7 @@ int gemm_run(const int8_t *xq, const float *s_tok, const int8_t *wq, const float
              int64_t M, int64_t N, int64_t K, uint16_t *y, int32_t *acc_out, void *workspace,
              const GemmPlan &p, const SiluOut *so, int dev, int sms, cudaStream_t st)
 {
-    const SiluOut none{nullptr, nullptr, 0};
+    const SiluOut none{nullptr, 0};
     if (p.variant == 1) {
         // tile_n: 128 -> 128 x 128, 256 -> 128 x 256, 512 -> 256 x 256 by a CTA pair
         const int bn = p.tile_n == 128 ? 128 : p.tile_n == 256 ? 256 : 128;
@@ -593,6 +612,87 @@ int gemm_run(const int8_t *xq, const float *s_tok, const int8_t *wq, const float
     if (so)
         return launch_decode_nt<true>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, *so, dev, st);
     return launch_decode_nt<false>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc_out, workspace, none, dev, st);
+}
+
+
+// ------------------------------------------------------------------ row entry points
+// (F8: E4M3 codes with scale amax / 448, else int8 codes with amax / 127)
+
+template <bool F8>
+int quantize_rows_impl(const uint16_t *x, const float *smooth_inv, int64_t M, int64_t K,
+                       int8_t *q, float *s_tok, w8a8_stream_t stream)
+{
+    if (!x || !q || !s_tok)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, K);
+    if (rc)
+        return rc;
+    if (!aligned16(x) || !aligned16(q) || (smooth_inv && !aligned16(smooth_inv)))
+        return W8A8_ERR_ALIGNMENT;
+    if (static_cast<const void *>(x) == static_cast<const void *>(q))
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    const RowLaunch L = row_launch(K);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (L.nch) {
+    case 1: return launch_quantize_rows<1, F8>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    case 2: return launch_quantize_rows<2, F8>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    default: return launch_quantize_rows<4, F8>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    }
+}
+
+template <bool F8>
+int rmsnorm_quant_impl(const uint16_t *x, const uint16_t *residual, uint16_t *h_out,
+                       const float *gamma_smoothed, float eps, int64_t M, int64_t K, int8_t *q,
+                       float *s_tok, w8a8_stream_t stream)
+{
+    if (!x || !gamma_smoothed || !q || !s_tok || ((residual == nullptr) != (h_out == nullptr)))
+        return W8A8_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f))
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, K);
+    if (rc)
+        return rc;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(gamma_smoothed) ||
+        (residual && (!aligned16(residual) || !aligned16(h_out))))
+        return W8A8_ERR_ALIGNMENT;
+    if (h_out && static_cast<const void *>(h_out) == static_cast<const void *>(x))
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    const RowLaunch L = row_launch(K);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (L.nch) {
+    case 1: return launch_rmsnorm<1, F8>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    case 2: return launch_rmsnorm<2, F8>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    default: return launch_rmsnorm<4, F8>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
+    }
+}
+
+template <bool F8>
+int silu_mul_quant_impl(const uint16_t *gate_up, int64_t M, int64_t I, int8_t *q, float *s_tok,
+                        w8a8_stream_t stream)
+{
+    if (!gate_up || !q || !s_tok)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_row_shape(M, I);
+    if (rc)
+        return rc;
+    if (!aligned16(gate_up) || !aligned16(q))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const RowLaunch L = row_launch(I);
+    switch (L.nch) {
+    case 1: return launch_silu<1, F8>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
+    case 2: return launch_silu<2, F8>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
+    default: return launch_silu<4, F8>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
+    }
 }
 
 } // namespace
@@ -644,28 +744,18 @@ const char *w8a8_status_string(int status)
     }
 }
 
+
 int w8a8_quantize_rows(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, int64_t K,
                        int8_t *q, float *s_tok, w8a8_stream_t stream)
 {
-    if (!x || !q || !s_tok)
-        return W8A8_ERR_INVALID_ARG;
-    int rc = check_row_shape(M, K);
-    if (rc)
-        return rc;
-    if (!aligned16(x) || !aligned16(q) || (smooth_inv && !aligned16(smooth_inv)))
-        return W8A8_ERR_ALIGNMENT;
-    if (static_cast<const void *>(x) == static_cast<const void *>(q))
-        return W8A8_ERR_INVALID_ARG;
-    int dev, sms;
-    if ((rc = current_device(&dev, &sms)))
-        return rc;
-    const RowLaunch L = row_launch(K);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    switch (L.nch) {
-    case 1: return launch_quantize_rows<1>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
-    case 2: return launch_quantize_rows<2>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
-    default: return launch_quantize_rows<4>(x, smooth_inv, M, (int)K, q, s_tok, L.threads, dev, sms, st);
-    }
+    return quantize_rows_impl<false>(x, smooth_inv, M, K, q, s_tok, stream);
+}
+
+int w8a8_quantize_rows_fp8(const w8a8_bf16 *x, const float *smooth_inv, int64_t M, int64_t K,
+                           uint8_t *q, float *s_tok, w8a8_stream_t stream)
+{
+    return quantize_rows_impl<true>(x, smooth_inv, M, K, reinterpret_cast<int8_t *>(q), s_tok,
+                                    stream);
 }
 
 int w8a8_quantize_rows_static(const w8a8_bf16 *x, const float *smooth_inv, float scale,
@@ -697,54 +787,35 @@ int w8a8_quantize_rows_static(const w8a8_bf16 *x, const float *smooth_inv, float
                          static_cast<int>(K), nvec_total, static_cast<int>(M), q, s_tok);
 }
 
+
+
 int w8a8_smooth_rmsnorm_quant(const w8a8_bf16 *x, const w8a8_bf16 *residual, w8a8_bf16 *h_out,
                               const float *gamma_smoothed, float eps, int64_t M, int64_t K,
                               int8_t *q, float *s_tok, w8a8_stream_t stream)
 {
-    if (!x || !gamma_smoothed || !q || !s_tok || ((residual == nullptr) != (h_out == nullptr)))
-        return W8A8_ERR_INVALID_ARG;
-    if (!(eps >= 0.0f))
-        return W8A8_ERR_INVALID_ARG;
-    int rc = check_row_shape(M, K);
-    if (rc)
-        return rc;
-    if (!aligned16(x) || !aligned16(q) || !aligned16(gamma_smoothed) ||
-        (residual && (!aligned16(residual) || !aligned16(h_out))))
-        return W8A8_ERR_ALIGNMENT;
-    if (h_out && static_cast<const void *>(h_out) == static_cast<const void *>(x))
-        return W8A8_ERR_INVALID_ARG;
-    int dev, sms;
-    if ((rc = current_device(&dev, &sms)))
-        return rc;
-    const RowLaunch L = row_launch(K);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    switch (L.nch) {
-    case 1: return launch_rmsnorm<1>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
-    case 2: return launch_rmsnorm<2>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
-    default: return launch_rmsnorm<4>(x, residual, h_out, gamma_smoothed, eps, M, (int)K, q, s_tok, L.threads, dev, sms, st);
-    }
+    return rmsnorm_quant_impl<false>(x, residual, h_out, gamma_smoothed, eps, M, K, q, s_tok,
+                                     stream);
+}
+
+int w8a8_smooth_rmsnorm_quant_fp8(const w8a8_bf16 *x, const w8a8_bf16 *residual,
+                                  w8a8_bf16 *h_out, const float *gamma_smoothed, float eps,
+                                  int64_t M, int64_t K, uint8_t *q, float *s_tok,
+                                  w8a8_stream_t stream)
+{
+    return rmsnorm_quant_impl<true>(x, residual, h_out, gamma_smoothed, eps, M, K,
+                                    reinterpret_cast<int8_t *>(q), s_tok, stream);
 }
 
 int w8a8_silu_mul_quant(const w8a8_bf16 *gate_up, int64_t M, int64_t I, int8_t *q, float *s_tok,
                         w8a8_stream_t stream)
 {
-    if (!gate_up || !q || !s_tok)
-        return W8A8_ERR_INVALID_ARG;
-    int rc = check_row_shape(M, I);
-    if (rc)
-        return rc;
-    if (!aligned16(gate_up) || !aligned16(q))
-        return W8A8_ERR_ALIGNMENT;
-    int dev, sms;
-    if ((rc = current_device(&dev, &sms)))
-        return rc;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const RowLaunch L = row_launch(I);
-    switch (L.nch) {
-    case 1: return launch_silu<1>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
-    case 2: return launch_silu<2>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
-    default: return launch_silu<4>(gate_up, M, (int)I, q, s_tok, L.threads, dev, sms, st);
-    }
+    return silu_mul_quant_impl<false>(gate_up, M, I, q, s_tok, stream);
+}
+
+int w8a8_silu_mul_quant_fp8(const w8a8_bf16 *gate_up, int64_t M, int64_t I, uint8_t *q,
+                            float *s_tok, w8a8_stream_t stream)
+{
+    return silu_mul_quant_impl<true>(gate_up, M, I, reinterpret_cast<int8_t *>(q), s_tok, stream);
 }
 
 size_t w8a8_gemm_silu_quant_workspace_size(int64_t M, int64_t I, int64_t K)
@@ -757,7 +828,7 @@ size_t w8a8_gemm_silu_quant_workspace_size(int64_t M, int64_t I, int64_t K)
     GemmPlan p;
     if (plan_gemm(M, 2 * I, K, 0, 0, 0, sms, &p))
         return 0;
-    return align16_size(p.ws_bytes) + align16_size(static_cast<size_t>(M) * 4u);
+    return p.ws_bytes;
 }
 
 int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_il,
@@ -781,20 +852,18 @@ int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_
     GemmPlan p;
     if ((rc = plan_gemm(M, 2 * I, K, 0, 0, 0, sms, &p)))
         return rc;
-    const size_t amax_off = align16_size(p.ws_bytes);
-    if (!workspace || workspace_bytes < amax_off + align16_size(static_cast<size_t>(M) * 4u))
+    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
         return W8A8_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const SiluOut so{a, reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + amax_off),
-                     static_cast<int>(I)};
+    const SiluOut so{a, static_cast<int>(I)};
     if ((rc = gemm_run(xq, s_tok, wq_il, s_ch_il, M, 2 * I, K, nullptr, nullptr, workspace, p,
                        &so, dev, sms, st)))
         return rc;
     const RowLaunch L = row_launch(I);
     switch (L.nch) {
-    case 1: return launch_quantize_f32<1>(a, so.amax, M, (int)I, q, s_out, L.threads, dev, sms, st);
-    case 2: return launch_quantize_f32<2>(a, so.amax, M, (int)I, q, s_out, L.threads, dev, sms, st);
-    default: return launch_quantize_f32<4>(a, so.amax, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    case 1: return launch_quantize_f32<1>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    case 2: return launch_quantize_f32<2>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    default: return launch_quantize_f32<4>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
     }
 }
 
@@ -849,6 +918,45 @@ int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq, co
 {
     return w8a8_gemm_dequant_ex(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace,
                                 workspace_bytes, 0, 0, 0, stream);
+}
+
+size_t w8a8_gemm_fp8_workspace_size(int64_t M, int64_t N, int64_t K, int variant, int ctas,
+                                    int tile_n)
+{
+    if (check_gemm_shape(M, N, K))
+        return 0;
+    int dev, sms = 148;
+    if (current_device(&dev, &sms))
+        sms = 148;
+    GemmPlan p;
+    if (plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p, true))
+        return 0;
+    return p.ws_bytes;
+}
+
+int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq,
+                          const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
+                          float *acc_out, void *workspace, size_t workspace_bytes, int variant,
+                          int ctas, int tile_n, w8a8_stream_t stream)
+{
+    if (!xq || !s_tok || !wq || !s_ch || !y)
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc)
+        return rc;
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(s_ch) || !aligned16(y) ||
+        (acc_out && !aligned16(acc_out)) || (workspace && !aligned16(workspace)))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    GemmPlan p;
+    if ((rc = plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p, true)))
+        return rc;
+    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
+        return W8A8_ERR_WORKSPACE;
+    return gemm_run_fp8(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace, p, dev, sms,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream)
@@ -985,5 +1093,5 @@ extern "C" int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, c
     if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
         return W8A8_ERR_CUDA;
     return launch_decode_nt<false>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, scratch,
-                                   SiluOut{nullptr, nullptr, 0}, dev, st);
+                                   SiluOut{nullptr, 0}, dev, st);
 }

@@ -41,7 +41,8 @@ def lib():
         L.oracle_quantize_row_f32_fp8.argtypes = [P, I64, P, P]
         L.oracle_quantize_rows_fp8.argtypes = [P, P, I64, I64, P, P, C.c_int]
         L.oracle_quantize_rows_f32_fp8.argtypes = [P, I64, I64, P, P, C.c_int]
-        L.oracle_gemm_fp8.argtypes = [P, P, P, P, I64, I64, I64, P, P, P]
+        L.oracle_dequant_f32acc.argtypes = [P, P, P, I64, I64, P]
+        L.oracle_gemm_fp8.argtypes = [P, P, P, P, I64, I64, I64, P, P, P, C.c_int]
         L.oracle_minmax_scale.restype = C.c_float
         L.oracle_minmax_scale.argtypes = [P, I64]
         L.oracle_quantize_rows_static.argtypes = [P, P, C.c_float, I64, I64, P, C.c_int]
@@ -190,7 +191,17 @@ def rtn_weights_fp8(w_bf16, s=None, nthreads=NTHREADS):
     return quantize_rows_f32_fp8(v, nthreads)
 
 
-def gemm_fp8(xq, s_tok, wq, s_ch):
+def dequant_f32acc(acc, s_tok, s_ch):
+    """bf16 bits of (acc * s_tok[m]) * s_ch[n] for binary32 accumulators acc [M, N]."""
+    acc = _c(acc, np.float32)
+    M, N = acc.shape
+    y = np.empty((M, N), dtype=np.uint16)
+    lib().oracle_dequant_f32acc(_p(acc), _p(_c(s_tok, np.float32)), _p(_c(s_ch, np.float32)),
+                                M, N, _p(y))
+    return y
+
+
+def gemm_fp8(xq, s_tok, wq, s_ch, nthreads=NTHREADS):
     """FP8 GEMM reference -> (y bf16 bits [M, N], exact acc float64, sum |products| float64)."""
     xq = _c(xq, np.uint8)
     wq = _c(wq, np.uint8)
@@ -201,7 +212,8 @@ def gemm_fp8(xq, s_tok, wq, s_ch):
     acc = np.empty((M, N), dtype=np.float64)
     absacc = np.empty((M, N), dtype=np.float64)
     y = np.empty((M, N), dtype=np.uint16)
-    lib().oracle_gemm_fp8(_p(xq), _p(st), _p(wq), _p(sc), M, N, K, _p(acc), _p(absacc), _p(y))
+    lib().oracle_gemm_fp8(_p(xq), _p(st), _p(wq), _p(sc), M, N, K, _p(acc), _p(absacc), _p(y),
+                          nthreads)
     return y, acc, absacc
 
 

@@ -358,14 +358,58 @@ int oracle_quantize_rows_f32_fp8(const float *y, int64_t M, int64_t K, uint8_t *
     return 0;
 }
 
+/* The FP8 epilogue applied to given binary32 accumulators [M, N]: y = bf16_RN((acc s_tok)
+ * s_ch). Used to check a device's epilogue against its own accumulators, whose rounding
+ * order is the tensor cores'. */
+int oracle_dequant_f32acc(const float *acc, const float *s_tok, const float *s_ch, int64_t M,
+                          int64_t N, uint16_t *y)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float f = acc[m * N + n] * s_tok[m];
+            f = f * s_ch[n];
+            y[m * N + n] = oracle_f32_to_bf16(f);
+        }
+    return 0;
+}
+
 /*
  * FP8 GEMM reference: acc[m,n] = sum_k e4m3(xq[m,k]) e4m3(wq[n,k]) computed exactly (each
  * product is exact in binary64 and the sum stays exact for K <= 2^15: the terms are
  * multiples of 2^-18 below 2^18), also sum_k |products| (the scale of the rounding error of
  * any binary32 accumulation), and y = bf16_RN((float(acc) s_tok) s_ch).
  */
+struct gemm8_ctx {
+    const float *xd, *wd;
+    const float *s_tok, *s_ch;
+    int64_t N, K;
+    double *acc, *absacc;
+    uint16_t *y;
+};
+
+static void gemm8_row(void *vctx, int64_t m)
+{
+    struct gemm8_ctx *c = (struct gemm8_ctx *)vctx;
+    const int64_t N = c->N, K = c->K;
+    for (int64_t n = 0; n < N; ++n) {
+        double a = 0.0, b = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double p = (double)c->xd[m * K + k] * (double)c->wd[n * K + k];
+            a += p;
+            b += fabs(p);
+        }
+        c->acc[m * N + n] = a;
+        c->absacc[m * N + n] = b;
+        float f = (float)a;
+        f = f * c->s_tok[m];
+        f = f * c->s_ch[n];
+        c->y[m * N + n] = oracle_f32_to_bf16(f);
+    }
+}
+
 int oracle_gemm_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const float *s_ch,
-                    int64_t M, int64_t N, int64_t K, double *acc, double *absacc, uint16_t *y)
+                    int64_t M, int64_t N, int64_t K, double *acc, double *absacc, uint16_t *y,
+                    int nthreads)
 {
     float *xd = (float *)malloc((size_t)(M * K) * sizeof(float));
     float *wd = (float *)malloc((size_t)(N * K) * sizeof(float));
@@ -373,21 +417,8 @@ int oracle_gemm_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, co
         xd[i] = oracle_e4m3_to_f32(xq[i]);
     for (int64_t i = 0; i < N * K; ++i)
         wd[i] = oracle_e4m3_to_f32(wq[i]);
-    for (int64_t m = 0; m < M; ++m)
-        for (int64_t n = 0; n < N; ++n) {
-            double a = 0.0, b = 0.0;
-            for (int64_t k = 0; k < K; ++k) {
-                const double p = (double)xd[m * K + k] * (double)wd[n * K + k];
-                a += p;
-                b += fabs(p);
-            }
-            acc[m * N + n] = a;
-            absacc[m * N + n] = b;
-            float f = (float)a;
-            f = f * s_tok[m];
-            f = f * s_ch[n];
-            y[m * N + n] = oracle_f32_to_bf16(f);
-        }
+    struct gemm8_ctx c = {xd, wd, s_tok, s_ch, N, K, acc, absacc, y};
+    parallel_rows(gemm8_row, &c, M, nthreads);
     free(xd);
     free(wd);
     return 0;

@@ -65,13 +65,14 @@ def bf16_ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(ordered(a) - ordered(b))
 
 
-def assert_rms_rows_match(got_q, got_s, x, gamma, eps, residual=None, ref=None):
+def assert_rms_rows_match(got_q, got_s, x, gamma, eps, residual=None, ref=None,
+                          ref_fn=oracle.smooth_rmsnorm_quant):
     """GPU smoothed-RMSNorm results against the oracle. Rows whose binary64 mean of squares
     lies so close to a binary32 rounding boundary that another summation order may round it
     the other way (oracle flag `ambiguous`) may match either neighbouring binary32 value;
     every other row must match exactly."""
     if ref is None:
-        ref = oracle.smooth_rmsnorm_quant(x, gamma, eps, residual=residual)
+        ref = ref_fn(x, gamma, eps, residual=residual)
     bad = np.where((got_s != ref["s"]) | (got_q != ref["q"]).any(axis=1))[0]
     for m in bad:
         assert ref["ambiguous"][m], f"row {m} differs and is not ambiguous"
@@ -79,7 +80,7 @@ def assert_rms_rows_match(got_q, got_s, x, gamma, eps, residual=None, ref=None):
         for direction in (np.inf, -np.inf):
             ms = ref["ms"].copy()
             ms[m] = np.nextafter(np.float32(ms[m]), np.float32(direction))
-            alt = oracle.smooth_rmsnorm_quant(x[m:m + 1], gamma, eps,
+            alt = ref_fn(x[m:m + 1], gamma, eps,
                                               residual=None if residual is None
                                               else residual[m:m + 1],
                                               ms_override=ms[m:m + 1])

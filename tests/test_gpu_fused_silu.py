@@ -59,6 +59,23 @@ def test_fused_equals_unfused_gpu_chain():
     assert torch.equal(q0, q1) and torch.equal(s0, s1)
 
 
+def test_shared_workspace_after_other_stream_k_calls():
+    """One workspace serves the fused call after stream-K GEMMs of other shapes, whose
+    partial-sum slots stay as they were left."""
+    ws = w8.Workspace()
+    for M, N in ((64, 16384), (7, 4096)):  # dirty the partial slots with two other shapes
+        xq, st, wq, sc = _inputs(M, N // 2, 4096, M)
+        w8.w8a8_gemm_dequant_ex(dev(xq), dev(st), dev(wq), dev(sc), variant=2, workspace=ws)
+    M, I, K = 16, 5120, 4096
+    xq, st, wq, sc = _inputs(M, I, K, 3)
+    a_ref, q_ref, s_ref = _reference(xq, st, wq, sc)
+    wq_il, sc_il = prep.interleave_gate_up(dev(wq), dev(sc))
+    q, s, a = w8.w8a8_gemm_silu_quant(dev(xq), dev(st), wq_il, sc_il, workspace=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(s), s_ref)
+    assert np.array_equal(host(q), q_ref)
+
+
 def test_interleave_is_a_row_permutation():
     I, K = 192, 32
     wq = torch.arange(2 * I, dtype=torch.int32).repeat_interleave(K).view(2 * I, K)

@@ -191,3 +191,19 @@ def test_gemm_fp8_brute_force():
     # transposed operands give the transposed accumulator
     _, acc_t, _ = oracle.gemm_fp8(wq, sc, xq, st)
     assert np.array_equal(acc_t, acc.T)
+
+
+def test_dequant_f32acc_matches_the_gemm_epilogue():
+    """With exactly representable accumulators the epilogue alone equals the GEMM's."""
+    rng = np.random.default_rng(12)
+    xq = rng.integers(0x20, 0x40, (4, 32)).astype(np.uint8)  # small codes: sums exact in f32
+    wq = rng.integers(0x20, 0x40, (6, 32)).astype(np.uint8)
+    st = rng.uniform(0.1, 1.0, 4).astype(np.float32)
+    sc = rng.uniform(0.1, 1.0, 6).astype(np.float32)
+    y, acc, _ = oracle.gemm_fp8(xq, st, wq, sc)
+    assert np.array_equal(acc.astype(np.float32).astype(np.float64), acc)
+    assert np.array_equal(oracle.dequant_f32acc(acc.astype(np.float32), st, sc), y)
+    a = np.float32(3.0)
+    want = torch.tensor([float(np.float32(np.float32(a * st[1]) * sc[2]))]).to(torch.bfloat16)
+    got = oracle.dequant_f32acc(np.full((4, 6), a, np.float32), st, sc)[1, 2]
+    assert int(got) == int(want.view(torch.int16).item()) & 0xFFFF
