@@ -42,6 +42,9 @@ def lib():
         L.oracle_quantize_rows_fp8.argtypes = [P, P, I64, I64, P, P, C.c_int]
         L.oracle_quantize_rows_f32_fp8.argtypes = [P, I64, I64, P, P, C.c_int]
         L.oracle_dequant_f32acc.argtypes = [P, P, P, I64, I64, P]
+        L.oracle_gptq_hessian.argtypes = [P, I64, I64, C.c_double, P, P]
+        L.oracle_gptq_hinv_chol.argtypes = [P, I64, P]
+        L.oracle_gptq_quantize.argtypes = [P, I64, I64, P, P, P, P, P, P, C.c_double, P, C.c_int]
         L.oracle_gemm_fp8.argtypes = [P, P, P, P, I64, I64, I64, P, P, P, C.c_int]
         L.oracle_minmax_scale.restype = C.c_float
         L.oracle_minmax_scale.argtypes = [P, I64]
@@ -401,3 +404,52 @@ def block_reference(inputs, prep, eps, nthreads=NTHREADS):
     out["down"], _ = gemm_dequant(out["q4"], out["s4"], prep["down"]["wq"],
                                   prep["down"]["s_ch"], want_acc=False, nthreads=nthreads)
     return out
+
+
+# ------------------------------------------------------------------ GPTQ
+
+
+def gptq_hessian(x_f32, damp=0.01):
+    """H = (2/T) X^T X with dead columns set to 1 and dampening -> (H float64 [K, K], dead)."""
+    x = _c(x_f32, np.float32)
+    T, K = x.shape
+    H = np.empty((K, K), dtype=np.float64)
+    dead = np.empty(K, dtype=np.uint8)
+    lib().oracle_gptq_hessian(_p(x), T, K, float(damp), _p(H), _p(dead))
+    return H, dead.astype(bool)
+
+
+def gptq_hinv_chol(H):
+    """U upper triangular with H^-1 = U^T U."""
+    H = _c(H, np.float64)
+    K = H.shape[0]
+    U = np.empty((K, K), dtype=np.float64)
+    if lib().oracle_gptq_hinv_chol(_p(H), K, _p(U)) != 0:
+        raise ValueError("H is not positive definite")
+    return U
+
+
+def gptq_quantize(w_f32, dead, U, q_follow=None, tie_tol=0.0, want_wcomp=False,
+                  nthreads=NTHREADS):
+    """Column-by-column GPTQ of the rows of w [N, K] -> dict(q, s, wcomp, status)."""
+    w = _c(w_f32, np.float32)
+    N, K = w.shape
+    d = _c(np.asarray(dead, dtype=np.uint8), np.uint8)
+    U = _c(U, np.float64)
+    q = np.empty((N, K), dtype=np.int8)
+    s = np.empty(N, dtype=np.float32)
+    wc = np.empty((N, K), dtype=np.float64) if want_wcomp else None
+    qf = _c(q_follow, np.int8)
+    st = np.empty((N, K), dtype=np.uint8) if q_follow is not None else None
+    lib().oracle_gptq_quantize(_p(w), N, K, _p(d), _p(U), _p(q), _p(s), _p(wc), _p(qf),
+                               float(tie_tol), _p(st), nthreads)
+    return dict(q=q, s=s, wcomp=wc, status=st)
+
+
+def gptq(w_f32, x_f32, damp=0.01, want_wcomp=False, nthreads=NTHREADS):
+    """GPTQ int8 weights of w [N, K] (binary32, smoothed) for calibration inputs x [T, K]."""
+    H, dead = gptq_hessian(x_f32, damp)
+    U = gptq_hinv_chol(H)
+    r = gptq_quantize(w_f32, dead, U, want_wcomp=want_wcomp, nthreads=nthreads)
+    r.update(H=H, dead=dead, U=U)
+    return r

@@ -13,6 +13,8 @@
  *   - bf16 values travel as raw 16-bit patterns; widening is exact, narrowing is RN-even.
  *
  * Sources (page title, section):
+ *   [P1] "Optimizing Llama 3 Inference Speed Using INT8 Quantization via AutoGPTQ"
+ *        (promptcube3), "Crucial Config Tips for Performance" -- GPTQ's dampening factor.
  *   [P2] "INT8 W8A8 ... using SmoothQuant and GPTQ" (arc-codex article 3619...):
  *        "At its core, quantizing a weight involves 2 steps" -- scale = max|col|/127,
  *        q = round(w/scale); "The problem with naive quantization" -- per-channel RTN and
@@ -20,7 +22,9 @@
  *        token, worked example [1.32, 0.75, 0.91, 153.0]; "How SmoothQuant prevents
  *        outliers" -- RMSNorm = divide by RMS then multiply by gamma, gamma folding;
  *        "How the SmoothQuant smoothing factor is computed" -- s_j from max|A_j|, max|W_j|,
- *        alpha (formula lost in the extract; the SmoothQuant paper's form is used).
+ *        alpha (formula lost in the extract; the SmoothQuant paper's form is used); "The
+ *        solution: How GPTQ improves on naive quantization" -- quantize a weight, measure the
+ *        error, redistribute it over the remaining weights guided by the Hessian.
  *   [P3] "INT8 Post-Training Quantization for LLM Inference on NVIDIA GPUs", section
  *        "1. Min-Max Calibration" -- S = max(|min|,|max|)/127, range [-127, 127].
  *   [P4] "W8A8 ... accuracy and serving results" (Red Hat developer article), section
@@ -779,5 +783,188 @@ int oracle_rtn_weights(const uint16_t *w, const float *s, int64_t N, int64_t K, 
 {
     struct rtn_ctx c = {w, s, K, wq, s_ch};
     parallel_rows(rtn_row, &c, N, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ GPTQ weights */
+
+/*
+ * GPTQ weight quantization [P2 "The solution: How GPTQ improves on naive quantization": after
+ * rounding each weight, measure the error it introduced and redistribute it over the weights
+ * not yet quantized, guided by a Hessian computed from the calibration activations; P1
+ * "Crucial Config Tips for Performance": a dampening factor]. The pages give the steps in
+ * prose only; the arithmetic is the GPTQ paper's (Frantar et al., 2022), which the pages
+ * follow: per output channel (a row of W [N, K]), columns in order j = 0 .. K-1,
+ *   q_j = clamp(rint(w_j / s), -127, 127)                (s: the row's RTN scale, kept fixed)
+ *   e_j = (w_j - q_j s) / U[j][j]
+ *   w_k = w_k - e_j U[j][k]  for every k > j             (the compensation)
+ * with U the upper-triangular Cholesky factor of H^-1 (H^-1 = U^T U), whose row j is the
+ * inverse Hessian of the columns not yet quantized, scaled, that the compensation needs.
+ * Everything is binary64 here; H is built, dampened and factored by the three functions
+ * below, in this order.
+ */
+
+/* Steps 1-3: H = (2 / T) X^T X from the calibration activations X [T, K] (binary32, as the
+ * layer receives them); a column with H_jj = 0 (an input channel that is always zero) gets
+ * H_jj = 1 and is flagged dead (its weights are zeroed before quantization); then
+ * H_jj += damp * mean_j(H_jj). H: [K, K] row-major. */
+int oracle_gptq_hessian(const float *x, int64_t T, int64_t K, double damp, double *H,
+                        uint8_t *dead)
+{
+    for (int64_t i = 0; i < K; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; ++t)
+                acc += (double)x[t * K + i] * (double)x[t * K + j];
+            H[i * K + j] = 2.0 * acc / (double)T;
+        }
+    double mean = 0.0;
+    for (int64_t j = 0; j < K; ++j) {
+        dead[j] = H[j * K + j] == 0.0;
+        if (dead[j])
+            H[j * K + j] = 1.0;
+        mean += H[j * K + j];
+    }
+    mean /= (double)K;
+    for (int64_t j = 0; j < K; ++j)
+        H[j * K + j] += damp * mean;
+    return 0;
+}
+
+/* Step 4: U with H^-1 = U^T U, U upper triangular, positive diagonal; computed as written:
+ * L = Cholesky factor of H (H = L L^T), H^-1 = L^-T L^-1, then the Cholesky factorization
+ * of H^-1 in the U^T U form. Returns -1 if H is not positive definite. */
+int oracle_gptq_hinv_chol(const double *H, int64_t K, double *U)
+{
+    double *L = (double *)calloc((size_t)(K * K), sizeof(double));
+    double *Li = (double *)calloc((size_t)(K * K), sizeof(double));
+    double *Hi = (double *)calloc((size_t)(K * K), sizeof(double));
+    int rc = 0;
+    for (int64_t j = 0; j < K && rc == 0; ++j) {
+        double d = H[j * K + j];
+        for (int64_t k = 0; k < j; ++k)
+            d -= L[j * K + k] * L[j * K + k];
+        if (!(d > 0.0)) {
+            rc = -1;
+            break;
+        }
+        L[j * K + j] = sqrt(d);
+        for (int64_t i = j + 1; i < K; ++i) {
+            double v = H[i * K + j];
+            for (int64_t k = 0; k < j; ++k)
+                v -= L[i * K + k] * L[j * K + k];
+            L[i * K + j] = v / L[j * K + j];
+        }
+    }
+    if (rc == 0) {
+        /* L^-1 by forward substitution, one unit vector (column c) at a time */
+        for (int64_t c = 0; c < K; ++c)
+            for (int64_t i = c; i < K; ++i) {
+                double v = i == c ? 1.0 : 0.0;
+                for (int64_t k = c; k < i; ++k)
+                    v -= L[i * K + k] * Li[k * K + c];
+                Li[i * K + c] = v / L[i * K + i];
+            }
+        /* H^-1 = (L^-1)^T L^-1 */
+        for (int64_t i = 0; i < K; ++i)
+            for (int64_t j = 0; j < K; ++j) {
+                double v = 0.0;
+                for (int64_t k = (i > j ? i : j); k < K; ++k)
+                    v += Li[k * K + i] * Li[k * K + j];
+                Hi[i * K + j] = v;
+            }
+        /* H^-1 = U^T U */
+        memset(U, 0, (size_t)(K * K) * sizeof(double));
+        for (int64_t i = 0; i < K && rc == 0; ++i) {
+            double d = Hi[i * K + i];
+            for (int64_t k = 0; k < i; ++k)
+                d -= U[k * K + i] * U[k * K + i];
+            if (!(d > 0.0)) {
+                rc = -1;
+                break;
+            }
+            U[i * K + i] = sqrt(d);
+            for (int64_t j = i + 1; j < K; ++j) {
+                double v = Hi[i * K + j];
+                for (int64_t k = 0; k < i; ++k)
+                    v -= U[k * K + i] * U[k * K + j];
+                U[i * K + j] = v / U[i * K + i];
+            }
+        }
+    }
+    free(L);
+    free(Li);
+    free(Hi);
+    return rc;
+}
+
+struct gptq_ctx {
+    const float *w;
+    int64_t K;
+    const uint8_t *dead;
+    const double *U;
+    int8_t *q;
+    float *s_ch;
+    double *wcomp;
+    const int8_t *q_follow;
+    double tie_tol;
+    uint8_t *status;
+};
+
+static void gptq_row(void *vctx, int64_t n)
+{
+    struct gptq_ctx *c = (struct gptq_ctx *)vctx;
+    const int64_t K = c->K;
+    /* the row's scale, from the weight as given (RTN's scale) */
+    float amax = 0.0f;
+    for (int64_t j = 0; j < K; ++j)
+        if (fabsf(c->w[n * K + j]) > amax)
+            amax = fabsf(c->w[n * K + j]);
+    const float s = amax / 127.0f;
+    c->s_ch[n] = s;
+    double *w = (double *)malloc((size_t)K * sizeof(double));
+    for (int64_t j = 0; j < K; ++j)
+        w[j] = c->dead[j] ? 0.0 : (double)c->w[n * K + j];
+    for (int64_t j = 0; j < K; ++j) {
+        if (c->wcomp)
+            c->wcomp[n * K + j] = w[j];
+        double qd = 0.0, r = 0.0;
+        if (s > 0.0f) {
+            r = w[j] / (double)s;
+            qd = rint(r);
+            qd = qd > 127.0 ? 127.0 : (qd < -127.0 ? -127.0 : qd);
+        }
+        if (c->q_follow) {
+            /* follow given codes: judge each against this step's own decision */
+            const double qf = (double)c->q_follow[n * K + j];
+            uint8_t st = 0;
+            if (qf != qd) {
+                /* admissible only across a rounding tie: |qf - qd| = 1 and r within tie_tol
+                 * of the half-integer between them */
+                const double mid = 0.5 * (qf + qd);
+                st = (fabs(qf - qd) == 1.0 && fabs(r - mid) <= c->tie_tol) ? 1 : 2;
+            }
+            c->status[n * K + j] = st;
+            qd = qf;
+        }
+        c->q[n * K + j] = (int8_t)qd;
+        const double e = (w[j] - qd * (double)s) / c->U[j * K + j];
+        for (int64_t k = j + 1; k < K; ++k)
+            w[k] -= e * c->U[j * K + k];
+    }
+    free(w);
+}
+
+/* Steps 5-6 for the rows of W [N, K] (binary32, the smoothed weight) given dead and U.
+ * wcomp (optional): the compensated value of every weight at the moment it is quantized.
+ * q_follow (optional): codes from elsewhere to propagate instead of this function's own;
+ * status[n, j] then says whether code j of row n equals the own decision (0), differs from
+ * it by one across a rounding tie within tie_tol (1), or differs otherwise (2). */
+int oracle_gptq_quantize(const float *w, int64_t N, int64_t K, const uint8_t *dead,
+                         const double *U, int8_t *q, float *s_ch, double *wcomp,
+                         const int8_t *q_follow, double tie_tol, uint8_t *status, int nthreads)
+{
+    struct gptq_ctx c = {w, K, dead, U, q, s_ch, wcomp, q_follow, tie_tol, status};
+    parallel_rows(gptq_row, &c, N, nthreads);
     return 0;
 }
