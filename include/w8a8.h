@@ -10,6 +10,7 @@
  *   [PTQ]   "INT8 Post-Training Quantization for LLM Inference on NVIDIA GPUs" (devtechtools)
  *   [SERVE] "W8A8 Llama 3.1 8B: accuracy and serving results" (Red Hat developers)
  *   [INFENG] "05 Quantization AWQ GPTQ FP8" (inference-engineering notes)
+ *   [AUTOGPTQ] "Optimizing Llama 3 Inference Speed Using INT8 Quantization via AutoGPTQ"
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller; row-major, contiguous.
@@ -55,7 +56,8 @@ enum w8a8_status {
     W8A8_ERR_WORKSPACE = -4,         /* workspace missing or smaller than required */
     W8A8_ERR_CUDA = -5,              /* a CUDA runtime/driver call failed */
     W8A8_ERR_TIMEOUT = -6,           /* a device-side bounded wait ran out */
-    W8A8_ERR_NO_DEVICE = -7          /* no sm_100 device is current */
+    W8A8_ERR_NO_DEVICE = -7,         /* no sm_100 device is current */
+    W8A8_ERR_NUMERIC = -8            /* a matrix that must be positive definite is not */
 };
 
 /*
@@ -285,6 +287,39 @@ W8A8_API int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const 
                                    w8a8_bf16 *y, float *acc_out, void *workspace,
                                    size_t workspace_bytes, int variant, int ctas, int tile_n,
                                    w8a8_stream_t stream);
+
+/*
+ * ---------------------------------------------------------------- GPTQ weights (offline)
+ *
+ * GPTQ quantization of one linear layer's weight to the int8 + per-channel-scale format of
+ * w8a8_gemm_dequant [W8A8 "The solution: How GPTQ improves on naive quantization": after
+ * rounding each weight, measure the error and redistribute it over the weights not yet
+ * quantized, guided by a Hessian from the calibration activations; AUTOGPTQ "Crucial Config
+ * Tips for Performance": the dampening factor]. In binary64 on the device:
+ *   W'[n,j] = float(w[n,j]) * smooth[j]   (binary32 product; W' = w if smooth == NULL)
+ *   s_ch[n] = max_j |W'[n,j]| / 127       (binary32, as RTN)
+ *   H       = (2/T) x^T x; H_jj = 0 (an input channel that is always zero) -> H_jj = 1 and
+ *             column j of W' is zeroed; then H_jj += damp * mean_j(H_jj)
+ *   U       = the upper Cholesky factor of H^-1 (H^-1 = U^T U)
+ *   for j = 0 .. K-1, every row n:  q = clamp(rint(W'[n,j] / s_ch[n]), -127, 127),
+ *             e = (W'[n,j] - q s_ch[n]) / U[j][j],  W'[n,k] -= e U[j][k] for k > j
+ * The column updates are applied in blocks of 64 (the lazy-batch form), so the binary64 sums
+ * run in another order than the column-by-column statement; a code can differ from that
+ * statement's only where W'/s lies within rounding distance of a half-integer.
+ * w: bf16 [N,K] (nn.Linear layout). smooth: fp32 [K] or NULL (SmoothQuant factors s_j).
+ * x_cal: fp32 [T,K], the layer's calibration inputs as the layer receives them (X diag(1/s)).
+ * damp > 0 (0.01 is GPTQ's usual value). wq: int8 [N,K]; s_ch: fp32 [N]. u_out: fp64 [K,K]
+ * or NULL (U, for checking). workspace: w8a8_gptq_workspace_size(N, K) bytes, 256-byte
+ * aligned, any contents. Requires K % 64 == 0, 64 <= K <= 32768, N >= 1, T >= 1.
+ * Unlike the rest of the library this call SYNCHRONIZES `stream` at its end (offline
+ * preparation): it returns W8A8_ERR_NUMERIC when H is not positive definite in binary64 (not
+ * possible with damp > 0 in exact arithmetic).
+ */
+W8A8_API size_t w8a8_gptq_workspace_size(int64_t N, int64_t K);
+W8A8_API int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_cal,
+                                int64_t N, int64_t K, int64_t T, double damp, int8_t *wq,
+                                float *s_ch, double *u_out, void *workspace,
+                                size_t workspace_bytes, w8a8_stream_t stream);
 
 /*
  * Measurement aid, not part of the W8A8 path (the pages have no counterpart): launches `ctas`

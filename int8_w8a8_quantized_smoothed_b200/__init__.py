@@ -25,6 +25,7 @@ __all__ = [
     "w8a8_status_string", "w8a8_version",
     "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
     "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size",
+    "w8a8_gptq_quantize", "w8a8_gptq_workspace_size",
     "Workspace", "FP8",
 ]
 
@@ -32,7 +33,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw8a8.so"
 
 STATUS = {0: "W8A8_OK", -1: "W8A8_ERR_INVALID_ARG", -2: "W8A8_ERR_ALIGNMENT",
           -3: "W8A8_ERR_UNSUPPORTED_SHAPE", -4: "W8A8_ERR_WORKSPACE", -5: "W8A8_ERR_CUDA",
-          -6: "W8A8_ERR_TIMEOUT", -7: "W8A8_ERR_NO_DEVICE"}
+          -6: "W8A8_ERR_TIMEOUT", -7: "W8A8_ERR_NO_DEVICE", -8: "W8A8_ERR_NUMERIC"}
 
 # (name, restype, argtypes) of every function declared in include/w8a8.h
 _P, _I64, _I, _F, _SZ = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
@@ -62,6 +63,9 @@ SIGNATURES = [
     ("w8a8_gemm_fp8_workspace_size", _SZ, [_I64, _I64, _I64, _I, _I, _I]),
     ("w8a8_gemm_dequant_fp8", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _I, _I,
                                    _I, _P]),
+    ("w8a8_gptq_workspace_size", _SZ, [_I64, _I64]),
+    ("w8a8_gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I64, C.c_double, _P, _P, _P, _P, _SZ,
+                                _P]),
 ]
 
 # FP8 codes are OCP E4M3 bit patterns, carried in torch.float8_e4m3fn tensors
@@ -455,3 +459,36 @@ def w8a8_gemm_dequant_noalloc(xq, s_tok, wq, s_ch, y=None, stream=None):
     _check("w8a8_gemm_dequant_noalloc", lib().w8a8_gemm_dequant_noalloc(
         _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _stream(stream)))
     return y
+
+
+def w8a8_gptq_workspace_size(N: int, K: int) -> int:
+    return int(lib().w8a8_gptq_workspace_size(N, K))
+
+
+def w8a8_gptq_quantize(w, x_cal, smooth=None, damp=0.01, wq=None, s_ch=None, want_u=False,
+                       workspace=None, stream=None):
+    """GPTQ int8 weights (offline): w bf16 [N, K] (times smooth [K] if given), calibration
+    inputs x_cal fp32 [T, K] as the layer receives them. Synchronizes the stream.
+    Returns (wq int8 [N, K], s_ch fp32 [N]) and, with want_u, U fp64 [K, K]."""
+    _need(w, "w", torch.bfloat16)
+    N, K = w.shape
+    _need(x_cal, "x_cal", torch.float32)
+    T, K2 = x_cal.shape
+    if K2 != K:
+        raise ValueError(f"w [N,K] and x_cal [T,K] disagree on K: {K} vs {K2}")
+    if smooth is not None:
+        _need(smooth, "smooth", torch.float32, (K,))
+    e = dict(device=w.device)
+    wq = torch.empty((N, K), dtype=torch.int8, **e) if wq is None else wq
+    s_ch = torch.empty(N, dtype=torch.float32, **e) if s_ch is None else s_ch
+    _need(wq, "wq", torch.int8, (N, K))
+    _need(s_ch, "s_ch", torch.float32, (N,))
+    u = torch.empty((K, K), dtype=torch.float64, **e) if want_u else None
+    need = w8a8_gptq_workspace_size(N, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, **e)
+    _check("w8a8_gptq_quantize", lib().w8a8_gptq_quantize(
+        _ptr(w), _ptr(smooth), _ptr(x_cal), N, K, T, float(damp), _ptr(wq), _ptr(s_ch),
+        _ptr(u), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return (wq, s_ch, u) if want_u else (wq, s_ch)

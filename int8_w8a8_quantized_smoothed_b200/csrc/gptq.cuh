@@ -1,0 +1,479 @@
+// GPTQ weight quantization on the GPU, in binary64 (offline preparation of the int8 weights).
+//
+// For each output channel (row of W [N, K]) the columns are quantized in order; after each
+// rounding the error is spread over the columns not yet quantized through U, the upper
+// Cholesky factor of the inverse Hessian (H^-1 = U^T U, H = (2/T) X^T X of the calibration
+// inputs, dampened). Pipeline, all on the device:
+//   hessian      H = (2/T) X^T X                         64 x 64 tiles of the lower half
+//   diag         dead channels (H_jj = 0 -> 1), H_jj += damp * mean(H_jj)
+//   UL Cholesky  H = V V^T with V upper, by 64-column blocks from the last to the first
+//                (diagonal block, panel solve, trailing update of the blocks above-left)
+//   inverse      U = V^-1 (upper): diagonal blocks inverted, then the off-diagonal blocks by
+//                distance from the diagonal (each needs only blocks nearer to it)
+//   quantize     64-column blocks in order: one warp per row runs the block's columns
+//                sequentially (quantize, error, compensate inside the block), then one
+//                tiled update applies the block's errors to every later column (the lazy
+//                batch form: the same sums as the column-by-column form, in another order)
+// U = V^-1 is the Cholesky factor GPTQ needs: H = V V^T gives H^-1 = V^-T V^-1 = U^T U.
+// The dense steps run on 64 x 64 tiles staged in shared memory, 256 threads each owning a
+// 4 x 4 micro-tile (rows ty + 16a, columns tx + 16b) with fused multiply-adds.
+#pragma once
+
+#include <stdint.h>
+
+namespace w8a8 {
+namespace gptq {
+
+constexpr int kT = 64;    // tile / column-block size
+constexpr int kLd = 65;   // padded shared-memory row (doubles)
+constexpr int kThreads = 256;
+// dynamic shared memory of the two-tile kernels
+constexpr int kTwoTileBytes = 2 * kT * kLd * 8;
+
+extern __shared__ __align__(16) double gptq_smem[];
+
+// acc[a][b] += sum_k A[ty + 16a][k] * Bt[tx + 16b][k]   (both tiles row-major in smem, [64][kLd])
+__device__ __forceinline__ void mm_abt(const double *A, const double *Bt, double (&acc)[4][4])
+{
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll 4
+    for (int k = 0; k < kT; ++k) {
+        double a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[i] = A[(ty + 16 * i) * kLd + k];
+            b[i] = Bt[(tx + 16 * i) * kLd + k];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
+}
+
+// acc[a][b] += sum_k A[ty + 16a][k] * B[k][tx + 16b]
+__device__ __forceinline__ void mm_ab(const double *A, const double *B, double (&acc)[4][4])
+{
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll 4
+    for (int k = 0; k < kT; ++k) {
+        double a[4], b[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[i] = A[(ty + 16 * i) * kLd + k];
+            b[i] = B[k * kLd + tx + 16 * i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
+}
+
+// 64 x 64 block (r0, c0) of a row-major matrix with leading dimension ld -> smem [64][kLd].
+__device__ __forceinline__ void load_tile(double *sm, const double *g, int64_t ld, int64_t r0,
+                                          int64_t c0)
+{
+    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
+        const int r = e >> 6, c = e & 63;
+        sm[r * kLd + c] = g[(r0 + r) * ld + c0 + c];
+    }
+}
+
+__device__ __forceinline__ void zero_acc(double (&acc)[4][4])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            acc[i][j] = 0.0;
+}
+
+// ------------------------------------------------------------------ Hessian
+
+// One CTA per 64 x 64 tile (ti >= tj) of H = (2/T) X^T X, X binary32 [T, K] (K % 64 == 0);
+// the tile and its mirror are written.
+__global__ void __launch_bounds__(kThreads) hessian_kernel(const float *__restrict__ x, int64_t T,
+                                                          int64_t K, double *__restrict__ H)
+{
+    __shared__ double sa[16][kT + 1], sb[16][kT + 1];
+    // blockIdx.x -> (ti, tj), ti >= tj, row-major over the lower triangle of tiles
+    int64_t b = blockIdx.x, ti = 0;
+    while (b > ti) {
+        b -= ti + 1;
+        ++ti;
+    }
+    const int64_t tj = b;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double acc[4][4];
+    zero_acc(acc);
+    for (int64_t t0 = 0; t0 < T; t0 += 16) {
+        for (int e = threadIdx.x; e < 16 * kT; e += kThreads) {
+            const int r = e >> 6, c = e & 63;
+            const bool ok = t0 + r < T;
+            sa[r][c] = ok ? static_cast<double>(x[(t0 + r) * K + ti * kT + c]) : 0.0;
+            sb[r][c] = ok ? static_cast<double>(x[(t0 + r) * K + tj * kT + c]) : 0.0;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int t = 0; t < 16; ++t) {
+            double a[4], bb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = sa[t][ty + 16 * i];
+                bb[i] = sb[t][tx + 16 * i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fma(a[i], bb[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t r = ti * kT + ty + 16 * i, c = tj * kT + tx + 16 * j;
+            const double h = 2.0 * acc[i][j] / static_cast<double>(T);
+            H[r * K + c] = h;
+            H[c * K + r] = h;
+        }
+}
+
+// Dead channels and dampening (one CTA): H_jj = 0 -> 1 and dead[j] = 1; then
+// H_jj += damp * mean_j H_jj.
+__global__ void __launch_bounds__(1024) diag_kernel(double *__restrict__ H, int64_t K,
+                                                   double damp, uint8_t *__restrict__ dead)
+{
+    __shared__ double red[32];
+    double sum = 0.0;
+    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) {
+        double h = H[j * K + j];
+        const bool d = h == 0.0;
+        dead[j] = d ? 1 : 0;
+        if (d) {
+            h = 1.0;
+            H[j * K + j] = h;
+        }
+        sum += h;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = sum;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        double v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (threadIdx.x == 0)
+            red[0] = v;
+    }
+    __syncthreads();
+    const double add = damp * (red[0] / static_cast<double>(K));
+    for (int64_t j = threadIdx.x; j < K; j += blockDim.x)
+        H[j * K + j] += add;
+}
+
+// ------------------------------------------------------------------ UL Cholesky H = V V^T
+
+// Diagonal block kb: D = V_kk V_kk^T, V_kk upper, right-looking from the last column; the
+// block's upper triangle is overwritten with V_kk. A non-positive pivot (H not positive
+// definite) is replaced by the smallest normal double and reported through *bad.
+__global__ void __launch_bounds__(kThreads) chol_diag_kernel(double *__restrict__ A, int64_t K,
+                                                            int kb, int *__restrict__ bad)
+{
+    __shared__ double d[kT * kLd];
+    const int64_t o = static_cast<int64_t>(kb) * kT;
+    load_tile(d, A, K, o, o);
+    __syncthreads();
+    for (int j = kT - 1; j >= 0; --j) {
+        double p = d[j * kLd + j];
+        if (!(p > 0.0)) {
+            if (threadIdx.x == 0)
+                atomicExch(bad, 1);
+            p = 2.2250738585072014e-308;
+        }
+        const double vjj = sqrt(p);
+        __syncthreads(); // every thread has read the pivot
+        // column j above the diagonal: V[i][j] = D[i][j] / V[j][j]
+        if (threadIdx.x < j)
+            d[threadIdx.x * kLd + j] = d[threadIdx.x * kLd + j] / vjj;
+        if (threadIdx.x == 0)
+            d[j * kLd + j] = vjj;
+        __syncthreads();
+        // D[i][i'] -= V[i][j] V[i'][j] for i <= i' < j (upper triangle of the rest)
+        for (int e = threadIdx.x; e < j * j; e += kThreads) {
+            const int i = e / j, i2 = e % j;
+            if (i <= i2)
+                d[i * kLd + i2] -= d[i * kLd + j] * d[i2 * kLd + j];
+        }
+        __syncthreads();
+    }
+    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
+        const int r = e >> 6, c = e & 63;
+        if (r <= c)
+            A[(o + r) * K + o + c] = d[r * kLd + c];
+    }
+}
+
+// Panel of block column kb: V[ib][kb] = A[ib][kb] V_kk^-T for every ib < kb (one CTA each):
+// X V_kk^T = A solved from the last column: x_j = a_j / V[j][j], then a_k -= x_j V[k][j]
+// for k < j.
+__global__ void __launch_bounds__(kThreads) chol_panel_kernel(double *__restrict__ A, int64_t K,
+                                                             int kb)
+{
+    double *a = gptq_smem, *v = gptq_smem + kT * kLd;
+    const int64_t oc = static_cast<int64_t>(kb) * kT, orow = static_cast<int64_t>(blockIdx.x) * kT;
+    load_tile(a, A, K, orow, oc);
+    load_tile(v, A, K, oc, oc);
+    __syncthreads();
+    for (int j = kT - 1; j >= 0; --j) {
+        if (threadIdx.x < kT)
+            a[threadIdx.x * kLd + j] = a[threadIdx.x * kLd + j] / v[j * kLd + j];
+        __syncthreads();
+        for (int e = threadIdx.x; e < kT * j; e += kThreads) {
+            const int r = e / j, k = e % j;
+            a[r * kLd + k] -= a[r * kLd + j] * v[k * kLd + j];
+        }
+        __syncthreads();
+    }
+    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
+        const int r = e >> 6, c = e & 63;
+        A[(orow + r) * K + oc + c] = a[r * kLd + c];
+    }
+}
+
+// Trailing update after block column kb: A[ib][jb] -= V[ib][kb] V[jb][kb]^T for
+// ib <= jb < kb (the upper triangle of the remaining blocks); one CTA per pair.
+__global__ void __launch_bounds__(kThreads) chol_update_kernel(double *__restrict__ A, int64_t K,
+                                                              int kb)
+{
+    double *p1 = gptq_smem, *p2 = gptq_smem + kT * kLd;
+    int64_t b = blockIdx.x, jb = 0;
+    while (b > jb) { // pairs (ib <= jb), enumerated jb-major
+        b -= jb + 1;
+        ++jb;
+    }
+    const int64_t ib = b;
+    const int64_t oc = static_cast<int64_t>(kb) * kT;
+    load_tile(p1, A, K, ib * kT, oc);
+    load_tile(p2, A, K, jb * kT, oc);
+    __syncthreads();
+    double acc[4][4];
+    zero_acc(acc);
+    mm_abt(p1, p2, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t r = ib * kT + ty + 16 * i, c = jb * kT + tx + 16 * j;
+            A[r * K + c] -= acc[i][j];
+        }
+}
+
+// ------------------------------------------------------------------ U = V^-1 (upper)
+
+// Diagonal blocks (one CTA each): U_kk = V_kk^-1 by back substitution, one column per
+// thread: U[c][c] = 1 / V[c][c], U[i][c] = -(sum_{k=i+1..c} V[i][k] U[k][c]) / V[i][i].
+// The block's lower triangle is written as zeros.
+__global__ void __launch_bounds__(kT) trtri_diag_kernel(const double *__restrict__ V,
+                                                       double *__restrict__ U, int64_t K)
+{
+    double *v = gptq_smem, *u = gptq_smem + kT * kLd;
+    const int64_t o = static_cast<int64_t>(blockIdx.x) * kT;
+    for (int e = threadIdx.x; e < kT * kT; e += blockDim.x) {
+        const int r = e >> 6, c = e & 63;
+        v[r * kLd + c] = r <= c ? V[(o + r) * K + o + c] : 0.0;
+        u[r * kLd + c] = 0.0;
+    }
+    __syncthreads();
+    const int c = threadIdx.x;
+    u[c * kLd + c] = 1.0 / v[c * kLd + c];
+    for (int i = c - 1; i >= 0; --i) {
+        double s = 0.0;
+        for (int k = i + 1; k <= c; ++k)
+            s = fma(v[i * kLd + k], u[k * kLd + c], s);
+        u[i * kLd + c] = -s / v[i * kLd + i];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kT * kT; e += blockDim.x) {
+        const int r = e >> 6, cc = e & 63;
+        U[(o + r) * K + o + cc] = u[r * kLd + cc];
+    }
+}
+
+// Off-diagonal blocks at distance dist (one CTA per block i, j = i + dist):
+// U[i][j] = -U_ii (sum_{k=i+1..j} V[i][k] U[k][j]); every U[k][j] used is nearer the diagonal.
+__global__ void __launch_bounds__(kThreads) trtri_off_kernel(const double *__restrict__ V,
+                                                            double *__restrict__ U, int64_t K,
+                                                            int dist)
+{
+    double *sa = gptq_smem, *sb = gptq_smem + kT * kLd;
+    const int64_t i = blockIdx.x, j = i + dist;
+    double acc[4][4];
+    zero_acc(acc);
+    for (int64_t k = i + 1; k <= j; ++k) {
+        load_tile(sa, V, K, i * kT, k * kT);
+        load_tile(sb, U, K, k * kT, j * kT);
+        __syncthreads();
+        mm_ab(sa, sb, acc);
+        __syncthreads();
+    }
+    // T -> sb, U_ii -> sa, then U[i][j] = -U_ii T
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            sb[(ty + 16 * a) * kLd + tx + 16 * b] = acc[a][b];
+    load_tile(sa, U, K, i * kT, i * kT);
+    __syncthreads();
+    zero_acc(acc);
+    mm_ab(sa, sb, acc);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            U[(i * kT + ty + 16 * a) * K + j * kT + tx + 16 * b] = -acc[a][b];
+}
+
+// Lower off-diagonal blocks of U are zero (U is returned whole to callers that ask for it).
+__global__ void __launch_bounds__(kThreads) zero_lower_kernel(double *__restrict__ U, int64_t K)
+{
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; e < K * K;
+         e += static_cast<int64_t>(gridDim.x) * kThreads) {
+        const int64_t r = e / K, c = e % K;
+        if (r / kT > c / kT)
+            U[e] = 0.0;
+    }
+}
+
+// ------------------------------------------------------------------ quantize and compensate
+
+// Working copy of the smoothed weight, binary64: W'[n][j] = bf16(w[n][j]) * s_j (binary32
+// product, as the RTN path computes it), 0 for dead channels; s_ch[n] = max_j |W'[n][j]| / 127
+// over the weight as given (binary32). One warp per row.
+__global__ void __launch_bounds__(kThreads) prep_kernel(const uint16_t *__restrict__ w,
+                                                       const float *__restrict__ smooth,
+                                                       const uint8_t *__restrict__ dead,
+                                                       int64_t N, int64_t K,
+                                                       double *__restrict__ wd,
+                                                       float *__restrict__ s_ch)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+         n < N; n += warps) {
+        float amax = 0.0f;
+        for (int64_t j = lane; j < K; j += 32) {
+            float f = __uint_as_float(static_cast<uint32_t>(w[n * K + j]) << 16);
+            if (smooth)
+                f = __fmul_rn(f, smooth[j]);
+            amax = fmaxf(amax, fabsf(f));
+            wd[n * K + j] = dead[j] ? 0.0 : static_cast<double>(f);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0)
+            s_ch[n] = __fdiv_rn(amax, 127.0f);
+    }
+}
+
+// Column block jb (columns j0 .. j0 + 63), one warp per row, lane l holding columns l and
+// l + 32: for each column j in order the lane that holds it rounds w_j / s, forms the error
+// e = (w_j - q s) / U[j][j] and broadcasts it; every lane subtracts e U[j][k] from its
+// columns k > j of the block. Codes go to wq, errors to err [N][64] for the update kernel.
+__global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restrict__ wd,
+                                                              const double *__restrict__ U,
+                                                              const float *__restrict__ s_ch,
+                                                              int64_t N, int64_t K, int jb,
+                                                              int8_t *__restrict__ wq,
+                                                              double *__restrict__ err)
+{
+    __shared__ double u[kT * kLd];
+    const int64_t j0 = static_cast<int64_t>(jb) * kT;
+    load_tile(u, U, K, j0, j0);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+         n < N; n += warps) {
+        const double s = static_cast<double>(s_ch[n]);
+        double w0 = wd[n * K + j0 + lane], w1 = wd[n * K + j0 + 32 + lane];
+        int q0 = 0, q1 = 0;
+        double e0 = 0.0, e1 = 0.0;
+        for (int j = 0; j < kT; ++j) {
+            const bool hi = j >= 32;
+            double e = 0.0;
+            if (lane == (j & 31)) {
+                const double wj = hi ? w1 : w0;
+                double q = 0.0;
+                if (s > 0.0) {
+                    q = rint(wj / s);
+                    q = fmin(fmax(q, -127.0), 127.0);
+                }
+                e = (wj - q * s) / u[j * kLd + j];
+                if (hi) {
+                    q1 = static_cast<int>(q);
+                    e1 = e;
+                } else {
+                    q0 = static_cast<int>(q);
+                    e0 = e;
+                }
+            }
+            e = __shfl_sync(0xffffffffu, e, j & 31);
+            if (lane > j)
+                w0 -= e * u[j * kLd + lane];
+            if (lane + 32 > j)
+                w1 -= e * u[j * kLd + lane + 32];
+        }
+        wq[n * K + j0 + lane] = static_cast<int8_t>(q0);
+        wq[n * K + j0 + 32 + lane] = static_cast<int8_t>(q1);
+        err[n * kT + lane] = e0;
+        err[n * kT + 32 + lane] = e1;
+    }
+}
+
+// Lazy batch update after column block jb: W'[n][c] -= sum_t err[n][t] U[j0 + t][c] for the
+// columns c >= j0 + 64; one CTA per 64 x 64 tile (rows beyond N skipped).
+__global__ void __launch_bounds__(kThreads) update_kernel(double *__restrict__ wd,
+                                                         const double *__restrict__ U,
+                                                         const double *__restrict__ err,
+                                                         int64_t N, int64_t K, int jb)
+{
+    double *se = gptq_smem, *su = gptq_smem + kT * kLd;
+    const int64_t j0 = static_cast<int64_t>(jb) * kT;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kT;
+    const int64_t c0 = j0 + kT + static_cast<int64_t>(blockIdx.x) * kT;
+    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
+        const int r = e >> 6, c = e & 63;
+        se[r * kLd + c] = r0 + r < N ? err[(r0 + r) * kT + c] : 0.0;
+    }
+    load_tile(su, U, K, j0, c0);
+    __syncthreads();
+    double acc[4][4];
+    zero_acc(acc);
+    mm_ab(se, su, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int64_t r = r0 + ty + 16 * a;
+        if (r < N) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                wd[r * K + c0 + tx + 16 * b] -= acc[a][b];
+        }
+    }
+}
+
+} // namespace gptq
+} // namespace w8a8

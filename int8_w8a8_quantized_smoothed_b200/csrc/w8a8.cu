@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "gemm.cuh"
+#include "gptq.cuh"
 #include "probe.cuh"
 #include "rowquant.cuh"
 #include "w8a8.h"
@@ -615,6 +616,33 @@ int gemm_run(const int8_t *xq, const float *s_tok, const int8_t *wq, const float
 }
 
 
+// ------------------------------------------------------------------ GPTQ workspace
+
+struct GptqLayout {
+    size_t a_off, u_off, w_off, e_off, d_off, b_off, total;
+};
+
+size_t round256(size_t b)
+{
+    return (b + 255) & ~static_cast<size_t>(255);
+}
+
+// H/V [K,K] fp64, U [K,K] fp64, working weight [N,K] fp64, block errors [N,64] fp64, dead
+// flags [K], the non-positive-pivot flag.
+GptqLayout gptq_layout(int64_t N, int64_t K)
+{
+    GptqLayout L;
+    const size_t kk = static_cast<size_t>(K) * static_cast<size_t>(K) * sizeof(double);
+    L.a_off = 0;
+    L.u_off = L.a_off + round256(kk);
+    L.w_off = L.u_off + round256(kk);
+    L.e_off = L.w_off + round256(static_cast<size_t>(N) * static_cast<size_t>(K) * sizeof(double));
+    L.d_off = L.e_off + round256(static_cast<size_t>(N) * 64 * sizeof(double));
+    L.b_off = L.d_off + round256(static_cast<size_t>(K));
+    L.total = L.b_off + 256;
+    return L;
+}
+
 // ------------------------------------------------------------------ row entry points
 // (F8: E4M3 codes with scale amax / 448, else int8 codes with amax / 127)
 
@@ -739,6 +767,8 @@ const char *w8a8_status_string(int status)
         return "device-side wait timed out";
     case W8A8_ERR_NO_DEVICE:
         return "no sm_100 device";
+    case W8A8_ERR_NUMERIC:
+        return "matrix not positive definite";
     default:
         return "unknown status";
     }
@@ -957,6 +987,90 @@ int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *
         return W8A8_ERR_WORKSPACE;
     return gemm_run_fp8(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace, p, dev, sms,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t w8a8_gptq_workspace_size(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 64 || K % 64 != 0 || K > 32768)
+        return 0;
+    const GptqLayout L = gptq_layout(N, K);
+    return L.total;
+}
+
+int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_cal, int64_t N,
+                       int64_t K, int64_t T, double damp, int8_t *wq, float *s_ch,
+                       double *u_out, void *workspace, size_t workspace_bytes,
+                       w8a8_stream_t stream)
+{
+    namespace g = w8a8::gptq;
+    if (!w || !x_cal || !wq || !s_ch || N < 1 || T < 1 || !(damp > 0.0) || !(damp < 1e300))
+        return W8A8_ERR_INVALID_ARG;
+    if (K < 64 || K % 64 != 0 || K > 32768 || N > 0x7fffffffLL || T > 0x7fffffffLL)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    const GptqLayout L = gptq_layout(N, K);
+    if (!workspace || workspace_bytes < L.total)
+        return W8A8_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 ||
+        reinterpret_cast<uintptr_t>(u_out) % 8 != 0)
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char *base = static_cast<char *>(workspace);
+    double *A = reinterpret_cast<double *>(base + L.a_off);   // H, then V in its upper part
+    double *U = reinterpret_cast<double *>(base + L.u_off);
+    double *wd = reinterpret_cast<double *>(base + L.w_off);
+    double *err = reinterpret_cast<double *>(base + L.e_off);
+    uint8_t *dead = reinterpret_cast<uint8_t *>(base + L.d_off);
+    int *bad = reinterpret_cast<int *>(base + L.b_off);
+    const int nb = static_cast<int>(K / g::kT);
+    const int sm2 = g::kTwoTileBytes;
+    for (const void *fn : {reinterpret_cast<const void *>(&g::chol_panel_kernel),
+                           reinterpret_cast<const void *>(&g::chol_update_kernel),
+                           reinterpret_cast<const void *>(&g::trtri_diag_kernel),
+                           reinterpret_cast<const void *>(&g::trtri_off_kernel),
+                           reinterpret_cast<const void *>(&g::update_kernel)})
+        if ((rc = ensure_smem(fn, dev, sm2)))
+            return rc;
+    if (cudaMemsetAsync(bad, 0, sizeof(int), st) != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    g::hessian_kernel<<<nb * (nb + 1) / 2, g::kThreads, 0, st>>>(x_cal, T, K, A);
+    g::diag_kernel<<<1, 1024, 0, st>>>(A, K, damp, dead);
+    for (int kb = nb - 1; kb >= 0; --kb) {
+        g::chol_diag_kernel<<<1, g::kThreads, 0, st>>>(A, K, kb, bad);
+        if (kb > 0) {
+            g::chol_panel_kernel<<<kb, g::kThreads, sm2, st>>>(A, K, kb);
+            g::chol_update_kernel<<<kb * (kb + 1) / 2, g::kThreads, sm2, st>>>(A, K, kb);
+        }
+    }
+    g::trtri_diag_kernel<<<nb, g::kT, sm2, st>>>(A, U, K);
+    for (int d = 1; d < nb; ++d)
+        g::trtri_off_kernel<<<nb - d, g::kThreads, sm2, st>>>(A, U, K, d);
+    const unsigned rows_grid =
+        static_cast<unsigned>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(sms) * 8));
+    g::prep_kernel<<<rows_grid, g::kThreads, 0, st>>>(w, smooth, dead, N, K, wd, s_ch);
+    const unsigned row_tiles = static_cast<unsigned>((N + g::kT - 1) / g::kT);
+    for (int jb = 0; jb < nb; ++jb) {
+        g::quant_block_kernel<<<rows_grid, g::kThreads, 0, st>>>(wd, U, s_ch, N, K, jb, wq, err);
+        if (jb + 1 < nb)
+            g::update_kernel<<<dim3(nb - 1 - jb, row_tiles), g::kThreads, sm2, st>>>(wd, U, err, N,
+                                                                                 K, jb);
+    }
+    if (u_out) {
+        g::zero_lower_kernel<<<sms * 4, g::kThreads, 0, st>>>(U, K);
+        if (cudaMemcpyAsync(u_out, U, static_cast<size_t>(K * K) * sizeof(double),
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+            return W8A8_ERR_CUDA;
+    }
+    if (cudaGetLastError() != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    int bad_h = 0;
+    if (cudaMemcpyAsync(&bad_h, bad, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    return bad_h ? W8A8_ERR_NUMERIC : W8A8_OK;
 }
 
 int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream)
