@@ -680,6 +680,61 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ single-kernel case
 
 
+def measure_f64_peak(iters=4000, reps=3):
+    """Binary64 FMA rate (TFLOP/s) of this device from w8a8_probe_f64_fma, best of reps."""
+    import int8_w8a8_quantized_smoothed_b200 as w8
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    ctas = props.multi_processor_count * 8
+    out = torch.empty(ctas * 256, dtype=torch.float64, device="cuda")
+    w8.w8a8_probe_f64_fma(iters, ctas, out)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        w8.w8a8_probe_f64_fma(iters, ctas, out)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, 2 * 8 * iters * 256 * ctas / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    return best
+
+
+def run_gptq_case(args, dims):
+    """`--case gptq:N:K:T`: GPTQ of one [N, K] weight with T calibration tokens, whole call
+    (Hessian, factor, quantize-and-compensate) timed with CUDA events; binary64 flops against
+    the FMA probe's rate."""
+    import int8_w8a8_quantized_smoothed_b200 as w8
+    from int8_w8a8_quantized_smoothed_b200 import build as wbuild, synth
+    wbuild.build()
+    N, K, T = dims
+    dev = torch.device("cuda", 0)
+    w = synth.weight_device(N, K, 1, dev)
+    x = synth.activation_device(T, K, 2, dev).float()
+    s = synth.gamma_device(K, 3, dev).float()
+    ws = torch.empty(w8.w8a8_gptq_workspace_size(N, K), dtype=torch.uint8, device=dev)
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    sch = torch.empty(N, dtype=torch.float32, device=dev)
+    w8.w8a8_gptq_quantize(w, x, s, wq=wq, s_ch=sch, workspace=ws)
+    times = []
+    for _ in range(max(1, args.steps)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        w8.w8a8_gptq_quantize(w, x, s, wq=wq, s_ch=sch, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(times)
+    flops = {"hessian": T * K * (K + 1), "cholesky": K ** 3 / 3, "inverse": K ** 3 / 3,
+             "quantize": N * K * K}
+    total = sum(flops.values())
+    peak = measure_f64_peak()
+    return {"case": args.case, "ms_per_call": round(t * 1e3, 3),
+            "fp64_tflops": round(total / t / 1e12, 2), "fp64_peak_tflops_measured": round(peak, 2),
+            "frac": round(total / t / 1e12 / peak, 4),
+            "flops": {k: float(v) for k, v in flops.items()},
+            "note": "median of K calls; each call synchronizes (offline preparation)"}
+
+
 def run_case(args):
     """`--case gemm:M:N:K[:variant]` (INT8), `gemm8:M:N:K[:variant]` (FP8), `rms:M:K`, `rmsres:M:K`, `quant:M:K`, `static:M:K` or
     `silu:M:I`:
@@ -689,6 +744,8 @@ def run_case(args):
     wbuild.build()
     parts = args.case.split(":")
     dev = torch.device("cuda", 0)
+    if parts[0] == "gptq":
+        return run_gptq_case(args, [int(v) for v in parts[1:4]])
     if parts[0] in ("gemm", "gemm8"):
         M, N, K = (int(v) for v in parts[1:4])
         variant = int(parts[4]) if len(parts) > 4 else 0

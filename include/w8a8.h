@@ -331,6 +331,14 @@ W8A8_API int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const f
 W8A8_API int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream);
 
 /*
+ * Measurement aid for the GPTQ kernels' roofline (no counterpart on the pages): `ctas` CTAs of
+ * 256 threads, each thread running 8 independent chains of `iters` binary64 fused
+ * multiply-adds, 2 * 8 * iters * 256 * ctas flops in all; out: fp64 [ctas * 256] (the chains'
+ * sums, written so the work is kept). W8A8_ERR_INVALID_ARG for iters < 1, ctas < 1, out NULL.
+ */
+W8A8_API int w8a8_probe_f64_fma(long long iters, int ctas, double *out, w8a8_stream_t stream);
+
+/*
  * Kernel overlap mode, process-wide (default 1). Results are identical in every mode.
  *   0: each kernel of this library starts after the previous work in its stream completes.
  *   1: programmatic dependent launch: a kernel may launch and run its prologue (barrier

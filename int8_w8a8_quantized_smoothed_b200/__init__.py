@@ -25,7 +25,7 @@ __all__ = [
     "w8a8_status_string", "w8a8_version",
     "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
     "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size",
-    "w8a8_gptq_quantize", "w8a8_gptq_workspace_size",
+    "w8a8_gptq_quantize", "w8a8_gptq_workspace_size", "w8a8_probe_f64_fma",
     "Workspace", "FP8",
 ]
 
@@ -64,6 +64,7 @@ SIGNATURES = [
     ("w8a8_gemm_dequant_fp8", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _I, _I,
                                    _I, _P]),
     ("w8a8_gptq_workspace_size", _SZ, [_I64, _I64]),
+    ("w8a8_probe_f64_fma", _I, [C.c_longlong, _I, _P, _P]),
     ("w8a8_gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I64, C.c_double, _P, _P, _P, _P, _SZ,
                                 _P]),
 ]
@@ -459,6 +460,15 @@ def w8a8_gemm_dequant_noalloc(xq, s_tok, wq, s_ch, y=None, stream=None):
     _check("w8a8_gemm_dequant_noalloc", lib().w8a8_gemm_dequant_noalloc(
         _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _stream(stream)))
     return y
+
+
+def w8a8_probe_f64_fma(iters: int, ctas: int, out=None, stream=None):
+    """Binary64 FMA throughput probe: 2 * 8 * iters * 256 * ctas flops. Returns out."""
+    if out is None:
+        out = torch.empty(ctas * 256, dtype=torch.float64, device="cuda")
+    _check("w8a8_probe_f64_fma", lib().w8a8_probe_f64_fma(int(iters), int(ctas), _ptr(out),
+                                                          _stream(stream)))
+    return out
 
 
 def w8a8_gptq_workspace_size(N: int, K: int) -> int:

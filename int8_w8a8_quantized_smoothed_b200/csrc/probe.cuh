@@ -54,6 +54,27 @@ __global__ void __launch_bounds__(128, 1) mma_i8_probe_kernel(long long iters,
     }
 }
 
+// Binary64 FMA throughput probe (the denominator of the GPTQ kernels' roofline): every thread
+// runs 8 independent chains of `iters` fused multiply-adds; the sums are written so that the
+// work is kept.
+__global__ void __launch_bounds__(256) fma_f64_probe_kernel(long long iters, double *out)
+{
+    double a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        a[i] = 1.0 + 1e-9 * (threadIdx.x + i);
+    const double m = 0.999999999, c = 1e-12;
+    for (long long it = 0; it < iters; ++it)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            a[i] = fma(a[i], m, c);
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        s += a[i];
+    out[static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x] = s;
+}
+
 // Failure-path self-test: one CTA whose waits can never be satisfied -- thread 0 on an
 // mbarrier nobody arrives at, thread 32 on a flag word nobody sets -- each bounded by
 // limit_ns, so both give up, raise the device status word and return. Shows that a wait that

@@ -1093,6 +1093,18 @@ int w8a8_probe_i8_mma(long long iters, int n, int ctas, w8a8_stream_t stream)
     }
 }
 
+int w8a8_probe_f64_fma(long long iters, int ctas, double *out, w8a8_stream_t stream)
+{
+    if (iters < 1 || ctas < 1 || !out)
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    fma_f64_probe_kernel<<<ctas, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(iters, out);
+    return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
 int w8a8_set_overlap(int mode)
 {
     if (mode < 0 || mode > 2)
