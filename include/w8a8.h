@@ -244,6 +244,55 @@ W8A8_API int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const in
                                   size_t workspace_bytes, w8a8_stream_t stream);
 
 /*
+ * ---------------------------------------------------------------- the fused decoder block
+ *
+ * One Llama decoder block's whole linear path at decode sizes (1 <= M <= 64 tokens) as a single
+ * persistent kernel (the fused block path: the row operations and the four GEMMs in one
+ * launch, a grid-wide barrier between dependent phases, the weight stream running on across
+ * phase boundaries). It computes what this chain of the separate entry points computes:
+ *   q1, s1      = w8a8_smooth_rmsnorm_quant(x, gamma1)
+ *   qkv_out     = w8a8_gemm_dequant(q1, s1, qkv)
+ *   q2, s2      = w8a8_quantize_rows(attn, sinv_o)
+ *   o_out       = w8a8_gemm_dequant(q2, s2, o)
+ *   q3, s3, h_out = w8a8_smooth_rmsnorm_quant(o_out, gamma2, residual = x)
+ *   q4, s4, a_out = w8a8_gemm_silu_quant(q3, s3, gate_up_il)
+ *   y_out       = w8a8_gemm_dequant(q4, s4, down)
+ * with identical results except that the binary64 sums of squares of the two RMSNorms are
+ * added in another order (the method leaves the order free; a row whose mean of squares lies
+ * within that order's effect of a binary32 rounding boundary may round to the neighbour).
+ * attn stands for the attention output (the o projection's input). Shapes: x, attn, o_out,
+ * h_out, y_out bf16 [M, H]; qkv_out bf16 [M, QKV]; a_out fp32 [M, I]; q1..q3 int8 [M, H], q4
+ * int8 [M, I], s1..s4 fp32 [M]; gamma1, gamma2, sinv_o fp32 [H] (sinv_o may not be NULL: pass
+ * ones for no smoothing); weights int8 [N, K] with fp32 scales [N]: qkv [QKV, H], o [H, H],
+ * gate_up_il [2I, H] interleaved as for w8a8_gemm_silu_quant, down [H, I]. Every pointer
+ * 16-byte aligned. Requires 1 <= M <= 64, H a multiple of 128 up to 8192, I a multiple of 128
+ * up to 32768, QKV a multiple of 8. workspace: w8a8_block_decode_workspace_size() bytes, 256-byte aligned, zero-filled
+ * before its first use; each call leaves it ready for the next call in stream order (a call
+ * that returned W8A8_ERR_TIMEOUT through w8a8_device_status leaves it to be zero-filled
+ * again). Launched as a cooperative grid of one CTA per SM.
+ */
+typedef struct w8a8_linear {
+    const int8_t *wq;  /* int8 [N, K] */
+    const float *s_ch; /* fp32 [N] */
+} w8a8_linear;
+
+typedef struct w8a8_block_io {
+    int64_t M, H, I, QKV;
+    float eps;
+    const w8a8_bf16 *x, *attn;
+    const float *gamma1, *sinv_o, *gamma2;
+    w8a8_linear qkv, o, gate_up_il, down;
+    w8a8_bf16 *qkv_out, *o_out, *h_out, *y_out;
+    float *a_out;
+    int8_t *q1, *q2, *q3, *q4;
+    float *s1, *s2, *s3, *s4;
+} w8a8_block_io;
+
+W8A8_API size_t w8a8_block_decode_workspace_size(int64_t M, int64_t H, int64_t I, int64_t QKV);
+W8A8_API int w8a8_block_decode(const w8a8_block_io *io, void *workspace, size_t workspace_bytes,
+                               w8a8_stream_t stream);
+
+/*
  * ---------------------------------------------------------------- FP8 (E4M3) variant
  *
  * W8A8 with 8-bit floating-point codes instead of int8, the variant for Hopper and Blackwell

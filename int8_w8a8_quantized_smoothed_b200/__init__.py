@@ -26,6 +26,7 @@ __all__ = [
     "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
     "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size",
     "w8a8_gptq_quantize", "w8a8_gptq_workspace_size", "w8a8_probe_f64_fma",
+    "w8a8_block_decode", "w8a8_block_decode_workspace_size", "BlockBuffers",
     "Workspace", "FP8",
 ]
 
@@ -64,6 +65,8 @@ SIGNATURES = [
     ("w8a8_gemm_dequant_fp8", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _SZ, _I, _I,
                                    _I, _P]),
     ("w8a8_gptq_workspace_size", _SZ, [_I64, _I64]),
+    ("w8a8_block_decode_workspace_size", _SZ, [_I64, _I64, _I64, _I64]),
+    ("w8a8_block_decode", _I, [_P, _P, _SZ, _P]),
     ("w8a8_probe_f64_fma", _I, [C.c_longlong, _I, _P, _P]),
     ("w8a8_gptq_quantize", _I, [_P, _P, _P, _I64, _I64, _I64, C.c_double, _P, _P, _P, _P, _SZ,
                                 _P]),
@@ -502,3 +505,75 @@ def w8a8_gptq_quantize(w, x_cal, smooth=None, damp=0.01, wq=None, s_ch=None, wan
         _ptr(u), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
     return (wq, s_ch, u) if want_u else (wq, s_ch)
+
+
+class _Linear(C.Structure):
+    _fields_ = [("wq", C.c_void_p), ("s_ch", C.c_void_p)]
+
+
+class _BlockIO(C.Structure):
+    """Mirror of w8a8_block_io (include/w8a8.h)."""
+    _fields_ = [("M", C.c_int64), ("H", C.c_int64), ("I", C.c_int64), ("QKV", C.c_int64),
+                ("eps", C.c_float),
+                ("x", C.c_void_p), ("attn", C.c_void_p),
+                ("gamma1", C.c_void_p), ("sinv_o", C.c_void_p), ("gamma2", C.c_void_p),
+                ("qkv", _Linear), ("o", _Linear), ("gate_up_il", _Linear), ("down", _Linear),
+                ("qkv_out", C.c_void_p), ("o_out", C.c_void_p), ("h_out", C.c_void_p),
+                ("y_out", C.c_void_p), ("a_out", C.c_void_p),
+                ("q1", C.c_void_p), ("q2", C.c_void_p), ("q3", C.c_void_p), ("q4", C.c_void_p),
+                ("s1", C.c_void_p), ("s2", C.c_void_p), ("s3", C.c_void_p), ("s4", C.c_void_p)]
+
+
+def w8a8_block_decode_workspace_size(M, H, I, QKV) -> int:
+    return int(lib().w8a8_block_decode_workspace_size(M, H, I, QKV))
+
+
+class BlockBuffers:
+    """Outputs and intermediates of one fused decoder-block call (allocated once, reused)."""
+
+    def __init__(self, M, H, I, QKV, device):
+        e = dict(device=device)
+        self.qkv = torch.empty((M, QKV), dtype=torch.bfloat16, **e)
+        self.o = torch.empty((M, H), dtype=torch.bfloat16, **e)
+        self.h = torch.empty((M, H), dtype=torch.bfloat16, **e)
+        self.y = torch.empty((M, H), dtype=torch.bfloat16, **e)
+        self.a = torch.empty((M, I), dtype=torch.float32, **e)
+        self.q = [torch.empty((M, H), dtype=torch.int8, **e) for _ in range(3)] + \
+                 [torch.empty((M, I), dtype=torch.int8, **e)]
+        self.s = [torch.empty(M, dtype=torch.float32, **e) for _ in range(4)]
+        need = w8a8_block_decode_workspace_size(M, H, I, QKV)
+        self.workspace = torch.zeros(max(need, 256), dtype=torch.uint8, **e)
+
+
+def w8a8_block_decode(x, attn, gamma1, sinv_o, gamma2, qkv, o, gate_up_il, down, eps,
+                      buffers=None, stream=None):
+    """One decoder block's linear path at decode sizes in a single persistent kernel.
+    qkv, o, gate_up_il, down: (wq int8 [N, K], s_ch fp32 [N]) with gate_up_il interleaved as
+    for w8a8_gemm_silu_quant. Returns the BlockBuffers (y = the down projection's output)."""
+    _need(x, "x", torch.bfloat16)
+    M, H = x.shape
+    _need(attn, "attn", torch.bfloat16, (M, H))
+    for t, n in ((gamma1, "gamma1"), (sinv_o, "sinv_o"), (gamma2, "gamma2")):
+        _need(t, n, torch.float32, (H,))
+    QKV = qkv[0].shape[0]
+    I = down[0].shape[1]
+    for (wq, sc), n, shape in ((qkv, "qkv", (QKV, H)), (o, "o", (H, H)),
+                               (gate_up_il, "gate_up_il", (2 * I, H)), (down, "down", (H, I))):
+        _need(wq, n + ".wq", torch.int8, shape)
+        _need(sc, n + ".s_ch", torch.float32, (shape[0],))
+    b = BlockBuffers(M, H, I, QKV, x.device) if buffers is None else buffers
+    io = _BlockIO(M=M, H=H, I=I, QKV=QKV, eps=float(eps),
+                  x=x.data_ptr(), attn=attn.data_ptr(), gamma1=gamma1.data_ptr(),
+                  sinv_o=sinv_o.data_ptr(), gamma2=gamma2.data_ptr(),
+                  qkv=_Linear(qkv[0].data_ptr(), qkv[1].data_ptr()),
+                  o=_Linear(o[0].data_ptr(), o[1].data_ptr()),
+                  gate_up_il=_Linear(gate_up_il[0].data_ptr(), gate_up_il[1].data_ptr()),
+                  down=_Linear(down[0].data_ptr(), down[1].data_ptr()),
+                  qkv_out=b.qkv.data_ptr(), o_out=b.o.data_ptr(), h_out=b.h.data_ptr(),
+                  y_out=b.y.data_ptr(), a_out=b.a.data_ptr(),
+                  q1=b.q[0].data_ptr(), q2=b.q[1].data_ptr(), q3=b.q[2].data_ptr(),
+                  q4=b.q[3].data_ptr(), s1=b.s[0].data_ptr(), s2=b.s[1].data_ptr(),
+                  s3=b.s[2].data_ptr(), s4=b.s[3].data_ptr())
+    _check("w8a8_block_decode", lib().w8a8_block_decode(
+        C.byref(io), _ptr(b.workspace), b.workspace.numel(), _stream(stream)))
+    return b

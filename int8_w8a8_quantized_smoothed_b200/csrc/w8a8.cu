@@ -13,6 +13,7 @@
 #include <tuple>
 #include <utility>
 
+#include "block.cuh"
 #include "gemm.cuh"
 #include "gptq.cuh"
 #include "probe.cuh"
@@ -616,6 +617,42 @@ int gemm_run(const int8_t *xq, const float *s_tok, const int8_t *wq, const float
 }
 
 
+// ------------------------------------------------------------------ fused decoder block
+
+// Workspace: the barrier counter and the SiLU maxima, then per GEMM phase a count word per
+// 128-channel block and an int32 accumulation tile [128 channels x Mp tokens] per block.
+size_t block_phase_bytes(int64_t M, int64_t N)
+{
+    const size_t Mp = static_cast<size_t>((M + 3) & ~3LL);
+    const size_t NB = static_cast<size_t>((N + kBM - 1) / kBM);
+    return (kFlagBytes + NB * kBM * Mp * 4u + 255) & ~static_cast<size_t>(255);
+}
+
+template <int NT, int STAGES, int KPS, int NV>
+int launch_block(const BlockMaps &maps, const BlockArgs &args, int dev, int sms, cudaStream_t st)
+{
+    using Cfg = BlockCfg<NT, STAGES, KPS>;
+    auto kernel = block_decode_kernel<NT, STAGES, KPS, NV>;
+    if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
+        return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative; // every CTA resident: they wait on each other
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, maps, args);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    return W8A8_OK;
+}
+
 // ------------------------------------------------------------------ GPTQ workspace
 
 struct GptqLayout {
@@ -987,6 +1024,106 @@ int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *
         return W8A8_ERR_WORKSPACE;
     return gemm_run_fp8(xq, s_tok, wq, s_ch, M, N, K, y, acc_out, workspace, p, dev, sms,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t w8a8_block_decode_workspace_size(int64_t M, int64_t H, int64_t I, int64_t QKV)
+{
+    if (M < 1 || M > 64 || H < 128 || H % 128 || I < 128 || I % 128 || QKV < 8 || QKV % 8)
+        return 0;
+    return 512 + block_phase_bytes(M, QKV) + 2 * block_phase_bytes(M, H) +
+           block_phase_bytes(M, 2 * I);
+}
+
+int w8a8_block_decode(const w8a8_block_io *io, void *workspace, size_t workspace_bytes,
+                      w8a8_stream_t stream)
+{
+    if (!io)
+        return W8A8_ERR_INVALID_ARG;
+    const w8a8_block_io &b = *io;
+    const void *ptrs[] = {b.x, b.attn, b.gamma1, b.sinv_o, b.gamma2, b.qkv.wq, b.qkv.s_ch, b.o.wq,
+                          b.o.s_ch, b.gate_up_il.wq, b.gate_up_il.s_ch, b.down.wq, b.down.s_ch,
+                          b.qkv_out, b.o_out, b.h_out, b.y_out, b.a_out, b.q1, b.q2, b.q3, b.q4,
+                          b.s1, b.s2, b.s3, b.s4};
+    for (const void *p : ptrs)
+        if (!p)
+            return W8A8_ERR_INVALID_ARG;
+    if (!(b.eps >= 0.0f))
+        return W8A8_ERR_INVALID_ARG;
+    if (b.M < 1 || b.M > 64 || b.H < 128 || b.H % 128 || b.I < 128 || b.I % 128 || b.QKV < 8 ||
+        b.QKV % 8 || b.H > 8192 || b.I > 32768 || b.QKV > 0x7fffffffLL)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return W8A8_ERR_ALIGNMENT;
+    if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return workspace ? W8A8_ERR_ALIGNMENT : W8A8_ERR_WORKSPACE;
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    if (sms > kMaxCtas || (2 * b.I + kBM - 1) / kBM > kMaxCtas || (b.QKV + kBM - 1) / kBM > kMaxCtas)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    const size_t need = 512 + block_phase_bytes(b.M, b.QKV) + 2 * block_phase_bytes(b.M, b.H) +
+                        block_phase_bytes(b.M, 2 * b.I);
+    if (workspace_bytes < need)
+        return W8A8_ERR_WORKSPACE;
+    const int M = static_cast<int>(b.M), H = static_cast<int>(b.H), I = static_cast<int>(b.I),
+              Q = static_cast<int>(b.QKV);
+    const int nt = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+    BlockMaps maps;
+    const int8_t *wq[4] = {b.qkv.wq, b.o.wq, b.gate_up_il.wq, b.down.wq};
+    const int8_t *xq[4] = {b.q1, b.q2, b.q3, b.q4};
+    const int Ns[4] = {Q, H, 2 * I, H}, Ks[4] = {H, H, H, I};
+    for (int p = 0; p < 4; ++p)
+        if (encode_kmajor_i8(&maps.w[p], wq[p], Ns[p], Ks[p], kBM) ||
+            encode_kmajor_i8(&maps.x[p], xq[p], M, Ks[p], nt))
+            return W8A8_ERR_CUDA;
+    BlockArgs a;
+    a.M = M;
+    a.H = H;
+    a.I = I;
+    a.eps = b.eps;
+    a.x = b.x;
+    a.attn = b.attn;
+    a.g1 = b.gamma1;
+    a.sinv_o = b.sinv_o;
+    a.g2 = b.gamma2;
+    int8_t *qs[4] = {b.q1, b.q2, b.q3, b.q4};
+    float *ss[4] = {b.s1, b.s2, b.s3, b.s4};
+    for (int p = 0; p < 4; ++p) {
+        a.q[p] = qs[p];
+        a.s[p] = ss[p];
+    }
+    a.h = b.h_out;
+    a.a = b.a_out;
+    const float *sch[4] = {b.qkv.s_ch, b.o.s_ch, b.gate_up_il.s_ch, b.down.s_ch};
+    uint16_t *ys[4] = {b.qkv_out, b.o_out, nullptr, b.y_out};
+    char *ws = static_cast<char *>(workspace);
+    size_t off = 512;
+    for (int p = 0; p < 4; ++p) {
+        char *base = ws + off;
+        a.g[p] = BlockGemm{sch[p], ys[p], Ns[p], Ks[p], reinterpret_cast<int32_t *>(base + kFlagBytes),
+                           reinterpret_cast<unsigned int *>(base)};
+        off += block_phase_bytes(b.M, Ns[p]);
+    }
+    a.bar = reinterpret_cast<unsigned long long *>(ws);
+    a.amax_w = reinterpret_cast<unsigned int *>(ws + 256);
+    a.limit_ns = kWaitLimitNs;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // two k-blocks per stage, as many stages as fit: the ring holds a CTA's whole share of the
+    // small projections
+    if (H <= 4096) {
+        switch (nt) {
+        case 16: return launch_block<16, 6, 2, 4>(maps, a, dev, sms, st);
+        case 32: return launch_block<32, 5, 2, 4>(maps, a, dev, sms, st);
+        default: return launch_block<64, 4, 2, 4>(maps, a, dev, sms, st);
+        }
+    }
+    switch (nt) {
+    case 16: return launch_block<16, 6, 2, 8>(maps, a, dev, sms, st);
+    case 32: return launch_block<32, 5, 2, 8>(maps, a, dev, sms, st);
+    default: return launch_block<64, 4, 2, 8>(maps, a, dev, sms, st);
+    }
 }
 
 size_t w8a8_gptq_workspace_size(int64_t N, int64_t K)
