@@ -218,7 +218,7 @@ class ClockSampler:
 class Layer:
     """One decoder block's linear path at M tokens: prepared weights, inputs, outputs."""
 
-    def __init__(self, arch, M, seed, device, fp8=False):
+    def __init__(self, arch, M, seed, device, fp8=False, block=False):
         import int8_w8a8_quantized_smoothed_b200 as w8
         from int8_w8a8_quantized_smoothed_b200 import prep, synth
         self.M, self.arch, self.fp8 = M, arch, fp8
@@ -279,6 +279,11 @@ class Layer:
         self.s4 = torch.empty(M, dtype=torch.float32, **e)
         self.down = torch.empty(M, H, dtype=torch.bfloat16, **e)
         self.down_host = torch.empty(M, H, dtype=torch.bfloat16).pin_memory()
+        # the fused decoder-block kernel: its own buffers; the block output is self.down
+        self.block = None
+        if block:
+            self.block = w8.BlockBuffers(M, H, I, P["qkv"][0], device)
+            self.down = self.block.y
 
     def rows(self):
         import int8_w8a8_quantized_smoothed_b200 as w8
@@ -289,6 +294,11 @@ class Layer:
         import int8_w8a8_quantized_smoothed_b200 as w8
         if self.fp8:
             return self.chain_fp8(ws, gemms, rows)
+        if self.block is not None:  # one launch for the whole block
+            w8.w8a8_block_decode(self.x, self.attn, self.g1f, self.sinv_o, self.g2f,
+                                 self.w["qkv"], self.w["o"], self.w_gu_il, self.w["down"], EPS,
+                                 buffers=self.block)
+            return
         fused = self.fused if fused is None else fused
         if rows:
             w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
@@ -415,8 +425,8 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     wl = WORKLOADS[args.workload]
     arch = wl["arch"]
-    layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev, fp8=args.fp8)
-              for i, M in enumerate(wl["Ms"])]
+    layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev, fp8=args.fp8,
+                    block=args.fused_block) for i, M in enumerate(wl["Ms"])]
     unfused = args.unfused or args.fp8  # the SiLU*up epilogue is INT8 only
     for L in layers:
         L.fused = not unfused
@@ -479,7 +489,7 @@ def run_ours(args, world, rank, local):
     nbytes = sum(layer_work(arch, L.M)[1] for L in layers)
     g_bytes = sum(layer_work(arch, L.M)[3] for L in layers)
 
-    launches_per_step = 8 * len(layers)
+    launches_per_step = (1 if args.fused_block else 8) * len(layers)
     h2d = sum(L.x.numel() * 2 + L.attn.numel() * 2 for L in layers)
     d2h = sum(L.down.numel() * 2 for L in layers)
 
@@ -503,13 +513,18 @@ def run_ours(args, world, rank, local):
     value, t_max = combine(nbytes, secs / args.steps, world)
     ms_per_step = t_max * 1e3
 
-    # dominant kernel: the GEMM launches of the step, timed alone as a graph
-    g_gemm = capture(step_gemms)
-    gsecs = time_graph(g_gemm, args.steps, args.warmup) / args.steps
-    g_rows = capture(step_rows)
-    rsecs = time_graph(g_rows, args.steps, args.warmup) / args.steps
+    # dominant kernel: the GEMM launches of the step, timed alone as a graph (the fused block
+    # kernel has no separate GEMM launches: its whole step stands in)
+    if args.fused_block:
+        g_gemm = g_rows = None
+        gsecs, rsecs = t_max, 0.0
+    else:
+        g_gemm = capture(step_gemms)
+        gsecs = time_graph(g_gemm, args.steps, args.warmup) / args.steps
+        g_rows = capture(step_rows)
+        rsecs = time_graph(g_rows, args.steps, args.warmup) / args.steps
     gfsecs = None
-    if not unfused:
+    if not unfused and not args.fused_block:
         g_gemm_f = capture(step_gemms_fused)
         gfsecs = time_graph(g_gemm_f, args.steps, args.warmup) / args.steps
         del g_gemm_f
@@ -540,13 +555,15 @@ def run_ours(args, world, rank, local):
                     "frac_of_nominal": round(gemm_tops / INT8_NOMINAL_TOPS, 4),
                     "traffic": None}
     else:
-        roofline = {"kernel": "gemm_decode_kernel" + ("<F8>" if args.fp8 else "") +
-                              " (all GEMM launches of the step, plain dequant epilogues, timed "
-                              "alone as a graph)",
+        roofline = {"kernel": ("block_decode_kernel (the fused block: the whole step, row "
+                               "phases included)") if args.fused_block else
+                              ("gemm_decode_kernel" + ("<F8>" if args.fp8 else "") +
+                               " (all GEMM launches of the step, plain dequant epilogues, timed "
+                               "alone as a graph)"),
                     "bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": hbm_peak,
                     "unit": "GB/s", "frac": round(gemm_gbs / hbm_peak, 4),
                     "peak_source": f"{peak_src} copy bandwidth (burst)", "traffic": None}
-    roofline["per_launch_us"] = round(gsecs / (4 * len(layers)) * 1e6, 3)
+    roofline["per_launch_us"] = round(gsecs / ((1 if args.fused_block else 4) * len(layers)) * 1e6, 3)
     result = {
         "metric": METRIC, "value": round(value / 1e9, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -835,6 +852,9 @@ def main(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="gate|up GEMM and SiLU*up+quant as separate launches instead of the "
                          "fused SiLU*up epilogue")
+    ap.add_argument("--fused-block", action="store_true",
+                    help="run each decoder block's linear path as the single fused persistent "
+                         "kernel (w8a8_block_decode; M <= 64)")
     ap.add_argument("--fp8", action="store_true",
                     help="the FP8 (E4M3) variant of the path: FP8 row kernels and GEMMs")
     ap.add_argument("--overlap", type=int, choices=[0, 1, 2], default=2,

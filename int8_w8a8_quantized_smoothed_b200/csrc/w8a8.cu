@@ -365,6 +365,16 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
     const int64_t U = NB * TT * KB;
     // every CTA must be resident at once (owners wait on later CTAs): at most one per SM
     int64_t G = (ctas == 0 || ctas > num_sms) ? num_sms : ctas;
+    if (ctas == 0) {
+        // Whole blocks per CTA when that keeps most SMs streaming: no block is split, so no
+        // partial sums cross CTAs (e.g. 224 channel blocks as 2 per CTA on 112 SMs beats the
+        // even split over 148 SMs at every decode size: the split-K tail costs more than the
+        // 36 idle SMs' share of the weight stream).
+        const int64_t blocks = NB * TT;
+        const int64_t per = (blocks + num_sms - 1) / num_sms;
+        if (per <= 2 && blocks % per == 0 && (blocks / per) * 10 >= static_cast<int64_t>(num_sms) * 7)
+            G = blocks / per;
+    }
     if (G > U)
         G = U;
     if (G > kMaxCtas)
