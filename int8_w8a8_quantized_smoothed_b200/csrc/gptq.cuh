@@ -8,8 +8,9 @@
 //   diag         dead channels (H_jj = 0 -> 1), H_jj += damp * mean(H_jj)
 //   UL Cholesky  H = V V^T with V upper, by 64-column blocks from the last to the first
 //                (diagonal block, panel solve, trailing update of the blocks above-left)
-//   inverse      U = V^-1 (upper): diagonal blocks inverted, then the off-diagonal blocks by
-//                distance from the diagonal (each needs only blocks nearer to it)
+//   inverse      U = V^-1 (upper): diagonal blocks inverted, then the off-diagonal blocks
+//                right-looking from the bottom block row (every finished block row adds its
+//                contributions to all pending blocks at once)
 //   quantize     64-column blocks in order: one warp per row runs the block's columns
 //                sequentially (quantize, error, compensate inside the block), then one
 //                tiled update applies the block's errors to every later column (the lazy
@@ -310,39 +311,52 @@ __global__ void __launch_bounds__(kT) trtri_diag_kernel(const double *__restrict
     }
 }
 
-// Off-diagonal blocks at distance dist (one CTA per block i, j = i + dist):
-// U[i][j] = -U_ii (sum_{k=i+1..j} V[i][k] U[k][j]); every U[k][j] used is nearer the diagonal.
-__global__ void __launch_bounds__(kThreads) trtri_off_kernel(const double *__restrict__ V,
-                                                            double *__restrict__ U, int64_t K,
-                                                            int dist)
+// Off-diagonal blocks, right-looking from the bottom block row: U[i][j] (i < j) is
+// -U_ii T[i][j] with T[i][j] = sum_{k=i+1..j} V[i][k] U[k][j]. The off-diagonal blocks of U hold
+// the running sums T (zero to begin with); once block row k is final (trtri_final_kernel),
+// trtri_update_kernel adds V[i][k] U[k][j] into T[i][j] for every i < k <= j, one product per
+// CTA, so each T[i][j] receives its terms in the fixed order k = j, j-1, .., i+1.
+__global__ void __launch_bounds__(kThreads) trtri_update_kernel(const double *__restrict__ V,
+                                                               double *__restrict__ U, int64_t K,
+                                                               int k)
 {
     double *sa = gptq_smem, *sb = gptq_smem + kT * kLd;
-    const int64_t i = blockIdx.x, j = i + dist;
+    const int64_t nb = K / kT;
+    const int64_t i = blockIdx.x % k, j = k + blockIdx.x / k; // i < k <= j < nb
+    if (j >= nb)
+        return;
+    load_tile(sa, V, K, i * kT, k * kT);
+    load_tile(sb, U, K, k * kT, j * kT);
+    __syncthreads();
     double acc[4][4];
     zero_acc(acc);
-    for (int64_t k = i + 1; k <= j; ++k) {
-        load_tile(sa, V, K, i * kT, k * kT);
-        load_tile(sb, U, K, k * kT, j * kT);
-        __syncthreads();
-        mm_ab(sa, sb, acc);
-        __syncthreads();
-    }
-    // T -> sb, U_ii -> sa, then U[i][j] = -U_ii T
+    mm_ab(sa, sb, acc);
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-            sb[(ty + 16 * a) * kLd + tx + 16 * b] = acc[a][b];
-    load_tile(sa, U, K, i * kT, i * kT);
+            U[(i * kT + ty + 16 * a) * K + j * kT + tx + 16 * b] += acc[a][b];
+}
+
+// Block row k final: U[k][j] = -U_kk T[k][j] for every j > k (one CTA per j).
+__global__ void __launch_bounds__(kThreads) trtri_final_kernel(double *__restrict__ U, int64_t K,
+                                                              int k)
+{
+    double *sa = gptq_smem, *sb = gptq_smem + kT * kLd;
+    const int64_t j = k + 1 + blockIdx.x;
+    load_tile(sa, U, K, static_cast<int64_t>(k) * kT, static_cast<int64_t>(k) * kT);
+    load_tile(sb, U, K, static_cast<int64_t>(k) * kT, j * kT);
     __syncthreads();
+    double acc[4][4];
     zero_acc(acc);
     mm_ab(sa, sb, acc);
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-            U[(i * kT + ty + 16 * a) * K + j * kT + tx + 16 * b] = -acc[a][b];
+            U[(static_cast<int64_t>(k) * kT + ty + 16 * a) * K + j * kT + tx + 16 * b] = -acc[a][b];
 }
 
 // Lower off-diagonal blocks of U are zero (U is returned whole to callers that ask for it).

@@ -1177,7 +1177,8 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     for (const void *fn : {reinterpret_cast<const void *>(&g::chol_panel_kernel),
                            reinterpret_cast<const void *>(&g::chol_update_kernel),
                            reinterpret_cast<const void *>(&g::trtri_diag_kernel),
-                           reinterpret_cast<const void *>(&g::trtri_off_kernel),
+                           reinterpret_cast<const void *>(&g::trtri_update_kernel),
+                           reinterpret_cast<const void *>(&g::trtri_final_kernel),
                            reinterpret_cast<const void *>(&g::update_kernel)})
         if ((rc = ensure_smem(fn, dev, sm2)))
             return rc;
@@ -1192,9 +1193,18 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
             g::chol_update_kernel<<<kb * (kb + 1) / 2, g::kThreads, sm2, st>>>(A, K, kb);
         }
     }
+    // U's off-diagonal blocks start as zero running sums
+    if (cudaMemsetAsync(U, 0, static_cast<size_t>(K * K) * sizeof(double), st) != cudaSuccess)
+        return W8A8_ERR_CUDA;
     g::trtri_diag_kernel<<<nb, g::kT, sm2, st>>>(A, U, K);
-    for (int d = 1; d < nb; ++d)
-        g::trtri_off_kernel<<<nb - d, g::kThreads, sm2, st>>>(A, U, K, d);
+    for (int k = nb - 1; k >= 1; --k) {
+        // block row k is final from here on (row nb-1 is its diagonal block only)
+        if (k < nb - 1)
+            g::trtri_final_kernel<<<nb - 1 - k, g::kThreads, sm2, st>>>(U, K, k);
+        g::trtri_update_kernel<<<k * (nb - k), g::kThreads, sm2, st>>>(A, U, K, k);
+    }
+    if (nb > 1)
+        g::trtri_final_kernel<<<nb - 1, g::kThreads, sm2, st>>>(U, K, 0);
     const unsigned rows_grid =
         static_cast<unsigned>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(sms) * 8));
     g::prep_kernel<<<rows_grid, g::kThreads, 0, st>>>(w, smooth, dead, N, K, wd, s_ch);
