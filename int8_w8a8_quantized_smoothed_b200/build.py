@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libw8a8.so")
 SOURCES = [os.path.join(CSRC, "w8a8.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "rowquant.cuh", "gemm.cuh", "probe.cuh")] + [
+DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(ROOT, "include", "w8a8.h")]
 
 NVCC_FLAGS = [

@@ -191,29 +191,44 @@ __global__ void __launch_bounds__(kThreads) chol_diag_kernel(double *__restrict_
                                                             int kb, int *__restrict__ bad)
 {
     __shared__ double d[kT * kLd];
+    __shared__ double piv[2]; // V[j][j] and its reciprocal, formed once per step
     const int64_t o = static_cast<int64_t>(kb) * kT;
     load_tile(d, A, K, o, o);
     __syncthreads();
     for (int j = kT - 1; j >= 0; --j) {
-        double p = d[j * kLd + j];
-        if (!(p > 0.0)) {
-            if (threadIdx.x == 0)
+        if (threadIdx.x == 0) {
+            double p = d[j * kLd + j];
+            if (!(p > 0.0)) {
                 atomicExch(bad, 1);
-            p = 2.2250738585072014e-308;
+                p = 2.2250738585072014e-308;
+            }
+            const double vjj = sqrt(p);
+            piv[0] = vjj;
+            piv[1] = 1.0 / vjj;
+            d[j * kLd + j] = vjj;
         }
-        const double vjj = sqrt(p);
-        __syncthreads(); // every thread has read the pivot
+        __syncthreads();
         // column j above the diagonal: V[i][j] = D[i][j] / V[j][j]
         if (threadIdx.x < j)
-            d[threadIdx.x * kLd + j] = d[threadIdx.x * kLd + j] / vjj;
-        if (threadIdx.x == 0)
-            d[j * kLd + j] = vjj;
+            d[threadIdx.x * kLd + j] = d[threadIdx.x * kLd + j] * piv[1];
         __syncthreads();
-        // D[i][i'] -= V[i][j] V[i'][j] for i <= i' < j (upper triangle of the rest)
-        for (int e = threadIdx.x; e < j * j; e += kThreads) {
-            const int i = e / j, i2 = e % j;
-            if (i <= i2)
-                d[i * kLd + i2] -= d[i * kLd + j] * d[i2 * kLd + j];
+        // D[i][i'] -= V[i][j] V[i'][j] for i <= i' < j (upper triangle of the rest); thread
+        // (ty, tx) owns rows ty + 16a and columns tx + 16b
+        {
+            const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int i = ty + 16 * a;
+                if (i < j) {
+                    const double vi = d[i * kLd + j];
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const int i2 = tx + 16 * b;
+                        if (i <= i2 && i2 < j)
+                            d[i * kLd + i2] -= vi * d[i2 * kLd + j];
+                    }
+                }
+            }
         }
         __syncthreads();
     }
@@ -232,16 +247,30 @@ __global__ void __launch_bounds__(kThreads) chol_panel_kernel(double *__restrict
 {
     double *a = gptq_smem, *v = gptq_smem + kT * kLd;
     const int64_t oc = static_cast<int64_t>(kb) * kT, orow = static_cast<int64_t>(blockIdx.x) * kT;
+    __shared__ double vinv[kT]; // 1 / V[j][j]
     load_tile(a, A, K, orow, oc);
     load_tile(v, A, K, oc, oc);
     __syncthreads();
+    if (threadIdx.x < kT)
+        vinv[threadIdx.x] = 1.0 / v[threadIdx.x * kLd + threadIdx.x];
+    __syncthreads();
     for (int j = kT - 1; j >= 0; --j) {
         if (threadIdx.x < kT)
-            a[threadIdx.x * kLd + j] = a[threadIdx.x * kLd + j] / v[j * kLd + j];
+            a[threadIdx.x * kLd + j] = a[threadIdx.x * kLd + j] * vinv[j];
         __syncthreads();
-        for (int e = threadIdx.x; e < kT * j; e += kThreads) {
-            const int r = e / j, k = e % j;
-            a[r * kLd + k] -= a[r * kLd + j] * v[k * kLd + j];
+        {
+            const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+            for (int aa = 0; aa < 4; ++aa) {
+                const int r = ty + 16 * aa;
+                const double xr = a[r * kLd + j];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int k = tx + 16 * b;
+                    if (k < j)
+                        a[r * kLd + k] -= xr * v[k * kLd + j];
+                }
+            }
         }
         __syncthreads();
     }
@@ -414,14 +443,19 @@ __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restric
                                                               double *__restrict__ err)
 {
     __shared__ double u[kT * kLd];
+    __shared__ double uinv[kT]; // 1 / U[j][j]
     const int64_t j0 = static_cast<int64_t>(jb) * kT;
     load_tile(u, U, K, j0, j0);
+    __syncthreads();
+    if (threadIdx.x < kT)
+        uinv[threadIdx.x] = 1.0 / u[threadIdx.x * kLd + threadIdx.x];
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
     for (int64_t n = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
          n < N; n += warps) {
         const double s = static_cast<double>(s_ch[n]);
+        const double sinv = s > 0.0 ? 1.0 / s : 0.0;
         double w0 = wd[n * K + j0 + lane], w1 = wd[n * K + j0 + 32 + lane];
         int q0 = 0, q1 = 0;
         double e0 = 0.0, e1 = 0.0;
@@ -432,10 +466,10 @@ __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restric
                 const double wj = hi ? w1 : w0;
                 double q = 0.0;
                 if (s > 0.0) {
-                    q = rint(wj / s);
+                    q = rint(wj * sinv);
                     q = fmin(fmax(q, -127.0), 127.0);
                 }
-                e = (wj - q * s) / u[j * kLd + j];
+                e = (wj - q * s) * uinv[j];
                 if (hi) {
                     q1 = static_cast<int>(q);
                     e1 = e;
