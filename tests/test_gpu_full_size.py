@@ -100,3 +100,62 @@ def test_row_kernels_full_size_sampled_rows(M, H, I):
     q, s = w8.w8a8_silu_mul_quant(dev_bf16(gu))
     q_ref, s_ref = oracle.silu_mul_quant(gu[rows])
     assert np.array_equal(host(q)[rows], q_ref) and np.array_equal(host(s)[rows], s_ref)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) at full size
+
+
+def _fp8_codes(shape, seed):
+    c = np.random.default_rng(seed).integers(0, 256, shape, dtype=np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x3C  # no NaN codes
+    return c
+
+
+def _dev_fp8(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda().view(w8.FP8)
+
+
+def _check_gemm_fp8(M, N, K, seed, wseed):
+    xq = _fp8_codes((M, K), seed)
+    wq = _fp8_codes((N, K), wseed)
+    st = synth.scales(M, seed + 2, 1e-3, 0.5)
+    sc = synth.scales(N, seed + 3, 1e-4, 2e-2)
+    acc = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    y = w8.w8a8_gemm_dequant_fp8(_dev_fp8(xq), dev(st), _dev_fp8(wq), dev(sc), acc_out=acc)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, M - 1], synth.row_sample(M, seed, count=6)]))
+    _, acc_ref, absacc = oracle.gemm_fp8(xq[rows], st[rows], wq, sc)
+    a = host(acc)[rows].astype(np.float64)
+    assert (np.abs(a - acc_ref) <= (K + 16) * 2.0 ** -24 * absacc).all()
+    assert np.array_equal(host_bf16(y)[rows], oracle.dequant_f32acc(host(acc)[rows], st[rows], sc))
+
+
+@pytest.mark.parametrize("M", [1, 64, 2048])
+@pytest.mark.parametrize("name,N,K", projections(LLAMA8B))
+def test_llama8b_gemm_fp8(M, name, N, K):
+    _check_gemm_fp8(M, N, K, _seed(name, M) + 3, _seed(name, 2))
+
+
+@pytest.mark.parametrize("M", [16, 4096])
+@pytest.mark.parametrize("name,N,K", projections(LLAMA70B))
+def test_llama70b_gemm_fp8(M, name, N, K):
+    _check_gemm_fp8(M, N, K, _seed(name, M) + 4, _seed(name, 3))
+
+
+@pytest.mark.parametrize("M,H,I", [(8192, 4096, 14336), (64, 4096, 14336)])
+def test_row_kernels_fp8_full_size_sampled_rows(M, H, I):
+    rows = synth.row_sample(M, 5, count=32)
+    x = synth.activation(M, H, 11)
+    res = synth.normal_bf16((M, H), 12)
+    gam = synth.gamma(H, 13)
+    q, s, h = w8.w8a8_smooth_rmsnorm_quant_fp8(dev_bf16(x), dev(gam), 1e-5,
+                                               residual=dev_bf16(res))
+    ref, _ = assert_rms_rows_match(q.view(torch.uint8).cpu().numpy()[rows], host(s)[rows],
+                                   x[rows], gam, 1e-5, residual=res[rows],
+                                   ref_fn=oracle.smooth_rmsnorm_quant_fp8)
+    assert np.array_equal(host_bf16(h)[rows], ref["h"])
+    gu = synth.normal_bf16((M, 2 * I), 15, std=2.0)
+    q, s = w8.w8a8_silu_mul_quant_fp8(dev_bf16(gu))
+    q_ref, s_ref = oracle.silu_mul_quant_fp8(gu[rows])
+    assert np.array_equal(q.view(torch.uint8).cpu().numpy()[rows], q_ref)
+    assert np.array_equal(host(s)[rows], s_ref)
