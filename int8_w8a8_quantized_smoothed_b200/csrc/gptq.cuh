@@ -12,9 +12,11 @@
 //                right-looking from the bottom block row (every finished block row adds its
 //                contributions to all pending blocks at once)
 //   quantize     64-column blocks in order: one warp per row runs the block's columns
-//                sequentially (quantize, error, compensate inside the block), then one
-//                tiled update applies the block's errors to every later column (the lazy
-//                batch form: the same sums as the column-by-column form, in another order)
+//                sequentially (quantize, error, compensate inside the block); the lazy
+//                batch form applies the errors later, in two levels: each block's errors
+//                go at once to the rest of its group of four blocks, and a group's 256
+//                columns of errors go to every column after the group in one tiled pass
+//                (the same sums as the column-by-column form, in another order)
 // U = V^-1 is the Cholesky factor GPTQ needs: H = V V^T gives H^-1 = V^-T V^-1 = U^T U.
 // The dense steps run on 64 x 64 tiles staged in shared memory, 256 threads each owning a
 // 4 x 4 micro-tile (rows ty + 16a, columns tx + 16b) with fused multiply-adds.
@@ -28,8 +30,9 @@ namespace gptq {
 constexpr int kT = 64;    // tile / column-block size
 constexpr int kLd = 65;   // padded shared-memory row (doubles)
 constexpr int kThreads = 256;
-// dynamic shared memory of the two-tile kernels
+// dynamic shared memory of the two- and three-tile kernels
 constexpr int kTwoTileBytes = 2 * kT * kLd * 8;
+constexpr int kThreeTileBytes = 3 * kT * kLd * 8;
 
 extern __shared__ __align__(16) double gptq_smem[];
 
@@ -73,13 +76,33 @@ __device__ __forceinline__ void mm_ab(const double *A, const double *B, double (
     }
 }
 
-// 64 x 64 block (r0, c0) of a row-major matrix with leading dimension ld -> smem [64][kLd].
+// asynchronous global -> shared copies (complete after cp_async_wait_all)
+__device__ __forceinline__ void cp_async8(double *smem, const double *gmem)
+{
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(a), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(double *smem, const double *gmem)
+{
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(a), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// 64 x 64 block (r0, c0) of a row-major matrix with leading dimension ld -> smem [64][kLd],
+// issued as asynchronous copies: the caller waits (cp_async_wait_all) and synchronizes.
 __device__ __forceinline__ void load_tile(double *sm, const double *g, int64_t ld, int64_t r0,
                                           int64_t c0)
 {
+#pragma unroll 4
     for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
         const int r = e >> 6, c = e & 63;
-        sm[r * kLd + c] = g[(r0 + r) * ld + c0 + c];
+        cp_async8(sm + r * kLd + c, g + (r0 + r) * ld + c0 + c);
     }
 }
 
@@ -187,46 +210,45 @@ __global__ void __launch_bounds__(1024) diag_kernel(double *__restrict__ H, int6
 // Diagonal block kb: D = V_kk V_kk^T, V_kk upper, right-looking from the last column; the
 // block's upper triangle is overwritten with V_kk. A non-positive pivot (H not positive
 // definite) is replaced by the smallest normal double and reported through *bad.
+// One barrier per column: every thread forms the pivot and its reciprocal itself, the scaled
+// column V[i][j] = D[i][j] / V[j][j] (i < j) goes to the unused lower triangle (d[j][i]) and
+// the pivot to dg[j], so nothing read in a step is written in it.
 __global__ void __launch_bounds__(kThreads) chol_diag_kernel(double *__restrict__ A, int64_t K,
                                                             int kb, int *__restrict__ bad)
 {
     __shared__ double d[kT * kLd];
-    __shared__ double piv[2]; // V[j][j] and its reciprocal, formed once per step
+    __shared__ double dg[kT];
     const int64_t o = static_cast<int64_t>(kb) * kT;
     load_tile(d, A, K, o, o);
+    cp_async_wait_all();
     __syncthreads();
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     for (int j = kT - 1; j >= 0; --j) {
+        double p = d[j * kLd + j];
+        const bool ok = p > 0.0;
+        if (!ok)
+            p = 2.2250738585072014e-308;
+        const double vjj = sqrt(p);
+        const double rinv = 1.0 / vjj;
         if (threadIdx.x == 0) {
-            double p = d[j * kLd + j];
-            if (!(p > 0.0)) {
+            if (!ok)
                 atomicExch(bad, 1);
-                p = 2.2250738585072014e-308;
-            }
-            const double vjj = sqrt(p);
-            piv[0] = vjj;
-            piv[1] = 1.0 / vjj;
-            d[j * kLd + j] = vjj;
+            dg[j] = vjj;
         }
-        __syncthreads();
-        // column j above the diagonal: V[i][j] = D[i][j] / V[j][j]
         if (threadIdx.x < j)
-            d[threadIdx.x * kLd + j] = d[threadIdx.x * kLd + j] * piv[1];
-        __syncthreads();
+            d[j * kLd + threadIdx.x] = d[threadIdx.x * kLd + j] * rinv;
         // D[i][i'] -= V[i][j] V[i'][j] for i <= i' < j (upper triangle of the rest); thread
         // (ty, tx) owns rows ty + 16a and columns tx + 16b
-        {
-            const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const int i = ty + 16 * a;
-                if (i < j) {
-                    const double vi = d[i * kLd + j];
+        for (int a = 0; a < 4; ++a) {
+            const int i = ty + 16 * a;
+            if (i < j) {
+                const double vi = d[i * kLd + j] * rinv;
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const int i2 = tx + 16 * b;
-                        if (i <= i2 && i2 < j)
-                            d[i * kLd + i2] -= vi * d[i2 * kLd + j];
-                    }
+                for (int b = 0; b < 4; ++b) {
+                    const int i2 = tx + 16 * b;
+                    if (i <= i2 && i2 < j)
+                        d[i * kLd + i2] -= vi * (d[i2 * kLd + j] * rinv);
                 }
             }
         }
@@ -235,48 +257,48 @@ __global__ void __launch_bounds__(kThreads) chol_diag_kernel(double *__restrict_
     for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
         const int r = e >> 6, c = e & 63;
         if (r <= c)
-            A[(o + r) * K + o + c] = d[r * kLd + c];
+            A[(o + r) * K + o + c] = r == c ? dg[r] : d[c * kLd + r];
     }
 }
 
 // Panel of block column kb: V[ib][kb] = A[ib][kb] V_kk^-T for every ib < kb (one CTA each):
 // X V_kk^T = A solved from the last column: x_j = a_j / V[j][j], then a_k -= x_j V[k][j]
-// for k < j.
+// for k < j. One barrier per column: x_j goes to its own tile, every thread that needs it
+// scales a_j itself.
 __global__ void __launch_bounds__(kThreads) chol_panel_kernel(double *__restrict__ A, int64_t K,
                                                              int kb)
 {
-    double *a = gptq_smem, *v = gptq_smem + kT * kLd;
+    double *a = gptq_smem, *v = gptq_smem + kT * kLd, *x = gptq_smem + 2 * kT * kLd;
     const int64_t oc = static_cast<int64_t>(kb) * kT, orow = static_cast<int64_t>(blockIdx.x) * kT;
     __shared__ double vinv[kT]; // 1 / V[j][j]
     load_tile(a, A, K, orow, oc);
     load_tile(v, A, K, oc, oc);
+    cp_async_wait_all();
     __syncthreads();
     if (threadIdx.x < kT)
         vinv[threadIdx.x] = 1.0 / v[threadIdx.x * kLd + threadIdx.x];
     __syncthreads();
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     for (int j = kT - 1; j >= 0; --j) {
-        if (threadIdx.x < kT)
-            a[threadIdx.x * kLd + j] = a[threadIdx.x * kLd + j] * vinv[j];
-        __syncthreads();
-        {
-            const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+        const double vi = vinv[j];
 #pragma unroll
-            for (int aa = 0; aa < 4; ++aa) {
-                const int r = ty + 16 * aa;
-                const double xr = a[r * kLd + j];
+        for (int aa = 0; aa < 4; ++aa) {
+            const int r = ty + 16 * aa;
+            const double xr = a[r * kLd + j] * vi;
+            if (tx == 0)
+                x[r * kLd + j] = xr;
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int k = tx + 16 * b;
-                    if (k < j)
-                        a[r * kLd + k] -= xr * v[k * kLd + j];
-                }
+            for (int b = 0; b < 4; ++b) {
+                const int k = tx + 16 * b;
+                if (k < j)
+                    a[r * kLd + k] -= xr * v[k * kLd + j];
             }
         }
         __syncthreads();
     }
     for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
         const int r = e >> 6, c = e & 63;
-        A[(orow + r) * K + oc + c] = a[r * kLd + c];
+        A[(orow + r) * K + oc + c] = x[r * kLd + c];
     }
 }
 
@@ -295,6 +317,7 @@ __global__ void __launch_bounds__(kThreads) chol_update_kernel(double *__restric
     const int64_t oc = static_cast<int64_t>(kb) * kT;
     load_tile(p1, A, K, ib * kT, oc);
     load_tile(p2, A, K, jb * kT, oc);
+    cp_async_wait_all();
     __syncthreads();
     double acc[4][4];
     zero_acc(acc);
@@ -356,6 +379,7 @@ __global__ void __launch_bounds__(kThreads) trtri_update_kernel(const double *__
         return;
     load_tile(sa, V, K, i * kT, k * kT);
     load_tile(sb, U, K, k * kT, j * kT);
+    cp_async_wait_all();
     __syncthreads();
     double acc[4][4];
     zero_acc(acc);
@@ -376,6 +400,7 @@ __global__ void __launch_bounds__(kThreads) trtri_final_kernel(double *__restric
     const int64_t j = k + 1 + blockIdx.x;
     load_tile(sa, U, K, static_cast<int64_t>(k) * kT, static_cast<int64_t>(k) * kT);
     load_tile(sb, U, K, static_cast<int64_t>(k) * kT, j * kT);
+    cp_async_wait_all();
     __syncthreads();
     double acc[4][4];
     zero_acc(acc);
@@ -431,89 +456,149 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const uint16_t *__restri
     }
 }
 
-// Column block jb (columns j0 .. j0 + 63), one warp per row, lane l holding columns l and
-// l + 32: for each column j in order the lane that holds it rounds w_j / s, forms the error
-// e = (w_j - q s) / U[j][j] and broadcasts it; every lane subtracts e U[j][k] from its
-// columns k > j of the block. Codes go to wq, errors to err [N][64] for the update kernel.
+// Column block jb (columns j0 .. j0 + 63), one warp per pair of rows, lane l holding columns
+// l and l + 32 of both: for each column j in order the lane that holds it rounds w_j / s,
+// forms the error e = (w_j - q s) / U[j][j] and broadcasts it; every lane subtracts e U[j][k]
+// from its columns of the block (a lane whose column is already quantized updates a value
+// that is never read again, so the update needs no predicate). The two rows' dependency
+// chains interleave and share the loads of U; the column loop is unrolled, so which lane
+// pivots and which half it reads are compile-time constants. Codes go to wq, errors to
+// err[n * err_ld + t] (t = 0..63) for the update kernel.
+constexpr int kQuantRows = 2; // rows per warp in flight
+
 __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restrict__ wd,
                                                               const double *__restrict__ U,
                                                               const float *__restrict__ s_ch,
                                                               int64_t N, int64_t K, int jb,
                                                               int8_t *__restrict__ wq,
-                                                              double *__restrict__ err)
+                                                              double *__restrict__ err,
+                                                              int64_t err_ld)
 {
+    constexpr int R = kQuantRows;
     __shared__ double u[kT * kLd];
-    __shared__ double uinv[kT]; // 1 / U[j][j]
     const int64_t j0 = static_cast<int64_t>(jb) * kT;
     load_tile(u, U, K, j0, j0);
-    __syncthreads();
-    if (threadIdx.x < kT)
-        uinv[threadIdx.x] = 1.0 / u[threadIdx.x * kLd + threadIdx.x];
+    cp_async_wait_all();
     __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-    for (int64_t n = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
-         n < N; n += warps) {
-        const double s = static_cast<double>(s_ch[n]);
-        const double sinv = s > 0.0 ? 1.0 / s : 0.0;
-        double w0 = wd[n * K + j0 + lane], w1 = wd[n * K + j0 + 32 + lane];
-        int q0 = 0, q1 = 0;
-        double e0 = 0.0, e1 = 0.0;
-        for (int j = 0; j < kT; ++j) {
-            const bool hi = j >= 32;
-            double e = 0.0;
-            if (lane == (j & 31)) {
-                const double wj = hi ? w1 : w0;
-                double q = 0.0;
-                if (s > 0.0) {
-                    q = rint(wj * sinv);
-                    q = fmin(fmax(q, -127.0), 127.0);
-                }
-                e = (wj - q * s) * uinv[j];
-                if (hi) {
-                    q1 = static_cast<int>(q);
-                    e1 = e;
-                } else {
-                    q0 = static_cast<int>(q);
-                    e0 = e;
-                }
-            }
-            e = __shfl_sync(0xffffffffu, e, j & 31);
-            if (lane > j)
-                w0 -= e * u[j * kLd + lane];
-            if (lane + 32 > j)
-                w1 -= e * u[j * kLd + lane + 32];
+    const double uinv0 = 1.0 / u[lane * kLd + lane];
+    const double uinv1 = 1.0 / u[(lane + 32) * kLd + lane + 32];
+    const int64_t step = static_cast<int64_t>(gridDim.x) * (kThreads / 32) * R;
+    for (int64_t n0 = (static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5)) * R;
+         n0 < N; n0 += step) {
+        double s[R], sinv[R], w0[R], w1[R], q0[R], q1[R], e0[R], e1[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t n = n0 + r < N ? n0 + r : N - 1; // a duplicate row is not stored
+            s[r] = static_cast<double>(s_ch[n]);
+            sinv[r] = s[r] > 0.0 ? 1.0 / s[r] : 0.0;
+            w0[r] = wd[n * K + j0 + lane];
+            w1[r] = wd[n * K + j0 + 32 + lane];
+            q0[r] = q1[r] = e0[r] = e1[r] = 0.0;
         }
-        wq[n * K + j0 + lane] = static_cast<int8_t>(q0);
-        wq[n * K + j0 + 32 + lane] = static_cast<int8_t>(q1);
-        err[n * kT + lane] = e0;
-        err[n * kT + 32 + lane] = e1;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const double ua = u[j * kLd + lane], ub = u[j * kLd + 32 + lane];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (lane == j) {
+                    q0[r] = s[r] > 0.0 ? fmin(fmax(rint(w0[r] * sinv[r]), -127.0), 127.0) : 0.0;
+                    e0[r] = (w0[r] - q0[r] * s[r]) * uinv0;
+                }
+                const double e = __shfl_sync(0xffffffffu, e0[r], j);
+                w0[r] -= e * ua;
+                w1[r] -= e * ub;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const double ub = u[(32 + j) * kLd + 32 + lane];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (lane == j) {
+                    q1[r] = s[r] > 0.0 ? fmin(fmax(rint(w1[r] * sinv[r]), -127.0), 127.0) : 0.0;
+                    e1[r] = (w1[r] - q1[r] * s[r]) * uinv1;
+                }
+                const double e = __shfl_sync(0xffffffffu, e1[r], j);
+                w1[r] -= e * ub;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t n = n0 + r;
+            if (n < N) {
+                wq[n * K + j0 + lane] = static_cast<int8_t>(static_cast<int>(q0[r]));
+                wq[n * K + j0 + 32 + lane] = static_cast<int8_t>(static_cast<int>(q1[r]));
+                err[n * err_ld + lane] = e0[r];
+                err[n * err_ld + 32 + lane] = e1[r];
+            }
+        }
     }
 }
 
-// Lazy batch update after column block jb: W'[n][c] -= sum_t err[n][t] U[j0 + t][c] for the
-// columns c >= j0 + 64; one CTA per 64 x 64 tile (rows beyond N skipped).
+// rows of one update tile; 16-byte-aligned padded rows of the update kernel's tiles; its
+// dynamic shared memory
+constexpr int kRT = 128;
+constexpr int kLdU = 66;
+constexpr int kUpdateBytes = (kRT + kT) * kLdU * 8;
+
+// Lazy batch update: W'[n][c] -= sum_t err[n][t] U[j0 + t][c] for t < 64 * chunks and the
+// columns c = c_first + 64 * blockIdx.x + (0..63). One CTA per 128 x 64 tile of W' (a tile
+// past row N reads row N - 1 and writes nothing there); each thread owns an 8 x 4
+// micro-tile (rows ty + 16a, columns tx + 16b) and the depth runs in 64-deep chunks of err
+// and U copied to shared memory with 16-byte asynchronous copies, all in flight at once.
+// err rows, U rows and c_first are multiples of 16 bytes apart (64-column blocks, binary64).
 __global__ void __launch_bounds__(kThreads) update_kernel(double *__restrict__ wd,
                                                          const double *__restrict__ U,
                                                          const double *__restrict__ err,
-                                                         int64_t N, int64_t K, int jb)
+                                                         int64_t err_ld, int64_t N, int64_t K,
+                                                         int64_t j0, int chunks,
+                                                         int64_t c_first)
 {
-    double *se = gptq_smem, *su = gptq_smem + kT * kLd;
-    const int64_t j0 = static_cast<int64_t>(jb) * kT;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kT;
-    const int64_t c0 = j0 + kT + static_cast<int64_t>(blockIdx.x) * kT;
-    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
-        const int r = e >> 6, c = e & 63;
-        se[r * kLd + c] = r0 + r < N ? err[(r0 + r) * kT + c] : 0.0;
-    }
-    load_tile(su, U, K, j0, c0);
-    __syncthreads();
-    double acc[4][4];
-    zero_acc(acc);
-    mm_ab(se, su, acc);
+    double *se = gptq_smem, *su = gptq_smem + kRT * kLdU;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kRT;
+    const int64_t c0 = c_first + static_cast<int64_t>(blockIdx.x) * kT;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double acc[8][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            acc[a][b] = 0.0;
+    for (int ci = 0; ci < chunks; ++ci) {
+        if (ci)
+            __syncthreads();
+#pragma unroll 4
+        for (int e = threadIdx.x; e < kRT * (kT / 2); e += kThreads) {
+            const int r = e >> 5, c = (e & 31) * 2;
+            const int64_t n = r0 + r < N ? r0 + r : N - 1;
+            cp_async16(se + r * kLdU + c, err + n * err_ld + ci * kT + c);
+        }
+#pragma unroll 4
+        for (int e = threadIdx.x; e < kT * (kT / 2); e += kThreads) {
+            const int r = e >> 5, c = (e & 31) * 2;
+            cp_async16(su + r * kLdU + c, U + (j0 + static_cast<int64_t>(ci) * kT + r) * K + c0 + c);
+        }
+        cp_async_wait_all();
+        __syncthreads();
+#pragma unroll 2
+        for (int k = 0; k < kT; ++k) {
+            double a[8], b[4];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                a[i] = se[(ty + 16 * i) * kLdU + k];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                b[i] = su[k * kLdU + tx + 16 * i];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
         const int64_t r = r0 + ty + 16 * a;
         if (r < N) {
 #pragma unroll

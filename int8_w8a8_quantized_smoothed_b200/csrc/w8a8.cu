@@ -674,8 +674,11 @@ size_t round256(size_t b)
     return (b + 255) & ~static_cast<size_t>(255);
 }
 
-// H/V [K,K] fp64, U [K,K] fp64, working weight [N,K] fp64, block errors [N,64] fp64, dead
-// flags [K], the non-positive-pivot flag.
+// column blocks whose errors are batched into one update of the later columns
+constexpr int kGptqGroup = 4;
+
+// H/V [K,K] fp64, U [K,K] fp64, working weight [N,K] fp64, the errors of one group of column
+// blocks [N, 64 * kGptqGroup] fp64, dead flags [K], the non-positive-pivot flag.
 GptqLayout gptq_layout(int64_t N, int64_t K)
 {
     GptqLayout L;
@@ -684,7 +687,7 @@ GptqLayout gptq_layout(int64_t N, int64_t K)
     L.u_off = L.a_off + round256(kk);
     L.w_off = L.u_off + round256(kk);
     L.e_off = L.w_off + round256(static_cast<size_t>(N) * static_cast<size_t>(K) * sizeof(double));
-    L.d_off = L.e_off + round256(static_cast<size_t>(N) * 64 * sizeof(double));
+    L.d_off = L.e_off + round256(static_cast<size_t>(N) * 64 * kGptqGroup * sizeof(double));
     L.b_off = L.d_off + round256(static_cast<size_t>(K));
     L.total = L.b_off + 256;
     return L;
@@ -1174,14 +1177,18 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     int *bad = reinterpret_cast<int *>(base + L.b_off);
     const int nb = static_cast<int>(K / g::kT);
     const int sm2 = g::kTwoTileBytes;
-    for (const void *fn : {reinterpret_cast<const void *>(&g::chol_panel_kernel),
-                           reinterpret_cast<const void *>(&g::chol_update_kernel),
+    if ((rc = ensure_smem(reinterpret_cast<const void *>(&g::chol_panel_kernel), dev,
+                          g::kThreeTileBytes)))
+        return rc;
+    for (const void *fn : {reinterpret_cast<const void *>(&g::chol_update_kernel),
                            reinterpret_cast<const void *>(&g::trtri_diag_kernel),
                            reinterpret_cast<const void *>(&g::trtri_update_kernel),
-                           reinterpret_cast<const void *>(&g::trtri_final_kernel),
-                           reinterpret_cast<const void *>(&g::update_kernel)})
+                           reinterpret_cast<const void *>(&g::trtri_final_kernel)})
         if ((rc = ensure_smem(fn, dev, sm2)))
             return rc;
+    if ((rc = ensure_smem(reinterpret_cast<const void *>(&g::update_kernel), dev,
+                          g::kUpdateBytes)))
+        return rc;
     if (cudaMemsetAsync(bad, 0, sizeof(int), st) != cudaSuccess)
         return W8A8_ERR_CUDA;
     g::hessian_kernel<<<nb * (nb + 1) / 2, g::kThreads, 0, st>>>(x_cal, T, K, A);
@@ -1189,7 +1196,7 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     for (int kb = nb - 1; kb >= 0; --kb) {
         g::chol_diag_kernel<<<1, g::kThreads, 0, st>>>(A, K, kb, bad);
         if (kb > 0) {
-            g::chol_panel_kernel<<<kb, g::kThreads, sm2, st>>>(A, K, kb);
+            g::chol_panel_kernel<<<kb, g::kThreads, g::kThreeTileBytes, st>>>(A, K, kb);
             g::chol_update_kernel<<<kb * (kb + 1) / 2, g::kThreads, sm2, st>>>(A, K, kb);
         }
     }
@@ -1208,12 +1215,36 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     const unsigned rows_grid =
         static_cast<unsigned>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(sms) * 8));
     g::prep_kernel<<<rows_grid, g::kThreads, 0, st>>>(w, smooth, dead, N, K, wd, s_ch);
-    const unsigned row_tiles = static_cast<unsigned>((N + g::kT - 1) / g::kT);
-    for (int jb = 0; jb < nb; ++jb) {
-        g::quant_block_kernel<<<rows_grid, g::kThreads, 0, st>>>(wd, U, s_ch, N, K, jb, wq, err);
-        if (jb + 1 < nb)
-            g::update_kernel<<<dim3(nb - 1 - jb, row_tiles), g::kThreads, sm2, st>>>(wd, U, err, N,
-                                                                                 K, jb);
+    // groups of kGptqGroup column blocks: inside a group each block's errors reach the
+    // group's later blocks at once; the group's errors then reach every later column in one
+    // pass over the working weight
+    const unsigned row_tiles = static_cast<unsigned>((N + g::kRT - 1) / g::kRT);
+    // one wave of the quantize kernel (8 warps of kQuantRows rows per CTA)
+    int quant_per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &quant_per_sm, g::quant_block_kernel, g::kThreads, 0) != cudaSuccess ||
+        quant_per_sm < 1)
+        return W8A8_ERR_CUDA;
+    const int64_t quant_rows = static_cast<int64_t>(g::kThreads / 32) * g::kQuantRows;
+    const unsigned quant_grid = static_cast<unsigned>(std::min<int64_t>(
+        (N + quant_rows - 1) / quant_rows, static_cast<int64_t>(sms) * quant_per_sm));
+    const int64_t eld = static_cast<int64_t>(g::kT) * kGptqGroup;
+    const int ub = g::kUpdateBytes;
+    for (int b0 = 0; b0 < nb; b0 += kGptqGroup) {
+        const int b1 = std::min(nb, b0 + kGptqGroup);
+        for (int jb = b0; jb < b1; ++jb) {
+            double *ej = err + static_cast<int64_t>(jb - b0) * g::kT;
+            g::quant_block_kernel<<<quant_grid, g::kThreads, 0, st>>>(wd, U, s_ch, N, K, jb, wq,
+                                                                       ej, eld);
+            if (jb + 1 < b1)
+                g::update_kernel<<<dim3(b1 - 1 - jb, row_tiles), g::kThreads, ub, st>>>(
+                    wd, U, ej, eld, N, K, static_cast<int64_t>(jb) * g::kT, 1,
+                    static_cast<int64_t>(jb + 1) * g::kT);
+        }
+        if (b1 < nb)
+            g::update_kernel<<<dim3(nb - b1, row_tiles), g::kThreads, ub, st>>>(
+                wd, U, err, eld, N, K, static_cast<int64_t>(b0) * g::kT, b1 - b0,
+                static_cast<int64_t>(b1) * g::kT);
     }
     if (u_out) {
         g::zero_lower_kernel<<<sms * 4, g::kThreads, 0, st>>>(U, K);
