@@ -460,10 +460,12 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const uint16_t *__restri
 // l and l + 32 of both: for each column j in order the lane that holds it rounds w_j / s,
 // forms the error e = (w_j - q s) / U[j][j] and broadcasts it; every lane subtracts e U[j][k]
 // from its columns of the block (a lane whose column is already quantized updates a value
-// that is never read again, so the update needs no predicate). The two rows' dependency
-// chains interleave and share the loads of U; the column loop is unrolled, so which lane
-// pivots and which half it reads are compile-time constants. Codes go to wq, errors to
-// err[n * err_ld + t] (t = 0..63) for the update kernel.
+// that is never read again, so the update needs no predicate). Every lane forms the code and
+// error of its own column and the pivot lane's pair is selected, so the loop has no branch
+// and the two rows' dependency chains interleave (they share the loads of U); the column
+// loop is unrolled, so which lane pivots is a compile-time constant. A zero scale has a zero
+// reciprocal, so its codes are 0. Codes go to wq, errors to err[n * err_ld + t] (t = 0..63)
+// for the update kernel.
 constexpr int kQuantRows = 2; // rows per warp in flight
 
 __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restrict__ wd,
@@ -501,11 +503,11 @@ __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restric
             const double ua = u[j * kLd + lane], ub = u[j * kLd + 32 + lane];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                if (lane == j) {
-                    q0[r] = s[r] > 0.0 ? fmin(fmax(rint(w0[r] * sinv[r]), -127.0), 127.0) : 0.0;
-                    e0[r] = (w0[r] - q0[r] * s[r]) * uinv0;
-                }
-                const double e = __shfl_sync(0xffffffffu, e0[r], j);
+                const double qc = fmin(fmax(rint(w0[r] * sinv[r]), -127.0), 127.0);
+                const double ec = (w0[r] - qc * s[r]) * uinv0;
+                q0[r] = lane == j ? qc : q0[r];
+                e0[r] = lane == j ? ec : e0[r];
+                const double e = __shfl_sync(0xffffffffu, ec, j);
                 w0[r] -= e * ua;
                 w1[r] -= e * ub;
             }
@@ -515,11 +517,11 @@ __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restric
             const double ub = u[(32 + j) * kLd + 32 + lane];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                if (lane == j) {
-                    q1[r] = s[r] > 0.0 ? fmin(fmax(rint(w1[r] * sinv[r]), -127.0), 127.0) : 0.0;
-                    e1[r] = (w1[r] - q1[r] * s[r]) * uinv1;
-                }
-                const double e = __shfl_sync(0xffffffffu, e1[r], j);
+                const double qc = fmin(fmax(rint(w1[r] * sinv[r]), -127.0), 127.0);
+                const double ec = (w1[r] - qc * s[r]) * uinv1;
+                q1[r] = lane == j ? qc : q1[r];
+                e1[r] = lane == j ? ec : e1[r];
+                const double e = __shfl_sync(0xffffffffu, ec, j);
                 w1[r] -= e * ub;
             }
         }
@@ -536,17 +538,21 @@ __global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restric
     }
 }
 
-// rows of one update tile; 16-byte-aligned padded rows of the update kernel's tiles; its
-// dynamic shared memory
+// Update tiles: 128 rows x 64 columns; the depth is staged 32 at a time (err [128][32] and
+// U [32][64], rows padded to 16-byte multiples), two stages in flight; dynamic shared memory.
 constexpr int kRT = 128;
-constexpr int kLdU = 66;
-constexpr int kUpdateBytes = (kRT + kT) * kLdU * 8;
+constexpr int kDC = 32;
+constexpr int kLdE = kDC + 2;
+constexpr int kLdU = kT + 2;
+constexpr int kStage = kRT * kLdE + kDC * kLdU; // doubles
+constexpr int kUpdateBytes = 2 * kStage * 8;
 
 // Lazy batch update: W'[n][c] -= sum_t err[n][t] U[j0 + t][c] for t < 64 * chunks and the
 // columns c = c_first + 64 * blockIdx.x + (0..63). One CTA per 128 x 64 tile of W' (a tile
 // past row N reads row N - 1 and writes nothing there); each thread owns an 8 x 4
-// micro-tile (rows ty + 16a, columns tx + 16b) and the depth runs in 64-deep chunks of err
-// and U copied to shared memory with 16-byte asynchronous copies, all in flight at once.
+// micro-tile (rows ty + 16a, columns tx + 16b). The depth runs in 32-deep stages copied to
+// shared memory with 16-byte asynchronous copies, the next stage's copies in flight while
+// the current one is multiplied; the tile of W' is prefetched into L2 at the start.
 // err rows, U rows and c_first are multiples of 16 bytes apart (64-column blocks, binary64).
 __global__ void __launch_bounds__(kThreads) update_kernel(double *__restrict__ wd,
                                                          const double *__restrict__ U,
@@ -555,38 +561,54 @@ __global__ void __launch_bounds__(kThreads) update_kernel(double *__restrict__ w
                                                          int64_t j0, int chunks,
                                                          int64_t c_first)
 {
-    double *se = gptq_smem, *su = gptq_smem + kRT * kLdU;
     const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kRT;
     const int64_t c0 = c_first + static_cast<int64_t>(blockIdx.x) * kT;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    // the W' tile: 128 rows of four 128-byte lines
+    for (int l = threadIdx.x; l < kRT * 4; l += kThreads) {
+        const int64_t r = r0 + (l >> 2);
+        if (r < N)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(wd + r * K + c0 + (l & 3) * 16));
+    }
+    auto stage = [&](int buf, int cc) {
+        double *se = gptq_smem + buf * kStage, *su = se + kRT * kLdE;
+#pragma unroll
+        for (int e = threadIdx.x; e < kRT * (kDC / 2); e += kThreads) {
+            const int r = e >> 4, c = (e & 15) * 2;
+            const int64_t n = r0 + r < N ? r0 + r : N - 1;
+            cp_async16(se + r * kLdE + c, err + n * err_ld + cc * kDC + c);
+        }
+#pragma unroll
+        for (int e = threadIdx.x; e < kDC * (kT / 2); e += kThreads) {
+            const int r = e >> 5, c = (e & 31) * 2;
+            cp_async16(su + r * kLdU + c,
+                       U + (j0 + static_cast<int64_t>(cc) * kDC + r) * K + c0 + c);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
     double acc[8][4];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b)
             acc[a][b] = 0.0;
-    for (int ci = 0; ci < chunks; ++ci) {
-        if (ci)
-            __syncthreads();
-#pragma unroll 4
-        for (int e = threadIdx.x; e < kRT * (kT / 2); e += kThreads) {
-            const int r = e >> 5, c = (e & 31) * 2;
-            const int64_t n = r0 + r < N ? r0 + r : N - 1;
-            cp_async16(se + r * kLdU + c, err + n * err_ld + ci * kT + c);
+    const int stages = chunks * (kT / kDC);
+    stage(0, 0);
+    for (int cc = 0; cc < stages; ++cc) {
+        if (cc + 1 < stages) {
+            stage((cc + 1) & 1, cc + 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-#pragma unroll 4
-        for (int e = threadIdx.x; e < kT * (kT / 2); e += kThreads) {
-            const int r = e >> 5, c = (e & 31) * 2;
-            cp_async16(su + r * kLdU + c, U + (j0 + static_cast<int64_t>(ci) * kT + r) * K + c0 + c);
-        }
-        cp_async_wait_all();
         __syncthreads();
-#pragma unroll 2
-        for (int k = 0; k < kT; ++k) {
+        const double *se = gptq_smem + (cc & 1) * kStage, *su = se + kRT * kLdE;
+#pragma unroll 4
+        for (int k = 0; k < kDC; ++k) {
             double a[8], b[4];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-                a[i] = se[(ty + 16 * i) * kLdU + k];
+                a[i] = se[(ty + 16 * i) * kLdE + k];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 b[i] = su[k * kLdU + tx + 16 * i];
@@ -596,6 +618,7 @@ __global__ void __launch_bounds__(kThreads) update_kernel(double *__restrict__ w
                 for (int j = 0; j < 4; ++j)
                     acc[i][j] = fma(a[i], b[j], acc[i][j]);
         }
+        __syncthreads(); // the buffer is refilled two stages on
     }
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
