@@ -18,8 +18,9 @@
 //                columns of errors go to every column after the group in one tiled pass
 //                (the same sums as the column-by-column form, in another order)
 // U = V^-1 is the Cholesky factor GPTQ needs: H = V V^T gives H^-1 = V^-T V^-1 = U^T U.
-// The dense steps run on 64 x 64 tiles staged in shared memory, 256 threads each owning a
-// 4 x 4 micro-tile (rows ty + 16a, columns tx + 16b) with fused multiply-adds.
+// The dense steps run on tiles staged in shared memory by asynchronous copies, each thread
+// owning a register micro-tile of the result (4 x 4 in the Hessian, 8 x 4 in the trailing
+// and lazy-batch updates) accumulated with fused multiply-adds.
 #pragma once
 
 #include <stdint.h>
@@ -36,44 +37,47 @@ constexpr int kThreeTileBytes = 3 * kT * kLd * 8;
 
 extern __shared__ __align__(16) double gptq_smem[];
 
-// acc[a][b] += sum_k A[ty + 16a][k] * Bt[tx + 16b][k]   (both tiles row-major in smem, [64][kLd])
-__device__ __forceinline__ void mm_abt(const double *A, const double *Bt, double (&acc)[4][4])
+// The trailing-update tile kernels run 128 threads, each owning an 8 x 4 micro-tile of the
+// 64 x 64 result (rows ty + 8a, columns tx + 16b): twelve shared-memory loads per 32 FMAs.
+constexpr int kTileThreads = 128;
+
+// acc[a][b] += sum_k A[ty + 8a][k] * B[k][tx + 16b], or B[tx + 16b][k] when BT
+template <bool BT>
+__device__ __forceinline__ void mm84(const double *A, const double *B, double (&acc)[8][4])
 {
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll 4
     for (int k = 0; k < kT; ++k) {
-        double a[4], b[4];
+        double a[8], b[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            a[i] = A[(ty + 16 * i) * kLd + k];
-            b[i] = Bt[(tx + 16 * i) * kLd + k];
-        }
+        for (int i = 0; i < 8; ++i)
+            a[i] = A[(ty + 8 * i) * kLd + k];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
+            b[i] = BT ? B[(tx + 16 * i) * kLd + k] : B[k * kLd + tx + 16 * i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
 }
 
-// acc[a][b] += sum_k A[ty + 16a][k] * B[k][tx + 16b]
-__device__ __forceinline__ void mm_ab(const double *A, const double *B, double (&acc)[4][4])
+__device__ __forceinline__ void zero_acc84(double (&acc)[8][4])
 {
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-#pragma unroll 4
-    for (int k = 0; k < kT; ++k) {
-        double a[4], b[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            a[i] = A[(ty + 16 * i) * kLd + k];
-            b[i] = B[k * kLd + tx + 16 * i];
-        }
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[i][j] = fma(a[i], b[j], acc[i][j]);
-    }
+        for (int j = 0; j < 4; ++j)
+            acc[i][j] = 0.0;
+}
+
+// the 64 x 64 block (r0, c0) of a row-major matrix into L2 (four 128-byte lines per row)
+__device__ __forceinline__ void prefetch_tile_l2(const double *g, int64_t ld, int64_t r0,
+                                                 int64_t c0)
+{
+    for (int l = threadIdx.x; l < kT * 4; l += blockDim.x)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(g + (r0 + (l >> 2)) * ld + c0 + (l & 3) * 16));
 }
 
 // asynchronous global -> shared copies (complete after cp_async_wait_all)
@@ -96,11 +100,12 @@ __device__ __forceinline__ void cp_async_wait_all()
 
 // 64 x 64 block (r0, c0) of a row-major matrix with leading dimension ld -> smem [64][kLd],
 // issued as asynchronous copies: the caller waits (cp_async_wait_all) and synchronizes.
+template <int NT = kThreads>
 __device__ __forceinline__ void load_tile(double *sm, const double *g, int64_t ld, int64_t r0,
                                           int64_t c0)
 {
 #pragma unroll 4
-    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
+    for (int e = threadIdx.x; e < kT * kT; e += NT) {
         const int r = e >> 6, c = e & 63;
         cp_async8(sm + r * kLd + c, g + (r0 + r) * ld + c0 + c);
     }
@@ -304,8 +309,8 @@ __global__ void __launch_bounds__(kThreads) chol_panel_kernel(double *__restrict
 
 // Trailing update after block column kb: A[ib][jb] -= V[ib][kb] V[jb][kb]^T for
 // ib <= jb < kb (the upper triangle of the remaining blocks); one CTA per pair.
-__global__ void __launch_bounds__(kThreads) chol_update_kernel(double *__restrict__ A, int64_t K,
-                                                              int kb)
+__global__ void __launch_bounds__(kTileThreads) chol_update_kernel(double *__restrict__ A,
+                                                                  int64_t K, int kb)
 {
     double *p1 = gptq_smem, *p2 = gptq_smem + kT * kLd;
     int64_t b = blockIdx.x, jb = 0;
@@ -315,19 +320,20 @@ __global__ void __launch_bounds__(kThreads) chol_update_kernel(double *__restric
     }
     const int64_t ib = b;
     const int64_t oc = static_cast<int64_t>(kb) * kT;
-    load_tile(p1, A, K, ib * kT, oc);
-    load_tile(p2, A, K, jb * kT, oc);
+    prefetch_tile_l2(A, K, ib * kT, jb * kT);
+    load_tile<kTileThreads>(p1, A, K, ib * kT, oc);
+    load_tile<kTileThreads>(p2, A, K, jb * kT, oc);
     cp_async_wait_all();
     __syncthreads();
-    double acc[4][4];
-    zero_acc(acc);
-    mm_abt(p1, p2, acc);
+    double acc[8][4];
+    zero_acc84(acc);
+    mm84<true>(p1, p2, acc);
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int64_t r = ib * kT + ty + 16 * i, c = jb * kT + tx + 16 * j;
+            const int64_t r = ib * kT + ty + 8 * i, c = jb * kT + tx + 16 * j;
             A[r * K + c] -= acc[i][j];
         }
 }
@@ -368,49 +374,50 @@ __global__ void __launch_bounds__(kT) trtri_diag_kernel(const double *__restrict
 // the running sums T (zero to begin with); once block row k is final (trtri_final_kernel),
 // trtri_update_kernel adds V[i][k] U[k][j] into T[i][j] for every i < k <= j, one product per
 // CTA, so each T[i][j] receives its terms in the fixed order k = j, j-1, .., i+1.
-__global__ void __launch_bounds__(kThreads) trtri_update_kernel(const double *__restrict__ V,
-                                                               double *__restrict__ U, int64_t K,
-                                                               int k)
+__global__ void __launch_bounds__(kTileThreads) trtri_update_kernel(const double *__restrict__ V,
+                                                                   double *__restrict__ U,
+                                                                   int64_t K, int k)
 {
     double *sa = gptq_smem, *sb = gptq_smem + kT * kLd;
     const int64_t nb = K / kT;
     const int64_t i = blockIdx.x % k, j = k + blockIdx.x / k; // i < k <= j < nb
     if (j >= nb)
         return;
-    load_tile(sa, V, K, i * kT, k * kT);
-    load_tile(sb, U, K, k * kT, j * kT);
+    prefetch_tile_l2(U, K, i * kT, j * kT);
+    load_tile<kTileThreads>(sa, V, K, i * kT, k * kT);
+    load_tile<kTileThreads>(sb, U, K, k * kT, j * kT);
     cp_async_wait_all();
     __syncthreads();
-    double acc[4][4];
-    zero_acc(acc);
-    mm_ab(sa, sb, acc);
+    double acc[8][4];
+    zero_acc84(acc);
+    mm84<false>(sa, sb, acc);
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-            U[(i * kT + ty + 16 * a) * K + j * kT + tx + 16 * b] += acc[a][b];
+            U[(i * kT + ty + 8 * a) * K + j * kT + tx + 16 * b] += acc[a][b];
 }
 
 // Block row k final: U[k][j] = -U_kk T[k][j] for every j > k (one CTA per j).
-__global__ void __launch_bounds__(kThreads) trtri_final_kernel(double *__restrict__ U, int64_t K,
-                                                              int k)
+__global__ void __launch_bounds__(kTileThreads) trtri_final_kernel(double *__restrict__ U,
+                                                                  int64_t K, int k)
 {
     double *sa = gptq_smem, *sb = gptq_smem + kT * kLd;
     const int64_t j = k + 1 + blockIdx.x;
-    load_tile(sa, U, K, static_cast<int64_t>(k) * kT, static_cast<int64_t>(k) * kT);
-    load_tile(sb, U, K, static_cast<int64_t>(k) * kT, j * kT);
+    load_tile<kTileThreads>(sa, U, K, static_cast<int64_t>(k) * kT, static_cast<int64_t>(k) * kT);
+    load_tile<kTileThreads>(sb, U, K, static_cast<int64_t>(k) * kT, j * kT);
     cp_async_wait_all();
     __syncthreads();
-    double acc[4][4];
-    zero_acc(acc);
-    mm_ab(sa, sb, acc);
+    double acc[8][4];
+    zero_acc84(acc);
+    mm84<false>(sa, sb, acc);
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b)
-            U[(static_cast<int64_t>(k) * kT + ty + 16 * a) * K + j * kT + tx + 16 * b] = -acc[a][b];
+            U[(static_cast<int64_t>(k) * kT + ty + 8 * a) * K + j * kT + tx + 16 * b] = -acc[a][b];
 }
 
 // Lower off-diagonal blocks of U are zero (U is returned whole to callers that ask for it).

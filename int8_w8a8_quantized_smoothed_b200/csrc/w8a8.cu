@@ -1197,7 +1197,7 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
         g::chol_diag_kernel<<<1, g::kThreads, 0, st>>>(A, K, kb, bad);
         if (kb > 0) {
             g::chol_panel_kernel<<<kb, g::kThreads, g::kThreeTileBytes, st>>>(A, K, kb);
-            g::chol_update_kernel<<<kb * (kb + 1) / 2, g::kThreads, sm2, st>>>(A, K, kb);
+            g::chol_update_kernel<<<kb * (kb + 1) / 2, g::kTileThreads, sm2, st>>>(A, K, kb);
         }
     }
     // U's off-diagonal blocks start as zero running sums
@@ -1207,11 +1207,11 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     for (int k = nb - 1; k >= 1; --k) {
         // block row k is final from here on (row nb-1 is its diagonal block only)
         if (k < nb - 1)
-            g::trtri_final_kernel<<<nb - 1 - k, g::kThreads, sm2, st>>>(U, K, k);
-        g::trtri_update_kernel<<<k * (nb - k), g::kThreads, sm2, st>>>(A, U, K, k);
+            g::trtri_final_kernel<<<nb - 1 - k, g::kTileThreads, sm2, st>>>(U, K, k);
+        g::trtri_update_kernel<<<k * (nb - k), g::kTileThreads, sm2, st>>>(A, U, K, k);
     }
     if (nb > 1)
-        g::trtri_final_kernel<<<nb - 1, g::kThreads, sm2, st>>>(U, K, 0);
+        g::trtri_final_kernel<<<nb - 1, g::kTileThreads, sm2, st>>>(U, K, 0);
     const unsigned rows_grid =
         static_cast<unsigned>(std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(sms) * 8));
     g::prep_kernel<<<rows_grid, g::kThreads, 0, st>>>(w, smooth, dead, N, K, wd, s_ch);
