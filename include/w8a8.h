@@ -395,9 +395,10 @@ W8A8_API int w8a8_probe_f64_fma(long long iters, int ctas, double *out, w8a8_str
  *      the stream is still running; it waits for that kernel to complete before it reads
  *      any input or writes any output.
  *   2: as 1, and the GEMMs also start streaming their int8 weights (wq) before that wait,
- *      so a GEMM's weight traffic overlaps the tail of the kernels before it. Only valid
- *      when no kernel enqueued on the stream since its last completed synchronization
- *      writes wq -- e.g. weights prepared once and synchronized before serving.
+ *      so a GEMM's weight traffic overlaps the tail of the kernels before it; likewise the
+ *      smoothed RMSNorm reads gamma_smoothed before it. Only valid when no kernel enqueued
+ *      on the stream since its last completed synchronization writes wq or gamma_smoothed
+ *      -- e.g. weights prepared once and synchronized before serving.
  * Returns the previous mode, or W8A8_ERR_INVALID_ARG for another value. Applies to launches
  * made after the call (a captured CUDA graph keeps the mode it was captured with).
  */

@@ -414,7 +414,7 @@ template <int NCH, bool RES, bool F8 = false>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsnorm_quant_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ res, uint16_t *__restrict__ h_out,
     const float *__restrict__ gamma, float eps, int K, int M, int8_t *__restrict__ q,
-    float *__restrict__ s_tok)
+    float *__restrict__ s_tok, bool gamma_early)
 {
     // the sum's and the max's buffers alternate, so each is rewritten only after the other's
     // barrier: two barriers per row
@@ -422,25 +422,41 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsno
     __shared__ float shf[32];
     if (threadIdx.x == 0)
         pdl_launch_dependents();
-    pdl_wait(); // every input may come from the previous kernel
     const int nvec = K >> 3;
-    // gamma' of this thread's vectors, the same for every row: for short rows read once,
-    // together with the first row (its latency then overlaps the row's), and kept in
-    // registers; for long rows re-read per row
+    // gamma' of this thread's vectors, the same for every row: for short rows read once and
+    // kept in registers, for long rows re-read per row. gamma_early (overlap mode 2: no
+    // kernel still in flight writes gamma') reads it, or brings it into L2, before the
+    // dependency wait; otherwise it is read together with the first row, so its latency
+    // overlaps the row's.
     constexpr bool kKeepGamma = NCH <= 2;
     float gk[kKeepGamma ? NCH : 1][8];
-    if constexpr (kKeepGamma) {
+    auto read_gamma = [&]() {
+        if constexpr (kKeepGamma) {
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            const int vi = c * blockDim.x + threadIdx.x;
-            const float4 a = vi < nvec ? __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 b = vi < nvec ? __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi + 1)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-            gk[c][0] = a.x; gk[c][1] = a.y; gk[c][2] = a.z; gk[c][3] = a.w;
-            gk[c][4] = b.x; gk[c][5] = b.y; gk[c][6] = b.z; gk[c][7] = b.w;
+            for (int c = 0; c < NCH; ++c) {
+                const int vi = c * blockDim.x + threadIdx.x;
+                const float4 a = vi < nvec ? __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 b = vi < nvec
+                                     ? __ldg(reinterpret_cast<const float4 *>(gamma) + 2 * vi + 1)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                gk[c][0] = a.x; gk[c][1] = a.y; gk[c][2] = a.z; gk[c][3] = a.w;
+                gk[c][4] = b.x; gk[c][5] = b.y; gk[c][6] = b.z; gk[c][7] = b.w;
+            }
+        }
+    };
+    if (gamma_early) {
+        if constexpr (kKeepGamma) {
+            read_gamma();
+        } else {
+            // one 128-byte line (32 values) per 4 vectors of gamma'
+            for (int l = threadIdx.x; l < (nvec + 3) / 4; l += blockDim.x)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(gamma + 32 * l));
         }
     }
+    pdl_wait(); // every other input may come from the previous kernel
+    if (!gamma_early)
+        read_gamma();
     int64_t row = blockIdx.x;
     for (; row < M; row += gridDim.x) {
         uint4 rx[NCH], rr[RES ? NCH : 1];

@@ -251,8 +251,10 @@ int launch_rmsnorm_t(const uint16_t *x, const uint16_t *r, uint16_t *h, const fl
     const void *fn = reinterpret_cast<const void *>(&rmsnorm_quant_kernel<NCH, RES, F8>);
     if (int rc = ensure_smem(fn, dev, 0))
         return rc;
+    const bool gamma_early = g_overlap.load(std::memory_order_relaxed) >= 2;
     return launch_kernel(rmsnorm_quant_kernel<NCH, RES, F8>, dim3(row_grid(fn, threads, M, dev, sms)),
-                         dim3(threads), 0, st, x, r, h, g, eps, K, static_cast<int>(M), q, s);
+                         dim3(threads), 0, st, x, r, h, g, eps, K, static_cast<int>(M), q, s,
+                         gamma_early);
 }
 
 template <int NCH, bool F8>
