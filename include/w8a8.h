@@ -352,14 +352,15 @@ W8A8_API int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const 
  *   U       = the upper Cholesky factor of H^-1 (H^-1 = U^T U)
  *   for j = 0 .. K-1, every row n:  q = clamp(rint(W'[n,j] / s_ch[n]), -127, 127),
  *             e = (W'[n,j] - q s_ch[n]) / U[j][j],  W'[n,k] -= e U[j][k] for k > j
- * The column updates are applied in blocks of 64 (the lazy-batch form), so the binary64 sums
- * run in another order than the column-by-column statement; a code can differ from that
+ * The column updates are applied in blocks of 64 and groups of four blocks (the lazy-batch
+ * form), so the binary64 sums run in another order than the column-by-column statement; a code can differ from that
  * statement's only where W'/s lies within rounding distance of a half-integer.
  * w: bf16 [N,K] (nn.Linear layout). smooth: fp32 [K] or NULL (SmoothQuant factors s_j).
  * x_cal: fp32 [T,K], the layer's calibration inputs as the layer receives them (X diag(1/s)).
- * damp > 0 (0.01 is GPTQ's usual value). wq: int8 [N,K]; s_ch: fp32 [N]. u_out: fp64 [K,K]
- * or NULL (U, for checking). workspace: w8a8_gptq_workspace_size(N, K) bytes, 256-byte
- * aligned, any contents. Requires K % 64 == 0, 64 <= K <= 32768, N >= 1, T >= 1.
+ * damp > 0 (0.01 is GPTQ's usual value). wq: int8 [N,K], 16-byte aligned; s_ch: fp32 [N].
+ * u_out: fp64 [K,K] or NULL (U, for checking), 8-byte aligned. workspace:
+ * w8a8_gptq_workspace_size(N, K) bytes, 256-byte aligned, any contents (W8A8_ERR_ALIGNMENT
+ * otherwise). Requires K % 64 == 0, 64 <= K <= 32768, N >= 1, T >= 1.
  * Unlike the rest of the library this call SYNCHRONIZES `stream` at its end (offline
  * preparation): it returns W8A8_ERR_NUMERIC when H is not positive definite in binary64 (not
  * possible with damp > 0 in exact arithmetic).

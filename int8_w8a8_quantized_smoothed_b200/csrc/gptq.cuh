@@ -11,7 +11,7 @@
 //   inverse      U = V^-1 (upper): diagonal blocks inverted, then the off-diagonal blocks
 //                right-looking from the bottom block row (every finished block row adds its
 //                contributions to all pending blocks at once)
-//   quantize     64-column blocks in order: one warp per row runs the block's columns
+//   quantize     64-column blocks in order: one thread per row runs the block's columns
 //                sequentially (quantize, error, compensate inside the block); the lazy
 //                batch form applies the errors later, in two levels: each block's errors
 //                go at once to the rest of its group of four blocks, and a group's 256
@@ -463,85 +463,73 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const uint16_t *__restri
     }
 }
 
-// Column block jb (columns j0 .. j0 + 63), one warp per pair of rows, lane l holding columns
-// l and l + 32 of both: for each column j in order the lane that holds it rounds w_j / s,
-// forms the error e = (w_j - q s) / U[j][j] and broadcasts it; every lane subtracts e U[j][k]
-// from its columns of the block (a lane whose column is already quantized updates a value
-// that is never read again, so the update needs no predicate). Every lane forms the code and
-// error of its own column and the pivot lane's pair is selected, so the loop has no branch
-// and the two rows' dependency chains interleave (they share the loads of U); the column
-// loop is unrolled, so which lane pivots is a compile-time constant. A zero scale has a zero
-// reciprocal, so its codes are 0. Codes go to wq, errors to err[n * err_ld + t] (t = 0..63)
-// for the update kernel.
-constexpr int kQuantRows = 2; // rows per warp in flight
-
-__global__ void __launch_bounds__(kThreads) quant_block_kernel(double *__restrict__ wd,
-                                                              const double *__restrict__ U,
-                                                              const float *__restrict__ s_ch,
-                                                              int64_t N, int64_t K, int jb,
-                                                              int8_t *__restrict__ wq,
-                                                              double *__restrict__ err,
-                                                              int64_t err_ld)
+// Column block jb (columns j0 .. j0 + 63), one thread per weight row with the row's 64
+// block columns in registers: for each column j in order it rounds w_j / s, forms the error
+// e = (w_j - q s) / U[j][j] and subtracts e U[j][k] from its columns k > j (U's rows are
+// shared-memory broadcasts: every thread of a warp reads the same word). The loops are
+// unrolled, so every register index is a compile-time constant; nothing crosses lanes, so the
+// only serial chain is one row's own column steps. A zero scale has a zero reciprocal, so its
+// codes are 0. Each error replaces its dead column value, so the row's 64 errors go to
+// err[n * err_ld + t] (t = 0..63) as vector stores, and its 64 codes to wq as four 16-byte
+// stores.
+__global__ void __launch_bounds__(128) quant_block_kernel(double *__restrict__ wd,
+                                                         const double *__restrict__ U,
+                                                         const float *__restrict__ s_ch,
+                                                         int64_t N, int64_t K, int jb,
+                                                         int8_t *__restrict__ wq,
+                                                         double *__restrict__ err,
+                                                         int64_t err_ld)
 {
-    constexpr int R = kQuantRows;
-    __shared__ double u[kT * kLd];
+    __shared__ __align__(16) double u[kT * kT]; // the diagonal block of U, unpadded
+    __shared__ double uinv[kT];                 // 1 / U[j][j]
     const int64_t j0 = static_cast<int64_t>(jb) * kT;
-    load_tile(u, U, K, j0, j0);
+    for (int e = threadIdx.x; e < kT * (kT / 2); e += blockDim.x) {
+        const int r = e >> 5, c = (e & 31) * 2;
+        cp_async16(u + r * kT + c, U + (j0 + r) * K + j0 + c);
+    }
     cp_async_wait_all();
     __syncthreads();
-    const int lane = threadIdx.x & 31;
-    const double uinv0 = 1.0 / u[lane * kLd + lane];
-    const double uinv1 = 1.0 / u[(lane + 32) * kLd + lane + 32];
-    const int64_t step = static_cast<int64_t>(gridDim.x) * (kThreads / 32) * R;
-    for (int64_t n0 = (static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5)) * R;
-         n0 < N; n0 += step) {
-        double s[R], sinv[R], w0[R], w1[R], q0[R], q1[R], e0[R], e1[R];
+    for (int t = threadIdx.x; t < kT; t += blockDim.x)
+        uinv[t] = 1.0 / u[t * kT + t];
+    __syncthreads();
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; n < N;
+         n += stride) {
+        double w[kT];
+        const double2 *src = reinterpret_cast<const double2 *>(wd + n * K + j0);
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t n = n0 + r < N ? n0 + r : N - 1; // a duplicate row is not stored
-            s[r] = static_cast<double>(s_ch[n]);
-            sinv[r] = s[r] > 0.0 ? 1.0 / s[r] : 0.0;
-            w0[r] = wd[n * K + j0 + lane];
-            w1[r] = wd[n * K + j0 + 32 + lane];
-            q0[r] = q1[r] = e0[r] = e1[r] = 0.0;
+        for (int i = 0; i < kT / 2; ++i) {
+            const double2 v = src[i];
+            w[2 * i] = v.x;
+            w[2 * i + 1] = v.y;
         }
+        const double s = static_cast<double>(s_ch[n]);
+        const double sinv = s > 0.0 ? 1.0 / s : 0.0;
+        uint32_t qp[kT / 4];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const double ua = u[j * kLd + lane], ub = u[j * kLd + 32 + lane];
+        for (int i = 0; i < kT / 4; ++i)
+            qp[i] = 0u;
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const double qc = fmin(fmax(rint(w0[r] * sinv[r]), -127.0), 127.0);
-                const double ec = (w0[r] - qc * s[r]) * uinv0;
-                q0[r] = lane == j ? qc : q0[r];
-                e0[r] = lane == j ? ec : e0[r];
-                const double e = __shfl_sync(0xffffffffu, ec, j);
-                w0[r] -= e * ua;
-                w1[r] -= e * ub;
-            }
+        for (int j = 0; j < kT; ++j) {
+            const double q = fmin(fmax(rint(w[j] * sinv), -127.0), 127.0);
+            const double e = (w[j] - q * s) * uinv[j];
+            qp[j >> 2] |= (static_cast<uint32_t>(static_cast<int>(q)) & 0xffu) << (8 * (j & 3));
+#pragma unroll
+            for (int k = 0; k < kT; ++k)
+                if (k > j)
+                    w[k] -= e * u[j * kT + k];
+            w[j] = e;
+            // keeps the next step's loads of U out of this one (register pressure)
+            asm volatile("" ::: "memory");
         }
+        double2 *eo = reinterpret_cast<double2 *>(err + n * err_ld);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const double ub = u[(32 + j) * kLd + 32 + lane];
+        for (int i = 0; i < kT / 2; ++i)
+            eo[i] = make_double2(w[2 * i], w[2 * i + 1]);
+        uint4 *qo = reinterpret_cast<uint4 *>(wq + n * K + j0);
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const double qc = fmin(fmax(rint(w1[r] * sinv[r]), -127.0), 127.0);
-                const double ec = (w1[r] - qc * s[r]) * uinv1;
-                q1[r] = lane == j ? qc : q1[r];
-                e1[r] = lane == j ? ec : e1[r];
-                const double e = __shfl_sync(0xffffffffu, ec, j);
-                w1[r] -= e * ub;
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t n = n0 + r;
-            if (n < N) {
-                wq[n * K + j0 + lane] = static_cast<int8_t>(static_cast<int>(q0[r]));
-                wq[n * K + j0 + 32 + lane] = static_cast<int8_t>(static_cast<int>(q1[r]));
-                err[n * err_ld + lane] = e0[r];
-                err[n * err_ld + 32 + lane] = e1[r];
-            }
-        }
+        for (int i = 0; i < kT / 16; ++i)
+            qo[i] = make_uint4(qp[4 * i], qp[4 * i + 1], qp[4 * i + 2], qp[4 * i + 3]);
     }
 }
 

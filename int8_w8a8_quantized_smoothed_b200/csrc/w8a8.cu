@@ -1163,7 +1163,7 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     if (!workspace || workspace_bytes < L.total)
         return W8A8_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0 ||
-        reinterpret_cast<uintptr_t>(u_out) % 8 != 0)
+        reinterpret_cast<uintptr_t>(u_out) % 8 != 0 || reinterpret_cast<uintptr_t>(wq) % 16 != 0)
         return W8A8_ERR_ALIGNMENT;
     int dev, sms;
     int rc = current_device(&dev, &sms);
@@ -1221,23 +1221,18 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     // group's later blocks at once; the group's errors then reach every later column in one
     // pass over the working weight
     const unsigned row_tiles = static_cast<unsigned>((N + g::kRT - 1) / g::kRT);
-    // one wave of the quantize kernel (8 warps of kQuantRows rows per CTA)
-    int quant_per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &quant_per_sm, g::quant_block_kernel, g::kThreads, 0) != cudaSuccess ||
-        quant_per_sm < 1)
-        return W8A8_ERR_CUDA;
-    const int64_t quant_rows = static_cast<int64_t>(g::kThreads / 32) * g::kQuantRows;
-    const unsigned quant_grid = static_cast<unsigned>(std::min<int64_t>(
-        (N + quant_rows - 1) / quant_rows, static_cast<int64_t>(sms) * quant_per_sm));
+    // the quantize kernel: one thread per row, CTAs of 32..128 threads spread over the SMs
+    const int quant_threads = static_cast<int>(
+        std::min<int64_t>(128, std::max<int64_t>(32, ((N + sms - 1) / sms + 31) / 32 * 32)));
+    const unsigned quant_grid = static_cast<unsigned>((N + quant_threads - 1) / quant_threads);
     const int64_t eld = static_cast<int64_t>(g::kT) * kGptqGroup;
     const int ub = g::kUpdateBytes;
     for (int b0 = 0; b0 < nb; b0 += kGptqGroup) {
         const int b1 = std::min(nb, b0 + kGptqGroup);
         for (int jb = b0; jb < b1; ++jb) {
             double *ej = err + static_cast<int64_t>(jb - b0) * g::kT;
-            g::quant_block_kernel<<<quant_grid, g::kThreads, 0, st>>>(wd, U, s_ch, N, K, jb, wq,
-                                                                       ej, eld);
+            g::quant_block_kernel<<<quant_grid, quant_threads, 0, st>>>(wd, U, s_ch, N, K, jb,
+                                                                         wq, ej, eld);
             if (jb + 1 < b1)
                 g::update_kernel<<<dim3(b1 - 1 - jb, row_tiles), g::kThreads, ub, st>>>(
                     wd, U, ej, eld, N, K, static_cast<int64_t>(jb) * g::kT, 1,

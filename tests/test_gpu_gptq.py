@@ -114,3 +114,7 @@ def test_gptq_argument_checks():
     x = torch.zeros((4, 128), dtype=torch.float32, device="cuda")
     with pytest.raises(w8.W8A8Error, match="INVALID"):
         w8.w8a8_gptq_quantize(w, x, damp=0.0)
+    # the codes are stored 16 bytes at a time: a misaligned wq is refused before any launch
+    buf = torch.empty(8 * 128 + 16, dtype=torch.int8, device="cuda")
+    with pytest.raises(w8.W8A8Error, match="ALIGNMENT"):
+        w8.w8a8_gptq_quantize(w, x, wq=buf[1:1 + 8 * 128].view(8, 128))
