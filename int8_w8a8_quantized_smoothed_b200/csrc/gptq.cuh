@@ -31,9 +31,8 @@ namespace gptq {
 constexpr int kT = 64;    // tile / column-block size
 constexpr int kLd = 65;   // padded shared-memory row (doubles)
 constexpr int kThreads = 256;
-// dynamic shared memory of the two- and three-tile kernels
+// dynamic shared memory of the two-tile kernels
 constexpr int kTwoTileBytes = 2 * kT * kLd * 8;
-constexpr int kThreeTileBytes = 3 * kT * kLd * 8;
 
 extern __shared__ __align__(16) double gptq_smem[];
 
@@ -268,43 +267,44 @@ __global__ void __launch_bounds__(kThreads) chol_diag_kernel(double *__restrict_
 
 // Panel of block column kb: V[ib][kb] = A[ib][kb] V_kk^-T for every ib < kb (one CTA each):
 // X V_kk^T = A solved from the last column: x_j = a_j / V[j][j], then a_k -= x_j V[k][j]
-// for k < j. One barrier per column: x_j goes to its own tile, every thread that needs it
-// scales a_j itself.
-__global__ void __launch_bounds__(kThreads) chol_panel_kernel(double *__restrict__ A, int64_t K,
-                                                             int kb)
+// for k < j. The rows are independent: one thread per row holds its 64 values in registers
+// (loops unrolled, constant register indices) and reads V's column j as a shared-memory
+// broadcast, so the column loop needs no barrier; a compiler barrier per column keeps the
+// next column's loads of V from being hoisted (register pressure).
+__global__ void __launch_bounds__(kT) chol_panel_kernel(double *__restrict__ A, int64_t K, int kb)
 {
-    double *a = gptq_smem, *v = gptq_smem + kT * kLd, *x = gptq_smem + 2 * kT * kLd;
+    __shared__ __align__(16) double v[kT * kT]; // V_kk, unpadded
+    __shared__ double vinv[kT];                 // 1 / V[j][j]
     const int64_t oc = static_cast<int64_t>(kb) * kT, orow = static_cast<int64_t>(blockIdx.x) * kT;
-    __shared__ double vinv[kT]; // 1 / V[j][j]
-    load_tile(a, A, K, orow, oc);
-    load_tile(v, A, K, oc, oc);
+    for (int e = threadIdx.x; e < kT * (kT / 2); e += kT) {
+        const int r = e >> 5, c = (e & 31) * 2;
+        cp_async16(v + r * kT + c, A + (oc + r) * K + oc + c);
+    }
     cp_async_wait_all();
     __syncthreads();
-    if (threadIdx.x < kT)
-        vinv[threadIdx.x] = 1.0 / v[threadIdx.x * kLd + threadIdx.x];
+    vinv[threadIdx.x] = 1.0 / v[threadIdx.x * kT + threadIdx.x];
     __syncthreads();
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double a[kT];
+    double2 *row = reinterpret_cast<double2 *>(A + (orow + threadIdx.x) * K + oc);
+#pragma unroll
+    for (int i = 0; i < kT / 2; ++i) {
+        const double2 t = row[i];
+        a[2 * i] = t.x;
+        a[2 * i + 1] = t.y;
+    }
+#pragma unroll
     for (int j = kT - 1; j >= 0; --j) {
-        const double vi = vinv[j];
+        const double x = a[j] * vinv[j];
+        a[j] = x;
 #pragma unroll
-        for (int aa = 0; aa < 4; ++aa) {
-            const int r = ty + 16 * aa;
-            const double xr = a[r * kLd + j] * vi;
-            if (tx == 0)
-                x[r * kLd + j] = xr;
+        for (int k = 0; k < kT; ++k)
+            if (k < j)
+                a[k] -= x * v[k * kT + j];
+        asm volatile("" ::: "memory");
+    }
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int k = tx + 16 * b;
-                if (k < j)
-                    a[r * kLd + k] -= xr * v[k * kLd + j];
-            }
-        }
-        __syncthreads();
-    }
-    for (int e = threadIdx.x; e < kT * kT; e += kThreads) {
-        const int r = e >> 6, c = e & 63;
-        A[(orow + r) * K + oc + c] = x[r * kLd + c];
-    }
+    for (int i = 0; i < kT / 2; ++i)
+        row[i] = make_double2(a[2 * i], a[2 * i + 1]);
 }
 
 // Trailing update after block column kb: A[ib][jb] -= V[ib][kb] V[jb][kb]^T for

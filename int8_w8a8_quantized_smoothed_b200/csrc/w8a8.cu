@@ -1179,9 +1179,6 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     int *bad = reinterpret_cast<int *>(base + L.b_off);
     const int nb = static_cast<int>(K / g::kT);
     const int sm2 = g::kTwoTileBytes;
-    if ((rc = ensure_smem(reinterpret_cast<const void *>(&g::chol_panel_kernel), dev,
-                          g::kThreeTileBytes)))
-        return rc;
     for (const void *fn : {reinterpret_cast<const void *>(&g::chol_update_kernel),
                            reinterpret_cast<const void *>(&g::trtri_diag_kernel),
                            reinterpret_cast<const void *>(&g::trtri_update_kernel),
@@ -1198,7 +1195,7 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     for (int kb = nb - 1; kb >= 0; --kb) {
         g::chol_diag_kernel<<<1, g::kThreads, 0, st>>>(A, K, kb, bad);
         if (kb > 0) {
-            g::chol_panel_kernel<<<kb, g::kThreads, g::kThreeTileBytes, st>>>(A, K, kb);
+            g::chol_panel_kernel<<<kb, g::kT, 0, st>>>(A, K, kb);
             g::chol_update_kernel<<<kb * (kb + 1) / 2, g::kTileThreads, sm2, st>>>(A, K, kb);
         }
     }
