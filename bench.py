@@ -571,10 +571,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": ("e4m3xe4m3->f32, fp32 scales, bf16 io" if args.fp8 else
                   "i8xi8->i32, fp32 scales, bf16 io"), "data": "synthetic",
-        "config": {"workload": f"{wl['desc']}, M in {wl['Ms']}: one decoder block's linear "
-                               f"path per M on its own layer's weights",
-                   "tokens": wl["Ms"], "hidden": arch["H"], "intermediate": arch["I"],
-                   "qkv_out": arch["QKV"], "alpha": ALPHA, "parallelism": f"replicas x{world}",
+        "config": {**workload_config(wl, arch), "parallelism": f"replicas x{world}",
                    "l2": "no flush: each step streams "
                          f"{sum(L.w[n][0].numel() for L in layers for n in L.w) / 1e6:.0f} MB "
                          "of int8 weights (> 126 MB L2)",
@@ -658,6 +655,14 @@ def cpu_baseline(arch, M=64, min_seconds=10.0):
                       f"threads of {os.cpu_count()} host cores"}
 
 
+def workload_config(wl, arch):
+    """The workload's description, the same in both arms' JSON lines."""
+    return {"workload": f"{wl['desc']}, M in {wl['Ms']}: one decoder block's linear path per M "
+                        f"on its own layer's weights",
+            "tokens": wl["Ms"], "hidden": arch["H"], "intermediate": arch["I"],
+            "qkv_out": arch["QKV"], "alpha": ALPHA}
+
+
 def run_reference(args, world, rank):
     """Reference arm: the CPU oracle timed on the host cores, each step a bounded sample
     (the M=1 block linear path of the workload's architecture)."""
@@ -685,8 +690,9 @@ def run_reference(args, world, rank):
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8xi8->i32, fp32 scales, bf16 io",
         "data": "synthetic",
-        "config": {"workload": f"{wl['desc']} (bounded CPU sample, M=1 per step)",
-                   "parallelism": "host cores"},
+        "config": {**workload_config(wl, arch), "parallelism": "host cores",
+                   "codes": "INT8 (scale absmax / 127)",
+                   "sample": f"each step: the M={M} member of the set through the CPU oracle"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": min(nth, M),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
