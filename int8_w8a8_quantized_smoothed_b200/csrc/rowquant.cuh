@@ -285,8 +285,9 @@ __device__ __forceinline__ void load_row(const uint4 *__restrict__ xr, int nvec,
 //
 // Rows of up to 4096 values run with at most 256 threads (NCH <= 2); those kernels are
 // compiled for several resident CTAs per SM (at most 40 registers for quantize_rows and
-// SiLU, 64 for RMSNorm, which keeps gamma' in registers), since with so little work per
-// thread the arithmetic and the reductions' latency, not HBM, set their pace.
+// SiLU, 85 for RMSNorm, which keeps gamma' in registers and loads the next row while it
+// reduces the current one), since with so little work per thread the arithmetic and the
+// reductions' latency, not HBM, set their pace.
 
 template <int NCH, bool F8 = false>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quantize_rows_kernel(const uint16_t *__restrict__ x,
@@ -411,7 +412,7 @@ __global__ void __launch_bounds__(256) quantize_rows_static_kernel(
 // ----------------------------------------------------------------- smoothed RMSNorm + quant
 
 template <int NCH, bool RES, bool F8 = false>
-__global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsnorm_quant_kernel(
+__global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 3 : 1) rmsnorm_quant_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ res, uint16_t *__restrict__ h_out,
     const float *__restrict__ gamma, float eps, int K, int M, int8_t *__restrict__ q,
     float *__restrict__ s_tok, bool gamma_early)
@@ -458,11 +459,37 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 4 : 1) rmsno
     if (!gamma_early)
         read_gamma();
     int64_t row = blockIdx.x;
+    // short rows: the next row's loads are issued before this row's reductions, so each CTA
+    // keeps a row in flight while it works on another
+    constexpr bool kPre = NCH <= 2;
+    uint4 nx[kPre ? NCH : 1], nr[kPre && RES ? NCH : 1];
+    if constexpr (kPre) {
+        if (row < M) {
+            load_row<NCH>(reinterpret_cast<const uint4 *>(x + row * K), nvec, nx);
+            if constexpr (RES)
+                load_row<NCH>(reinterpret_cast<const uint4 *>(res + row * K), nvec, nr);
+        }
+    }
     for (; row < M; row += gridDim.x) {
         uint4 rx[NCH], rr[RES ? NCH : 1];
-        load_row<NCH>(reinterpret_cast<const uint4 *>(x + row * K), nvec, rx);
-        if constexpr (RES)
-            load_row<NCH>(reinterpret_cast<const uint4 *>(res + row * K), nvec, rr);
+        if constexpr (kPre) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                rx[c] = nx[c];
+                if constexpr (RES)
+                    rr[c] = nr[c];
+            }
+            const int64_t next = row + gridDim.x;
+            if (next < M) {
+                load_row<NCH>(reinterpret_cast<const uint4 *>(x + next * K), nvec, nx);
+                if constexpr (RES)
+                    load_row<NCH>(reinterpret_cast<const uint4 *>(res + next * K), nvec, nr);
+            }
+        } else {
+            load_row<NCH>(reinterpret_cast<const uint4 *>(x + row * K), nvec, rx);
+            if constexpr (RES)
+                load_row<NCH>(reinterpret_cast<const uint4 *>(res + row * K), nvec, rr);
+        }
         float v[NCH][8];
         double ss = 0.0;
 #pragma unroll
