@@ -11,8 +11,9 @@
 //   inverse      U = V^-1 (upper): diagonal blocks inverted, then the off-diagonal blocks
 //                right-looking from the bottom block row (every finished block row adds its
 //                contributions to all pending blocks at once)
-//   quantize     64-column blocks in order: one thread per row runs the block's columns
-//                sequentially (quantize, error, compensate inside the block); the lazy
+//   quantize     64-column blocks in order: four lanes per row (one thread per row when
+//                the rows exceed one wave) run the block's columns sequentially
+//                (quantize, error, compensate inside the block); the lazy
 //                batch form applies the errors later, in two levels: each block's errors
 //                go at once to the rest of its group of four blocks, and a group's 256
 //                columns of errors go to every column after the group in one tiled pass
@@ -463,8 +464,86 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const uint16_t *__restri
     }
 }
 
-// Column block jb (columns j0 .. j0 + 63), one thread per weight row with the row's 64
-// block columns in registers: for each column j in order it rounds w_j / s, forms the error
+// Column block jb (columns j0 .. j0 + 63), four lanes per weight row: lane l of a quad holds
+// columns 4i + l (i = 0..15) in registers. For each column j = 4i + o in order the quad's
+// lane o rounds w_j / s and forms the error e = (w_j - q s) / U[j][j]; a quad shuffle hands e
+// to the other three, and each lane subtracts e U[j][k] from its columns k > j (U's rows
+// are read from shared memory, four distinct words per warp access). Every lane forms the
+// code and error of its own column i and lane o's are kept, so the loop has no branch; the
+// loops are unrolled, so register indices and o are compile-time constants, and a compiler
+// barrier per column keeps the next column's loads of U from being hoisted. A zero scale has
+// a zero reciprocal, so its codes are 0. Errors go to err[n * err_ld + t] (t = 0..63),
+// codes to wq. The whole warp walks its 8 rows together (shuffles need every lane); a row
+// past N repeats row N - 1 and stores nothing.
+constexpr int kQuantThreads = 128;
+
+__global__ void __launch_bounds__(kQuantThreads) quant_block_kernel(
+    double *__restrict__ wd, const double *__restrict__ U, const float *__restrict__ s_ch,
+    int64_t N, int64_t K, int jb, int8_t *__restrict__ wq, double *__restrict__ err,
+    int64_t err_ld)
+{
+    __shared__ __align__(16) double u[kT * kT]; // the diagonal block of U, unpadded
+    __shared__ double uinv[kT];                 // 1 / U[j][j]
+    const int64_t j0 = static_cast<int64_t>(jb) * kT;
+    for (int e = threadIdx.x; e < kT * (kT / 2); e += blockDim.x) {
+        const int r = e >> 5, c = (e & 31) * 2;
+        cp_async16(u + r * kT + c, U + (j0 + r) * K + j0 + c);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    for (int t = threadIdx.x; t < kT; t += blockDim.x)
+        uinv[t] = 1.0 / u[t * kT + t];
+    __syncthreads();
+    const int l = threadIdx.x & 3, lane = threadIdx.x & 31;
+    const int qbase = lane & ~3;
+    double ui[kT / 4]; // 1 / U[c][c] of this lane's columns
+#pragma unroll
+    for (int i = 0; i < kT / 4; ++i)
+        ui[i] = uinv[4 * i + l];
+    const int64_t warp = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    for (int64_t n0 = warp * 8; n0 < N; n0 += warps * 8) {
+        const int64_t n = n0 + (lane >> 2);
+        const int64_t nr = n < N ? n : N - 1;
+        double w[kT / 4];
+#pragma unroll
+        for (int i = 0; i < kT / 4; ++i)
+            w[i] = wd[nr * K + j0 + 4 * i + l];
+        const double s = static_cast<double>(s_ch[nr]);
+        const double sinv = s > 0.0 ? 1.0 / s : 0.0;
+        uint32_t qp[kT / 16];
+#pragma unroll
+        for (int i = 0; i < kT / 16; ++i)
+            qp[i] = 0u;
+#pragma unroll
+        for (int j = 0; j < kT; ++j) {
+            const int i = j >> 2, o = j & 3;
+            const double qc = fmin(fmax(rint(w[i] * sinv), -127.0), 127.0);
+            const double ec = (w[i] - qc * s) * ui[i];
+            const double e = __shfl_sync(0xffffffffu, ec, qbase | o);
+            if (l == o)
+                qp[i >> 2] |= (static_cast<uint32_t>(static_cast<int>(qc)) & 0xffu)
+                              << (8 * (i & 3));
+#pragma unroll
+            for (int ii = 0; ii < kT / 4; ++ii)
+                if (ii > i || (ii == i && l > o))
+                    w[ii] -= e * u[j * kT + 4 * ii + l];
+            if (l == o)
+                w[i] = e;
+            asm volatile("" ::: "memory");
+        }
+        if (n < N) {
+#pragma unroll
+            for (int i = 0; i < kT / 4; ++i) {
+                err[n * err_ld + 4 * i + l] = w[i];
+                wq[n * K + j0 + 4 * i + l] = static_cast<int8_t>((qp[i >> 2] >> (8 * (i & 3))) & 0xffu);
+            }
+        }
+    }
+}
+
+// Column block jb for many rows (one wave of the four-lane form does not hold them): one
+// thread per weight row with the row's 64 block columns in registers: for each column j in order it rounds w_j / s, forms the error
 // e = (w_j - q s) / U[j][j] and subtracts e U[j][k] from its columns k > j (U's rows are
 // shared-memory broadcasts: every thread of a warp reads the same word). The loops are
 // unrolled, so every register index is a compile-time constant; nothing crosses lanes, so the
@@ -472,7 +551,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const uint16_t *__restri
 // codes are 0. Each error replaces its dead column value, so the row's 64 errors go to
 // err[n * err_ld + t] (t = 0..63) as vector stores, and its 64 codes to wq as four 16-byte
 // stores.
-__global__ void __launch_bounds__(128) quant_block_kernel(double *__restrict__ wd,
+__global__ void __launch_bounds__(128) quant_block_rows_kernel(double *__restrict__ wd,
                                                          const double *__restrict__ U,
                                                          const float *__restrict__ s_ch,
                                                          int64_t N, int64_t K, int jb,

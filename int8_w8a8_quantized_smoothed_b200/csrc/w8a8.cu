@@ -1218,18 +1218,30 @@ int w8a8_gptq_quantize(const w8a8_bf16 *w, const float *smooth, const float *x_c
     // group's later blocks at once; the group's errors then reach every later column in one
     // pass over the working weight
     const unsigned row_tiles = static_cast<unsigned>((N + g::kRT - 1) / g::kRT);
-    // the quantize kernel: one thread per row, CTAs of 32..128 threads spread over the SMs
-    const int quant_threads = static_cast<int>(
+    // the quantize kernel: four lanes per row (32 rows per CTA) while one wave holds the
+    // rows; beyond that one thread per row (CTAs of 32..128 threads)
+    int quad_per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&quad_per_sm, g::quant_block_kernel,
+                                                      g::kQuantThreads, 0) != cudaSuccess)
+        return W8A8_ERR_CUDA;
+    const int64_t quad_ctas = (N + g::kQuantThreads / 4 - 1) / (g::kQuantThreads / 4);
+    const bool quad = quad_ctas <= static_cast<int64_t>(sms) * std::max(quad_per_sm, 1);
+    const int row_threads = static_cast<int>(
         std::min<int64_t>(128, std::max<int64_t>(32, ((N + sms - 1) / sms + 31) / 32 * 32)));
-    const unsigned quant_grid = static_cast<unsigned>((N + quant_threads - 1) / quant_threads);
+    const unsigned quant_grid = static_cast<unsigned>(
+        quad ? quad_ctas : (N + row_threads - 1) / row_threads);
     const int64_t eld = static_cast<int64_t>(g::kT) * kGptqGroup;
     const int ub = g::kUpdateBytes;
     for (int b0 = 0; b0 < nb; b0 += kGptqGroup) {
         const int b1 = std::min(nb, b0 + kGptqGroup);
         for (int jb = b0; jb < b1; ++jb) {
             double *ej = err + static_cast<int64_t>(jb - b0) * g::kT;
-            g::quant_block_kernel<<<quant_grid, quant_threads, 0, st>>>(wd, U, s_ch, N, K, jb,
-                                                                         wq, ej, eld);
+            if (quad)
+                g::quant_block_kernel<<<quant_grid, g::kQuantThreads, 0, st>>>(wd, U, s_ch, N, K,
+                                                                                jb, wq, ej, eld);
+            else
+                g::quant_block_rows_kernel<<<quant_grid, row_threads, 0, st>>>(wd, U, s_ch, N, K,
+                                                                               jb, wq, ej, eld);
             if (jb + 1 < b1)
                 g::update_kernel<<<dim3(b1 - 1 - jb, row_tiles), g::kThreads, ub, st>>>(
                     wd, U, ej, eld, N, K, static_cast<int64_t>(jb) * g::kT, 1,

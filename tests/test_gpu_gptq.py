@@ -57,7 +57,10 @@ def _follow(wf, dead, U, q, rows=None):
 @pytest.mark.parametrize("N,K,T", [(96, 256, 512), (200, 512, 256), (64, 1024, 1024),
                                    (8, 64, 16),
                                    # ragged groups of column blocks: 4 + 1 and 4 + 3 blocks
-                                   (33, 320, 128), (1, 448, 64), (130, 448, 300)])
+                                   (33, 320, 128), (1, 448, 64), (130, 448, 300),
+                                   # more rows than one wave of the four-lane quantize
+                                   # kernel holds: the one-thread-per-row kernel
+                                   (20000, 128, 64)])
 def test_gptq_matches_oracle(N, K, T):
     w, wf, x, q, sch, u = _run(N, K, T, seed=N + K)
     r = oracle.gptq(wf, x, damp=0.01)
