@@ -759,7 +759,8 @@ def run_gptq_case(args, dims):
 
 
 def run_case(args):
-    """`--case gemm:M:N:K[:variant]` (INT8), `gemm8:M:N:K[:variant]` (FP8), `rms:M:K`, `rmsres:M:K`, `quant:M:K`, `static:M:K` or
+    """`--case gemm:M:N:K[:variant[:ctas[:tile_n]]]` (INT8; ctas and tile_n as in
+    w8a8_gemm_dequant_ex), `gemm8:M:N:K[:variant[:ctas[:tile_n]]]` (FP8), `rms:M:K`, `rmsres:M:K`, `quant:M:K`, `static:M:K` or
     `silu:M:I`:
     one kernel launched repeatedly (a CUDA graph of back-to-back launches)."""
     import int8_w8a8_quantized_smoothed_b200 as w8
@@ -772,6 +773,8 @@ def run_case(args):
     if parts[0] in ("gemm", "gemm8"):
         M, N, K = (int(v) for v in parts[1:4])
         variant = int(parts[4]) if len(parts) > 4 else 0
+        ctas = int(parts[5]) if len(parts) > 5 else 0
+        tile_n = int(parts[6]) if len(parts) > 6 else 0
         fp8 = parts[0] == "gemm8"
         copies = max(1, math.ceil(4 * 126e6 / (N * K)))  # rotate weights through > 4x L2
 
@@ -790,7 +793,8 @@ def run_case(args):
         gemm = w8.w8a8_gemm_dequant_fp8 if fp8 else w8.w8a8_gemm_dequant_ex
 
         def launch(i):
-            gemm(xq, st, ws_[i % copies], sc, y=y, workspace=wsp, variant=variant)
+            gemm(xq, st, ws_[i % copies], sc, y=y, workspace=wsp, variant=variant, ctas=ctas,
+                 tile_n=tile_n)
         work = gemm_bytes(M, N, K)
         flops = 2 * M * N * K
     else:
