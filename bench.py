@@ -255,7 +255,7 @@ class Layer:
                 self.w[name] = (p["wq"], p["s_ch"])
             del wb, p
         # the gate|up weight in the row order of the fused SiLU*up epilogue
-        self.w_gu_il = None if fp8 else prep.interleave_gate_up(*self.w["gate_up"])
+        self.w_gu_il = prep.interleave_gate_up(*self.w["gate_up"])
         torch.cuda.synchronize()
         # inputs (device) and their pinned host copies for the end-to-end measurement
         self.x = synth.activation_device(M, H, seed + 20, device)
@@ -292,14 +292,14 @@ class Layer:
 
     def chain(self, ws, gemms=True, rows=True, fused=None):
         import int8_w8a8_quantized_smoothed_b200 as w8
+        fused = self.fused if fused is None else fused
         if self.fp8:
-            return self.chain_fp8(ws, gemms, rows)
+            return self.chain_fp8(ws, gemms, rows, fused)
         if self.block is not None:  # one launch for the whole block
             w8.w8a8_block_decode(self.x, self.attn, self.g1f, self.sinv_o, self.g2f,
                                  self.w["qkv"], self.w["o"], self.w_gu_il, self.w["down"], EPS,
                                  buffers=self.block)
             return
-        fused = self.fused if fused is None else fused
         if rows:
             w8.w8a8_smooth_rmsnorm_quant(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
         if gemms:
@@ -326,8 +326,8 @@ class Layer:
             w8.w8a8_gemm_dequant(self.q4, self.s4, *self.w["down"], y=self.down, workspace=ws)
 
 
-    def chain_fp8(self, ws, gemms=True, rows=True):
-        """The same block with E4M3 codes: FP8 row kernels and FP8 GEMMs (SiLU*up unfused)."""
+    def chain_fp8(self, ws, gemms=True, rows=True, fused=True):
+        """The same block with E4M3 codes: FP8 row kernels and FP8 GEMMs."""
         import int8_w8a8_quantized_smoothed_b200 as w8
         if rows:
             w8.w8a8_smooth_rmsnorm_quant_fp8(self.x, self.g1f, EPS, q=self.q1, s_tok=self.s1)
@@ -340,11 +340,16 @@ class Layer:
         if rows:
             w8.w8a8_smooth_rmsnorm_quant_fp8(self.o, self.g2f, EPS, residual=self.x,
                                              h_out=self.h, q=self.q3, s_tok=self.s3)
-        if gemms:
-            w8.w8a8_gemm_dequant_fp8(self.q3, self.s3, *self.w["gate_up"], y=self.gu,
-                                     workspace=ws)
-        if rows:
-            w8.w8a8_silu_mul_quant_fp8(self.gu, q=self.q4, s_tok=self.s4)
+        if fused:
+            if gemms:
+                w8.w8a8_gemm_silu_quant_fp8(self.q3, self.s3, *self.w_gu_il, a=self.a,
+                                            q=self.q4, s_out=self.s4, workspace=ws)
+        else:
+            if gemms:
+                w8.w8a8_gemm_dequant_fp8(self.q3, self.s3, *self.w["gate_up"], y=self.gu,
+                                         workspace=ws)
+            if rows:
+                w8.w8a8_silu_mul_quant_fp8(self.gu, q=self.q4, s_tok=self.s4)
         if gemms:
             w8.w8a8_gemm_dequant_fp8(self.q4, self.s4, *self.w["down"], y=self.down,
                                      workspace=ws)
@@ -427,7 +432,7 @@ def run_ours(args, world, rank, local):
     arch = wl["arch"]
     layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev, fp8=args.fp8,
                     block=args.fused_block) for i, M in enumerate(wl["Ms"])]
-    unfused = args.unfused or args.fp8  # the SiLU*up epilogue is INT8 only
+    unfused = args.unfused
     for L in layers:
         L.fused = not unfused
     ws = w8.Workspace(dev)
@@ -436,6 +441,8 @@ def run_ours(args, world, rank, local):
                  [w8.w8a8_gemm_fp8_workspace_size(L.M, N, K) for L in layers
                   for (N, K) in projections(arch).values()] +
                  [w8.w8a8_gemm_silu_quant_workspace_size(L.M, arch["I"], arch["H"])
+                  for L in layers] +
+                 [w8.w8a8_gemm_silu_quant_fp8_workspace_size(L.M, arch["I"], arch["H"])
                   for L in layers])
     ws.get(max_ws)
     # the weights are prepared and synchronized: from here on no kernel writes them, so the

@@ -338,6 +338,25 @@ W8A8_API int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const 
                                    w8a8_stream_t stream);
 
 /*
+ * The fused gate|up GEMM + SiLU(gate)*up + per-token quantization of w8a8_gemm_silu_quant
+ * with FP8 operands and codes: the same interleaved weight layout and arguments (xq, wq_il
+ * E4M3 codes as uint8; q: E4M3 codes [M,I] as uint8, s_out = max_i |a[m,i]| / 448). The
+ * epilogue rounds the dequantized gate and up values to bf16 exactly as w8a8_gemm_dequant_fp8
+ * stores them and continues as w8a8_silu_mul_quant_fp8, so the result is bit-identical to
+ * those two calls whenever the GEMM's binary32 accumulators are the same; that holds for the
+ * same kernel plan on the interleaved weight. The plan is the GEMM's automatic one, with
+ * stream-K in place of the cluster split-K (it has no SiLU epilogue). Workspace:
+ * w8a8_gemm_silu_quant_fp8_workspace_size(M, I, K) bytes, under w8a8_gemm_workspace_size's
+ * rules.
+ */
+W8A8_API size_t w8a8_gemm_silu_quant_fp8_workspace_size(int64_t M, int64_t I, int64_t K);
+W8A8_API int w8a8_gemm_silu_quant_fp8(const uint8_t *xq, const float *s_tok,
+                                      const uint8_t *wq_il, const float *s_ch_il, int64_t M,
+                                      int64_t I, int64_t K, float *a, uint8_t *q, float *s_out,
+                                      void *workspace, size_t workspace_bytes,
+                                      w8a8_stream_t stream);
+
+/*
  * ---------------------------------------------------------------- GPTQ weights (offline)
  *
  * GPTQ quantization of one linear layer's weight to the int8 + per-channel-scale format of

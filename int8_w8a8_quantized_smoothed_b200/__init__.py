@@ -24,7 +24,8 @@ __all__ = [
     "w8a8_get_overlap", "w8a8_device_status",
     "w8a8_status_string", "w8a8_version",
     "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
-    "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size",
+    "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size", "w8a8_gemm_silu_quant_fp8",
+    "w8a8_gemm_silu_quant_fp8_workspace_size",
     "w8a8_gptq_quantize", "w8a8_gptq_workspace_size", "w8a8_probe_f64_fma",
     "w8a8_block_decode", "w8a8_block_decode_workspace_size", "BlockBuffers",
     "Workspace", "FP8",
@@ -51,6 +52,9 @@ SIGNATURES = [
     ("w8a8_gemm_dequant_noalloc", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("w8a8_gemm_silu_quant_workspace_size", _SZ, [_I64, _I64, _I64]),
     ("w8a8_gemm_silu_quant", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    ("w8a8_gemm_silu_quant_fp8_workspace_size", _SZ, [_I64, _I64, _I64]),
+    ("w8a8_gemm_silu_quant_fp8", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ,
+                                      _P]),
     ("w8a8_probe_i8_mma", _I, [C.c_longlong, _I, _I, _P]),
     ("w8a8_selftest_wait_timeout", _I, [C.c_ulonglong, _P]),
     ("w8a8_set_overlap", _I, [_I]),
@@ -438,6 +442,44 @@ def w8a8_gemm_silu_quant(xq, s_tok, wq_il, s_ch_il, a=None, q=None, s_out=None,
         wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
                                    * workspace.element_size())
     _check("w8a8_gemm_silu_quant", lib().w8a8_gemm_silu_quant(
+        _ptr(xq), _ptr(s_tok), _ptr(wq_il), _ptr(s_ch_il), M, I, K, _ptr(a), _ptr(q),
+        _ptr(s_out), _ptr(wbuf), wbytes, _stream(stream)))
+    return q, s_out, a
+
+
+def w8a8_gemm_silu_quant_fp8_workspace_size(M: int, I: int, K: int) -> int:
+    return int(lib().w8a8_gemm_silu_quant_fp8_workspace_size(M, I, K))
+
+
+def w8a8_gemm_silu_quant_fp8(xq, s_tok, wq_il, s_ch_il, a=None, q=None, s_out=None,
+                             workspace=None, stream=None):
+    """w8a8_gemm_silu_quant with FP8 operands and codes (xq, wq_il, q as
+    torch.float8_e4m3fn; s_out = max |a| / 448). Returns (q, s_out, a)."""
+    _need(xq, "xq", FP8)
+    _need(wq_il, "wq_il", FP8)
+    M, K = xq.shape
+    N, K2 = wq_il.shape
+    if K != K2 or N % 2:
+        raise ValueError(f"xq [M,K] and wq_il [2I,K] disagree: {tuple(xq.shape)} {tuple(wq_il.shape)}")
+    I = N // 2
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _need(s_ch_il, "s_ch_il", torch.float32, (N,))
+    e = dict(device=xq.device)
+    a = torch.empty((M, I), dtype=torch.float32, **e) if a is None else a
+    q = torch.empty((M, I), dtype=FP8, **e) if q is None else q
+    s_out = torch.empty(M, dtype=torch.float32, **e) if s_out is None else s_out
+    _need(a, "a", torch.float32, (M, I))
+    _need(q, "q", FP8, (M, I))
+    _need(s_out, "s_out", torch.float32, (M,))
+    need = w8a8_gemm_silu_quant_fp8_workspace_size(M, I, K)
+    if workspace is None:
+        workspace = _workspace_for(xq.device)
+    if isinstance(workspace, Workspace):
+        wbuf, wbytes = workspace.get(need)
+    else:
+        wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
+                                   * workspace.element_size())
+    _check("w8a8_gemm_silu_quant_fp8", lib().w8a8_gemm_silu_quant_fp8(
         _ptr(xq), _ptr(s_tok), _ptr(wq_il), _ptr(s_ch_il), M, I, K, _ptr(a), _ptr(q),
         _ptr(s_out), _ptr(wbuf), wbytes, _stream(stream)))
     return q, s_out, a

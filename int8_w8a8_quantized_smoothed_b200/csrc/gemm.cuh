@@ -24,7 +24,8 @@
 // channels 64b..64b+63), so every 128-row group of weight rows holds the gate and up rows of
 // the same 64 output channels. The epilogue rounds both dequantized values to bf16 (exactly
 // what the plain epilogue stores), forms a = silu(g) * u in binary32 as the SiLU*up row
-// kernel does, and stores a; a following row pass takes each token's max |a| and quantizes.
+// kernel does, and stores a; a following row pass takes each token's max |a| and quantizes
+// (to int8, or to E4M3 for FP8 operands; the FP8 form has no cluster split-K variant).
 #pragma once
 
 #include "ptx.cuh"
@@ -52,6 +53,7 @@ __device__ __forceinline__ float bf16_round(float f)
 // One thread's row: 32 gate columns (rg, channel scales scg) and the 32 up columns of the
 // same output channels (ru, scu) -> a = silu(bf16(g)) * bf16(u), stored at dst (32 floats,
 // 16-byte stores).
+template <bool F8 = false>
 __device__ __forceinline__ void silu_row_chunk(const uint32_t (&rg)[32], const uint32_t (&ru)[32],
                                                 float st, const float *scg, const float *scu,
                                                 float *__restrict__ dst)
@@ -67,8 +69,8 @@ __device__ __forceinline__ void silu_row_chunk(const uint32_t (&rg)[32], const u
         const float cu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            g[i] = bf16_round(dequant_f32(static_cast<int32_t>(rg[8 * e + i]), st, cg[i]));
-            u[i] = bf16_round(dequant_f32(static_cast<int32_t>(ru[8 * e + i]), st, cu[i]));
+            g[i] = bf16_round(dequant_acc<F8>(rg[8 * e + i], st, cg[i]));
+            u[i] = bf16_round(dequant_acc<F8>(ru[8 * e + i], st, cu[i]));
         }
         silu_mul8(g, u, a);
         reinterpret_cast<float4 *>(dst)[2 * e] = make_float4(a[0], a[1], a[2], a[3]);
@@ -197,7 +199,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         uint16_t *__restrict__ y, int32_t *__restrict__ acc_out, SiluOut so,
                         int prefetch_static, unsigned long long limit_ns)
 {
-    static_assert(!(SILU && F8), "the fused SiLU epilogue is INT8 only");
     using Cfg = PrefillCfg<BN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
                     tmem_ld_wait();
                     if (row_ok && ch0 < so.I)
-                        silu_row_chunk(rg, ru, st, sh_sch + buf * BN + cg * 32,
+                        silu_row_chunk<F8>(rg, ru, st, sh_sch + buf * BN + cg * 32,
                                        sh_sch + buf * BN + (cg + 2) * 32,
                                        so.a + static_cast<int64_t>(row) * so.I + ch0);
                 }
@@ -418,7 +419,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              int32_t *__restrict__ acc_out, SiluOut so, int prefetch_static,
                              unsigned long long limit_ns)
 {
-    static_assert(!(SILU && F8), "the fused SiLU epilogue is INT8 only");
     using Cfg = PairCfg<STAGES>;
     constexpr int TN = 256, TM = 256;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
                     tmem_ld_wait();
                     if (row_ok && ch0 < so.I)
-                        silu_row_chunk(rg, ru, st, sh_sch + buf * TN + cg * 32,
+                        silu_row_chunk<F8>(rg, ru, st, sh_sch + buf * TN + cg * 32,
                                        sh_sch + buf * TN + (cg + 2) * 32,
                                        so.a + static_cast<int64_t>(row) * so.I + ch0);
                 }
@@ -735,7 +735,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                        int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
                        SiluOut so, int prefetch_static, unsigned long long limit_ns)
 {
-    static_assert(!(SILU && F8), "the fused SiLU epilogue is INT8 only");
+    static_assert(!(SILU && F8 && CLUSTER), "the fused SiLU epilogue of the FP8 cluster split-K is not built");
     using Cfg = DecodeCfg<NT, STAGES, KPS, CLUSTER>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(

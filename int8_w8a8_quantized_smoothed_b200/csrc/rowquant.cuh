@@ -673,7 +673,7 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) silu_
 // is quantized per token with s = max_j |a[m, j]| / 127, exactly as the SiLU*up row kernel
 // quantizes the same values.
 
-template <int NCH>
+template <int NCH, bool F8 = false>
 __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quantize_f32_rows_kernel(
     const float *__restrict__ a, int I, int M, int8_t *__restrict__ q, float *__restrict__ s_tok)
 {
@@ -707,7 +707,7 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quant
             for (int i = 0; i < 8; ++i)
                 amax = fmaxf(amax, fabsf(v[c][i]));
         amax = block_max(amax, sh[it & 1u]);
-        quantize_and_store<NCH>(v, amax, 0, nvec, q + row * I, s_tok + row);
+        quantize_and_store<NCH, F8>(v, amax, 0, nvec, q + row * I, s_tok + row);
     }
 }
 

@@ -278,14 +278,14 @@ int launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int t
                          dim3(threads), 0, st, gu, I, static_cast<int>(M), q, s);
 }
 
-template <int NCH>
+template <int NCH, bool F8 = false>
 int launch_quantize_f32(const float *a, int64_t M, int I, int8_t *q, float *s, int threads,
                         int dev, int sms, cudaStream_t st)
 {
-    const void *fn = reinterpret_cast<const void *>(&quantize_f32_rows_kernel<NCH>);
+    const void *fn = reinterpret_cast<const void *>(&quantize_f32_rows_kernel<NCH, F8>);
     if (int rc = ensure_smem(fn, dev, 0))
         return rc;
-    return launch_kernel(quantize_f32_rows_kernel<NCH>, dim3(row_grid(fn, threads, M, dev, sms)),
+    return launch_kernel(quantize_f32_rows_kernel<NCH, F8>, dim3(row_grid(fn, threads, M, dev, sms)),
                          dim3(threads), 0, st, a, I, static_cast<int>(M), q, s);
 }
 
@@ -524,7 +524,10 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
                   uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev, cudaStream_t st)
 {
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
-    if (p.variant == 3) {
+    if constexpr (SILU && F8) {
+        if (p.variant == 3) // the FP8 cluster split-K has no SiLU epilogue: planned away
+            return W8A8_ERR_UNSUPPORTED_SHAPE;
+    } else if (p.variant == 3) {
         using Cfg = DecodeCfg<NT, STAGES, KPS, true>;
         auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU, F8>;
         if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
@@ -570,10 +573,11 @@ int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *
     }
 }
 
-// The FP8 GEMM launch for a plan (plain dequant epilogue, variants 1 and 2).
+// The FP8 GEMM launch for a plan: plain dequant epilogue (so == nullptr) or the fused
+// SiLU*up epilogue (tile kernels and stream-K; not the cluster split-K).
 int gemm_run_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const float *s_ch,
                  int64_t M, int64_t N, int64_t K, uint16_t *y, float *acc_out, void *workspace,
-                 const GemmPlan &p, int dev, int sms, cudaStream_t st)
+                 const GemmPlan &p, int dev, int sms, cudaStream_t st, const SiluOut *so = nullptr)
 {
     const SiluOut none{nullptr, 0};
     int32_t *acc = reinterpret_cast<int32_t *>(acc_out); // raw binary32 words
@@ -582,6 +586,13 @@ int gemm_run_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const
         CUtensorMap ta, tb;
         if (encode_kmajor_i8(&ta, xq, M, K, kBM) || encode_kmajor_i8(&tb, wq, N, K, bn))
             return W8A8_ERR_CUDA;
+        if (so) {
+            if (p.tile_n == 512)
+                return launch_prefill_pair<6, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, dev, sms, st);
+            if (p.tile_n == 256)
+                return launch_prefill<256, 4, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, dev, sms, st);
+            return launch_prefill<128, 6, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, dev, sms, st);
+        }
         if (p.tile_n == 512)
             return launch_prefill_pair<6, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
         if (p.tile_n == 256)
@@ -591,6 +602,8 @@ int gemm_run_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const
     CUtensorMap tw, tx;
     if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
         return W8A8_ERR_CUDA;
+    if (so)
+        return launch_decode_nt<true, true>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, workspace, *so, dev, st);
     return launch_decode_nt<false, true>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, workspace, none, dev, st);
 }
 
@@ -946,6 +959,66 @@ int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_
     case 1: return launch_quantize_f32<1>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
     case 2: return launch_quantize_f32<2>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
     default: return launch_quantize_f32<4>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
+    }
+}
+
+// The FP8 fused gate|up plan: as the GEMM's own, with stream-K in place of the cluster
+// split-K (which has no SiLU epilogue).
+int plan_silu_fp8(int64_t M, int64_t I, int64_t K, int sms, GemmPlan *p)
+{
+    int rc = plan_gemm(M, 2 * I, K, 0, 0, 0, sms, p, true);
+    if (rc == W8A8_OK && p->variant == 3)
+        rc = plan_gemm(M, 2 * I, K, 2, 0, 0, sms, p, true);
+    return rc;
+}
+
+size_t w8a8_gemm_silu_quant_fp8_workspace_size(int64_t M, int64_t I, int64_t K)
+{
+    if (I < 64 || I % 64 != 0 || check_gemm_shape(M, 2 * I, K))
+        return 0;
+    int dev, sms = 148;
+    if (current_device(&dev, &sms))
+        sms = 148;
+    GemmPlan p;
+    if (plan_silu_fp8(M, I, K, sms, &p))
+        return 0;
+    return p.ws_bytes;
+}
+
+int w8a8_gemm_silu_quant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq_il,
+                             const float *s_ch_il, int64_t M, int64_t I, int64_t K, float *a,
+                             uint8_t *q, float *s_out, void *workspace, size_t workspace_bytes,
+                             w8a8_stream_t stream)
+{
+    if (!xq || !s_tok || !wq_il || !s_ch_il || !a || !q || !s_out)
+        return W8A8_ERR_INVALID_ARG;
+    if (I < 64 || I % 64 != 0)
+        return W8A8_ERR_UNSUPPORTED_SHAPE;
+    int rc = check_gemm_shape(M, 2 * I, K);
+    if (rc || (rc = check_row_shape(M, I)))
+        return rc;
+    if (!aligned16(xq) || !aligned16(wq_il) || !aligned16(s_ch_il) || !aligned16(a) ||
+        !aligned16(q) || (workspace && !aligned16(workspace)))
+        return W8A8_ERR_ALIGNMENT;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    GemmPlan p;
+    if ((rc = plan_silu_fp8(M, I, K, sms, &p)))
+        return rc;
+    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
+        return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const SiluOut so{a, static_cast<int>(I)};
+    if ((rc = gemm_run_fp8(xq, s_tok, wq_il, s_ch_il, M, 2 * I, K, nullptr, nullptr, workspace,
+                           p, dev, sms, st, &so)))
+        return rc;
+    int8_t *qc = reinterpret_cast<int8_t *>(q);
+    const RowLaunch L = row_launch(I);
+    switch (L.nch) {
+    case 1: return launch_quantize_f32<1, true>(a, M, (int)I, qc, s_out, L.threads, dev, sms, st);
+    case 2: return launch_quantize_f32<2, true>(a, M, (int)I, qc, s_out, L.threads, dev, sms, st);
+    default: return launch_quantize_f32<4, true>(a, M, (int)I, qc, s_out, L.threads, dev, sms, st);
     }
 }
 

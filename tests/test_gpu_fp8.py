@@ -14,7 +14,7 @@ import torch
 
 import int8_w8a8_quantized_smoothed_b200 as w8
 import oracle
-from int8_w8a8_quantized_smoothed_b200 import synth
+from int8_w8a8_quantized_smoothed_b200 import prep, synth
 from helpers import assert_rms_rows_match, dev, dev_bf16, f32_out, host, host_bf16, with_canary
 
 pytestmark = pytest.mark.gpu
@@ -221,3 +221,55 @@ def test_fp8_linear_chain_matches_oracle():
     ref, _ = assert_rms_rows_match(codes(q), host(s), x, gamma, 1e-5,
                                    ref_fn=oracle.smooth_rmsnorm_quant_fp8)
     _check_gemm(codes(q), host(s), wq, s_ch)
+
+
+# ---------------------------------------------------------------- fused gate|up + SiLU*up
+#
+# The fused call's binary32 accumulators equal the plain FP8 GEMM's on the same interleaved
+# weight under the same plan (the automatic one; the fused call takes stream-K where that
+# plan is the cluster split-K, so the reference is asked for stream-K there): SiLU*up and
+# the E4M3 quantization of the plain GEMM's bf16 output, by the oracle, must then match the
+# fused result bit for bit.
+
+def _gate_up_fp8(M, I, K, seed):
+    xq, s_tok = oracle.quantize_rows_fp8(synth.activation(M, K, seed))
+    wq, s_ch = oracle.rtn_weights_fp8(synth.weight(2 * I, K, seed + 1))
+    return xq, s_tok, wq, s_ch
+
+
+FUSED_SHAPES = [(1, 1024, 512), (16, 5120, 1024), (64, 14336, 4096), (33, 2048, 1024),
+                (8, 128, 4112), (300, 1024, 512), (129, 512, 400), (512, 2048, 1024)]
+
+
+@pytest.mark.parametrize("M,I,K", FUSED_SHAPES)
+def test_fused_gate_up_silu_quant_fp8(M, I, K):
+    xq, st, wq, sc = _gate_up_fp8(M, I, K, seed=M + I + K)
+    wq_il, sc_il = prep.interleave_gate_up(dev_fp8(wq), dev(sc))
+    NB = (2 * I + 127) // 128
+    cluster = M <= 64 and 2 * NB <= torch.cuda.get_device_properties(0).multi_processor_count \
+        and K > 128
+    y_il = w8.w8a8_gemm_dequant_fp8(dev_fp8(xq), dev(st), wq_il, sc_il,
+                                    variant=2 if cluster else 0)
+    y = host_bf16(y_il).reshape(M, I // 64, 2, 64)
+    gu = np.concatenate([y[:, :, 0, :].reshape(M, I), y[:, :, 1, :].reshape(M, I)], axis=1)
+    a_ref = oracle.silu_mul(gu)
+    q_ref, s_ref = oracle.quantize_rows_f32_fp8(a_ref)
+    ws = w8.Workspace()
+    for _ in range(2):  # the second call checks that the workspace came back zeroed
+        q, s, a = w8.w8a8_gemm_silu_quant_fp8(dev_fp8(xq), dev(st), wq_il, sc_il, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(a).view(np.uint32), a_ref.view(np.uint32))
+        assert np.array_equal(host(s), s_ref)
+        assert np.array_equal(codes(q), q_ref)
+
+
+def test_fused_fp8_equals_unfused_gpu_chain():
+    """Whole channel blocks per CTA (the decode plan for this weight): every accumulator is
+    one CTA's sum over all of K in the same order, interleaved or not."""
+    M, I, K = 16, 14336, 4096
+    xq, st, wq, sc = _gate_up_fp8(M, I, K, 7)
+    y = w8.w8a8_gemm_dequant_fp8(dev_fp8(xq), dev(st), dev_fp8(wq), dev(sc))
+    q0, s0 = w8.w8a8_silu_mul_quant_fp8(y)
+    wq_il, sc_il = prep.interleave_gate_up(dev_fp8(wq), dev(sc))
+    q1, s1, _ = w8.w8a8_gemm_silu_quant_fp8(dev_fp8(xq), dev(st), wq_il, sc_il)
+    assert torch.equal(q0.view(torch.uint8), q1.view(torch.uint8)) and torch.equal(s0, s1)
