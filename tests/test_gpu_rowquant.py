@@ -172,6 +172,34 @@ def test_smooth_rmsnorm_quant_persistent_loop(M, K, with_residual):
         assert np.array_equal(host_bf16(h), ref["h"])
 
 
+@pytest.mark.parametrize("M,K", [(3, 4096), (600, 4096), (5, 8192), (300, 16384)])
+@pytest.mark.parametrize("with_residual", [False, True])
+def test_smooth_rmsnorm_quant_same_in_every_overlap_mode(M, K, with_residual):
+    """Overlap mode 2 reads gamma' before the dependency wait (into registers for rows of up
+    to 4096 values, into L2 for longer rows): the results are those of modes 0 and 1."""
+    x = dev_bf16(synth.activation(M, K, seed=M + K))
+    gf = dev(synth.gamma(K, seed=K + 3))
+    res = dev_bf16(synth.normal_bf16((M, K), seed=M + 5)) if with_residual else None
+    prev = w8.w8a8_get_overlap()
+    out = {}
+    try:
+        for mode in (0, 1, 2):
+            w8.w8a8_set_overlap(mode)
+            h = torch.empty(M, K, dtype=torch.bfloat16, device="cuda") if with_residual else None
+            r = w8.w8a8_smooth_rmsnorm_quant(x, gf, 1e-5, residual=res, h_out=h)
+            torch.cuda.synchronize()
+            out[mode] = [host(t) if t.dtype != torch.bfloat16 else host_bf16(t) for t in r]
+    finally:
+        w8.w8a8_set_overlap(prev)
+    for mode in (1, 2):
+        for a, b in zip(out[0], out[mode]):
+            assert np.array_equal(a, b), f"overlap mode {mode}"
+    ref, _ = assert_rms_rows_match(out[2][0], out[2][1], synth.activation(M, K, seed=M + K),
+                                   synth.gamma(K, seed=K + 3), 1e-5,
+                                   residual=synth.normal_bf16((M, K), seed=M + 5)
+                                   if with_residual else None)
+
+
 @pytest.mark.parametrize("M,I", [(5000, 128), (700, 14336), (300, 28672)])
 def test_silu_mul_quant_persistent_loop(M, I):
     gu = synth.normal_bf16((M, 2 * I), seed=M + I + 5, std=2.5)
