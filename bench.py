@@ -880,6 +880,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.case is None:
         ap.error("--warmup must be at least 3")
+    if args.fp8 and args.fused_block:
+        ap.error("the fused block kernel (--fused-block) has INT8 codes only")
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
