@@ -121,6 +121,26 @@ def test_extreme_accumulators():
         _compare(y, acc, y_ref, acc_ref)
 
 
+@pytest.mark.parametrize("variant", [1, 2, 3])
+def test_largest_k_accumulators_near_int32_limit(variant):
+    # K = 133136, the largest multiple of 16 within the library's bound (127^2 K < 2^31):
+    # every product is +-127*127 and the sums come within 2^22 of the int32 limit, in the
+    # tile kernel, across stream-K CTAs and across an 8-CTA cluster
+    M, N, K = 3, 16, 133136
+    xq = np.full((M, K), 127, np.int8)
+    xq[1] = -127
+    xq[2, ::2] = -127
+    wq = np.full((N, K), 127, np.int8)
+    wq[5] = -127
+    st = synth.scales(M, 3)
+    sc = synth.scales(N, 4)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    top = int(acc_ref[0, 0])
+    assert top == 127 * 127 * K and 2 ** 31 - top < 2 ** 22
+    y, acc = _run(xq, st, wq, sc, variant=variant)
+    _compare(y, acc, y_ref, acc_ref)
+
+
 def test_auto_variant_and_workspace_reuse():
     # the stream-K workspace must come back ready for the next call (flags zero): run twice
     # through one workspace, with the automatic choice and forced stream-K
