@@ -312,7 +312,7 @@ int decode_nt(int64_t M)
 
 
 int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
-              GemmPlan *p, bool f8 = false)
+              GemmPlan *p)
 {
     if (variant < 0 || variant > 3 || ctas < 0 ||
         (tile_n != 0 && tile_n != 128 && tile_n != 256 && tile_n != 512))
@@ -966,9 +966,9 @@ int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_
 // split-K (which has no SiLU epilogue).
 int plan_silu_fp8(int64_t M, int64_t I, int64_t K, int sms, GemmPlan *p)
 {
-    int rc = plan_gemm(M, 2 * I, K, 0, 0, 0, sms, p, true);
+    int rc = plan_gemm(M, 2 * I, K, 0, 0, 0, sms, p);
     if (rc == W8A8_OK && p->variant == 3)
-        rc = plan_gemm(M, 2 * I, K, 2, 0, 0, sms, p, true);
+        rc = plan_gemm(M, 2 * I, K, 2, 0, 0, sms, p);
     return rc;
 }
 
@@ -1084,7 +1084,7 @@ size_t w8a8_gemm_fp8_workspace_size(int64_t M, int64_t N, int64_t K, int variant
     if (current_device(&dev, &sms))
         sms = 148;
     GemmPlan p;
-    if (plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p, true))
+    if (plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p))
         return 0;
     return p.ws_bytes;
 }
@@ -1106,7 +1106,7 @@ int w8a8_gemm_dequant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *
     if ((rc = current_device(&dev, &sms)))
         return rc;
     GemmPlan p;
-    if ((rc = plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p, true)))
+    if ((rc = plan_gemm(M, N, K, variant, ctas, tile_n, sms, &p)))
         return rc;
     if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
         return W8A8_ERR_WORKSPACE;
