@@ -422,13 +422,47 @@ def time_graph(g, steps, warmup):
     return e0.elapsed_time(e1) / 1e3
 
 
+def replay_latencies(g, n):
+    """Per-replay device times (microseconds) of n back-to-back replays: an event pair
+    around every replay on the launching stream (the replays still follow one another
+    without host synchronization). Returns p50, p95 and mean."""
+    st = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    ev[0].record(st)
+    for i in range(n):
+        g.replay()
+        ev[i + 1].record(st)
+    torch.cuda.synchronize()
+    t = sorted(ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(n))
+    return {"p50_us": round(statistics.median(t), 2),
+            "p95_us": round(t[min(n - 1, math.ceil(0.95 * n) - 1)], 2),
+            "mean_us": round(sum(t) / n, 2), "n": n,
+            "how": "one CUDA event pair per graph replay, replays back to back"}
+
+
 def run_ours(args, world, rank, local):
+    """The workload's JSON line; with the default decode workload it also carries a record
+    of each --extra workload (prefill8b by default), measured the same way in this run."""
     import int8_w8a8_quantized_smoothed_b200 as w8
     from int8_w8a8_quantized_smoothed_b200 import build as wbuild
     wbuild.build()
     w8.lib()
+    result = measure_workload(args, args.workload, world, rank, local, primary=True)
+    extras = [] if args.extra in ("", "none") else [
+        e for e in args.extra.split(",") if e != args.workload]
+    for name in extras:
+        torch.cuda.empty_cache()
+        result[name] = measure_workload(args, name, world, rank, local, primary=False)
+    return result
+
+
+def measure_workload(args, name, world, rank, local, primary):
+    """Times one workload's step (and its GEMM launches and row launches alone). The primary
+    workload's record is the JSON line itself (with e2e and the CPU baseline); a secondary
+    one is a nested record with the same timing, roofline and clock keys."""
+    import int8_w8a8_quantized_smoothed_b200 as w8
     dev = torch.device("cuda", local)
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS[name]
     arch = wl["arch"]
     layers = [Layer(arch, M, seed=1000 * (i + 1), device=dev, fp8=args.fp8,
                     block=args.fused_block) for i, M in enumerate(wl["Ms"])]
@@ -535,9 +569,12 @@ def run_ours(args, world, rank, local):
         g_gemm_f = capture(step_gemms_fused)
         gfsecs = time_graph(g_gemm_f, args.steps, args.warmup) / args.steps
         del g_gemm_f
-    g_e2e = capture(step_e2e)
-    esecs = time_graph(g_e2e, args.steps, args.warmup) / args.steps
-    e_value, _ = combine(nbytes, esecs, world)
+    latency = replay_latencies(g_step, max(100, min(args.steps, 1000)))
+    g_e2e = esecs = e_value = None
+    if primary:
+        g_e2e = capture(step_e2e)
+        esecs = time_graph(g_e2e, args.steps, args.warmup) / args.steps
+        e_value, _ = combine(nbytes, esecs, world)
     assert w8.w8a8_device_status(reset=True) == 0, "device-side wait ran out"
 
     hbm_peak, peak_src = read_peaks()
@@ -589,6 +626,7 @@ def run_ours(args, world, rank, local):
                    "codes": "FP8 E4M3 (scale absmax / 448)" if args.fp8 else
                             "INT8 (scale absmax / 127)"},
         "tops": round(ops / t_max / 1e12, 3),
+        "latency_us": latency,
         "roofline_step": {"t_roof_us": round(t_roof * 1e6, 2),
                           "t_us": round(t_max * 1e6, 2), "frac": round(t_roof / t_max, 4),
                           "frac_vs_measured_int8": round(t_roof_meas / t_max, 4),
@@ -602,23 +640,28 @@ def run_ours(args, world, rank, local):
                          "note": "gemms: plain epilogues; row_kernels: the step's row "
                                  "launches" + ("" if unfused else
                                                " (SiLU*up is fused into the gate|up GEMM)")},
-        "e2e": {"value": round(e_value / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(esecs * 1e3, 5),
-                "how": "CUDA graph per step: pinned-host inputs H2D and outputs D2H on a copy "
-                       "stream overlapping the other layers' C-ABI calls"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(t_wall0, time.perf_counter()),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
+    if primary:
+        result["e2e"] = {"value": round(e_value / 1e9, 2), "unit": "GB/s",
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                         "ms_per_step": round(esecs * 1e3, 5),
+                         "how": "CUDA graph per step: pinned-host inputs H2D and outputs D2H on "
+                                "a copy stream overlapping the other layers' C-ABI calls"}
+    else:  # a nested record: the JSON line's own keys stay the primary workload's
+        for k in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling",
+                  "vs_baseline", "data", "gpu_launches"):
+            result.pop(k)
+    if primary and rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
         result["cpu_baseline"] = cpu_baseline(arch)
-    traffic = args.traffic if args.traffic is not None else (
-        None if args.fp8 else NCU_GEMM_TRAFFIC.get(args.workload))
+    traffic = args.traffic if (args.traffic is not None and primary) else (
+        None if args.fp8 else NCU_GEMM_TRAFFIC.get(name))
     if traffic is not None:
         result["roofline"]["traffic"] = traffic
         result["roofline"]["traffic_per"] = "GEMM launch (ncu DRAM read + write bytes)"
         result["roofline"]["algorithmic_bytes_per_launch"] = round(g_bytes / (4 * len(layers)))
-    del g_step, g_gemm, g_rows, g_e2e
+    del g_step, g_gemm, g_rows, g_e2e, layers
     return result
 
 
@@ -862,6 +905,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode8b")
+    ap.add_argument("--extra", default=None,
+                    help="comma-separated further workloads measured in the same run and "
+                         "reported as nested records of the line (default: prefill8b with the "
+                         "decode8b workload, else none; 'none' disables)")
     ap.add_argument("--case", default=None)
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if measured")
@@ -882,6 +929,12 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.fp8 and args.fused_block:
         ap.error("the fused block kernel (--fused-block) has INT8 codes only")
+    if args.extra is None:
+        args.extra = "prefill8b" if (args.workload == "decode8b" and not args.fused_block) \
+            else "none"
+    for e in args.extra.split(","):
+        if e not in WORKLOADS and e not in ("", "none"):
+            ap.error(f"--extra: unknown workload {e}")
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -194,7 +194,7 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
  *
  * Computes exactly what w8a8_gemm_dequant computes, always with its small-M swap-AB kernels
  * (M <= 256), and allocates nothing. Only the stream-K kernel, used when the weight has many
- * 128-channel blocks, needs scratch; it is a file-scope device array of
+ * 128-channel blocks, needs scratch; it is a file-scope static device array of
  * W8A8_NOALLOC_SCRATCH_BYTES (8 MiB) inside the library; every GPU on which the library is
  * loaded holds that array until the process exits. The caller still owns and passes every
  * input and output. Arguments and requirements are those of w8a8_gemm_dequant without
@@ -206,8 +206,10 @@ W8A8_API size_t w8a8_gemm_workspace_size_ex(int64_t M, int64_t N, int64_t K, int
  *     M <= 108 always fits. W8A8_ERR_UNSUPPORTED_SHAPE for M > 256.
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
- *   - Each call clears the part of the array it uses (cudaMemsetAsync on `stream`) before
- *     its kernel runs, so an earlier failed call leaves no stale state.
+ *   - Each call that needs the scratch clears its 4 KiB of flag words (cudaMemsetAsync on
+ *     `stream`) before its kernel runs, so flags left raised by an earlier call whose wait
+ *     ran out cannot leak into it; the partial sums need no clearing (each is written
+ *     before its flag is raised).
  *   - All calls on a device share the one array and it keeps the last call's contents:
  *     calls whose kernels can overlap on the GPU (different streams without ordering
  *     between them) race on it and give wrong results. Serialize them.
@@ -432,6 +434,17 @@ W8A8_API int w8a8_get_overlap(void);
  * reset != 0 clears the word. Returns W8A8_ERR_CUDA if synchronization fails.
  */
 W8A8_API int w8a8_device_status(int reset);
+
+/*
+ * Stream status: waits until `stream` has finished the work queued on it so far (not the
+ * whole device), then returns W8A8_OK, or W8A8_ERR_TIMEOUT if a kernel of this library on
+ * the current device gave up a bounded wait since the device word was last cleared. The word
+ * is per device, not per stream: a timeout in a kernel of another stream on the same device
+ * shows here too once that kernel has run. It is not cleared here (w8a8_device_status(1)
+ * clears it). Returns W8A8_ERR_CUDA if the stream's work failed. [No counterpart on the
+ * pages: the failure-detection side of every call above.]
+ */
+W8A8_API int w8a8_last_device_status(w8a8_stream_t stream);
 
 /*
  * Self-test of the failure path (no counterpart on the pages): launches one small kernel

@@ -21,7 +21,7 @@ __all__ = [
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
     "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_gemm_silu_quant",
     "w8a8_gemm_silu_quant_workspace_size", "w8a8_probe_i8_mma", "w8a8_selftest_wait_timeout", "w8a8_set_overlap",
-    "w8a8_get_overlap", "w8a8_device_status",
+    "w8a8_get_overlap", "w8a8_device_status", "w8a8_last_device_status",
     "w8a8_status_string", "w8a8_version",
     "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
     "w8a8_gemm_dequant_fp8", "w8a8_gemm_fp8_workspace_size", "w8a8_gemm_silu_quant_fp8",
@@ -60,6 +60,7 @@ SIGNATURES = [
     ("w8a8_set_overlap", _I, [_I]),
     ("w8a8_get_overlap", _I, []),
     ("w8a8_device_status", _I, [_I]),
+    ("w8a8_last_device_status", _I, [_P]),
     ("w8a8_status_string", C.c_char_p, [_I]),
     ("w8a8_version", _I, []),
     ("w8a8_quantize_rows_fp8", _I, [_P, _P, _I64, _I64, _P, _P, _P]),
@@ -175,6 +176,12 @@ def w8a8_get_overlap() -> int:
 def w8a8_device_status(reset: bool = False) -> int:
     """Synchronizes the current device; returns 0 or -6 (a bounded wait ran out)."""
     return lib().w8a8_device_status(1 if reset else 0)
+
+
+def w8a8_last_device_status(stream=None) -> int:
+    """Waits for `stream` (default: the current stream) only; returns 0 or -6 (a bounded
+    wait of a kernel on this device ran out; the word is not cleared)."""
+    return lib().w8a8_last_device_status(_stream(stream))
 
 
 def w8a8_quantize_rows(x, smooth_inv=None, q=None, s_tok=None, stream=None):

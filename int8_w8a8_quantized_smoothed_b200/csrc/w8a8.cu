@@ -1398,6 +1398,25 @@ int w8a8_selftest_wait_timeout(unsigned long long limit_ns, w8a8_stream_t stream
     return W8A8_OK;
 }
 
+int w8a8_last_device_status(w8a8_stream_t stream)
+{
+    int dev, sms;
+    int rc = current_device(&dev, &sms);
+    if (rc)
+        return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the read is ordered after this stream's work; the host copy target is pageable, so the
+    // call returns once the stream has reached it
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbolAsync(&word, g_status_word, sizeof(word), 0,
+                                  cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+    }
+    return (word & kStatusTimeout) ? W8A8_ERR_TIMEOUT : W8A8_OK;
+}
+
 int w8a8_device_status(int reset)
 {
     int dev, sms;
@@ -1421,13 +1440,13 @@ int w8a8_device_status(int reset)
 
 // ------------------------------------------------------------------ no-allocation GEMM
 
-namespace {
-
-// Split-K scratch of w8a8_gemm_dequant_noalloc: accumulators and tickets live here instead
+// Split-K scratch of w8a8_gemm_dequant_noalloc: flag words and partial sums live here instead
 // of in a caller-provided workspace. Host code must not pass `g_noalloc_scratch` itself to a
 // kernel (on the host it names a host-side shadow, not device memory); it passes the device
 // address looked up by noalloc_scratch().
-__device__ __align__(256) unsigned char g_noalloc_scratch[W8A8_NOALLOC_SCRATCH_BYTES];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[W8A8_NOALLOC_SCRATCH_BYTES];
+
+namespace {
 
 void *g_noalloc_ptr[kMaxDevices];
 
@@ -1478,7 +1497,12 @@ extern "C" int w8a8_gemm_dequant_noalloc(const int8_t *xq, const float *s_tok, c
             return rc;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (p.ws_bytes > 0 && cudaMemsetAsync(scratch, 0, p.ws_bytes, st) != cudaSuccess) {
+    // Only the flag words must be zero when the kernel starts (each contributor writes its
+    // partial sums before raising its flag, and the owner lowers the flags it consumed);
+    // clearing them on every call also drops flags left raised by a call whose wait ran out.
+    if (p.ws_bytes > 0 &&
+        cudaMemsetAsync(static_cast<char *>(scratch) + p.flag_off, 0, kFlagBytes, st) !=
+            cudaSuccess) {
         cudaGetLastError();
         return W8A8_ERR_CUDA;
     }

@@ -88,3 +88,37 @@ def assert_rms_rows_match(got_q, got_s, x, gamma, eps, residual=None, ref=None,
                 ok = True
         assert ok, f"row {m} matches neither admissible mean of squares"
     return ref, len(bad)
+
+
+def check_block_rows(rows, x, attn, pr, eps, got):
+    """One decoder block's chain on sampled rows, stage by stage: every stage's GPU result
+    against the oracle applied to the GPU's own inputs of that stage, each of which the
+    previous check has tied to the oracle. An order-ambiguous RMSNorm row, where the GPU may
+    take the other admissible neighbouring mean of squares, is thus checked through the
+    whole chain instead of being left out. `got` maps q1 s1 qkv q2 s2 o h q3 s3 q4 s4 down
+    (and optionally gate_up, a) to host arrays (bf16 as uint16 bits, a as float32); returns
+    how many RMSNorm rows took the other neighbour."""
+    xr, ar = x[rows], attn[rows]
+    g = {k: v[rows] for k, v in got.items()}
+
+    def gemm(q, s, name):
+        y, _ = oracle.gemm_dequant(q, s, pr[name]["wq"], pr[name]["s_ch"], want_acc=False)
+        return y
+
+    _, n1 = assert_rms_rows_match(g["q1"], g["s1"], xr, pr["gamma1f"], eps)
+    assert np.array_equal(g["qkv"], gemm(g["q1"], g["s1"], "qkv"))
+    q2, s2 = oracle.quantize_rows(ar, pr.get("s_inv_o"))
+    assert np.array_equal(g["q2"], q2) and np.array_equal(g["s2"], s2)
+    assert np.array_equal(g["o"], gemm(g["q2"], g["s2"], "o"))
+    ref3, n3 = assert_rms_rows_match(g["q3"], g["s3"], g["o"], pr["gamma2f"], eps,
+                                     residual=xr)
+    assert np.array_equal(g["h"], ref3["h"])
+    gu = gemm(g["q3"], g["s3"], "gate_up")
+    if "gate_up" in g:
+        assert np.array_equal(g["gate_up"], gu)
+    if "a" in g:
+        assert np.array_equal(g["a"].view(np.uint32), oracle.silu_mul(gu).view(np.uint32))
+    q4, s4 = oracle.silu_mul_quant(gu)
+    assert np.array_equal(g["q4"], q4) and np.array_equal(g["s4"], s4)
+    assert np.array_equal(g["down"], gemm(g["q4"], g["s4"], "down"))
+    return n1 + n3

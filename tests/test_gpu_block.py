@@ -10,7 +10,7 @@ import torch
 import int8_w8a8_quantized_smoothed_b200 as w8
 import oracle
 from int8_w8a8_quantized_smoothed_b200 import prep, synth
-from helpers import assert_rms_rows_match, dev, dev_bf16, host, host_bf16
+from helpers import assert_rms_rows_match, check_block_rows, dev, dev_bf16, host, host_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -105,7 +105,12 @@ def test_decoder_block_chain_m512_sampled_rows():
     torch.cuda.synchronize()
     assert w8.w8a8_device_status() == 0
 
-    # oracle on the sampled rows
+    # every sampled row, stage by stage (ambiguous RMSNorm rows by the neighbour rule)
+    got = dict(q1=host(q1), s1=host(s1), qkv=host_bf16(qkv), q2=host(q2), s2=host(s2),
+               o=host_bf16(o), h=host_bf16(h), q3=host(q3), s3=host(s3),
+               gate_up=host_bf16(gu), q4=host(q4), s4=host(s4), down=host_bf16(down))
+    check_block_rows(rows, x, attn, pr, EPS, got)
+    # and end to end from the inputs through the oracle's own chain
     ref = oracle.block_reference({"x": x[rows], "attn": attn[rows]}, pr, EPS)
     ambiguous = ref["amb1"] | ref["amb3"]
     assert ambiguous.sum() <= 1

@@ -127,6 +127,8 @@ def _check_gemm_fp8(M, N, K, seed, wseed):
     _, acc_ref, absacc = oracle.gemm_fp8(xq[rows], st[rows], wq, sc)
     a = host(acc)[rows].astype(np.float64)
     assert (np.abs(a - acc_ref) <= (K + 16) * 2.0 ** -24 * absacc).all()
+    # empirical guard (measured at most 14 units of 2^-24 * sum|products| on B200)
+    assert (np.abs(a - acc_ref) <= 64 * 2.0 ** -24 * absacc).all()
     assert np.array_equal(host_bf16(y)[rows], oracle.dequant_f32acc(host(acc)[rows], st[rows], sc))
 
 

@@ -283,3 +283,17 @@ def test_wait_timeout_reports_status_and_context_stays_usable():
     assert np.array_equal(host(q), q_ref) and np.array_equal(host(s), s_ref)
     with pytest.raises(w8.W8A8Error):
         w8.w8a8_selftest_wait_timeout(10)  # below the allowed range
+
+
+def test_stream_status_reports_timeout_of_that_streams_kernel():
+    # w8a8_last_device_status waits for one stream only and reads the device word without
+    # clearing it
+    assert w8.w8a8_device_status(reset=True) == 0
+    s = torch.cuda.Stream()
+    assert w8.w8a8_last_device_status(s) == 0
+    w8.w8a8_selftest_wait_timeout(2_000_000, stream=s)
+    assert w8.w8a8_last_device_status(s) == -6
+    assert w8.w8a8_last_device_status(s) == -6  # not cleared by reading
+    assert w8.w8a8_device_status(reset=True) == -6
+    assert w8.w8a8_last_device_status(s) == 0
+    assert w8.w8a8_last_device_status() == 0

@@ -263,6 +263,91 @@ def test_exp_against_binary64():
     assert all(b >= a for a, b in zip(sweep, sweep[1:]))
 
 
+def _rn32(q):
+    """Round an exact rational to the nearest binary32 value, ties to even, with gradual
+    underflow (quantum 2^-149) and overflow to infinity. Returns a Fraction or +-inf."""
+    q = Fraction(q)
+    if q == 0:
+        return Fraction(0)
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (max(e, -126) - 23)
+    n = a / quantum
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    v = fl * quantum
+    if v >= Fraction(2) ** 128:
+        return math.inf if q > 0 else -math.inf
+    return v if q > 0 else -v
+
+
+def _exp_spec(x):
+    """The binary32 exp exactly as the header writes it down, each operation evaluated in
+    exact rational arithmetic and rounded once to binary32 (an fma rounds once): Cody-Waite
+    reduction with k = rint(RN(x * RN(1/ln 2))), r = fma(-k, ln2_hi, x), r = fma(-k, ln2_lo, r)
+    (ln2_hi = ln 2 to 16 significant bits, ln2_lo = RN(ln 2 - ln2_hi)); the degree-7 Taylor
+    polynomial with coefficients RN(1/i!) by Horner's rule in fma; then times 2^(k/2) and
+    2^(k - k/2) (k/2 truncated toward zero); x > 89 -> +inf, x < -104 -> +0."""
+    import decimal
+    ctx = decimal.Context(prec=60)
+    ln2_dec = ctx.ln(decimal.Decimal(2))
+    ln2 = Fraction(ln2_dec)
+    x = Fraction(float(x))
+    if x > 89:
+        return math.inf
+    if x < -104:
+        return 0.0
+    log2e = _rn32(Fraction(ctx.divide(decimal.Decimal(1), ln2_dec)))
+    ln2_hi = Fraction(math.floor(ln2 * 2 ** 16), 2 ** 16)  # bit 17 of ln 2 is 0: floor = RN
+    ln2_lo = _rn32(ln2 - ln2_hi)
+    k = round(_rn32(x * log2e))  # Fraction.__round__ rounds half to even, as rint does
+    r = _rn32(-k * ln2_hi + x)
+    r = _rn32(-k * ln2_lo + r)
+    c = [_rn32(Fraction(1, math.factorial(i))) for i in range(8)]
+    p = c[7]
+    for i in range(6, -1, -1):
+        p = _rn32(p * r + c[i])
+    k1 = int(k / 2) if k >= 0 else -int(-k / 2)
+    k2 = k - k1
+    v = _rn32(p * Fraction(2) ** k1)
+    if v in (math.inf, -math.inf):
+        return v
+    v = _rn32(v * Fraction(2) ** k2)
+    return float(v)
+
+
+def test_exp_bits_match_an_exact_evaluation_of_its_written_definition():
+    # Pins every bit of the oracle's exp (and so of the SiLU the GPU must reproduce) to the
+    # header's written definition, evaluated independently with exact rationals: a dropped
+    # Horner term, a wrong constant or a different scaling split changes many of these bits.
+    rng = np.random.default_rng(11)
+    f32 = np.float32
+    ln2 = math.log(2.0)
+    xs = [f32(0.0), f32(-0.0), f32(89.0), np.nextafter(f32(89.0), f32(100)), f32(-104.0),
+          np.nextafter(f32(-104.0), f32(-200)), f32(88.72283), f32(88.7228394),
+          f32(-87.33654), f32(-87.336548), f32(-103.278931), f32(-103.97), f32(1e-8),
+          f32(-1e-8), f32(2.0 ** -30), f32(0.5), f32(-0.5), f32(1.0), f32(-1.0)]
+    for j in range(-150, 129, 3):  # arguments where k changes, and their neighbours
+        t = f32((j + 0.5) * ln2)
+        xs += [t, np.nextafter(t, f32(200)), np.nextafter(t, f32(-200))]
+    xs += list(np.linspace(-104, 89, 1200, dtype=np.float32))
+    xs += list(rng.uniform(-104, 89, 1500).astype(np.float32))
+    xs += list(rng.uniform(-1, 1, 500).astype(np.float32))
+    mismatches = []
+    for x in xs:
+        got = f32(oracle.exp(x))
+        want = f32(_exp_spec(x))
+        if got.view(np.uint32) != want.view(np.uint32):
+            mismatches.append((float(x), float(got), float(want)))
+    assert not mismatches, mismatches[:5]
+
+
 def test_silu_special_values_and_accuracy():
     assert oracle.silu(0.0) == 0.0
     for g in (20.0, 50.0, 88.0, 100.0):
