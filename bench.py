@@ -820,7 +820,26 @@ def run_case(args):
     dev = torch.device("cuda", 0)
     if parts[0] == "gptq":
         return run_gptq_case(args, [int(v) for v in parts[1:4]])
-    if parts[0] in ("gemm", "gemm8"):
+    if parts[0] == "silug":
+        # the fused gate|up GEMM + SiLU*up + quantization call, silug:M:I:K
+        M, I, K = (int(v) for v in parts[1:4])
+        copies = max(1, math.ceil(4 * 126e6 / (2 * I * K)))
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+        st = torch.rand(M, device=dev) * 1e-2
+        ws_ = [torch.randint(-127, 128, (2 * I, K), dtype=torch.int8, device=dev)
+               for _ in range(copies)]
+        sc = torch.rand(2 * I, device=dev) * 1e-3
+        a = torch.empty(M, I, dtype=torch.float32, device=dev)
+        q = torch.empty(M, I, dtype=torch.int8, device=dev)
+        s_out = torch.empty(M, dtype=torch.float32, device=dev)
+        wsp = w8.Workspace(dev)
+
+        def launch(i):
+            w8.w8a8_gemm_silu_quant(xq, st, ws_[i % copies], sc, a=a, q=q, s_out=s_out,
+                                    workspace=wsp)
+        work = gemm_bytes(M, 2 * I, K) - 2 * M * 2 * I + 5 * M * I + 4 * M
+        flops = 2 * M * 2 * I * K
+    elif parts[0] in ("gemm", "gemm8"):
         M, N, K = (int(v) for v in parts[1:4])
         variant = int(parts[4]) if len(parts) > 4 else 0
         ctas = int(parts[5]) if len(parts) > 5 else 0
@@ -893,7 +912,7 @@ def run_case(args):
     out = {"case": args.case, "us_per_launch": round(t * 1e6, 3),
            "GBps_algorithmic": round(work / t / 1e9, 1),
            "note": "CUDA graph of back-to-back launches"}
-    if parts[0] in ("gemm", "gemm8"):
+    if parts[0] in ("gemm", "gemm8", "silug"):
         out["TOPS"] = round(flops / t / 1e12, 1)
     return out
 

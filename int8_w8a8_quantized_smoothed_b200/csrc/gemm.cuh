@@ -39,10 +39,14 @@ constexpr int kBM = 128;  // MMA M: TMEM lanes
 constexpr int kBK = 128;  // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kUmmaK = 32; // K of one kind::i8 MMA
 
-// Output of the fused SiLU*up epilogue: a [M, I] binary32.
+// Output of the fused SiLU*up epilogue: a [M, I] binary32. With amax non-null (the small-M
+// kernels), also the max |a| of every (token, group of 64 output channels): amax[m * (I / 64)
+// + group], from which the quantization pass takes each token's scale without re-reading
+// the row.
 struct SiluOut {
     float *a;
     int I;
+    float *amax = nullptr;
 };
 
 __device__ __forceinline__ float bf16_round(float f)
@@ -715,14 +719,31 @@ template <typename GateUp>
 __device__ __forceinline__ void silu_block_rows(int m0, int mt, int t, int etid, const SiluOut &so,
                                                 GateUp gate_up)
 {
-    for (int v = etid; v < mt * 8; v += 128) {
+    // every lane of a warp runs the same trips (the group max is a shuffle over the 8 lanes
+    // that hold one token's 64 channels)
+    for (int base = 0; base < mt * 8; base += 128) {
+        const int v = base + etid;
+        const bool act = v < mt * 8;
         const int m = m0 + (v >> 3), j0 = (v & 7) * 8;
-        float g[8], u[8], a[8];
-        gate_up(m, j0, g, u);
-        silu_mul8(g, u, a);
-        float *dst = so.a + static_cast<int64_t>(m) * so.I + static_cast<int64_t>(t) * 64 + j0;
-        reinterpret_cast<float4 *>(dst)[0] = make_float4(a[0], a[1], a[2], a[3]);
-        reinterpret_cast<float4 *>(dst)[1] = make_float4(a[4], a[5], a[6], a[7]);
+        float mx = 0.0f;
+        if (act) {
+            float g[8], u[8], a[8];
+            gate_up(m, j0, g, u);
+            silu_mul8(g, u, a);
+            float *dst = so.a + static_cast<int64_t>(m) * so.I + static_cast<int64_t>(t) * 64 + j0;
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(a[0], a[1], a[2], a[3]);
+            reinterpret_cast<float4 *>(dst)[1] = make_float4(a[4], a[5], a[6], a[7]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mx = fmaxf(mx, fabsf(a[i]));
+        }
+        if (so.amax != nullptr) {
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1)
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (act && (v & 7) == 0)
+                so.amax[static_cast<int64_t>(m) * (so.I / 64) + t] = mx;
+        }
     }
 }
 
@@ -1184,7 +1205,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         if constexpr (SILU) {
-            if (warp >= 2 && mbar_wait(bar_red, 0, limit_ns)) {
+            // a warp takes part as a whole (the group maxima are warp shuffles)
+            if (warp >= 2 && __all_sync(0xffffffffu, mbar_wait(bar_red, 0, limit_ns))) {
                 const int etid = threadIdx.x - 64;
                 const int32_t *P = reinterpret_cast<const int32_t *>(smem);
                 // this CTA's tokens only: rows m0 .. m1 - 1 of the summed tile

@@ -711,4 +711,45 @@ __global__ void __launch_bounds__(NCH <= 2 ? 256 : 1024, NCH <= 2 ? 6 : 1) quant
     }
 }
 
+// The same quantization of a when the SiLU*up epilogue has already taken the max |a| of
+// every (token, group of 64 channels) (SiluOut::amax): a token's scale is the max of its I / 64
+// partial maxima divided by 127 (448 for E4M3). The max is exact and order-free, so the scale,
+// and with it every code, is bit-identical to a pass over the whole row. With the row's range
+// known, a row no longer has to sit in one CTA: CTA (x, m) codes the x-th slice of
+// 8 * blockDim values of row m, so a pass over few tokens still spreads over many SMs; the
+// CTAs of slice 0 write the scales.
+template <bool F8 = false>
+__global__ void __launch_bounds__(256) quantize_f32_parts_kernel(
+    const float *__restrict__ a, const float *__restrict__ amax_part, int I, int M,
+    int8_t *__restrict__ q, float *__restrict__ s_tok)
+{
+    __shared__ float sh[32];
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+    pdl_wait(); // a and the maxima come from the previous kernel
+    const int64_t m = blockIdx.y;
+    const int groups = I >> 6;
+    const int nvec = I >> 3;
+    const int v0 = blockIdx.x * blockDim.x;
+    const int vi = v0 + threadIdx.x;
+    // this thread's 8 values, requested before the reduction so that the two overlap
+    float v[1][8];
+    if (vi < nvec) {
+        const float4 *ar = reinterpret_cast<const float4 *>(a + m * I);
+        const float4 lo = __ldcs(ar + 2 * vi);
+        const float4 hi = __ldcs(ar + 2 * vi + 1);
+        v[0][0] = lo.x; v[0][1] = lo.y; v[0][2] = lo.z; v[0][3] = lo.w;
+        v[0][4] = hi.x; v[0][5] = hi.y; v[0][6] = hi.z; v[0][7] = hi.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            v[0][i] = 0.0f;
+    }
+    float mx = 0.0f;
+    for (int j = threadIdx.x; j < groups; j += blockDim.x)
+        mx = fmaxf(mx, __ldcg(amax_part + m * groups + j));
+    mx = block_max(mx, sh);
+    quantize_and_store<1, F8>(v, mx, v0, nvec, q + m * I, blockIdx.x == 0 ? s_tok + m : nullptr);
+}
+
 } // namespace w8a8

@@ -278,6 +278,18 @@ int launch_silu(const uint16_t *gu, int64_t M, int I, int8_t *q, float *s, int t
                          dim3(threads), 0, st, gu, I, static_cast<int>(M), q, s);
 }
 
+template <bool F8 = false>
+int launch_quantize_f32_parts(const float *a, const float *parts, int64_t M, int I, int8_t *q,
+                              float *s, int dev, cudaStream_t st)
+{
+    const void *fn = reinterpret_cast<const void *>(&quantize_f32_parts_kernel<F8>);
+    if (int rc = ensure_smem(fn, dev, 0))
+        return rc;
+    const unsigned slices = static_cast<unsigned>((I / 8 + 255) / 256);
+    return launch_kernel(quantize_f32_parts_kernel<F8>, dim3(slices, static_cast<unsigned>(M)),
+                         dim3(256), 0, st, a, parts, I, static_cast<int>(M), q, s);
+}
+
 template <int NCH, bool F8 = false>
 int launch_quantize_f32(const float *a, int64_t M, int I, int8_t *q, float *s, int threads,
                         int dev, int sms, cudaStream_t st)
@@ -309,6 +321,21 @@ int decode_nt(int64_t M)
 {
     return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
 }
+
+// Bytes of the per-(token, 64-channel group) maxima the fused SiLU*up call keeps in its
+// workspace after the GEMM's own part (small-M plans only), and where they start: never
+// inside the flag words, which every later stream-K call on the same workspace must find zero
+// (the maxima are written before they are read in every call, so they need no clearing).
+size_t silu_parts_off(const GemmPlan &p)
+{
+    const size_t base = p.ws_bytes > kFlagBytes ? p.ws_bytes : kFlagBytes;
+    return (base + 255) & ~static_cast<size_t>(255);
+}
+size_t silu_parts_bytes(const GemmPlan &p, int64_t M, int64_t I)
+{
+    return p.variant == 1 ? 0 : static_cast<size_t>(M) * static_cast<size_t>(I / 64) * 4u;
+}
+
 
 
 int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n, int num_sms,
@@ -923,7 +950,8 @@ size_t w8a8_gemm_silu_quant_workspace_size(int64_t M, int64_t I, int64_t K)
     GemmPlan p;
     if (plan_gemm(M, 2 * I, K, 0, 0, 0, sms, &p))
         return 0;
-    return p.ws_bytes;
+    const size_t parts = silu_parts_bytes(p, M, I);
+    return parts ? silu_parts_off(p) + parts : p.ws_bytes;
 }
 
 int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_il,
@@ -947,13 +975,20 @@ int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_
     GemmPlan p;
     if ((rc = plan_gemm(M, 2 * I, K, 0, 0, 0, sms, &p)))
         return rc;
-    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
+    const size_t parts = silu_parts_bytes(p, M, I);
+    const size_t need = parts ? silu_parts_off(p) + parts : p.ws_bytes;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
         return W8A8_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const SiluOut so{a, static_cast<int>(I)};
+    float *amax = parts ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                    silu_parts_off(p))
+                        : nullptr;
+    const SiluOut so{a, static_cast<int>(I), amax};
     if ((rc = gemm_run(xq, s_tok, wq_il, s_ch_il, M, 2 * I, K, nullptr, nullptr, workspace, p,
                        &so, dev, sms, st)))
         return rc;
+    if (amax) // small M: each token's range from the epilogue's group maxima
+        return launch_quantize_f32_parts(a, amax, M, static_cast<int>(I), q, s_out, dev, st);
     const RowLaunch L = row_launch(I);
     switch (L.nch) {
     case 1: return launch_quantize_f32<1>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
@@ -982,7 +1017,8 @@ size_t w8a8_gemm_silu_quant_fp8_workspace_size(int64_t M, int64_t I, int64_t K)
     GemmPlan p;
     if (plan_silu_fp8(M, I, K, sms, &p))
         return 0;
-    return p.ws_bytes;
+    const size_t parts = silu_parts_bytes(p, M, I);
+    return parts ? silu_parts_off(p) + parts : p.ws_bytes;
 }
 
 int w8a8_gemm_silu_quant_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq_il,
@@ -1006,14 +1042,21 @@ int w8a8_gemm_silu_quant_fp8(const uint8_t *xq, const float *s_tok, const uint8_
     GemmPlan p;
     if ((rc = plan_silu_fp8(M, I, K, sms, &p)))
         return rc;
-    if (p.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < p.ws_bytes))
+    const size_t parts = silu_parts_bytes(p, M, I);
+    const size_t need = parts ? silu_parts_off(p) + parts : p.ws_bytes;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
         return W8A8_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const SiluOut so{a, static_cast<int>(I)};
+    float *amax = parts ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                    silu_parts_off(p))
+                        : nullptr;
+    const SiluOut so{a, static_cast<int>(I), amax};
     if ((rc = gemm_run_fp8(xq, s_tok, wq_il, s_ch_il, M, 2 * I, K, nullptr, nullptr, workspace,
                            p, dev, sms, st, &so)))
         return rc;
     int8_t *qc = reinterpret_cast<int8_t *>(q);
+    if (amax)
+        return launch_quantize_f32_parts<true>(a, amax, M, static_cast<int>(I), qc, s_out, dev, st);
     const RowLaunch L = row_launch(I);
     switch (L.nch) {
     case 1: return launch_quantize_f32<1, true>(a, M, (int)I, qc, s_out, L.threads, dev, sms, st);

@@ -76,6 +76,26 @@ def test_shared_workspace_after_other_stream_k_calls():
     assert np.array_equal(host(q), q_ref)
 
 
+def test_stream_k_after_fused_calls_on_the_same_workspace():
+    """Small-M fused calls keep each token's group maxima in the workspace past its flag
+    words: split stream-K GEMMs issued after them on the same workspace still find their
+    flags zero and give the oracle's result."""
+    ws = w8.Workspace()
+    ws.get(8 << 20)  # one buffer for every call below
+    for M, I, K in ((1, 14336, 4096), (16, 5120, 1024)):  # without and with split-K parts
+        xq, st, wq, sc = _inputs(M, I, K, 5 + M)
+        wq_il, sc_il = prep.interleave_gate_up(dev(wq), dev(sc))
+        w8.w8a8_gemm_silu_quant(dev(xq), dev(st), wq_il, sc_il, workspace=ws)
+        M2, N2, K2 = 16, 20480, 1024
+        assert w8.w8a8_gemm_workspace_size(M2, N2, K2) > 0  # a split stream-K plan
+        xq2, st2, wq2, sc2 = _inputs(M2, N2 // 2, K2, 9 + M)
+        y = w8.w8a8_gemm_dequant(dev(xq2), dev(st2), dev(wq2), dev(sc2), workspace=ws)
+        torch.cuda.synchronize()
+        y_ref, _ = oracle.gemm_dequant(xq2, st2, wq2, sc2, want_acc=False)
+        assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), y_ref)
+    assert w8.w8a8_device_status(reset=True) == 0
+
+
 def test_interleave_is_a_row_permutation():
     I, K = 192, 32
     wq = torch.arange(2 * I, dtype=torch.int32).repeat_interleave(K).view(2 * I, K)
