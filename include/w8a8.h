@@ -156,7 +156,11 @@ W8A8_API size_t w8a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * Small M (at most 64 tokens by default, up to 256 on request) runs a swap-AB kernel that
  * streams the weight: split-K over thread-block clusters (partials summed in distributed
  * shared memory) when the weight has few 128-channel blocks, persistent stream-K over all SMs
- * otherwise; larger M runs a persistent tile kernel. All give identical results.
+ * otherwise; larger M runs a persistent tile kernel (256 x 256 tiles on CTA pairs, or 128-row
+ * tiles), which splits the tiles' k-blocks evenly over the CTA pairs (stream-K: a tile shared
+ * by several pairs is finished by the one holding its first k-blocks, after adding the
+ * others' int32 partials from the workspace) when there are few, long tiles (at most one per
+ * two CTA pairs, K >= 8192). All give identical results.
  */
 W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_t *wq,
                       const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
@@ -170,10 +174,12 @@ W8A8_API int w8a8_gemm_dequant(const int8_t *xq, const float *s_tok, const int8_
  * the tokens are taken 256 at a time, each channel block once per such tile). ctas:
  * variant 2 = persistent CTAs sharing the weight stream (0 = one per SM, at most one per SM);
  * variant 3 = cluster size, the number of K splits per 128-channel block (0 = automatic,
- * at most 8, fewer if the clusters would not all fit on the GPU at once). tile_n (variant 1)
- * = 0 automatic, 128 (128 x 128 output tiles), 256 (128 x 256) or 512 (256 x 256). The
- * workspace needed is w8a8_gemm_workspace_size_ex() of the same arguments (only variant 2
- * uses one).
+ * at most 8, fewer if the clusters would not all fit on the GPU at once); variant 1 with
+ * tile_n 512 = CTA pairs of the stream-K schedule (0 = whole tiles; at most one pair per two
+ * SMs, and at most three pairs per tile so that a split tile has at most three later pieces).
+ * tile_n (variant 1) = 0 automatic, 128 (128 x 128 output tiles), 256 (128 x 256) or 512
+ * (256 x 256). The workspace needed is w8a8_gemm_workspace_size_ex() of the same arguments
+ * (variant 2, and variant 1 on the stream-K schedule, use one).
  */
 W8A8_API int w8a8_gemm_dequant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
                          const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,

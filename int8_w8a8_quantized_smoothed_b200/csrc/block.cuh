@@ -122,10 +122,6 @@ __device__ __forceinline__ void st_release_cta_shared(uint32_t *p, uint32_t v)
     asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_global()
-{
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 // Waits (bounded) until the barrier counter reaches target; false if the wait ran out.
 __device__ __forceinline__ bool grid_wait(const unsigned long long *bar, unsigned long long target,

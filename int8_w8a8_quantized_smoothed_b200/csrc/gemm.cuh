@@ -402,26 +402,77 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ---------------------------------------------------------------- prefill, CTA pairs
 
+// ---- stream-K: U units split evenly over G workers, worker g taking [g U / G, (g+1) U / G)
+
+// CTA holding unit v under the even split of U units over G CTAs.
+__host__ __device__ __forceinline__ int64_t sk_owner_of(int64_t v, int64_t U, int64_t G)
+{
+    int64_t c = (v * G) / U;
+    while (c + 1 < G && ((c + 1) * U) / G <= v)
+        ++c;
+    while (c > 0 && (c * U) / G > v)
+        --c;
+    return c;
+}
+
+struct SkSegment {
+    int64_t t;    // block (decode: channel block t / tiles, token tile t % tiles) or tile
+    int kb0, kb1; // k-block range [kb0, kb1)
+};
+
+// The segment of [u, u1) that starts at u.
+__device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
+{
+    SkSegment sg;
+    sg.t = u / KB;
+    sg.kb0 = static_cast<int>(u - sg.t * KB);
+    const int64_t left = u1 - u;
+    sg.kb1 = static_cast<int>(min(static_cast<int64_t>(KB), sg.kb0 + left));
+    return sg;
+}
+
 template <int STAGES> struct PairCfg {
     static constexpr int kHalf = 128;             // rows of A and of B per CTA
     static constexpr int kABytes = kHalf * kBK;   // 16 KB
     static constexpr int kBBytes = kHalf * kBK;   // 16 KB
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kBarOff = STAGES * kStageBytes;
-    static constexpr int kSchOff = (kBarOff + (2 * STAGES + 4) * 8 + 16 + 15) & ~15;
+    // full[S], empty[S], tmem_full[2], tmem_empty[2], tmem slot (16 B), the stream-K fixup
+    // barrier and a word for the epilogue group
+    static constexpr int kFixBarOff = kBarOff + (2 * STAGES + 4) * 8 + 16;
+    static constexpr int kSchOff = (kFixBarOff + 16 + 15) & ~15;
     static constexpr int kSmemBytes = kSchOff + 4 * 2 * 256 * 4 + 1024; // + scales [4][2][256]
     static constexpr int kTmemCols = 512;         // two 128 x 256 accumulators per CTA
+    // stream-K: a CTA's partial of a split tile, 128 rows x 256 columns of accumulator words,
+    // stored as [64 column quads][128 rows][4] so that the rows of a warp are consecutive
+    static constexpr int kPartBytes = kHalf * 256 * 4;
+    static constexpr int kPartHalf = kPartBytes / 2; // columns 0..127 or 128..255
+    static constexpr int kMaxContrib = 3;            // contributors per split tile
+    static_assert(kMaxContrib * kPartHalf <= STAGES * kStageBytes,
+                  "the fixup stages contributor halves in the idle ring");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
+// Persistent 256 x 256 tiles on CTA pairs (cta_group::2). Two schedules:
+//   tile-persistent (ws_flag == nullptr): pair p takes tiles p, p + P, ...;
+//   stream-K (ws_flag != nullptr): the tiles x k-blocks units are split evenly over the P
+//     pairs; a pair walks its range in segments (the part inside one tile). A tile split
+//     between pairs is finished by its owner, the pair holding its k-block 0 (that segment is
+//     the owner's last, so it completes last); the later pairs sharing the tile (at most
+//     kMaxContrib; the host sizes shares so) store their int32 partial (binary32 for FP8)
+//     halves in their CTA's workspace slot and raise the CTA's flag. The owner, whose ring is
+//     idle by then, brings the contributors' column halves into it with bulk copies, adds
+//     them to its accumulator chunk by chunk and finishes the tile; it lowers the flags, so
+//     the workspace is ready for the next call.
 template <int STAGES, bool SILU = false, bool F8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmB,
                              const float *__restrict__ s_tok, const float *__restrict__ s_ch,
                              int M, int N, int K, uint16_t *__restrict__ y,
-                             int32_t *__restrict__ acc_out, SiluOut so, int prefetch_static,
-                             unsigned long long limit_ns)
+                             int32_t *__restrict__ acc_out, SiluOut so,
+                             int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
+                             int prefetch_static, unsigned long long limit_ns)
 {
     using Cfg = PairCfg<STAGES>;
     constexpr int TN = 256, TM = 256;
@@ -436,7 +487,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t bar_tfull = bar_empty + 8 * STAGES;  // both CTAs
     const uint32_t bar_tempty = bar_tfull + 16;         // used in the even CTA
     const uint32_t tslot = bar_tempty + 16;
+    const uint32_t bar_fix = sbase + Cfg::kFixBarOff;
     uint32_t *tslot_ptr = reinterpret_cast<uint32_t *>(smem + Cfg::kBarOff + (2 * STAGES + 4) * 8);
+    volatile uint32_t *sh_word = reinterpret_cast<volatile uint32_t *>(smem + Cfg::kFixBarOff + 8);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -447,6 +500,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int num_n = (N + TN - 1) / TN;
     const int tiles = num_m * num_n;
     const int kblocks = (K + kBK - 1) / kBK;
+    const bool sk = ws_flag != nullptr;
+    const int64_t U = static_cast<int64_t>(tiles) * kblocks;
+    const int64_t u_begin = sk ? (static_cast<int64_t>(pair) * U) / npairs : pair;
+    const int64_t u_end = sk ? (static_cast<int64_t>(pair + 1) * U) / npairs : tiles;
+    // The segments of this pair's work, in order: (tile, k-blocks [kb0, kb1)). cursor starts
+    // at u_begin; every role walks the same sequence.
+    auto next_seg = [&](int64_t &cursor, int &t, int &kb0, int &kb1) -> bool {
+        if (cursor >= u_end)
+            return false;
+        if (sk) {
+            const SkSegment sg = sk_segment(cursor, u_end, kblocks);
+            t = static_cast<int>(sg.t);
+            kb0 = sg.kb0;
+            kb1 = sg.kb1;
+            cursor += kb1 - kb0;
+        } else {
+            t = static_cast<int>(cursor);
+            kb0 = 0;
+            kb1 = kblocks;
+            cursor += npairs;
+        }
+        return true;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -457,6 +533,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(bar_tfull + 8 * b, 1);
             mbar_init(bar_tempty + 8 * b, 8); // 4 epilogue warps in each CTA of the pair
         }
+        mbar_init(bar_fix, 1);
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -480,10 +557,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t full0 = map_peer_smem(bar_full, 0); // the leader's full barriers
             uint32_t npre = 0;
             if (prefetch_static) {
-                for (int tile = pair; tile < tiles && npre < STAGES; tile += npairs) {
+                int64_t cur = u_begin;
+                int t, kb0, kb1;
+                while (npre < STAGES && next_seg(cur, t, kb0, kb1)) {
                     int mb, nb;
-                    tile_coords(tile, num_m, num_n, mb, nb);
-                    for (int kb = 0; kb < kblocks && npre < STAGES; ++kb, ++npre) {
+                    tile_coords(t, num_m, num_n, mb, nb);
+                    for (int kb = kb0; kb < kb1 && npre < STAGES; ++kb, ++npre) {
                         if (rank == 0)
                             mbar_expect_tx(bar_full + 8 * npre, 2 * Cfg::kStageBytes);
                         tma_load_2d_pair(sB + npre * Cfg::kBBytes, &tmB, full0 + 8 * npre,
@@ -493,11 +572,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             pdl_wait();
             uint32_t it = 0;
-            for (int tile = pair; tile < tiles; tile += npairs) {
+            bool ok = true;
+            int64_t cur = u_begin;
+            int t, kb0, kb1;
+            while (ok && next_seg(cur, t, kb0, kb1)) {
                 int mb, nb;
-                tile_coords(tile, num_m, num_n, mb, nb);
-                bool ok = true;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                tile_coords(t, num_m, num_n, mb, nb);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const uint32_t s = it % STAGES;
                     if (it < npre) {
                         tma_load_2d_pair(sA + s * Cfg::kABytes, &tmA, full0 + 8 * s, kb * kBK,
@@ -516,29 +597,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tma_load_2d_pair(sB + s * Cfg::kBBytes, &tmB, full0 + 8 * s, kb * kBK,
                                      nb * TN + rank * Cfg::kHalf);
                 }
-                if (!ok) {
-                    it = 0; // leave the tail: a stage wait already ran out
-                    break;
-                }
             }
             // Producer tail (each CTA): the leader's multicast commits have released every
-            // stage of this CTA's ring before it may exit.
-            drain_ring(bar_empty, it, STAGES, limit_ns);
+            // stage of this CTA's ring before it may exit (a stage wait that ran out leaves
+            // it at once).
+            if (ok)
+                drain_ring(bar_empty, it, STAGES, limit_ns);
             pdl_launch_dependents(); // the pair's main loop is done in this CTA
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
             constexpr uint32_t idesc = idesc_8bit<F8>(TM, TN);
-            uint32_t it = 0, t = 0;
+            uint32_t it = 0, seg = 0;
             bool ok = true;
-            for (int tile = pair; tile < tiles && ok; tile += npairs, ++t) {
-                const uint32_t buf = t & 1u;
-                const uint32_t aph = (t >> 1) & 1u;
+            int64_t cur = u_begin;
+            int t, kb0, kb1;
+            while (ok && next_seg(cur, t, kb0, kb1)) {
+                const uint32_t buf = seg & 1u;
+                const uint32_t aph = (seg >> 1) & 1u;
+                ++seg;
                 if (!mbar_wait(bar_tempty + 8 * buf, aph ^ 1u, limit_ns))
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * TN;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const uint32_t s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
                     if (!mbar_wait(bar_full + 8 * s, ph, limit_ns)) {
@@ -552,7 +634,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int k = 0; k < kBK / kUmmaK; ++k)
                         umma_8bit_pair<F8>(d, sw128_kmajor_desc(a0 + k * kUmmaK),
                                            sw128_kmajor_desc(b0 + k * kUmmaK), idesc,
-                                     (kb > 0 || k > 0) ? 1u : 0u);
+                                           (kb > kb0 || k > 0) ? 1u : 0u);
                     umma_commit_pair(bar_empty + 8 * s, 0x3); // frees the stage in both CTAs
                 }
                 if (ok)
@@ -563,59 +645,164 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // epilogue warps 2..5: this CTA's 128 accumulator rows of the 256-row tile
         pdl_wait();
         const int quarter = warp & 3;
+        const int etid = threadIdx.x - 64;
+        const int rl = quarter * 32 + lane; // row within this CTA's half of the tile
         const uint32_t tempty0 = map_peer_smem(bar_tempty, 0);
-        const int row_in_tile = static_cast<int>(rank) * Cfg::kHalf + quarter * 32 + lane;
+        const int row_in_tile = static_cast<int>(rank) * Cfg::kHalf + rl;
         float *sh_sch = reinterpret_cast<float *>(smem + Cfg::kSchOff) + (warp - 2) * 2 * TN;
+        const int4 *ring = reinterpret_cast<const int4 *>(smem);
+        int4 *my_slot = sk ? reinterpret_cast<int4 *>(ws_part) +
+                                 static_cast<int64_t>(blockIdx.x) * (Cfg::kPartBytes / 16)
+                           : nullptr;
         TileScales<TN> nxt;
         auto fetch = [&](int tile) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
             nxt.fetch(s_ch, s_tok, nb * TN, N, mb * TM + row_in_tile, M, lane);
         };
-        if (pair < tiles)
-            fetch(pair);
-        uint32_t t = 0;
-        for (int tile = pair; tile < tiles; tile += npairs, ++t) {
+        int64_t peek = u_begin, cur = u_begin;
+        int pt, pk0, pk1, t, kb0, kb1;
+        if (next_seg(peek, pt, pk0, pk1))
+            fetch(pt);
+        uint32_t seg = 0;
+        while (next_seg(cur, t, kb0, kb1)) {
             int mb, nb;
-            tile_coords(tile, num_m, num_n, mb, nb);
-            const uint32_t buf = t & 1u;
-            const uint32_t aph = (t >> 1) & 1u;
-            // this tile's scales to the warp's shared memory, the next tile's requested
+            tile_coords(t, num_m, num_n, mb, nb);
+            const uint32_t buf = seg & 1u;
+            const uint32_t aph = (seg >> 1) & 1u;
+            ++seg;
+            // this segment's scales to the warp's shared memory, the next segment's requested
             nxt.publish(sh_sch + buf * TN, lane);
             const float st = nxt.st;
-            if (tile + npairs < tiles)
-                fetch(tile + npairs);
+            if (next_seg(peek, pt, pk0, pk1))
+                fetch(pt);
             if (!mbar_wait(bar_tfull + 8 * buf, aph, limit_ns))
                 break;
             tc_fence_after();
-            const int row = mb * TM + row_in_tile;
-            const bool row_ok = row < M;
             const uint32_t tbase = tmem_base + buf * TN + (static_cast<uint32_t>(quarter * 32) << 16);
-            if constexpr (SILU) {
-#pragma unroll 1
-                for (int p = 0; p < TN / 64; ++p) {
-                    const int cg = (p >> 1) * 4 + (p & 1);
-                    const int ch0 = nb * (TN / 2) + (p >> 1) * 64 + (p & 1) * 32;
-                    uint32_t rg[32], ru[32];
-                    tmem_ld_32x32b_x32(tbase + cg * 32, rg);
-                    tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
-                    tmem_ld_wait();
-                    if (row_ok && ch0 < so.I)
-                        silu_row_chunk<F8>(rg, ru, st, sh_sch + buf * TN + cg * 32,
-                                       sh_sch + buf * TN + (cg + 2) * 32,
-                                       so.a + static_cast<int64_t>(row) * so.I + ch0);
-                }
-            } else {
+            if (kb0 > 0) {
+                // a later piece of a split tile: the partial to this CTA's slot, then its flag
 #pragma unroll 1
                 for (int c = 0; c < TN / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, r);
                     tmem_ld_wait();
-                    if (row_ok)
-                        store_row_chunk<F8>(r, row, nb * TN + c * 32, N, st,
-                                        sh_sch + buf * TN + c * 32, y, acc_out);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        __stcg(my_slot + (c * 8 + i) * Cfg::kHalf + rl,
+                               make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_cluster(tempty0 + 8 * buf);
+                named_bar_sync(1, 128);
+                if (etid == 0) {
+                    fence_acq_rel_gpu();
+                    st_relaxed_gpu(ws_flag + blockIdx.x, 1u);
+                }
+                continue;
             }
+            // The tile's first piece: whole, or owned with ncon later pieces to add.
+            int ncon = 0;
+            if (kb1 < kblocks) {
+                ncon = static_cast<int>(
+                    sk_owner_of(static_cast<int64_t>(t) * kblocks + kblocks - 1, U, npairs) - pair);
+                if (etid == 0) {
+                    bool all = true;
+                    for (int j = 1; j <= ncon && all; ++j) {
+                        const unsigned int *f = ws_flag + 2 * (pair + j) + rank;
+                        if (ld_acquire_gpu(f) == 0u) {
+                            const uint64_t t0 = globaltimer_ns();
+                            while (ld_acquire_gpu(f) == 0u) {
+                                if (globaltimer_ns() - t0 > limit_ns) {
+                                    flag_timeout();
+                                    all = false;
+                                    break;
+                                }
+                            }
+                        }
+                    }
+                    fence_proxy_async_global(); // the partials came from generic stores
+                    *sh_word = all ? 1u : 0u;
+                }
+                named_bar_sync(1, 128);
+                if (*sh_word == 0u)
+                    ncon = -1; // a wait ran out: leave the tile unwritten
+            }
+            const int row = mb * TM + row_in_tile;
+            const bool row_ok = row < M && ncon >= 0;
+            // nadd is uniform over the epilogue group (it guards a named barrier); a fixup wait
+            // that runs out only keeps this thread from storing
+            const int nadd = ncon > 0 ? ncon : 0;
+            // adds the contributors' words of chunk c (staged in the ring for half h) to r
+            auto add_parts = [&](uint32_t (&r)[32], int c, int h) {
+                for (int j = 0; j < nadd; ++j) {
+                    const int4 *src = ring + j * (Cfg::kPartHalf / 16) +
+                                      (c * 8 - h * 32) * Cfg::kHalf + rl;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int4 v = src[i * Cfg::kHalf];
+                        r[4 * i] = acc_add<F8>(r[4 * i], static_cast<uint32_t>(v.x));
+                        r[4 * i + 1] = acc_add<F8>(r[4 * i + 1], static_cast<uint32_t>(v.y));
+                        r[4 * i + 2] = acc_add<F8>(r[4 * i + 2], static_cast<uint32_t>(v.z));
+                        r[4 * i + 3] = acc_add<F8>(r[4 * i + 3], static_cast<uint32_t>(v.w));
+                    }
+                }
+            };
+            for (int h = 0; h < 2; ++h) {
+                bool ok_h = ncon >= 0;
+                if (nadd > 0) {
+                    // the contributors' column half h into the (idle) ring
+                    if (etid == 0) {
+                        fence_proxy_async_smem(); // earlier reads of the ring, before the copies
+                        mbar_expect_tx(bar_fix, static_cast<uint32_t>(ncon) * Cfg::kPartHalf);
+                        for (int j = 0; j < ncon; ++j)
+                            bulk_load_g2s(sbase + j * Cfg::kPartHalf,
+                                          ws_part + (static_cast<int64_t>(2 * (pair + 1 + j) + rank) *
+                                                         Cfg::kPartBytes + h * Cfg::kPartHalf) / 4,
+                                          Cfg::kPartHalf, bar_fix);
+                    }
+                    if (!mbar_wait(bar_fix, static_cast<uint32_t>(h), limit_ns))
+                        ok_h = false;
+                }
+                if constexpr (SILU) {
+#pragma unroll 1
+                    for (int p = 2 * h; p < 2 * h + 2; ++p) {
+                        const int cg = (p >> 1) * 4 + (p & 1);
+                        const int ch0 = nb * (TN / 2) + (p >> 1) * 64 + (p & 1) * 32;
+                        uint32_t rg[32], ru[32];
+                        tmem_ld_32x32b_x32(tbase + cg * 32, rg);
+                        tmem_ld_32x32b_x32(tbase + (cg + 2) * 32, ru);
+                        tmem_ld_wait();
+                        if (nadd > 0) {
+                            add_parts(rg, cg, h);
+                            add_parts(ru, cg + 2, h);
+                        }
+                        if (row_ok && ok_h && ch0 < so.I)
+                            silu_row_chunk<F8>(rg, ru, st, sh_sch + buf * TN + cg * 32,
+                                               sh_sch + buf * TN + (cg + 2) * 32,
+                                               so.a + static_cast<int64_t>(row) * so.I + ch0);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = 4 * h; c < 4 * h + 4; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tbase + c * 32, r);
+                        tmem_ld_wait();
+                        if (nadd > 0)
+                            add_parts(r, c, h);
+                        if (row_ok && ok_h)
+                            store_row_chunk<F8>(r, row, nb * TN + c * 32, N, st,
+                                                sh_sch + buf * TN + c * 32, y, acc_out);
+                    }
+                }
+                if (nadd > 0)
+                    named_bar_sync(1, 128); // every thread is done with this half in the ring
+            }
+            if (ncon > 0 && etid == 0) // the contributors' flags down for the next call
+                for (int j = 1; j <= ncon; ++j)
+                    st_relaxed_gpu(ws_flag + 2 * (pair + j) + rank, 0u);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -684,32 +871,6 @@ template <int NT, int STAGES, int KPS, bool CLUSTER> struct DecodeCfg {
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
-// CTA holding unit v under the even split of U units over G CTAs.
-__host__ __device__ __forceinline__ int64_t sk_owner_of(int64_t v, int64_t U, int64_t G)
-{
-    int64_t c = (v * G) / U;
-    while (c + 1 < G && ((c + 1) * U) / G <= v)
-        ++c;
-    while (c > 0 && (c * U) / G > v)
-        --c;
-    return c;
-}
-
-struct SkSegment {
-    int64_t t;    // block: channel block t / tiles, token tile t % tiles
-    int kb0, kb1; // k-block range [kb0, kb1)
-};
-
-// The segment of [u, u1) that starts at u.
-__device__ __forceinline__ SkSegment sk_segment(int64_t u, int64_t u1, int KB)
-{
-    SkSegment sg;
-    sg.t = u / KB;
-    sg.kb0 = static_cast<int>(u - sg.t * KB);
-    const int64_t left = u1 - u;
-    sg.kb1 = static_cast<int>(min(static_cast<int64_t>(KB), sg.kb0 + left));
-    return sg;
-}
 
 // The SiLU*up form of the final step of a block (see SiluOut): the block's 128 weight rows
 // are gate rows 0..63 and up rows 64..127 of output channels [64 t, 64 t + 64); v8 = (token,

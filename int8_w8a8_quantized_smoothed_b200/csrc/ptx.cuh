@@ -457,6 +457,24 @@ __device__ __forceinline__ void bulk_reduce_add_s32_peer(uint32_t dst_cluster, u
                  : "memory");
 }
 
+// Global data written by the generic proxy (ordinary stores, made visible by an acquire),
+// before an async-proxy (bulk copy / TMA) read of it.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global memory into
+// this CTA's shared memory, completing `bar`'s transaction count.
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -308,6 +308,7 @@ struct GemmPlan {
     int tile_n = 256;  // prefill tile width
     int nt = 16;       // decode token tile
     int ctas = 1;      // stream-K persistent grid, or cluster size
+    int sk_pairs = 0;  // pair tile kernel: stream-K over this many CTA pairs (0: whole tiles)
     size_t ws_bytes = 0;
     size_t flag_off = 0;
     size_t part_off = 0;
@@ -316,6 +317,8 @@ struct GemmPlan {
 // stream-K workspace: one flag word per CTA (at most kMaxCtas) in the first kFlagBytes
 constexpr int kMaxCtas = 1024;
 constexpr size_t kFlagBytes = kMaxCtas * 4;
+// the pair tile kernel's partial slot per CTA (128 x 256 accumulator words)
+constexpr size_t kPairPartBytes = 128 * 256 * 4;
 
 int decode_nt(int64_t M)
 {
@@ -375,9 +378,32 @@ int plan_gemm(int64_t M, int64_t N, int64_t K, int variant, int ctas, int tile_n
                 }
             }
             tile_n = best == 0 ? 128 : best == 1 ? 256 : 512;
+            // Stream-K over the pairs for few, long tiles: at most half the pairs would have a
+            // whole tile, each of at least 64 k-blocks. Every pair then takes an equal share
+            // of the tiles' k-blocks; a split tile's owner adds the later pieces at its end,
+            // a fixed cost of a few microseconds that only tiles this long amortize
+            // (measured: 512 x 4096 x 14336 38.3 -> 34.0 us; with K = 4096 stream-K was
+            // slower than whole tiles at M = 512 and 2048).
+            const int64_t P = num_sms / 2;
+            const int64_t tp = ((M + 255) / 256) * ((N + 255) / 256);
+            if (2 * tp <= P && KB >= 64) {
+                tile_n = 512;
+                ctas = static_cast<int>(P);
+            }
         }
         p->tile_n = tile_n;
         p->ws_bytes = 0;
+        if (tile_n == 512 && ctas > 0) {
+            // at most kMaxContrib (3) later pieces per split tile: shares of >= KB / 3 units
+            const int64_t tp = ((M + 255) / 256) * ((N + 255) / 256);
+            int64_t P = ctas < num_sms / 2 ? ctas : num_sms / 2;
+            if (P > 3 * tp)
+                P = 3 * tp;
+            p->sk_pairs = static_cast<int>(P < 1 ? 1 : P);
+            p->flag_off = 0;
+            p->part_off = kFlagBytes;
+            p->ws_bytes = kFlagBytes + static_cast<size_t>(2 * p->sk_pairs) * kPairPartBytes;
+        }
         return W8A8_OK;
     }
     p->nt = decode_nt(M);
@@ -487,9 +513,11 @@ int pair_clusters(const void *kernel, int smem, int dev, int num_sms)
 template <int STAGES, bool SILU, bool F8 = false>
 int launch_prefill_pair(const CUtensorMap &ta, const CUtensorMap &tb, const float *s_tok,
                         const float *s_ch, int64_t M, int64_t N, int64_t K, uint16_t *y,
-                        int32_t *acc, const SiluOut &so, int dev, int num_sms, cudaStream_t st)
+                        int32_t *acc, const SiluOut &so, const GemmPlan &p, void *ws, int dev,
+                        int num_sms, cudaStream_t st)
 {
     using Cfg = PairCfg<STAGES>;
+    static_assert(Cfg::kPartBytes == kPairPartBytes, "pair partial slot");
     auto kernel = gemm_prefill_pair_kernel<STAGES, SILU, F8>;
     int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes);
     if (rc)
@@ -497,13 +525,21 @@ int launch_prefill_pair(const CUtensorMap &ta, const CUtensorMap &tb, const floa
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
     int64_t pairs = pair_clusters(reinterpret_cast<const void *>(kernel), Cfg::kSmemBytes, dev,
                                   num_sms);
-    if (pairs > tiles)
+    int32_t *ws_part = nullptr;
+    unsigned int *ws_flag = nullptr;
+    if (p.sk_pairs > 0) { // stream-K: every pair resident, each with a partial slot
+        if (pairs > p.sk_pairs)
+            pairs = p.sk_pairs;
+        ws_part = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + p.part_off);
+        ws_flag = reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.flag_off);
+    } else if (pairs > tiles) {
         pairs = tiles;
+    }
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
     return launch_kernel_cluster(kernel, dim3(static_cast<unsigned>(2 * pairs)),
                                  dim3(kGemmThreads), Cfg::kSmemBytes, st, 2u, ta, tb, s_tok, s_ch,
                                  static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), y,
-                                 acc, so, prefetch, kWaitLimitNs);
+                                 acc, so, ws_part, ws_flag, prefetch, kWaitLimitNs);
 }
 
 // Largest cluster size <= want whose clusters can all be resident at once (one wave).
@@ -615,13 +651,13 @@ int gemm_run_fp8(const uint8_t *xq, const float *s_tok, const uint8_t *wq, const
             return W8A8_ERR_CUDA;
         if (so) {
             if (p.tile_n == 512)
-                return launch_prefill_pair<6, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, dev, sms, st);
+                return launch_prefill_pair<6, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, p, workspace, dev, sms, st);
             if (p.tile_n == 256)
                 return launch_prefill<256, 4, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, dev, sms, st);
             return launch_prefill<128, 6, true, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, *so, dev, sms, st);
         }
         if (p.tile_n == 512)
-            return launch_prefill_pair<6, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
+            return launch_prefill_pair<6, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, p, workspace, dev, sms, st);
         if (p.tile_n == 256)
             return launch_prefill<256, 4, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
         return launch_prefill<128, 6, false, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc, none, dev, sms, st);
@@ -649,13 +685,13 @@ int gemm_run(const int8_t *xq, const float *s_tok, const int8_t *wq, const float
             return W8A8_ERR_CUDA;
         if (so) {
             if (p.tile_n == 512)
-                return launch_prefill_pair<6, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, dev, sms, st);
+                return launch_prefill_pair<6, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, p, workspace, dev, sms, st);
             if (p.tile_n == 256)
                 return launch_prefill<256, 4, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, dev, sms, st);
             return launch_prefill<128, 6, true>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, *so, dev, sms, st);
         }
         if (p.tile_n == 512)
-            return launch_prefill_pair<6, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, dev, sms, st);
+            return launch_prefill_pair<6, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, p, workspace, dev, sms, st);
         if (p.tile_n == 256)
             return launch_prefill<256, 4, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, dev, sms, st);
         return launch_prefill<128, 6, false>(ta, tb, s_tok, s_ch, M, N, K, y, acc_out, none, dev, sms, st);

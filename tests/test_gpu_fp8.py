@@ -169,7 +169,11 @@ def _check_gemm(xq, s_tok, wq, s_ch, variant=0, ctas=0, tile_n=0, exact=False):
 
 
 GEMM_CASES = [
-    # (M, N, K, variant, ctas, tile_n)
+    # (M, N, K, variant, ctas, tile_n); tile_n 512 with ctas > 0: stream-K over that many
+    # CTA pairs (binary32 partials of split tiles added by the owner pair)
+    (300, 1000, 512, 1, 24, 512),
+    (512, 4096, 4096, 1, 74, 512),
+    (257, 264, 4112, 1, 5, 512),
     (1, 4096, 4096, 0, 0, 0),
     (16, 6144, 4096, 0, 0, 0),
     (37, 1024, 4112, 2, 0, 0),

@@ -96,6 +96,21 @@ def test_stream_k_after_fused_calls_on_the_same_workspace():
     assert w8.w8a8_device_status(reset=True) == 0
 
 
+@pytest.mark.parametrize("M,I,K", [(512, 2048, 8192), (300, 512, 16384), (257, 640, 8208)])
+def test_fused_silu_on_pair_stream_k(M, I, K):
+    """The SiLU*up epilogue on split tiles (these shapes plan stream-K over CTA pairs: few
+    tiles, K >= 8192): the owner pair adds the later pieces before it forms a."""
+    assert w8.w8a8_gemm_workspace_size(M, 2 * I, K) > 0
+    xq, st, wq, sc = _inputs(M, I, K, seed=M + I)
+    a_ref, q_ref, s_ref = _reference(xq, st, wq, sc)
+    wq_il, sc_il = prep.interleave_gate_up(dev(wq), dev(sc))
+    for _ in range(2):
+        q, s, a = w8.w8a8_gemm_silu_quant(dev(xq), dev(st), wq_il, sc_il)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(a).view(np.uint32), a_ref.view(np.uint32))
+        assert np.array_equal(host(q), q_ref) and np.array_equal(host(s), s_ref)
+
+
 def test_interleave_is_a_row_permutation():
     I, K = 192, 32
     wq = torch.arange(2 * I, dtype=torch.int32).repeat_interleave(K).view(2 * I, K)

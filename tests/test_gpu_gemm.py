@@ -229,3 +229,32 @@ def test_overlap_modes_give_identical_results(M):
     finally:
         w8.w8a8_set_overlap(prev)
     assert w8.w8a8_device_status(reset=True) == 0
+
+
+# Stream-K on the CTA-pair tile kernel (variant 1, tile_n 512, ctas = pairs): tiles split
+# between pairs are finished by the pair holding their first k-blocks after adding up to three
+# later pieces staged through its idle ring. Pair counts that leave 1..3 contributors per
+# tile, pairs with empty shares (tiny K), ragged M, N and K tails, and repeated calls on one
+# workspace (the owners lower the contributors' flags).
+PAIR_SK_CASES = [(300, 1000, 512, 24), (300, 1000, 512, 5), (257, 264, 4112, 5),
+                 (512, 4096, 4096, 74), (512, 4096, 14336, 74), (512, 6144, 4096, 74),
+                 (129, 264, 16, 6), (520, 256, 1024, 9), (65, 512, 4096, 6),
+                 (1000, 4096, 256, 74), (600, 1032, 1040, 37), (256, 256, 384, 3)]
+
+
+@pytest.mark.parametrize("M,N,K,pairs", PAIR_SK_CASES)
+def test_pair_stream_k_bit_exact(M, N, K, pairs):
+    xq, st, wq, sc = _inputs(M, N, K, seed=M + 2 * N + K)
+    y_ref, acc_ref = oracle.gemm_dequant(xq, st, wq, sc)
+    for _ in range(2):
+        y, acc = _run(xq, st, wq, sc, variant=1, ctas=pairs, tile_n=512)
+        _compare(y, acc, y_ref, acc_ref)
+    assert w8.w8a8_device_status(reset=True) == 0
+
+
+def test_pair_stream_k_is_the_plan_for_few_long_tiles():
+    # the M = 512 decoder block's down projection: 32 tiles of 112 k-blocks on 74 pairs
+    assert w8.w8a8_gemm_workspace_size(512, 4096, 14336) > 0
+    # short tiles, or tiles that fill the pairs, keep the whole-tile schedules
+    assert w8.w8a8_gemm_workspace_size(512, 6144, 4096) == 0
+    assert w8.w8a8_gemm_workspace_size(8192, 28672, 4096) == 0
