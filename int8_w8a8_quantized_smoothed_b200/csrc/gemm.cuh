@@ -73,12 +73,51 @@ __device__ __forceinline__ void silu_row_chunk(const uint32_t (&rg)[32], const u
         const float cu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            g[i] = bf16_round(dequant_acc<F8>(rg[8 * e + i], st, cg[i]));
-            u[i] = bf16_round(dequant_acc<F8>(ru[8 * e + i], st, cu[i]));
+            g[i] = dequant_acc<F8>(rg[8 * e + i], st, cg[i]);
+            u[i] = dequant_acc<F8>(ru[8 * e + i], st, cu[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) { // to bf16 and back, two values per conversion
+            bf16_round2(g[i], g[i + 1]);
+            bf16_round2(u[i], u[i + 1]);
         }
         silu_mul8(g, u, a);
         reinterpret_cast<float4 *>(dst)[2 * e] = make_float4(a[0], a[1], a[2], a[3]);
         reinterpret_cast<float4 *>(dst)[2 * e + 1] = make_float4(a[4], a[5], a[6], a[7]);
+    }
+}
+
+// silu_row_chunk's 32 values of a, as 8 16-byte words instead of stores.
+template <bool F8 = false>
+__device__ __forceinline__ void silu_row_chunk_regs(const uint32_t (&rg)[32],
+                                                    const uint32_t (&ru)[32], float st,
+                                                    const float *scg, const float *scu,
+                                                    uint4 (&out)[8])
+{
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float g[8], u[8], a[8];
+        const float4 g0 = reinterpret_cast<const float4 *>(scg)[2 * e];
+        const float4 g1 = reinterpret_cast<const float4 *>(scg)[2 * e + 1];
+        const float4 u0 = reinterpret_cast<const float4 *>(scu)[2 * e];
+        const float4 u1 = reinterpret_cast<const float4 *>(scu)[2 * e + 1];
+        const float cg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float cu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            g[i] = dequant_acc<F8>(rg[8 * e + i], st, cg[i]);
+            u[i] = dequant_acc<F8>(ru[8 * e + i], st, cu[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) { // to bf16 and back, two values per conversion
+            bf16_round2(g[i], g[i + 1]);
+            bf16_round2(u[i], u[i + 1]);
+        }
+        silu_mul8(g, u, a);
+        out[2 * e] = make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]),
+                                __float_as_uint(a[2]), __float_as_uint(a[3]));
+        out[2 * e + 1] = make_uint4(__float_as_uint(a[4]), __float_as_uint(a[5]),
+                                    __float_as_uint(a[6]), __float_as_uint(a[7]));
     }
 }
 
@@ -166,6 +205,62 @@ __device__ __forceinline__ void store_row_chunk(const uint32_t (&r)[32], int row
             }
         }
     }
+}
+
+// The bf16 words of 32 dequantized accumulator columns of one output row (4 x 16 bytes).
+template <bool F8>
+__device__ __forceinline__ void dequant_chunk_bf16(const uint32_t (&r)[32], float st,
+                                                   const float *sc, uint4 *o)
+{
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const float4 c0 = reinterpret_cast<const float4 *>(sc)[2 * g];
+        const float4 c1 = reinterpret_cast<const float4 *>(sc)[2 * g + 1];
+        const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            f[i] = dequant_acc<F8>(r[8 * g + i], st, cs[i]);
+        o[g] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+    }
+}
+
+// The int32 accumulators of 32 columns of one output row, written as they are (the check
+// output): columns at or past N are skipped in groups of 8 (N % 8 == 0).
+__device__ __forceinline__ void store_acc_chunk(const uint32_t (&r)[32], int row, int n0, int N,
+                                                int32_t *__restrict__ acc_out)
+{
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+        if (n0 + 8 * g < N) {
+            int4 *ap = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + n0 + 8 * g);
+            ap[0] = make_int4(r[8 * g + 0], r[8 * g + 1], r[8 * g + 2], r[8 * g + 3]);
+            ap[1] = make_int4(r[8 * g + 4], r[8 * g + 5], r[8 * g + 6], r[8 * g + 7]);
+        }
+}
+
+// One warp's 32 output rows of 128 bytes each (lane l holds row l's 8 16-byte chunks in v),
+// stored so that every store instruction writes 4 rows x 128 contiguous bytes instead of 32
+// rows x 16: the chunks pass through the warp's 4 KB shared buffer, their slots XOR-swizzled
+// by row so that neither the writes nor the reads conflict. dst: row 0's first byte; stride:
+// bytes from row to row; rows at or past rows_valid and bytes at or past bytes_valid (a
+// multiple of 16) of a row are not written.
+__device__ __forceinline__ void warp_store_rows(uint4 *stage, const uint4 (&v)[8], int lane,
+                                                char *dst, int64_t stride, int rows_valid,
+                                                int bytes_valid)
+{
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        stage[lane * 8 + (j ^ (lane & 7))] = v[j];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = i * 4 + (lane >> 3), j = lane & 7;
+        if (r < rows_valid && j * 16 < bytes_valid)
+            *reinterpret_cast<uint4 *>(dst + r * stride + j * 16) = stage[r * 8 + (j ^ (r & 7))];
+    }
+    __syncwarp();
 }
 
 // Scales of one output tile for the prefill epilogues, fetched one tile ahead by each
@@ -375,10 +470,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
+                for (int c = 0; c < BN / 32; c += 2) {
+                    // two chunks requested together: one wait for their latency
+                    uint32_t r[32], r2[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, r);
+                    tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r2);
                     tmem_ld_wait();
+                    if (row_ok)
+                        store_row_chunk<F8>(r2, row, nb * BN + (c + 1) * 32, N, st,
+                                            sh_sch + buf * BN + (c + 1) * 32, y, acc_out);
                     if (row_ok)
                         store_row_chunk<F8>(r, row, nb * BN + c * 32, N, st,
                                         sh_sch + buf * BN + c * 32, y, acc_out);
@@ -441,7 +541,9 @@ template <int STAGES> struct PairCfg {
     // barrier and a word for the epilogue group
     static constexpr int kFixBarOff = kBarOff + (2 * STAGES + 4) * 8 + 16;
     static constexpr int kSchOff = (kFixBarOff + 16 + 15) & ~15;
-    static constexpr int kSmemBytes = kSchOff + 4 * 2 * 256 * 4 + 1024; // + scales [4][2][256]
+    // channel scales [4 warps][2][256], then each epilogue warp's 4 KB store staging buffer
+    static constexpr int kOutOff = kSchOff + 4 * 2 * 256 * 4;
+    static constexpr int kSmemBytes = kOutOff + 4 * 4096 + 1024;
     static constexpr int kTmemCols = 512;         // two 128 x 256 accumulators per CTA
     // stream-K: a CTA's partial of a split tile, 128 rows x 256 columns of accumulator words,
     // stored as [64 column quads][128 rows][4] so that the rows of a warp are consecutive
@@ -651,6 +753,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int row_in_tile = static_cast<int>(rank) * Cfg::kHalf + rl;
         float *sh_sch = reinterpret_cast<float *>(smem + Cfg::kSchOff) + (warp - 2) * 2 * TN;
         const int4 *ring = reinterpret_cast<const int4 *>(smem);
+        uint4 *stage_w = reinterpret_cast<uint4 *>(smem + Cfg::kOutOff) + (warp - 2) * 256;
         int4 *my_slot = sk ? reinterpret_cast<int4 *>(ws_part) +
                                  static_cast<int64_t>(blockIdx.x) * (Cfg::kPartBytes / 16)
                            : nullptr;
@@ -732,6 +835,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             const int row = mb * TM + row_in_tile;
             const bool row_ok = row < M && ncon >= 0;
+            const int wrow0 = mb * TM + static_cast<int>(rank) * Cfg::kHalf + quarter * 32;
             // nadd is uniform over the epilogue group (it guards a named barrier); a fixup wait
             // that runs out only keeps this thread from storing
             const int nadd = ncon > 0 ? ncon : 0;
@@ -766,6 +870,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (!mbar_wait(bar_fix, static_cast<uint32_t>(h), limit_ns))
                         ok_h = false;
                 }
+                // the warp's 32 rows go out together (staged stores): which of them are rows
+                // of the output, and whether every lane's values are good
+                const bool ok_w = __all_sync(0xffffffffu, ok_h) && ncon >= 0;
+                const int rows_valid = ok_w ? min(32, M - wrow0) : 0;
                 if constexpr (SILU) {
 #pragma unroll 1
                     for (int p = 2 * h; p < 2 * h + 2; ++p) {
@@ -779,22 +887,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             add_parts(rg, cg, h);
                             add_parts(ru, cg + 2, h);
                         }
-                        if (row_ok && ok_h && ch0 < so.I)
-                            silu_row_chunk<F8>(rg, ru, st, sh_sch + buf * TN + cg * 32,
-                                               sh_sch + buf * TN + (cg + 2) * 32,
-                                               so.a + static_cast<int64_t>(row) * so.I + ch0);
+                        uint4 v[8];
+                        silu_row_chunk_regs<F8>(rg, ru, st, sh_sch + buf * TN + cg * 32,
+                                                sh_sch + buf * TN + (cg + 2) * 32, v);
+                        warp_store_rows(stage_w, v, lane,
+                                        reinterpret_cast<char *>(so.a + static_cast<int64_t>(wrow0) * so.I + ch0),
+                                        static_cast<int64_t>(so.I) * 4, rows_valid,
+                                        min(128, (so.I - ch0) * 4));
                     }
                 } else {
-#pragma unroll 1
-                    for (int c = 4 * h; c < 4 * h + 4; ++c) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(tbase + c * 32, r);
-                        tmem_ld_wait();
-                        if (nadd > 0)
-                            add_parts(r, c, h);
-                        if (row_ok && ok_h)
-                            store_row_chunk<F8>(r, row, nb * TN + c * 32, N, st,
-                                                sh_sch + buf * TN + c * 32, y, acc_out);
+                    // the half's four chunks requested together: one wait for their latency
+                    uint32_t r[4][32];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+                        tmem_ld_32x32b_x32(tbase + (4 * h + cc) * 32, r[cc]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        uint4 v[8];
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int c = 4 * h + 2 * c2 + cc;
+                            if (nadd > 0)
+                                add_parts(r[2 * c2 + cc], c, h);
+                            dequant_chunk_bf16<F8>(r[2 * c2 + cc], st, sh_sch + buf * TN + c * 32,
+                                                   v + 4 * cc);
+                            if (acc_out && row_ok && ok_h)
+                                store_acc_chunk(r[2 * c2 + cc], row, nb * TN + c * 32, N, acc_out);
+                        }
+                        const int n0 = nb * TN + (2 * h + c2) * 64;
+                        warp_store_rows(stage_w, v, lane,
+                                        reinterpret_cast<char *>(y + static_cast<int64_t>(wrow0) * N + n0),
+                                        static_cast<int64_t>(N) * 2, rows_valid, min(128, (N - n0) * 2));
                     }
                 }
                 if (nadd > 0)
@@ -1226,16 +1350,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                     }
                 }
-                // dequantize into the staged output tile [m][128] bf16
+                // dequantize into the staged output tile [m][128] bf16 (two tokens per
+                // conversion instruction)
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < 16; j += 2) {
                     const int m = c0 + j;
                     if (m < mt) {
-                        ysm[m * kBM + r] = static_cast<uint16_t>(
-                            bf16_bits(dequant_acc<F8>(a[j], sh_stok[mbase + m], sc)));
-                        if (acc_out && n_ok)
+                        const uint32_t pr = pack_bf16x2(
+                            dequant_acc<F8>(a[j], sh_stok[mbase + m], sc),
+                            dequant_acc<F8>(a[j + 1], sh_stok[mbase + m + 1], sc));
+                        ysm[m * kBM + r] = static_cast<uint16_t>(pr & 0xFFFFu);
+                        if (m + 1 < mt)
+                            ysm[(m + 1) * kBM + r] = static_cast<uint16_t>(pr >> 16);
+                        if (acc_out && n_ok) {
                             acc_out[static_cast<int64_t>(mbase + m) * N + n] =
                                 static_cast<int32_t>(a[j]);
+                            if (m + 1 < mt)
+                                acc_out[static_cast<int64_t>(mbase + m + 1) * N + n] =
+                                    static_cast<int32_t>(a[j + 1]);
+                        }
                     }
                 }
             };

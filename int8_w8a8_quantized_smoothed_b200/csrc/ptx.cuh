@@ -503,9 +503,21 @@ __device__ __forceinline__ uint32_t bf16_bits(float f)
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
+// Two values to bf16 (round to nearest even) in one conversion instruction: lo in bits 0..15,
+// hi in bits 16..31. The same bits as two bf16_bits, at half the conversion-pipe cost.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
-    return bf16_bits(lo) | (bf16_bits(hi) << 16);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// a and b rounded to bf16 and back (exact), with one conversion instruction.
+__device__ __forceinline__ void bf16_round2(float &a, float &b)
+{
+    const uint32_t r = pack_bf16x2(a, b);
+    a = bf16_lo(r);
+    b = bf16_hi(r);
 }
 
 // y = bf16( (float(acc) * s_tok) * s_ch ), every step binary32 round-to-nearest-even.
