@@ -235,6 +235,8 @@ class Layer:
         a_gu = prep.column_absmax(prep.rmsnorm_calibration(h_cal, g2, EPS))
         self.w = {}
         self.fused = True
+        self.o_norm = True  # o GEMM + residual RMSNorm + quant through one entry point (INT8)
+        self.o_norm_one_launch = False  # ... as the GEMM's row tail (decode sizes)
         for i, (name, (N, K)) in enumerate(P.items()):
             wb = synth.weight_device(N, K, seed + 10 + i, device)
             if name == "qkv":
@@ -306,11 +308,17 @@ class Layer:
             w8.w8a8_gemm_dequant(self.q1, self.s1, *self.w["qkv"], y=self.qkv, workspace=ws)
         if rows:
             w8.w8a8_quantize_rows(self.attn, self.sinv_o, q=self.q2, s_tok=self.s2)
-        if gemms:
-            w8.w8a8_gemm_dequant(self.q2, self.s2, *self.w["o"], y=self.o, workspace=ws)
-        if rows:
-            w8.w8a8_smooth_rmsnorm_quant(self.o, self.g2f, EPS, residual=self.x, h_out=self.h,
-                                         q=self.q3, s_tok=self.s3)
+        if gemms and rows and self.o_norm:
+            # o projection, residual add and the next RMSNorm + quant: one call
+            w8.w8a8_gemm_rmsnorm_quant(self.q2, self.s2, *self.w["o"], self.x, self.g2f, EPS,
+                                       y=self.o, h_out=self.h, q=self.q3, s_out=self.s3,
+                                       workspace=ws, one_launch=self.o_norm_one_launch)
+        else:
+            if gemms:
+                w8.w8a8_gemm_dequant(self.q2, self.s2, *self.w["o"], y=self.o, workspace=ws)
+            if rows:
+                w8.w8a8_smooth_rmsnorm_quant(self.o, self.g2f, EPS, residual=self.x,
+                                             h_out=self.h, q=self.q3, s_tok=self.s3)
         if fused:
             # gate|up GEMM with the SiLU*up epilogue, then its per-token quantization pass
             if gemms:
@@ -469,12 +477,15 @@ def measure_workload(args, name, world, rank, local, primary):
     unfused = args.unfused
     for L in layers:
         L.fused = not unfused
+        L.o_norm_one_launch = args.o_norm_one_launch and L.M <= 64
     ws = w8.Workspace(dev)
     max_ws = max([w8.w8a8_gemm_workspace_size(L.M, N, K) for L in layers
                   for (N, K) in projections(arch).values()] +
                  [w8.w8a8_gemm_fp8_workspace_size(L.M, N, K) for L in layers
                   for (N, K) in projections(arch).values()] +
                  [w8.w8a8_gemm_silu_quant_workspace_size(L.M, arch["I"], arch["H"])
+                  for L in layers] +
+                 [w8.w8a8_gemm_rmsnorm_quant_workspace_size(L.M, arch["H"], arch["H"])
                   for L in layers] +
                  [w8.w8a8_gemm_silu_quant_fp8_workspace_size(L.M, arch["I"], arch["H"])
                   for L in layers])
@@ -530,7 +541,11 @@ def measure_workload(args, name, world, rank, local, primary):
     nbytes = sum(layer_work(arch, L.M)[1] for L in layers)
     g_bytes = sum(layer_work(arch, L.M)[3] for L in layers)
 
-    launches_per_step = (1 if args.fused_block else 8) * len(layers)
+    if args.fused_block:
+        launches_per_step = len(layers)
+    else:  # 8 per layer, 7 where the o GEMM runs the RMSNorm tail in the same launch
+        launches_per_step = sum(8 - (1 if L.o_norm_one_launch and not args.fp8 else 0)
+                                for L in layers)
     h2d = sum(L.x.numel() * 2 + L.attn.numel() * 2 for L in layers)
     d2h = sum(L.down.numel() * 2 for L in layers)
 
@@ -623,6 +638,9 @@ def measure_workload(args, name, world, rank, local, primary):
                    "overlap": args.overlap,
                    "silu_mul_quant": ("separate launch" if unfused else
                                       "fused into the gate|up GEMM epilogue + quantization pass"),
+                   "o_norm": ("residual add + RMSNorm + quant in the o GEMM's row tail "
+                              "(M <= 64)" if args.o_norm_one_launch and not args.fp8 else
+                              "separate launch (the faster form)"),
                    "codes": "FP8 E4M3 (scale absmax / 448)" if args.fp8 else
                             "INT8 (scale absmax / 127)"},
         "tops": round(ops / t_max / 1e12, 3),
@@ -935,6 +953,9 @@ def main(argv=None):
     ap.add_argument("--unfused", action="store_true",
                     help="gate|up GEMM and SiLU*up+quant as separate launches instead of the "
                          "fused SiLU*up epilogue")
+    ap.add_argument("--o-norm-one-launch", action="store_true",
+                    help="the residual RMSNorm + quant in the o GEMM's row tail at M <= 64 "
+                         "(w8a8_gemm_rmsnorm_quant one_launch) instead of a second launch")
     ap.add_argument("--fused-block", action="store_true",
                     help="run each decoder block's linear path as the single fused persistent "
                          "kernel (w8a8_block_decode; M <= 64)")

@@ -252,6 +252,57 @@ W8A8_API int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const in
                                   size_t workspace_bytes, w8a8_stream_t stream);
 
 /*
+ * The o projection's GEMM followed by the residual add and the next smoothed RMSNorm with its
+ * per-token quantization [W8A8 "How we compressed the model" (the INT8 linear); SERVE
+ * "Inter-token latency (ITL)" (the per-layer quantize steps between the GEMMs at decode);
+ * W8A8 "How SmoothQuant prevents outliers in activation tensors" (RMSNorm with gamma / s)].
+ * It computes exactly what this chain of two calls computes:
+ *   y            = w8a8_gemm_dequant(xq, s_tok, wq, s_ch)             bf16 [M, N]
+ *   h_out, q, s_out = w8a8_smooth_rmsnorm_quant(y, residual, h_out, gamma_smoothed, eps)
+ * i.e. h = bf16(y + residual), then the RMSNorm of h (row length N) with gamma_smoothed, then
+ * per-token INT8 codes. Two forms, with identical results:
+ *   one_launch = 0 (w8a8_gemm_rmsnorm_quant): the GEMM, then the row kernel, which the
+ *     dependent launch starts while the GEMM drains. The faster form on B200 at every size
+ *     measured, and the default.
+ *   one_launch = 1: at decode sizes (the cluster split-K plan of w8a8_gemm_dequant: at most 64
+ *     tokens, N <= 8192, few 128-channel blocks; w8a8_gemm_rmsnorm_quant_one_launch_ok(M, N,
+ *     K) returns 1) a single launch: the GEMM's CTAs take a ticket in the workspace once
+ *     their outputs are stored, and the last min(M, 64) of them run the row pass over y (read
+ *     back through L2). Other shapes return W8A8_ERR_UNSUPPORTED_SHAPE. Measured ~1.2-1.9 us
+ *     slower per call than the two launches: the ticket handshake (a release fence, an atomic
+ *     and a poll) costs more than the kernel boundary it removes.
+ * xq, s_tok, wq, s_ch, y: as for w8a8_gemm_dequant (y is written; it must not alias residual
+ * or h_out). residual, h_out: bf16 [M, N], 16-byte aligned; h_out may alias residual.
+ * gamma_smoothed: fp32 [N], 16-byte aligned. q: int8 [M, N], 16-byte aligned; s_out: fp32 [M].
+ * eps >= 0. N must also satisfy the row rules of w8a8_smooth_rmsnorm_quant (N % 16 == 0,
+ * N <= 32768).
+ * workspace: w8a8_gemm_rmsnorm_quant_workspace_size(M, N, K) bytes (at least 4 KiB: the
+ * GEMM's own workspace with its flag words, two of which, words 1022 and 1023, hold the
+ * one-launch form's counters), 16-byte aligned, zero-filled before first use; every completed
+ * call leaves the flag words zero again, so one buffer serves this entry point and
+ * w8a8_gemm_dequant alike, calls issued in order on one stream. After a call that reported
+ * W8A8_ERR_TIMEOUT through w8a8_last_device_status, zero the workspace again.
+ * Errors: W8A8_ERR_INVALID_ARG (NULL pointer, eps < 0 or NaN, y aliasing residual or h_out,
+ * one_launch not 0 or 1), W8A8_ERR_ALIGNMENT, W8A8_ERR_UNSUPPORTED_SHAPE (as for the two
+ * calls, or one_launch = 1 for a shape without the one-launch form), W8A8_ERR_WORKSPACE.
+ */
+W8A8_API size_t w8a8_gemm_rmsnorm_quant_workspace_size(int64_t M, int64_t N, int64_t K);
+W8A8_API int w8a8_gemm_rmsnorm_quant_one_launch_ok(int64_t M, int64_t N, int64_t K);
+W8A8_API int w8a8_gemm_rmsnorm_quant(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                                     const float *s_ch, int64_t M, int64_t N, int64_t K,
+                                     w8a8_bf16 *y, const w8a8_bf16 *residual, w8a8_bf16 *h_out,
+                                     const float *gamma_smoothed, float eps, int8_t *q,
+                                     float *s_out, void *workspace, size_t workspace_bytes,
+                                     w8a8_stream_t stream);
+W8A8_API int w8a8_gemm_rmsnorm_quant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                                        const float *s_ch, int64_t M, int64_t N, int64_t K,
+                                        w8a8_bf16 *y, const w8a8_bf16 *residual,
+                                        w8a8_bf16 *h_out, const float *gamma_smoothed, float eps,
+                                        int8_t *q, float *s_out, void *workspace,
+                                        size_t workspace_bytes, int one_launch,
+                                        w8a8_stream_t stream);
+
+/*
  * ---------------------------------------------------------------- the fused decoder block
  *
  * One Llama decoder block's whole linear path at decode sizes (1 <= M <= 64 tokens) as a single

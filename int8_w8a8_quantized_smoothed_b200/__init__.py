@@ -20,7 +20,9 @@ __all__ = [
     "w8a8_quantize_rows", "w8a8_quantize_rows_static", "w8a8_smooth_rmsnorm_quant", "w8a8_silu_mul_quant",
     "w8a8_gemm_dequant", "w8a8_gemm_dequant_ex", "w8a8_gemm_workspace_size",
     "w8a8_gemm_workspace_size_ex", "w8a8_gemm_dequant_noalloc", "w8a8_gemm_silu_quant",
-    "w8a8_gemm_silu_quant_workspace_size", "w8a8_probe_i8_mma", "w8a8_selftest_wait_timeout", "w8a8_set_overlap",
+    "w8a8_gemm_silu_quant_workspace_size", "w8a8_gemm_rmsnorm_quant",
+    "w8a8_gemm_rmsnorm_quant_workspace_size", "w8a8_gemm_rmsnorm_quant_one_launch_ok",
+    "w8a8_probe_i8_mma", "w8a8_selftest_wait_timeout", "w8a8_set_overlap",
     "w8a8_get_overlap", "w8a8_device_status", "w8a8_last_device_status",
     "w8a8_status_string", "w8a8_version",
     "w8a8_quantize_rows_fp8", "w8a8_smooth_rmsnorm_quant_fp8", "w8a8_silu_mul_quant_fp8",
@@ -52,6 +54,12 @@ SIGNATURES = [
     ("w8a8_gemm_dequant_noalloc", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("w8a8_gemm_silu_quant_workspace_size", _SZ, [_I64, _I64, _I64]),
     ("w8a8_gemm_silu_quant", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    ("w8a8_gemm_rmsnorm_quant_workspace_size", _SZ, [_I64, _I64, _I64]),
+    ("w8a8_gemm_rmsnorm_quant_one_launch_ok", _I, [_I64, _I64, _I64]),
+    ("w8a8_gemm_rmsnorm_quant", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _F, _P,
+                                     _P, _P, _SZ, _P]),
+    ("w8a8_gemm_rmsnorm_quant_ex", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _F,
+                                        _P, _P, _P, _SZ, _I, _P]),
     ("w8a8_gemm_silu_quant_fp8_workspace_size", _SZ, [_I64, _I64, _I64]),
     ("w8a8_gemm_silu_quant_fp8", _I, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ,
                                       _P]),
@@ -452,6 +460,57 @@ def w8a8_gemm_silu_quant(xq, s_tok, wq_il, s_ch_il, a=None, q=None, s_out=None,
         _ptr(xq), _ptr(s_tok), _ptr(wq_il), _ptr(s_ch_il), M, I, K, _ptr(a), _ptr(q),
         _ptr(s_out), _ptr(wbuf), wbytes, _stream(stream)))
     return q, s_out, a
+
+
+def w8a8_gemm_rmsnorm_quant_workspace_size(M: int, N: int, K: int) -> int:
+    return int(lib().w8a8_gemm_rmsnorm_quant_workspace_size(M, N, K))
+
+
+def w8a8_gemm_rmsnorm_quant_one_launch_ok(M: int, N: int, K: int) -> bool:
+    """Whether the one-launch form (the GEMM with the RMSNorm tail) applies to the shape."""
+    return bool(lib().w8a8_gemm_rmsnorm_quant_one_launch_ok(M, N, K))
+
+
+def w8a8_gemm_rmsnorm_quant(xq, s_tok, wq, s_ch, residual, gamma_smoothed, eps, y=None,
+                            h_out=None, q=None, s_out=None, workspace=None, one_launch=False,
+                            stream=None):
+    """The GEMM + dequant into y, then h = bf16(y + residual) and the smoothed RMSNorm of h
+    with per-token quantization: the same y, h, q, s as w8a8_gemm_dequant followed by
+    w8a8_smooth_rmsnorm_quant(y, ..., residual=residual). h_out may be residual (in place).
+    one_launch: the GEMM's last CTAs run the row pass (decode sizes only) instead of a second
+    launch. Returns (q, s_out, h_out, y)."""
+    _need(xq, "xq", torch.int8)
+    _need(wq, "wq", torch.int8)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2:
+        raise ValueError(f"xq [M,K] and wq [N,K] disagree: {tuple(xq.shape)} {tuple(wq.shape)}")
+    _need(s_tok, "s_tok", torch.float32, (M,))
+    _need(s_ch, "s_ch", torch.float32, (N,))
+    _need(residual, "residual", torch.bfloat16, (M, N))
+    _need(gamma_smoothed, "gamma_smoothed", torch.float32, (N,))
+    e = dict(device=xq.device)
+    y = torch.empty((M, N), dtype=torch.bfloat16, **e) if y is None else y
+    h_out = torch.empty((M, N), dtype=torch.bfloat16, **e) if h_out is None else h_out
+    q = torch.empty((M, N), dtype=torch.int8, **e) if q is None else q
+    s_out = torch.empty(M, dtype=torch.float32, **e) if s_out is None else s_out
+    _need(y, "y", torch.bfloat16, (M, N))
+    _need(h_out, "h_out", torch.bfloat16, (M, N))
+    _need(q, "q", torch.int8, (M, N))
+    _need(s_out, "s_out", torch.float32, (M,))
+    need = w8a8_gemm_rmsnorm_quant_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = _workspace_for(xq.device)
+    if isinstance(workspace, Workspace):
+        wbuf, wbytes = workspace.get(need)
+    else:
+        wbuf, wbytes = workspace, (0 if workspace is None else workspace.numel()
+                                   * workspace.element_size())
+    _check("w8a8_gemm_rmsnorm_quant_ex", lib().w8a8_gemm_rmsnorm_quant_ex(
+        _ptr(xq), _ptr(s_tok), _ptr(wq), _ptr(s_ch), M, N, K, _ptr(y), _ptr(residual),
+        _ptr(h_out), _ptr(gamma_smoothed), float(eps), _ptr(q), _ptr(s_out), _ptr(wbuf), wbytes,
+        1 if one_launch else 0, _stream(stream)))
+    return q, s_out, h_out, y
 
 
 def w8a8_gemm_silu_quant_fp8_workspace_size(M: int, I: int, K: int) -> int:

@@ -30,6 +30,7 @@
 
 #include "ptx.cuh"
 #include "rowquant.cuh"
+#include "rowpass.cuh"
 
 namespace w8a8 {
 
@@ -47,6 +48,20 @@ struct SiluOut {
     float *a;
     int I;
     float *amax = nullptr;
+};
+
+// The residual RMSNorm tail of the decode GEMM (cluster split-K): with y [M, N] the GEMM's
+// output, h = bf16(y + res) (written to h, which may alias res), then the smoothed RMSNorm of
+// h with gamma' (gamma divided by the next layer's smoothing factors) quantized per token
+// into q [M, N], s [M]. bar: two zero-initialized counter words (tickets, then departures).
+struct RowNormOut {
+    const uint16_t *res = nullptr;
+    uint16_t *h = nullptr;
+    const float *gamma = nullptr;
+    float eps = 0.0f;
+    int8_t *q = nullptr;
+    float *s = nullptr;
+    unsigned int *bar = nullptr;
 };
 
 __device__ __forceinline__ float bf16_round(float f)
@@ -1032,16 +1047,20 @@ __device__ __forceinline__ void silu_block_rows(int m0, int mt, int t, int etid,
     }
 }
 
-template <int NT, int STAGES, int KPS, bool CLUSTER, bool SILU = false, bool F8 = false>
+template <int NT, int STAGES, int KPS, bool CLUSTER, bool SILU = false, bool F8 = false,
+          int RNV = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmX, const float *__restrict__ s_tok,
                        const float *__restrict__ s_ch, int M, int N, int K,
                        uint16_t *__restrict__ y, int32_t *__restrict__ acc_out,
                        int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
-                       SiluOut so, int prefetch_static, unsigned long long limit_ns)
+                       SiluOut so, RowNormOut rn, int prefetch_static, unsigned long long limit_ns)
 {
     static_assert(!(SILU && F8 && CLUSTER), "the fused SiLU epilogue of the FP8 cluster split-K is not built");
+    // RNV > 0: the residual RMSNorm tail, rows of up to 8 * 128 * RNV values (INT8 cluster
+    // split-K with the plain epilogue only)
+    static_assert(RNV == 0 || (CLUSTER && !SILU && !F8), "the RMSNorm tail is built for the INT8 cluster split-K");
     using Cfg = DecodeCfg<NT, STAGES, KPS, CLUSTER>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -1551,6 +1570,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+    if constexpr (RNV > 0) {
+        // The residual RMSNorm of the output rows, by the last CTAs to finish. Every CTA takes
+        // a ticket once its output stores are done (the barrier above orders them before
+        // thread 0's release); the CTAs holding the last R tickets (R = min(M, 64, grid))
+        // wait until every ticket is taken, then run rows slot, slot + R, ... reading y back
+        // through L2. The others exit at once. The last row CTA to finish zeroes both
+        // counters for the next call.
+        const unsigned int total = gridDim.x * gridDim.y;
+        const unsigned int R = min(min(static_cast<unsigned int>(M), 64u), total);
+        volatile uint32_t *sh_ok = tslot_ptr + 5;
+        if (threadIdx.x == 0) {
+            fence_acq_rel_gpu();
+            *sh_word = atomicAdd(rn.bar, 1u);
+        }
+        __syncthreads();
+        const unsigned int ticket = *sh_word;
+        if (ticket + R >= total && warp >= 2) {
+            const int etid = threadIdx.x - 64;
+            const int slot = static_cast<int>(ticket - (total - R));
+            // the first row's residual and gamma' do not depend on y: requested before the wait
+            RmsRow<RNV> row;
+            rms_row_load_side<RNV>(rn.res + static_cast<int64_t>(slot) * N, rn.gamma, N, etid, row);
+            if (etid == 0) {
+                bool all = true;
+                if (ld_acquire_gpu(rn.bar) < total) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(rn.bar) < total) {
+                        if (globaltimer_ns() - t0 > limit_ns) {
+                            flag_timeout();
+                            all = false;
+                            break;
+                        }
+                    }
+                }
+                *sh_ok = all ? 1u : 0u;
+            }
+            named_bar_sync(1, 128);
+            // reductions' scratch: the (idle) stage ring
+            double *shd = reinterpret_cast<double *>(smem);
+            float *shf = reinterpret_cast<float *>(smem + 64);
+            if (*sh_ok != 0u) {
+                for (int m = slot; m < M; m += static_cast<int>(R)) {
+                    const int64_t off = static_cast<int64_t>(m) * N;
+                    if (m != slot)
+                        rms_row_load_side<RNV>(rn.res + off, rn.gamma, N, etid, row);
+                    rms_row_load_x<RNV>(y + off, true, N, etid, row);
+                    rms_row_finish<RNV>(row, true, rn.h + off, rn.eps, N, rn.q + off, rn.s + m,
+                                        etid, shd, shf);
+                }
+            }
+            named_bar_sync(1, 128);
+            if (etid == 0 && atom_add_acq_rel_gpu(rn.bar + 1, 1u) == R - 1) {
+                // every ticket is taken and every row CTA is past its wait
+                rn.bar[0] = 0u;
+                rn.bar[1] = 0u;
+            }
+        }
     }
 }
 

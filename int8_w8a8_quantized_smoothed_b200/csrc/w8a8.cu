@@ -581,18 +581,25 @@ int fit_cluster(Kern kernel, int want, int64_t clusters_needed, int smem, int de
     return 1;
 }
 
-template <int NT, int STAGES, int KPS, bool SILU, bool F8 = false>
+// RNV > 0: the cluster split-K with the residual RMSNorm tail (rn), rows of up to 1024 RNV
+// values; only the INT8 plain-epilogue cluster plans take it.
+template <int NT, int STAGES, int KPS, bool SILU, bool F8 = false, int RNV = 0>
 int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
                   const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
-                  uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev, cudaStream_t st)
+                  uint16_t *y, int32_t *acc, void *ws, const SiluOut &so, int dev, cudaStream_t st,
+                  const RowNormOut &rn = RowNormOut{})
 {
     const int prefetch = g_overlap.load(std::memory_order_relaxed) >= 2 ? 1 : 0;
+    if constexpr (RNV > 0) {
+        if (p.variant != 3)
+            return W8A8_ERR_UNSUPPORTED_SHAPE;
+    }
     if constexpr (SILU && F8) {
         if (p.variant == 3) // the FP8 cluster split-K has no SiLU epilogue: planned away
             return W8A8_ERR_UNSUPPORTED_SHAPE;
     } else if (p.variant == 3) {
         using Cfg = DecodeCfg<NT, STAGES, KPS, true>;
-        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU, F8>;
+        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, true, SILU, F8, RNV>;
         if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
             return rc;
         const int64_t NB = ((N + kBM - 1) / kBM) * ((M + NT - 1) / NT); // x token tiles
@@ -601,22 +608,25 @@ int launch_decode(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_t
                                      Cfg::kSmemBytes, st, static_cast<unsigned>(S), tw, tx, s_tok,
                                      s_ch, static_cast<int>(M), static_cast<int>(N),
                                      static_cast<int>(K), y, acc, static_cast<int32_t *>(nullptr),
-                                     static_cast<unsigned int *>(nullptr), so, prefetch,
+                                     static_cast<unsigned int *>(nullptr), so, rn, prefetch,
                                      kWaitLimitNs);
     }
-    using Cfg = DecodeCfg<NT, STAGES, KPS, false>;
-    auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false, SILU, F8>;
-    if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
-        return rc;
-    int32_t *ws_part =
-        p.ws_bytes ? reinterpret_cast<int32_t *>(static_cast<char *>(ws) + p.part_off) : nullptr;
-    unsigned int *ws_flag =
-        p.ws_bytes ? reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.flag_off)
-                   : nullptr;
-    return launch_kernel(kernel, dim3(p.ctas), dim3(kGemmThreads), Cfg::kSmemBytes, st, tw, tx,
-                         s_tok, s_ch, static_cast<int>(M), static_cast<int>(N),
-                         static_cast<int>(K), y, acc, ws_part, ws_flag, so, prefetch,
-                         kWaitLimitNs);
+    if constexpr (RNV == 0) {
+        using Cfg = DecodeCfg<NT, STAGES, KPS, false>;
+        auto kernel = gemm_decode_kernel<NT, STAGES, KPS, false, SILU, F8>;
+        if (int rc = ensure_smem(reinterpret_cast<const void *>(kernel), dev, Cfg::kSmemBytes))
+            return rc;
+        int32_t *ws_part =
+            p.ws_bytes ? reinterpret_cast<int32_t *>(static_cast<char *>(ws) + p.part_off) : nullptr;
+        unsigned int *ws_flag =
+            p.ws_bytes ? reinterpret_cast<unsigned int *>(static_cast<char *>(ws) + p.flag_off)
+                       : nullptr;
+        return launch_kernel(kernel, dim3(p.ctas), dim3(kGemmThreads), Cfg::kSmemBytes, st, tw, tx,
+                             s_tok, s_ch, static_cast<int>(M), static_cast<int>(N),
+                             static_cast<int>(K), y, acc, ws_part, ws_flag, so, RowNormOut{},
+                             prefetch, kWaitLimitNs);
+    }
+    return W8A8_ERR_UNSUPPORTED_SHAPE;
 }
 
 // Decode launch by token tile: (stages, k-blocks per stage) keep ~200 KB of weight and
@@ -633,6 +643,25 @@ int launch_decode_nt(const CUtensorMap &tw, const CUtensorMap &tx, const float *
     case 64: return launch_decode<64, 4, 2, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
     case 128: return launch_decode<128, 5, 1, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
     default: return launch_decode<256, 3, 1, SILU, F8>(tw, tx, s_tok, s_ch, M, N, K, p, y, acc, ws, so, dev, st);
+    }
+}
+
+// The INT8 cluster split-K GEMM with the residual RMSNorm tail: token tiles of at most 64,
+// rows of at most 8192 values.
+int launch_decode_rn(const CUtensorMap &tw, const CUtensorMap &tx, const float *s_tok,
+                     const float *s_ch, int64_t M, int64_t N, int64_t K, const GemmPlan &p,
+                     uint16_t *y, const RowNormOut &rn, int dev, cudaStream_t st)
+{
+    const SiluOut none{nullptr, 0};
+    const bool wide = N > 4096;
+    switch (p.nt) {
+    case 16: return wide ? launch_decode<16, 3, 4, false, false, 8>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, nullptr, none, dev, st, rn)
+                         : launch_decode<16, 3, 4, false, false, 4>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, nullptr, none, dev, st, rn);
+    case 32: return wide ? launch_decode<32, 5, 2, false, false, 8>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, nullptr, none, dev, st, rn)
+                         : launch_decode<32, 5, 2, false, false, 4>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, nullptr, none, dev, st, rn);
+    case 64: return wide ? launch_decode<64, 4, 2, false, false, 8>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, nullptr, none, dev, st, rn)
+                         : launch_decode<64, 4, 2, false, false, 4>(tw, tx, s_tok, s_ch, M, N, K, p, y, nullptr, nullptr, none, dev, st, rn);
+    default: return W8A8_ERR_UNSUPPORTED_SHAPE;
     }
 }
 
@@ -1031,6 +1060,111 @@ int w8a8_gemm_silu_quant(const int8_t *xq, const float *s_tok, const int8_t *wq_
     case 2: return launch_quantize_f32<2>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
     default: return launch_quantize_f32<4>(a, M, (int)I, q, s_out, L.threads, dev, sms, st);
     }
+}
+
+// ------------------------------------------------------------------ GEMM + residual RMSNorm
+
+// The RMSNorm tail's two counter words: the last two flag words, which no stream-K plan
+// reaches (its CTAs, at most one per SM, use the words 0 .. grid - 1).
+constexpr size_t kRowBarWord = kMaxCtas - 2;
+
+// Whether the one-launch form (the cluster split-K with the RMSNorm tail) applies.
+bool gemm_rn_fused(const GemmPlan &p, int64_t N, int sms)
+{
+    return p.variant == 3 && p.nt <= 64 && N <= 8192 && sms <= static_cast<int>(kRowBarWord);
+}
+
+size_t w8a8_gemm_rmsnorm_quant_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    if (check_gemm_shape(M, N, K) || check_row_shape(M, N))
+        return 0;
+    int dev, sms = 148;
+    if (current_device(&dev, &sms))
+        sms = 148;
+    GemmPlan p;
+    if (plan_gemm(M, N, K, 0, 0, 0, sms, &p))
+        return 0;
+    return p.ws_bytes > kFlagBytes ? p.ws_bytes : kFlagBytes;
+}
+
+int w8a8_gemm_rmsnorm_quant_one_launch_ok(int64_t M, int64_t N, int64_t K)
+{
+    if (check_gemm_shape(M, N, K) || check_row_shape(M, N))
+        return 0;
+    int dev, sms = 148;
+    if (current_device(&dev, &sms))
+        sms = 148;
+    GemmPlan p;
+    if (plan_gemm(M, N, K, 0, 0, 0, sms, &p))
+        return 0;
+    return gemm_rn_fused(p, N, sms) ? 1 : 0;
+}
+
+int w8a8_gemm_rmsnorm_quant_ex(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                               const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
+                               const w8a8_bf16 *residual, w8a8_bf16 *h_out,
+                               const float *gamma_smoothed, float eps, int8_t *q, float *s_out,
+                               void *workspace, size_t workspace_bytes, int one_launch,
+                               w8a8_stream_t stream)
+{
+    if (one_launch != 0 && one_launch != 1)
+        return W8A8_ERR_INVALID_ARG;
+    if (!xq || !s_tok || !wq || !s_ch || !y || !residual || !h_out || !gamma_smoothed || !q ||
+        !s_out || !(eps >= 0.0f))
+        return W8A8_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc || (rc = check_row_shape(M, N)))
+        return rc;
+    if (!aligned16(xq) || !aligned16(wq) || !aligned16(s_ch) || !aligned16(y) ||
+        !aligned16(residual) || !aligned16(h_out) || !aligned16(gamma_smoothed) ||
+        !aligned16(q) || (workspace && !aligned16(workspace)))
+        return W8A8_ERR_ALIGNMENT;
+    // h_out may alias residual (in place); y is written by the GEMM and read by the row pass
+    if (static_cast<const void *>(h_out) == static_cast<const void *>(y) ||
+        static_cast<const void *>(residual) == static_cast<const void *>(y))
+        return W8A8_ERR_INVALID_ARG;
+    int dev, sms;
+    if ((rc = current_device(&dev, &sms)))
+        return rc;
+    GemmPlan p;
+    if ((rc = plan_gemm(M, N, K, 0, 0, 0, sms, &p)))
+        return rc;
+    const size_t need = p.ws_bytes > kFlagBytes ? p.ws_bytes : kFlagBytes;
+    if (workspace == nullptr || workspace_bytes < need)
+        return W8A8_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (one_launch) {
+        if (!gemm_rn_fused(p, N, sms))
+            return W8A8_ERR_UNSUPPORTED_SHAPE;
+        CUtensorMap tw, tx;
+        if (encode_kmajor_i8(&tw, wq, N, K, kBM) || encode_kmajor_i8(&tx, xq, M, K, p.nt))
+            return W8A8_ERR_CUDA;
+        RowNormOut rn;
+        rn.res = residual;
+        rn.h = h_out;
+        rn.gamma = gamma_smoothed;
+        rn.eps = eps;
+        rn.q = q;
+        rn.s = s_out;
+        rn.bar = static_cast<unsigned int *>(workspace) + kRowBarWord;
+        return launch_decode_rn(tw, tx, s_tok, s_ch, M, N, K, p, y, rn, dev, st);
+    }
+    if ((rc = gemm_run(xq, s_tok, wq, s_ch, M, N, K, y, nullptr, workspace, p, nullptr, dev, sms,
+                       st)))
+        return rc;
+    return rmsnorm_quant_impl<false>(y, residual, h_out, gamma_smoothed, eps, M, N, q, s_out,
+                                     stream);
+}
+
+int w8a8_gemm_rmsnorm_quant(const int8_t *xq, const float *s_tok, const int8_t *wq,
+                            const float *s_ch, int64_t M, int64_t N, int64_t K, w8a8_bf16 *y,
+                            const w8a8_bf16 *residual, w8a8_bf16 *h_out,
+                            const float *gamma_smoothed, float eps, int8_t *q, float *s_out,
+                            void *workspace, size_t workspace_bytes, w8a8_stream_t stream)
+{
+    return w8a8_gemm_rmsnorm_quant_ex(xq, s_tok, wq, s_ch, M, N, K, y, residual, h_out,
+                                      gamma_smoothed, eps, q, s_out, workspace, workspace_bytes,
+                                      0, stream);
 }
 
 // The FP8 fused gate|up plan: as the GEMM's own, with stream-K in place of the cluster
