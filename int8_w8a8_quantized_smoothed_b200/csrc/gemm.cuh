@@ -176,15 +176,21 @@ template <int BN, int STAGES> struct PrefillCfg {
 // at the same time share A row-panels and B column-panels in L2.
 constexpr int kGroupM = 16;
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int &mb, int &nb)
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int &mb,
+                                            int &nb)
 {
-    const int per_group = kGroupM * num_n;
+    const int per_group = group_m * num_n;
     const int group = tile / per_group;
-    const int first_m = group * kGroupM;
-    const int gm = min(kGroupM, num_m - first_m);
+    const int first_m = group * group_m;
+    const int gm = min(group_m, num_m - first_m);
     const int local = tile - group * per_group;
     mb = first_m + local % gm;
     nb = local / gm;
+}
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int &mb, int &nb)
+{
+    tile_coords(tile, num_m, num_n, kGroupM, mb, nb);
 }
 
 // Dequantizes 32 accumulator columns of one output row and stores them as bf16 (16-byte
@@ -589,7 +595,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              int M, int N, int K, uint16_t *__restrict__ y,
                              int32_t *__restrict__ acc_out, SiluOut so,
                              int32_t *__restrict__ ws_part, unsigned int *__restrict__ ws_flag,
-                             int prefetch_static, unsigned long long limit_ns)
+                             int group_m, int prefetch_static, unsigned long long limit_ns)
 {
     using Cfg = PairCfg<STAGES>;
     constexpr int TN = 256, TM = 256;
@@ -678,7 +684,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 int t, kb0, kb1;
                 while (npre < STAGES && next_seg(cur, t, kb0, kb1)) {
                     int mb, nb;
-                    tile_coords(t, num_m, num_n, mb, nb);
+                    tile_coords(t, num_m, num_n, group_m, mb, nb);
                     for (int kb = kb0; kb < kb1 && npre < STAGES; ++kb, ++npre) {
                         if (rank == 0)
                             mbar_expect_tx(bar_full + 8 * npre, 2 * Cfg::kStageBytes);
@@ -694,7 +700,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int t, kb0, kb1;
             while (ok && next_seg(cur, t, kb0, kb1)) {
                 int mb, nb;
-                tile_coords(t, num_m, num_n, mb, nb);
+                tile_coords(t, num_m, num_n, group_m, mb, nb);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const uint32_t s = it % STAGES;
                     if (it < npre) {
@@ -775,7 +781,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         TileScales<TN> nxt;
         auto fetch = [&](int tile) {
             int mb, nb;
-            tile_coords(tile, num_m, num_n, mb, nb);
+            tile_coords(tile, num_m, num_n, group_m, mb, nb);
             nxt.fetch(s_ch, s_tok, nb * TN, N, mb * TM + row_in_tile, M, lane);
         };
         int64_t peek = u_begin, cur = u_begin;
@@ -785,7 +791,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t seg = 0;
         while (next_seg(cur, t, kb0, kb1)) {
             int mb, nb;
-            tile_coords(t, num_m, num_n, mb, nb);
+            tile_coords(t, num_m, num_n, group_m, mb, nb);
             const uint32_t buf = seg & 1u;
             const uint32_t aph = (seg >> 1) & 1u;
             ++seg;
