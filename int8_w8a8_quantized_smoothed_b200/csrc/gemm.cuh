@@ -1127,6 +1127,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(tslot_ptr);
+    // Cluster split-K: an owner thread dequantizes 4 channels, the same 4 for every row it
+    // handles; their scales are read when the epilogue starts, not after the reduction.
+    float4 cl_sc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -1232,6 +1235,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int r = quarter * 32 + lane; // channel within the block
         for (int i = etid; i < M; i += 128)
             sh_stok[i] = __ldg(s_tok + i);
+        if constexpr (CLUSTER) {
+            const int n = static_cast<int>((blockIdx.y / TT) * kBM) + (etid % (kBM / 4)) * 4;
+            if (n < N)
+                cl_sc = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
+        }
         named_bar_sync(1, 128);
         // tokens of block b's tile held in the accumulator (tile b % TT)
         auto tile_tokens = [&](int64_t b) {
@@ -1481,7 +1489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         s4.z = acc_add<true>(s4.z, p4.z);
                         s4.w = acc_add<true>(s4.w, p4.w);
                     }
-                    const float4 c4 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
+                    const float4 c4 = cl_sc; // the scales of channels n .. n + 3
                     const float st = sh_stok[m];
                     uint2 o;
                     o.x = bf16_bits(dequant_acc<true>(s4.x, st, c4.x)) |
@@ -1553,7 +1561,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int n = tch * kBM + c;
                 if (n < N) { // N % 8 == 0: the 4 channels are all valid or all past N
                     const int4 s4 = *reinterpret_cast<const int4 *>(P + ml * kBM + c);
-                    const float4 c4 = __ldg(reinterpret_cast<const float4 *>(s_ch + n));
+                    const float4 c4 = cl_sc; // the scales of channels n .. n + 3
                     const float st = sh_stok[m];
                     uint2 o;
                     o.x = bf16_bits(dequant_f32(s4.x, st, c4.x)) |
