@@ -51,7 +51,7 @@ WORKLOADS = {
 # DRAM bytes (read + write, ncu dram__bytes_read.sum + dram__bytes_write.sum) per GEMM launch,
 # averaged over the GEMM launches of one step of the workload, as captured with the current
 # GEMM kernels; None where no capture exists. Re-capture whenever a GEMM kernel changes.
-NCU_GEMM_TRAFFIC = {"decode8b": 54.86e6, "prefill8b": 235.5e6}
+NCU_GEMM_TRAFFIC = {"decode8b": 54.86e6, "prefill8b": 226.2e6}
 
 # Measured peaks (driver-written); fallbacks are the pool's earlier measurements.
 FALLBACK_HBM_GBS = 6650.0
