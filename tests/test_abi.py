@@ -101,6 +101,42 @@ def test_valid_call_without_gpu_reports_no_device(L):
     assert L.w8a8_device_status(0) == -7
 
 
+def test_gemm_rmsnorm_quant_host_checks(L):
+    # the o projection + residual RMSNorm entry point: argument checks, then the device
+    Y, R, H, G, Q, S, W = (_p(A + i * 0x100000) for i in range(7))
+    ws = 1 << 20
+
+    def call(M=4, N=1024, K=512, y=Y, res=R, h=H, eps=1e-5, one=0, wbytes=ws, g=G):
+        return L.w8a8_gemm_rmsnorm_quant_ex(_p(A), _p(A), _p(A), _p(A), M, N, K, y, res, h, g,
+                                            C.c_float(eps), Q, S, W, wbytes, one, None)
+
+    assert call(g=None) == -1                      # a null pointer
+    assert call(eps=-1.0) == -1                    # eps < 0
+    assert call(eps=float("nan")) == -1
+    assert call(one=2) == -1                       # the form selector
+    assert call(y=R) == -1                         # y may not alias the residual ...
+    assert call(h=Y) == -1                         # ... nor h_out
+    assert call(N=1032) == -3                      # rows of N % 16 != 0
+    assert call(K=40) == -3                        # the GEMM's K % 16
+    assert call(h=_p(A + 0x600008)) == -2          # a misaligned output
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == -7                        # valid: no device here
+        assert call(h=R) == -7                     # h_out may alias the residual
+
+
+def test_gemm_rmsnorm_quant_one_launch_plan(L):
+    # the one-launch form is the cluster split-K plan (M <= 64, few channel blocks, N <= 8192)
+    ok = L.w8a8_gemm_rmsnorm_quant_one_launch_ok
+    assert ok(1, 4096, 4096) == 1 and ok(64, 4096, 4096) == 1 and ok(5, 8192, 1024) == 1
+    assert ok(65, 4096, 4096) == 0                 # tile kernels
+    assert ok(4, 12288, 512) == 0                  # rows wider than 8192
+    assert ok(3, 1024, 128) == 0                   # one k-block: the stream-K plan
+    assert ok(4, 1032, 512) == 0                   # invalid row length
+    assert L.w8a8_gemm_rmsnorm_quant_workspace_size(16, 4096, 4096) >= 4096
+    assert L.w8a8_gemm_rmsnorm_quant_workspace_size(4, 1032, 512) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
